@@ -1,0 +1,421 @@
+"""Benchmark: paged GQA decode (Llama-3.1-70B shapes) through libsplitkv on B200.
+
+One step = the decode workload run twice, as the configuration states: K/V with identical
+strides, then V as a strided column slice of a 2x-wide buffer (independent strides).  Each run is
+the attention kernel (split-KV partials) followed by the plan's merge pass.  Batch 64, q_len 1,
+64 query / 8 KV heads, head_dim 128, page_size 16, KV lengths U[1024, 8192], permuted pages,
+bf16 N(0,1) data (seeded, synthetic).  The KV cache is resident device state (uploaded once);
+the KV working set (2 x 1.2 GB) is far larger than the 126 MB L2, so every step reads it from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...     (one rank per GPU, weak scaling)
+
+Prints ONE JSON line (rank 0).  ``value`` = achieved KV GB/s over all ranks (algorithmic KV bytes:
+exactly L_r tokens x Hk x D x 2 tensors x 2 bytes per request, per run) / max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: achieved KV GB/s (% of HBM peak), µs per decode step"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+KERNEL_SOURCES = ["split_kv_merge_b200/csrc/gqa_tc_decode.cu", "split_kv_merge_b200/csrc/gqa_simt.cu"]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def _kernel_hash(paths):
+    h = hashlib.sha256()
+    for rel in paths:
+        p = os.path.join(ROOT, rel)
+        if os.path.exists(p):
+            with open(p, "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_record(kernel_name, src_hash):
+    """DRAM bytes per launch from the committed ncu summary, only if it was taken on this exact
+    kernel source (else null)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        recs = json.load(f)
+    r = recs.get(kernel_name)
+    if not r or r.get("source_hash") != src_hash:
+        return None
+    return r
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() in ("active", "1", "yes"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _physical_gpu(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in vis.split(",") if x.strip()]
+    if local < len(ids) and ids[local].isdigit():
+        return int(ids[local])
+    return local
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _kv_bytes(case):
+    L = case.kv_lengths()
+    return int(L.sum()) * case.num_kv_heads * case.head_dim * 2 * 2
+
+
+def _cpu_baseline(cases, budget_s=12.0):
+    """The oracle as it stands, on the host cores, over a bounded sample of the same workload:
+    requests of both stride variants in order until ~budget_s seconds have passed."""
+    import oracle.attention as OA
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    done_bytes, n_req, t0 = 0, 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        for c in cases:
+            for r in range(c.batch):
+                OA.paged_attention(c.q, c.k, c.v, c.qo_indptr, c.kv_indptr, c.kv_indices, c.kv_last_page_len,
+                                   c.page_size, c.sm_scale, requests=[r])
+                L = int(c.kv_lengths()[r])
+                done_bytes += L * c.num_kv_heads * c.head_dim * 4
+                n_req += 1
+                if time.perf_counter() - t0 >= budget_s:
+                    break
+            if time.perf_counter() - t0 >= budget_s:
+                break
+    dt = time.perf_counter() - t0
+    return {"value": done_bytes / dt / 1e9, "unit": "GB/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"{n_req} requests of the same decode workload (float64 numpy oracle, "
+                      f"{dt:.1f} s, {os.cpu_count()} host cores visible)"}
+
+
+def _make_cases(rank: int):
+    from workloads import llama70b_decode_case
+    seed = 2 + 1000 * rank   # each rank holds its own batch of 64 requests (weak scaling)
+    return [llama70b_decode_case(independent_v=False, seed=seed), llama70b_decode_case(independent_v=True, seed=seed)]
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    cases = _make_cases(0)
+    per_step = []
+    budget = max(0.2, min(args.ref_budget, 150.0 / (args.steps + args.warmup)))   # whole run ~ minutes
+    for _ in range(args.warmup):
+        _cpu_baseline(cases, budget_s=budget)
+    for _ in range(args.steps):
+        per_step.append(_cpu_baseline(cases, budget_s=budget))
+    value = statistics.median(x["value"] for x in per_step)
+    kv = sum(_kv_bytes(c) for c in cases)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": kv / (value * 1e9) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(cases, None),
+            "cpu_baseline": {**per_step[-1], "value": value},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(cases, plans):
+    c = cases[0]
+    L = c.kv_lengths()
+    cfg = {"workload": "Llama-3.1-70B-shaped paged decode, run twice per step (equal K/V strides; V a column "
+                       "slice of a 2x-wide buffer)",
+           "batch": c.batch, "q_len": 1, "num_qo_heads": c.num_qo_heads, "num_kv_heads": c.num_kv_heads,
+           "head_dim": c.head_dim, "page_size": c.page_size, "kv_len_range": [1024, 8192],
+           "kv_tokens_per_run": int(L.sum()), "kv_bytes_per_step": sum(_kv_bytes(x) for x in cases),
+           "l2": "no flush: 2.4 GB KV working set per step > 126 MB L2", "parallelism": "replicas (independent "
+                                                                                    "request batches per GPU)"}
+    if plans is not None:
+        cfg["split_policy"] = "balanced"
+        cfg["plans"] = [p.info.as_dict() for p in plans]
+    return cfg
+
+
+def run_ours(args):
+    import torch
+    import split_kv_merge_b200 as skv
+    from workloads.device import paged_to_device
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cases = _make_cases(rank)
+    kv_bytes_step = sum(_kv_bytes(c) for c in cases)
+    runs = []
+    for c in cases:
+        d = paged_to_device(c, dev)
+        plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, c.page_size, c.num_qo_heads,
+                              c.num_kv_heads, c.head_dim, "balanced", 0).to(dev)
+        n_part = plan.info.num_partial_rows
+        o = torch.empty(c.q.shape[0], c.num_qo_heads, c.head_dim, dtype=torch.float32, device=dev)
+        lse = torch.empty(c.q.shape[0], c.num_qo_heads, dtype=torch.float32, device=dev)
+        o_part = torch.empty(max(1, n_part), c.num_qo_heads, c.head_dim, dtype=torch.float32, device=dev)
+        lse_part = torch.empty(max(1, n_part), c.num_qo_heads, dtype=torch.float32, device=dev)
+        runs.append(dict(c=c, d=d, plan=plan, o=o, lse=lse, o_part=o_part, lse_part=lse_part))
+    stream = torch.cuda.current_stream(dev)
+
+    def launch(run, ev=None):
+        c, d = run["c"], run["d"]
+        skv.paged_attn_fwd(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"], d["kv_last_page_len"],
+                           run["plan"], run["o"], run["lse"], run["o_part"], run["lse_part"], None, c.sm_scale,
+                           c.num_pages, stream, phase="partial")
+        if ev is not None:
+            ev.record(stream)
+        skv.merge_plan(run["o_part"], run["lse_part"], run["plan"], c.num_qo_heads, c.head_dim, run["o"],
+                       run["lse"], stream)
+
+    for _ in range(args.warmup):
+        for run in runs:
+            launch(run)
+    torch.cuda.synchronize(dev)
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    # ---------------------------------------------------------------- device-timed region
+    n_ev = args.steps * len(runs)
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(_physical_gpu(local)) as clk:
+        time.sleep(0.15)
+        start.record(stream)
+        i = 0
+        for _ in range(args.steps):
+            for run in runs:
+                ev_a[i].record(stream)
+                launch(run, ev_b[i])
+                ev_c[i].record(stream)
+                i += 1
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        time.sleep(0.1)
+    barrier()
+    total_ms = start.elapsed_time(end)
+    attn_ms = [ev_a[j].elapsed_time(ev_b[j]) for j in range(n_ev)]
+    merge_ms = [ev_b[j].elapsed_time(ev_c[j]) for j in range(n_ev)]
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    total_bytes = kv_bytes_step * args.steps * ws
+    value = total_bytes / (total_ms * 1e-3) / 1e9
+    ms_per_step = total_ms / args.steps
+
+    # ---------------------------------------------------------------- end-to-end through the public API
+    e2e = _e2e(args, runs, dev, stream, skv, torch)
+
+    if rank != 0:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+    peaks, peak_src = _peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]))
+    attn_avg_ms = statistics.mean(attn_ms)
+    per_launch_bytes = kv_bytes_step / len(runs)
+    achieved = per_launch_bytes / (attn_avg_ms * 1e-3) / 1e9
+    kernel = "gqa_tc_decode" if runs[0]["plan"].info.kernel == 2 else "gqa_simt_kernel"
+    src_hash = _kernel_hash(KERNEL_SOURCES)
+    tr = _traffic_record(kernel, src_hash)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(cases, [r["plan"] for r in runs]),
+        "us_per_step": round(ms_per_step * 1e3, 2),
+        "us_per_run": {"equal_strides": round(statistics.median(
+            [a + m for a, m in zip(attn_ms[0::2], merge_ms[0::2])]) * 1e3, 2),
+            "independent_v_strides": round(statistics.median(
+                [a + m for a, m in zip(attn_ms[1::2], merge_ms[1::2])]) * 1e3, 2)},
+        "pct_hbm": {"of_nominal_8TBps": round(100 * value / ws / NOMINAL_HBM_GBS, 2),
+                    f"of_{peak_src}_{hbm:.0f}GBps": round(100 * value / ws / hbm, 2)},
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6650 GB/s",
+                     "traffic": None if tr is None else tr["bytes_per_launch"],
+                     "algorithmic_bytes_per_launch": int(per_launch_bytes),
+                     "avg_launch_us": round(attn_avg_ms * 1e3, 2),
+                     "merge_avg_us": round(statistics.mean(merge_ms) * 1e3, 2)},
+        "e2e": e2e,
+        "gpu_launches": args.steps * sum(1 + (1 if r["plan"].info.num_merge_rows > 0 else 0) for r in runs),
+        "clocks": clk.summary(),
+        "kernel_source_hash": src_hash,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = _cpu_baseline(cases)
+    print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def _e2e(args, runs, dev, stream, skv, torch):
+    """Same metric through the public API with host buffers: every step plans on the host (C ABI),
+    copies q, the page table and the plan from pinned host memory, runs both phases, and copies O
+    and LSE back to pinned host memory."""
+    host = []
+    for run in runs:
+        c = run["c"]
+        hq = torch.from_numpy(np.ascontiguousarray(c.q).view(np.int16)).view(torch.bfloat16).pin_memory()
+        tabs = [torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).pin_memory()
+                for a in (c.kv_indptr, c.kv_indices, c.kv_last_page_len)]
+        o_h = torch.empty(run["o"].shape, dtype=run["o"].dtype).pin_memory()
+        l_h = torch.empty(run["lse"].shape, dtype=torch.float32).pin_memory()
+        q_d = torch.empty_like(run["d"]["q"])
+        tab_d = [torch.empty(t.shape, dtype=torch.int32, device=dev) for t in tabs]
+        host.append(dict(hq=hq, tabs=tabs, o_h=o_h, l_h=l_h, q_d=q_d, tab_d=tab_d))
+    steps = max(3, min(args.steps, args.e2e_steps))
+    h2d = d2h = 0
+
+    def one_step(count):
+        nonlocal h2d, d2h
+        for run, h in zip(runs, host):
+            c = run["c"]
+            plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, c.page_size, c.num_qo_heads,
+                                  c.num_kv_heads, c.head_dim, "balanced", 0)
+            plan.to(dev, non_blocking=True)
+            h["q_d"].copy_(h["hq"], non_blocking=True)
+            for src, dst in zip(h["tabs"], h["tab_d"]):
+                dst.copy_(src, non_blocking=True)
+            skv.paged_attn_fwd(h["q_d"], run["d"]["k"], run["d"]["v"], h["tab_d"][0], h["tab_d"][1], h["tab_d"][2],
+                               plan, run["o"], run["lse"], run["o_part"], run["lse_part"], None, c.sm_scale,
+                               c.num_pages, stream)
+            h["o_h"].copy_(run["o"], non_blocking=True)
+            h["l_h"].copy_(run["lse"], non_blocking=True)
+            if count:
+                h2d += h["hq"].numel() * 2 + sum(t.numel() * 4 for t in h["tabs"]) + plan.words.nbytes
+                d2h += h["o_h"].numel() * 4 + h["l_h"].numel() * 4
+        torch.cuda.synchronize(dev)
+
+    one_step(False)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one_step(True)
+    dt = time.perf_counter() - t0
+    kv = sum(_kv_bytes(r["c"]) for r in runs)
+    return {"value": round(kv * steps / dt / 1e9, 2), "unit": "GB/s", "steps": steps,
+            "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps,
+            "ms_per_step": round(dt / steps * 1e3, 4)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--ref-budget", type=float, default=8.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,250 @@
+/*
+ * splitkv.h -- C ABI of libsplitkv: batched attention over a paged KV cache with split-KV
+ * partials and an exact log-sum-exp merge, for NVIDIA B200 (sm_100a).
+ *
+ * Operations and where they are defined
+ *   skv_paged_attn_fwd  GQA attention over a paged KV cache whose K and V may have equal or
+ *                       independent strides (FlashInfer PR #4736 page, section 1
+ *                       "batch_pod.cu: flexible stride handling" and section 2 "SAME_KV_STRIDES
+ *                       template specialisation"); one KV sequence may be listed by many query
+ *                       batches (PyTorch MPS FlexAttention page, "KV batch broadcast").
+ *   skv_mla_decode_fwd  Multi-head latent attention decode: every head reads one 512+64-d latent
+ *                       row per token, V is the 512-d latent; seqlen_q is folded into heads to
+ *                       fill the MMA M tile (FlashInfer PR #3309 page, sections 1-2 and "why it
+ *                       is good": M tile 128, 2D/3D LSE layouts).
+ *   skv_merge_states    Exact merge of partial (O, LSE) states of KV splits (route primitive:
+ *                       partial attention at the KV holder merged "via online softmax",
+ *                       "Move the Query, Not the Cache", Methodology; in-CTA split with
+ *                       shared-memory merge, FlashInfer PR #5597 page, section 3).
+ *
+ * Semantics shared by all calls (natural-log LSE of the scaled logits):
+ *   s_t = sm_scale * q . k_t ;  O = sum_t softmax(s)_t v_t ;  LSE = ln sum_t exp(s_t).
+ *   A request with no KV tokens gives O = 0, LSE = -inf.  No causal mask: every query token
+ *   of a request attends to all of the request's KV tokens.
+ *
+ * Page table (device int32 arrays): request r owns pages kv_indices[kv_indptr[r] ..
+ *   kv_indptr[r+1]); its length is L_r = (n_r - 1) * page_size + kv_last_page_len[r] with
+ *   kv_last_page_len[r] in [1, page_size] (L_r = 0 when n_r = 0).  Token t of request r is
+ *   slot t % page_size of physical page kv_indices[kv_indptr[r] + t / page_size].
+ *
+ * Conventions
+ *   - Pure C.  Every pointer argument is a DEVICE pointer unless its name ends in _h (host).
+ *   - The caller owns every buffer; the library never allocates, never synchronises, never
+ *     prints.  Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Host-detectable errors return a status before anything is launched.
+ *   - Device-detected errors (a page id >= num_pages, a barrier wait that timed out) are
+ *     written to the optional device int32 word `status` (first error wins; 0 = ok) and the
+ *     affected outputs are unspecified.  Kernels never trap.
+ *   - Calls are asynchronous: buffers must stay valid until the stream reaches the work.
+ */
+#ifndef SPLITKV_H_
+#define SPLITKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SKV_API __attribute__((visibility("default")))
+#else
+#define SKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* skv_stream_t; /* same handle type as cudaStream_t */
+
+typedef enum {
+  SKV_OK = 0,
+  SKV_ERR_INVALID = 1,     /* bad argument: null pointer, negative size, inconsistent table   */
+  SKV_ERR_UNSUPPORTED = 2, /* valid but not implemented: head_dim, group size, dtype          */
+  SKV_ERR_ALIGNMENT = 3,   /* base pointer / stride not 16-byte aligned (TMA requirement)     */
+  SKV_ERR_WORKSPACE = 4,   /* plan or partial buffers too small for the plan                  */
+  SKV_ERR_CUDA = 5         /* a CUDA runtime call (attribute set, launch) failed              */
+} skv_status;
+
+/* codes written to the device status word */
+#define SKV_DEV_OK 0
+#define SKV_DEV_TIMEOUT 16   /* an mbarrier wait exceeded its iteration cap                  */
+#define SKV_DEV_PAGE_OOB 17  /* a page id outside [0, num_pages)                              */
+#define SKV_DEV_PLAN_BAD 18  /* a work item outside the request's pages / query rows          */
+
+typedef enum { SKV_BF16 = 0, SKV_F32 = 1, SKV_E4M3 = 2 } skv_dtype;
+
+/* split policies for the planners */
+typedef enum {
+  SKV_SPLIT_NONE = 0,     /* one split per request                                           */
+  SKV_SPLIT_FIXED = 1,    /* `param` splits per request (earlier splits take the extra page)  */
+  SKV_SPLIT_BALANCED = 2, /* chunk sizes chosen so all SMs stay busy; `param` = SM count       */
+                          /* (0 = query the current device)                                    */
+  SKV_SPLIT_EXPLICIT = 3  /* boundaries given in split_indptr_h / split_bounds_h               */
+} skv_split_policy;
+
+/* Summary of a plan.  The plan itself is an int32 array the caller copies to the device. */
+typedef struct {
+  int32_t num_work;         /* work items (CTAs per KV head for GQA, per split for MLA)       */
+  int32_t num_partial_rows; /* rows the o_part / lse_part buffers must hold (0: no split)     */
+  int32_t num_merge_rows;   /* output rows combined from >1 split by the merge pass           */
+  int32_t kernel;           /* kernel variant the dispatcher picked (informational)           */
+  int32_t q_tile;           /* query tokens per work item (MLA: the fold ratio F)             */
+  int32_t plan_words;       /* int32 words of the plan actually used                          */
+  int32_t max_splits;       /* largest split count of any request                             */
+  int32_t total_splits;     /* sum over requests of their split counts                        */
+} skv_plan_info;
+
+/* -------------------------------------------------------------------------------------------
+ * skv_plan_paged -- host-side planner for skv_paged_attn_fwd.
+ *   qo_indptr_h [batch+1]      query tokens of request r are rows qo_indptr_h[r] ..
+ *   kv_indptr_h [batch+1], kv_last_page_len_h [batch]   host copies of the page-table shape
+ *   page_size, num_qo_heads, num_kv_heads (divides num_qo_heads), head_dim in {64, 128}
+ *   policy / param              see skv_split_policy
+ *   split_indptr_h [batch+1], split_bounds_h   only for SKV_SPLIT_EXPLICIT: request r has
+ *       S_r = split_indptr_h[r+1] - split_indptr_h[r] splits whose S_r + 1 request-relative
+ *       page boundaries are split_bounds_h[split_indptr_h[r] + r ...] (non-decreasing, first 0,
+ *       last n_r; empty splits allowed).  Pass NULL otherwise.
+ *   plan_h / plan_capacity      output int32 buffer (host); SKV_ERR_WORKSPACE if too small,
+ *                               with info->plan_words set to the size needed.
+ *   info                        output summary.
+ * With S_r > 1 the split partials of query token i, split j of request r are row
+ *   part_base_r + i * S_r + j of o_part / lse_part; requests with S_r = 1 write O directly.
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
+                          const int32_t* kv_last_page_len_h, int32_t page_size,
+                          int32_t num_qo_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t policy, int32_t param, const int32_t* split_indptr_h,
+                          const int32_t* split_bounds_h, int32_t* plan_h,
+                          int64_t plan_capacity, skv_plan_info* info);
+
+/* Arguments of skv_paged_attn_fwd.  All pointers are device pointers. */
+typedef struct {
+  const void* q;            /* bf16 [total_q, Hq, D], contiguous                              */
+  const void* k_cache;      /* bf16: K(page, slot, head, d) = k_cache[page*k_stride[0] +       */
+  const void* v_cache;      /*   slot*k_stride[1] + head*k_stride[2] + d]; V likewise with      */
+  int64_t k_stride[3];      /*   v_stride.  Strides in elements, each a multiple of 8 (16 B);  */
+  int64_t v_stride[3];      /*   when all three are equal the SAME_KV_STRIDES kernel runs.     */
+  const int32_t* kv_indptr;         /* [batch+1]                                              */
+  const int32_t* kv_indices;        /* [kv_indptr[batch]] physical page ids                   */
+  const int32_t* kv_last_page_len;  /* [batch]                                                */
+  int32_t batch;
+  int32_t total_q;          /* rows of q / o                                                  */
+  int32_t num_pages;        /* physical pages in the cache (device bound check)               */
+  int32_t page_size;
+  int32_t num_qo_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;         /* 64 or 128                                                       */
+  float sm_scale;
+  void* o;                  /* [total_q, Hq, D] of o_dtype                                     */
+  int32_t o_dtype;          /* SKV_F32 or SKV_BF16                                             */
+  float* lse;               /* [total_q, Hq] fp32 (may be NULL)                                */
+  float* o_part;            /* [num_partial_rows, Hq, D] fp32, needed when the plan splits     */
+  float* lse_part;          /* [num_partial_rows, Hq] fp32                                     */
+  int32_t* status;          /* device status word (may be NULL)                                */
+} skv_paged_params;
+
+/* -------------------------------------------------------------------------------------------
+ * skv_paged_attn_fwd -- O, LSE (and split partials) of GQA attention over the paged cache.
+ *   plan_d: device copy of the plan from skv_plan_paged for the same shapes; info: its summary.
+ *   Query head h reads KV head h / (Hq / Hk).  Split partials are written to o_part/lse_part
+ *   and merged into o/lse on the same stream.
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_paged_attn_fwd(const skv_paged_params* p, const int32_t* plan_d,
+                              const skv_plan_info* info, skv_stream_t stream);
+
+/* The two phases of skv_paged_attn_fwd, for callers that schedule (or time) them separately:
+ *   skv_paged_attn_partial  the attention kernel only: writes o / lse of requests with one
+ *                           split and o_part / lse_part of split requests;
+ *   skv_merge_plan          the plan's merge pass: combines o_part / lse_part into o / lse
+ *                           (num_heads, head_dim: 512 for MLA).  A no-op for plans without
+ *                           merge rows.  Calling both in order equals skv_paged_attn_fwd. */
+SKV_API skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan_d,
+                                          const skv_plan_info* info, skv_stream_t stream);
+SKV_API skv_status skv_merge_plan(const float* o_part, const float* lse_part, const int32_t* plan_d,
+                                  const skv_plan_info* info, int32_t num_heads, int32_t head_dim,
+                                  void* o, int32_t o_dtype, float* lse, skv_stream_t stream);
+
+/* -------------------------------------------------------------------------------------------
+ * skv_plan_mla -- host-side planner for skv_mla_decode_fwd (same split policies).  The fold
+ *   ratio F (seqlen_q tokens folded into the head/row dimension) is skv_mla_fold_ratio(H,
+ *   q_len, 128) and is reported in info->q_tile.
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
+                        const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_heads,
+                        int32_t policy, int32_t param, const int32_t* split_indptr_h,
+                        const int32_t* split_bounds_h, int32_t* plan_h, int64_t plan_capacity,
+                        skv_plan_info* info);
+
+/* Arguments of skv_mla_decode_fwd.  All pointers are device pointers. */
+typedef struct {
+  const void* q_nope;       /* bf16 [B, q_len, H, 512], contiguous                            */
+  const void* q_pe;         /* bf16 [B, q_len, H, 64], contiguous                             */
+  const void* ckv;          /* latent: ckv(page, slot, d) = ckv[page*ckv_stride[0] +           */
+  const void* kpe;          /*   slot*ckv_stride[1] + d], d < 512; kpe likewise, d < 64        */
+  int64_t ckv_stride[2];    /* elements; multiples of 16 bytes                                 */
+  int64_t kpe_stride[2];
+  int32_t kv_dtype;         /* SKV_BF16 or SKV_E4M3 (OCP e4m3fn codes)                          */
+  float kv_scale;           /* per-tensor dequantisation scale (1 for bf16)                    */
+  const int32_t* kv_indptr;
+  const int32_t* kv_indices;
+  const int32_t* kv_last_page_len;
+  int32_t batch;
+  int32_t q_len;
+  int32_t num_heads;
+  int32_t num_pages;
+  int32_t page_size;
+  float sm_scale;
+  void* o;                  /* [B, q_len, H, 512] of o_dtype                                   */
+  int32_t o_dtype;          /* SKV_F32 or SKV_BF16                                             */
+  float* lse;               /* [B, q_len, H] fp32 (== 2D [B*q_len, H]); may be NULL            */
+  float* o_part;            /* [num_partial_rows, H, 512] fp32 when the plan splits            */
+  float* lse_part;          /* [num_partial_rows, H]                                           */
+  int32_t* status;
+} skv_mla_params;
+
+/* skv_mla_decode_fwd -- MLA decode: s = sm_scale (q_nope . ckv + q_pe . kpe), V = ckv (times
+ *   kv_scale for e4m3).  Partial rows follow the skv_plan_paged layout with query "token" =
+ *   (decode position i) of the request. */
+SKV_API skv_status skv_mla_decode_fwd(const skv_mla_params* p, const int32_t* plan_d,
+                              const skv_plan_info* info, skv_stream_t stream);
+/* First phase of skv_mla_decode_fwd (attention kernel only); finish with skv_merge_plan. */
+SKV_API skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d,
+                                          const skv_plan_info* info, skv_stream_t stream);
+
+/* -------------------------------------------------------------------------------------------
+ * skv_merge_states -- exact merge of partial states.
+ *   For each output row r and head h, over its states j:
+ *     M = max_j LSE_j, LSE = M + ln sum_j exp(LSE_j - M), O = sum_j exp(LSE_j - LSE) O_j;
+ *     no state, or all LSE_j = -inf: O = 0, LSE = -inf.
+ *   State layout: with state_indptr (device [num_rows+1]) the states of row r are rows
+ *   state_indptr[r] .. state_indptr[r+1] of o_states [*, H, D] / lse_states [*, H]; with
+ *   state_indptr == NULL there are `num_states` states per row stored state-major:
+ *   o_states [num_states, num_rows, H, D], lse_states [num_states, num_rows, H] (for example
+ *   one buffer per KV chunk holder).  head_dim a multiple of 4; o_out of o_dtype
+ *   [num_rows, H, D]; lse_out [num_rows, H] (may be NULL).
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_merge_states(const float* o_states, const float* lse_states,
+                            const int32_t* state_indptr, int32_t num_states, int64_t num_rows,
+                            int32_t num_heads, int32_t head_dim, void* o_out, int32_t o_dtype,
+                            float* lse_out, skv_stream_t stream);
+
+/* -------------------------------------------------------------------------------------------
+ * skv_paged_kv_gather -- test hook for the page-table walk: copies the logical K and V of every
+ *   request, through the same address generation the attention kernels use, into dense
+ *   k_out / v_out [sum_r L_r, Hk, D] bf16 (request r's tokens start at row token_indptr[r],
+ *   token_indptr device [batch+1] = prefix sums of L_r).  Bit-exact by construction.
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_paged_kv_gather(const skv_paged_params* p, const int32_t* token_indptr,
+                               int64_t total_tokens, void* k_out, void* v_out,
+                               skv_stream_t stream);
+
+/* Fold ratio used by the MLA kernels: the largest divisor F of q_len with num_heads * F <=
+ * tile_m (F >= 1).  Rows per work item = num_heads * F; work items per request = q_len / F. */
+SKV_API int32_t skv_mla_fold_ratio(int32_t num_heads, int32_t q_len, int32_t tile_m);
+
+SKV_API const char* skv_status_str(int32_t status);
+SKV_API int32_t skv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPLITKV_H_ */

@@ -1,0 +1,317 @@
+"""Python binding of libsplitkv (paged attention + split-KV + exact LSE merge on B200).
+
+Argument marshalling only: every step of the attention path runs in the CUDA kernels of
+``libsplitkv.so``.  Device buffers are torch CUDA tensors (PyTorch is used for memory and
+streams); host arrays are numpy.  Importing this package without the built library raises --
+there is no fallback path.
+
+Functions mirror the C ABI in include/splitkv.h:
+``plan_paged``, ``paged_attn_fwd``, ``plan_mla``, ``mla_decode_fwd``, ``merge_states``,
+``paged_kv_gather``, ``mla_fold_ratio``, ``status_str``, ``version``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsplitkv.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libsplitkv.so not built at {_LIB_PATH}: run `python split_kv_merge_b200/build.py`")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+# ----------------------------------------------------------------------------- constants
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA = range(6)
+DEV_OK, DEV_TIMEOUT, DEV_PAGE_OOB, DEV_PLAN_BAD = 0, 16, 17, 18
+BF16, F32, E4M3 = 0, 1, 2
+SPLIT_NONE, SPLIT_FIXED, SPLIT_BALANCED, SPLIT_EXPLICIT = 0, 1, 2, 3
+_POLICY = {"none": SPLIT_NONE, "fixed": SPLIT_FIXED, "balanced": SPLIT_BALANCED, "explicit": SPLIT_EXPLICIT}
+
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_vp = ctypes.c_void_p
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("num_work", ctypes.c_int32), ("num_partial_rows", ctypes.c_int32),
+                ("num_merge_rows", ctypes.c_int32), ("kernel", ctypes.c_int32),
+                ("q_tile", ctypes.c_int32), ("plan_words", ctypes.c_int32),
+                ("max_splits", ctypes.c_int32), ("total_splits", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class PagedParams(ctypes.Structure):
+    _fields_ = [("q", _vp), ("k_cache", _vp), ("v_cache", _vp),
+                ("k_stride", ctypes.c_int64 * 3), ("v_stride", ctypes.c_int64 * 3),
+                ("kv_indptr", _vp), ("kv_indices", _vp), ("kv_last_page_len", _vp),
+                ("batch", ctypes.c_int32), ("total_q", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_qo_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+                ("o", _vp), ("o_dtype", ctypes.c_int32), ("lse", _vp), ("o_part", _vp), ("lse_part", _vp),
+                ("status", _vp)]
+
+
+class MlaParams(ctypes.Structure):
+    _fields_ = [("q_nope", _vp), ("q_pe", _vp), ("ckv", _vp), ("kpe", _vp),
+                ("ckv_stride", ctypes.c_int64 * 2), ("kpe_stride", ctypes.c_int64 * 2),
+                ("kv_dtype", ctypes.c_int32), ("kv_scale", ctypes.c_float),
+                ("kv_indptr", _vp), ("kv_indices", _vp), ("kv_last_page_len", _vp),
+                ("batch", ctypes.c_int32), ("q_len", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("page_size", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+                ("o", _vp), ("o_dtype", ctypes.c_int32), ("lse", _vp), ("o_part", _vp), ("lse_part", _vp),
+                ("status", _vp)]
+
+
+def _proto(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_plan_paged = _proto("skv_plan_paged", ctypes.c_int, [ctypes.c_int32, _i32p, _i32p, _i32p, ctypes.c_int32,
+                                                       ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                       ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, _i32p,
+                                                       ctypes.c_int64, ctypes.POINTER(PlanInfo)])
+_plan_mla = _proto("skv_plan_mla", ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32,
+                                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _i32p, _i32p,
+                                                   _i32p, ctypes.c_int64, ctypes.POINTER(PlanInfo)])
+_paged_fwd = _proto("skv_paged_attn_fwd", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp,
+                                                          ctypes.POINTER(PlanInfo), _vp])
+_mla_fwd = _proto("skv_mla_decode_fwd", ctypes.c_int, [ctypes.POINTER(MlaParams), _vp,
+                                                        ctypes.POINTER(PlanInfo), _vp])
+_paged_partial = _proto("skv_paged_attn_partial", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp,
+                                                                  ctypes.POINTER(PlanInfo), _vp])
+_mla_partial = _proto("skv_mla_decode_partial", ctypes.c_int, [ctypes.POINTER(MlaParams), _vp,
+                                                                ctypes.POINTER(PlanInfo), _vp])
+_merge_plan = _proto("skv_merge_plan", ctypes.c_int, [_vp, _vp, _vp, ctypes.POINTER(PlanInfo), ctypes.c_int32,
+                                                       ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp])
+_merge = _proto("skv_merge_states", ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                                    ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp])
+_gather = _proto("skv_paged_kv_gather", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp, ctypes.c_int64, _vp,
+                                                        _vp, _vp])
+_fold = _proto("skv_mla_fold_ratio", ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32])
+_status_str = _proto("skv_status_str", ctypes.c_char_p, [ctypes.c_int32])
+_version = _proto("skv_version", ctypes.c_int32, [])
+
+SYMBOLS = ["skv_plan_paged", "skv_paged_attn_fwd", "skv_paged_attn_partial", "skv_merge_plan", "skv_plan_mla",
+           "skv_mla_decode_fwd", "skv_mla_decode_partial", "skv_merge_states", "skv_paged_kv_gather",
+           "skv_mla_fold_ratio", "skv_status_str", "skv_version"]
+
+
+class SkvError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {status_str(code)} (status {code})")
+        self.code = code
+
+
+def status_str(code: int) -> str:
+    return _status_str(int(code)).decode()
+
+
+def version() -> int:
+    return int(_version())
+
+
+def mla_fold_ratio(num_heads: int, q_len: int, tile_m: int = 128) -> int:
+    return int(_fold(num_heads, q_len, tile_m))
+
+
+def _check(code: int, where: str) -> None:
+    if code != OK:
+        raise SkvError(code, where)
+
+
+# ----------------------------------------------------------------------------- helpers
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _ptr_i32(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(_i32p)
+
+
+def _dptr(t) -> Optional[int]:
+    """Device pointer of a torch tensor (None passes NULL)."""
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.bfloat16: BF16, torch.float32: F32, torch.float8_e4m3fn: E4M3, torch.uint8: E4M3}[t.dtype]
+
+
+def _split_args(policy, split_page_start):
+    if policy != SPLIT_EXPLICIT:
+        return None, None
+    sizes = [len(b) - 1 for b in split_page_start]
+    indptr = _i32(np.concatenate([[0], np.cumsum(sizes)]))
+    bounds = _i32(np.concatenate([np.asarray(b, np.int64) for b in split_page_start]))
+    return indptr, bounds
+
+
+@dataclass
+class Plan:
+    """Host plan words, its summary, and (after ``to``) the device copy."""
+    words: np.ndarray
+    info: PlanInfo
+    device: Optional[object] = None
+
+    def to(self, device, non_blocking: bool = False):
+        import torch
+        src = torch.from_numpy(self.words)
+        if non_blocking:
+            src = src.pin_memory()
+        self.device = src.to(device, non_blocking=non_blocking)
+        return self
+
+
+def _plan(fn, args, policy, split_page_start, where):
+    pol = _POLICY[policy] if isinstance(policy, str) else int(policy)
+    si, sb = _split_args(pol, split_page_start)
+    info = PlanInfo()
+    cap = 0
+    code = fn(*args(pol), _ptr_i32(si), _ptr_i32(sb), None, 0, ctypes.byref(info))
+    if code not in (OK, ERR_WORKSPACE):
+        _check(code, where)
+    words = np.zeros(max(1, info.plan_words), dtype=np.int32)
+    cap = words.size
+    _check(fn(*args(pol), _ptr_i32(si), _ptr_i32(sb), _ptr_i32(words), cap, ctypes.byref(info)), where)
+    return Plan(words[: info.plan_words] if info.plan_words else words[:0], info)
+
+
+# ----------------------------------------------------------------------------- planners
+def plan_paged(qo_indptr, kv_indptr, kv_last_page_len, page_size: int, num_qo_heads: int,
+               num_kv_heads: int, head_dim: int, policy="balanced", param: int = 0,
+               split_page_start: Optional[Sequence[Sequence[int]]] = None) -> Plan:
+    """Host planner (skv_plan_paged).  Host int arrays in, Plan out."""
+    qo, ki, la = _i32(qo_indptr), _i32(kv_indptr), _i32(kv_last_page_len)
+    b = len(ki) - 1
+    return _plan(_plan_paged, lambda pol: (b, _ptr_i32(qo), _ptr_i32(ki), _ptr_i32(la), page_size, num_qo_heads,
+                                           num_kv_heads, head_dim, pol, param),
+                 policy, split_page_start, "skv_plan_paged")
+
+
+def plan_mla(batch_q_len: int, kv_indptr, kv_last_page_len, page_size: int, num_heads: int,
+             policy="balanced", param: int = 0,
+             split_page_start: Optional[Sequence[Sequence[int]]] = None) -> Plan:
+    """Host planner (skv_plan_mla).  ``batch_q_len`` is the query length of every request."""
+    ki, la = _i32(kv_indptr), _i32(kv_last_page_len)
+    b = len(ki) - 1
+    return _plan(_plan_mla, lambda pol: (b, batch_q_len, _ptr_i32(ki), _ptr_i32(la), page_size, num_heads, pol,
+                                         param),
+                 policy, split_page_start, "skv_plan_mla")
+
+
+# ----------------------------------------------------------------------------- launches
+def _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, o, lse, o_part, lse_part,
+                  status, sm_scale, num_pages, page_size=None):
+    if k_cache.stride(-1) != 1 or v_cache.stride(-1) != 1:
+        raise ValueError("the innermost (head_dim) stride of K and V must be 1")
+    p = PagedParams()
+    p.q, p.k_cache, p.v_cache = _dptr(q), _dptr(k_cache), _dptr(v_cache)
+    for i in range(3):
+        p.k_stride[i] = k_cache.stride(i)
+        p.v_stride[i] = v_cache.stride(i)
+    p.kv_indptr, p.kv_indices, p.kv_last_page_len = _dptr(kv_indptr), _dptr(kv_indices), _dptr(kv_last_page_len)
+    p.batch = kv_indptr.shape[0] - 1
+    p.total_q = q.shape[0] if q is not None else 0
+    p.num_pages = k_cache.shape[0] if num_pages is None else num_pages
+    p.page_size = k_cache.shape[1] if page_size is None else page_size
+    p.num_qo_heads = q.shape[1] if q is not None else k_cache.shape[2]
+    p.num_kv_heads = k_cache.shape[2]
+    p.head_dim = k_cache.shape[3]
+    p.sm_scale = float(p.head_dim ** -0.5 if sm_scale is None else sm_scale)
+    p.o = _dptr(o)
+    p.o_dtype = _dtype_code(o) if o is not None else F32
+    p.lse, p.o_part, p.lse_part, p.status = _dptr(lse), _dptr(o_part), _dptr(lse_part), _dptr(status)
+    return p
+
+
+def paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan: Plan, o, lse=None,
+                   o_part=None, lse_part=None, status=None, sm_scale: Optional[float] = None,
+                   num_pages: Optional[int] = None, stream=None, phase: str = "all") -> None:
+    """skv_paged_attn_fwd.  q [total_q, Hq, D] bf16; k_cache / v_cache [num_pages, P, Hk, D] bf16
+    views (any page/slot/head strides, head_dim contiguous); page-table tensors int32 on the
+    device; o [total_q, Hq, D] f32|bf16; lse [total_q, Hq] f32; o_part / lse_part sized by
+    ``plan.info.num_partial_rows`` when the plan splits."""
+    p = _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, o, lse, o_part, lse_part,
+                      status, sm_scale, num_pages)
+    fn = {"all": _paged_fwd, "partial": _paged_partial}[phase]
+    _check(fn(ctypes.byref(p), _dptr(plan.device), ctypes.byref(plan.info), _stream_ptr(stream)),
+           "skv_paged_attn_fwd" if phase == "all" else "skv_paged_attn_partial")
+
+
+def mla_decode_fwd(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len, plan: Plan, o, lse=None,
+                   o_part=None, lse_part=None, status=None, sm_scale: Optional[float] = None,
+                   kv_scale: float = 1.0, num_pages: Optional[int] = None, stream=None, phase: str = "all") -> None:
+    """skv_mla_decode_fwd.  q_nope [B, q_len, H, 512], q_pe [B, q_len, H, 64] bf16; ckv
+    [num_pages, P, 512], kpe [num_pages, P, 64] views (bf16, or uint8 / float8_e4m3fn codes);
+    o [B, q_len, H, 512]; lse [B, q_len, H]."""
+    if ckv.stride(-1) != 1 or kpe.stride(-1) != 1:
+        raise ValueError("the innermost stride of ckv and kpe must be 1")
+    p = MlaParams()
+    p.q_nope, p.q_pe, p.ckv, p.kpe = _dptr(q_nope), _dptr(q_pe), _dptr(ckv), _dptr(kpe)
+    for i in range(2):
+        p.ckv_stride[i] = ckv.stride(i)
+        p.kpe_stride[i] = kpe.stride(i)
+    p.kv_dtype = _dtype_code(ckv)
+    p.kv_scale = float(kv_scale)
+    p.kv_indptr, p.kv_indices, p.kv_last_page_len = _dptr(kv_indptr), _dptr(kv_indices), _dptr(kv_last_page_len)
+    p.batch = kv_indptr.shape[0] - 1
+    p.q_len = q_nope.shape[1]
+    p.num_heads = q_nope.shape[2]
+    p.num_pages = ckv.shape[0] if num_pages is None else num_pages
+    p.page_size = ckv.shape[1]
+    p.sm_scale = float(192.0 ** -0.5 if sm_scale is None else sm_scale)
+    p.o, p.o_dtype = _dptr(o), _dtype_code(o)
+    p.lse, p.o_part, p.lse_part, p.status = _dptr(lse), _dptr(o_part), _dptr(lse_part), _dptr(status)
+    fn = {"all": _mla_fwd, "partial": _mla_partial}[phase]
+    _check(fn(ctypes.byref(p), _dptr(plan.device), ctypes.byref(plan.info), _stream_ptr(stream)),
+           "skv_mla_decode_fwd" if phase == "all" else "skv_mla_decode_partial")
+
+
+def merge_plan(o_part, lse_part, plan: Plan, num_heads: int, head_dim: int, o, lse=None, stream=None) -> None:
+    """skv_merge_plan: the plan's merge pass (second phase of paged_attn_fwd / mla_decode_fwd)."""
+    _check(_merge_plan(_dptr(o_part), _dptr(lse_part), _dptr(plan.device), ctypes.byref(plan.info), num_heads,
+                       head_dim, _dptr(o), _dtype_code(o), _dptr(lse), _stream_ptr(stream)), "skv_merge_plan")
+
+
+def merge_states(o_states, lse_states, o_out, lse_out=None, state_indptr=None, num_states: int = 0,
+                 stream=None) -> None:
+    """skv_merge_states.  With ``state_indptr`` (device int32 [rows+1]): o_states [*, H, D],
+    lse_states [*, H].  Without: state-major o_states [S, rows, H, D], lse_states [S, rows, H]."""
+    if state_indptr is None:
+        num_states = o_states.shape[0]
+        rows, H, D = o_states.shape[1], o_states.shape[2], o_states.shape[3]
+    else:
+        rows, H, D = state_indptr.shape[0] - 1, o_states.shape[-2], o_states.shape[-1]
+    _check(_merge(_dptr(o_states), _dptr(lse_states), _dptr(state_indptr), num_states, rows, H, D, _dptr(o_out),
+                  _dtype_code(o_out), _dptr(lse_out), _stream_ptr(stream)), "skv_merge_states")
+
+
+def paged_kv_gather(k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, token_indptr, total_tokens: int,
+                    k_out, v_out, status=None, num_pages: Optional[int] = None, stream=None) -> None:
+    """skv_paged_kv_gather (test hook): dense copies of every request's logical K and V."""
+    p = _paged_params(None, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, None, None, None, None,
+                      status, None, num_pages)
+    _check(_gather(ctypes.byref(p), _dptr(token_indptr), total_tokens, _dptr(k_out), _dptr(v_out),
+                   _stream_ptr(stream)), "skv_paged_kv_gather")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+from .runner import RouteMerge, mla_decode, paged_attention  # noqa: E402,F401

@@ -1,0 +1,360 @@
+// C ABI of libsplitkv: argument validation, the split planner and kernel dispatch.
+//
+// Host-side dispatch picks the kernel variant (and the SAME_KV_STRIDES specialisation) before
+// launch instead of branching inside the kernel (FlashInfer PR #4736 page, conclusion 1
+// "host-side dispatch"; section 2 for the specialisation).  Split-KV planning turns each
+// request's page list into chunks so every SM has work at small batch; the partials of a split
+// request are merged exactly afterwards (route primitive, "Move the Query, Not the Cache").
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "skv_internal.h"
+
+using namespace skv;
+
+namespace {
+
+constexpr int32_t kVersion = 1;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct ReqShape {
+  int32_t q_start, q_len, n_pages;
+};
+
+// Shared planner: work items over (request, query tile, split) and merge items for split rows.
+skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t q_tile,
+                       int64_t units_per_page, int32_t policy, int32_t param,
+                       const int32_t* split_indptr_h, const int32_t* split_bounds_h,
+                       int32_t kernel, int32_t* plan_h, int64_t plan_capacity,
+                       skv_plan_info* info) {
+  if (info == nullptr) return SKV_ERR_INVALID;
+  std::memset(info, 0, sizeof(*info));
+  if (q_tile < 1) return SKV_ERR_INVALID;
+  // per-request split counts
+  int64_t chunk = 0;
+  if (policy == SKV_SPLIT_BALANCED) {
+    int sms = param;
+    if (sms <= 0) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+      cudaGetLastError();
+    }
+    int64_t total_units = 0;
+    for (const auto& q : req) {
+      const int64_t tiles = (q.q_len + q_tile - 1) / q_tile;
+      total_units += tiles * q.n_pages * units_per_page;
+    }
+    // aim for ~8 work items per SM-slot pair of waves; never below 8 pages per chunk
+    const int64_t target_items = (int64_t)sms * 8;
+    chunk = std::max<int64_t>(8, (total_units + target_items - 1) / std::max<int64_t>(1, target_items));
+  } else if (policy == SKV_SPLIT_FIXED) {
+    if (param < 1) return SKV_ERR_INVALID;
+  } else if (policy == SKV_SPLIT_EXPLICIT) {
+    if (split_indptr_h == nullptr || split_bounds_h == nullptr) return SKV_ERR_INVALID;
+    if (split_indptr_h[0] != 0) return SKV_ERR_INVALID;
+  } else if (policy != SKV_SPLIT_NONE) {
+    return SKV_ERR_INVALID;
+  }
+
+  std::vector<WorkItem> work;
+  std::vector<MergeItem> merges;
+  int32_t part_base = 0, max_splits = 0, total_splits = 0;
+  std::vector<int32_t> bounds;
+  for (int32_t r = 0; r < batch; ++r) {
+    const ReqShape& q = req[r];
+    int32_t S = 1;
+    bounds.clear();
+    if (policy == SKV_SPLIT_EXPLICIT) {
+      S = split_indptr_h[r + 1] - split_indptr_h[r];
+      if (S < 1) return SKV_ERR_INVALID;
+      const int32_t* b = split_bounds_h + split_indptr_h[r] + r;
+      if (b[0] != 0 || b[S] != q.n_pages) return SKV_ERR_INVALID;
+      for (int j = 0; j <= S; ++j) {
+        if (j > 0 && b[j] < b[j - 1]) return SKV_ERR_INVALID;
+        bounds.push_back(b[j]);
+      }
+    } else {
+      if (policy == SKV_SPLIT_FIXED) S = param;
+      if (policy == SKV_SPLIT_BALANCED) {
+        const int64_t units = (int64_t)q.n_pages * units_per_page;
+        S = (int32_t)std::max<int64_t>(1, (units + chunk - 1) / chunk);
+        S = std::min<int32_t>(S, std::max<int32_t>(1, q.n_pages));
+      }
+      bounds.push_back(0);
+      for (int j = 0; j < S; ++j) {
+        const int32_t rem = q.n_pages - bounds.back();
+        bounds.push_back(bounds.back() + (rem + (S - j) - 1) / (S - j));  // ceil first
+      }
+    }
+    max_splits = std::max(max_splits, S);
+    total_splits += S;
+    if (q.q_len == 0) continue;
+    for (int32_t q0 = 0; q0 < q.q_len; q0 += q_tile) {
+      const int32_t qc = std::min(q_tile, q.q_len - q0);
+      for (int j = 0; j < S; ++j) {
+        WorkItem w;
+        w.r = r;
+        w.q_start = q.q_start + q0;
+        w.q_count = qc;
+        w.page_begin = bounds[j];
+        w.page_end = bounds[j + 1];
+        w.part_row = S > 1 ? part_base + q0 * S + j : -1;
+        w.part_stride = S;
+        w.split = j;
+        work.push_back(w);
+      }
+    }
+    if (S > 1) {
+      for (int32_t i = 0; i < q.q_len; ++i) merges.push_back(MergeItem{q.q_start + i, part_base + i * S, S, 0});
+      part_base += q.q_len * S;
+    }
+  }
+  // longest items first: the hardware hands out CTAs roughly in index order
+  std::stable_sort(work.begin(), work.end(), [](const WorkItem& a, const WorkItem& b) {
+    return (a.page_end - a.page_begin) * a.q_count > (b.page_end - b.page_begin) * b.q_count;
+  });
+  info->num_work = (int32_t)work.size();
+  info->num_partial_rows = part_base;
+  info->num_merge_rows = (int32_t)merges.size();
+  info->kernel = kernel;
+  info->q_tile = q_tile;
+  info->max_splits = max_splits;
+  info->total_splits = total_splits;
+  const int64_t words = plan_words(info->num_work, info->num_merge_rows);
+  if (words > INT32_MAX) return SKV_ERR_INVALID;
+  info->plan_words = (int32_t)words;
+  if (plan_h == nullptr || plan_capacity < words) return SKV_ERR_WORKSPACE;
+  if (!work.empty()) std::memcpy(plan_h, work.data(), work.size() * sizeof(WorkItem));
+  if (!merges.empty())
+    std::memcpy(plan_h + 8 * work.size(), merges.data(), merges.size() * sizeof(MergeItem));
+  return SKV_OK;
+}
+
+skv_status check_table_h(int32_t batch, const int32_t* kv_indptr_h, const int32_t* last_h,
+                         int32_t page_size, std::vector<ReqShape>& req) {
+  if (batch < 0 || page_size < 1 || kv_indptr_h == nullptr || last_h == nullptr) return SKV_ERR_INVALID;
+  if (batch > 0 && kv_indptr_h[0] != 0) return SKV_ERR_INVALID;
+  req.resize(batch);
+  for (int32_t r = 0; r < batch; ++r) {
+    const int32_t n = kv_indptr_h[r + 1] - kv_indptr_h[r];
+    if (n < 0) return SKV_ERR_INVALID;
+    if (n > 0 && (last_h[r] < 1 || last_h[r] > page_size)) return SKV_ERR_INVALID;
+    if ((int64_t)n * page_size > INT32_MAX) return SKV_ERR_INVALID;
+    req[r].n_pages = n;
+  }
+  return SKV_OK;
+}
+
+skv_status cuda_status(int e) { return e == 0 ? SKV_OK : SKV_ERR_CUDA; }
+
+skv_status check_plan(const int32_t* plan_d, const skv_plan_info* info) {
+  if (info == nullptr) return SKV_ERR_INVALID;
+  if (info->num_work < 0 || info->num_merge_rows < 0 || info->num_partial_rows < 0) return SKV_ERR_INVALID;
+  if (info->num_work > 0 && plan_d == nullptr) return SKV_ERR_INVALID;
+  if (info->q_tile < 1) return SKV_ERR_INVALID;
+  return SKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t skv_version(void) { return kVersion; }
+
+const char* skv_status_str(int32_t s) {
+  switch (s) {
+    case SKV_OK: return "ok";
+    case SKV_ERR_INVALID: return "invalid argument";
+    case SKV_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case SKV_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case SKV_ERR_WORKSPACE: return "plan or partial buffer too small";
+    case SKV_ERR_CUDA: return "CUDA launch failed";
+    case SKV_DEV_TIMEOUT: return "device: barrier wait timed out";
+    case SKV_DEV_PAGE_OOB: return "device: page id out of range";
+    case SKV_DEV_PLAN_BAD: return "device: work item outside the request";
+    default: return "unknown status";
+  }
+}
+
+int32_t skv_mla_fold_ratio(int32_t num_heads, int32_t q_len, int32_t tile_m) {
+  if (num_heads < 1 || q_len < 1 || tile_m < 1) return 1;
+  int32_t best = 1;
+  for (int32_t f = 1; f <= q_len; ++f)
+    if (q_len % f == 0 && (int64_t)num_heads * f <= tile_m) best = f;
+  return best;
+}
+
+skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
+                          const int32_t* kv_last_page_len_h, int32_t page_size,
+                          int32_t num_qo_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t policy, int32_t param, const int32_t* split_indptr_h,
+                          const int32_t* split_bounds_h, int32_t* plan_h,
+                          int64_t plan_capacity, skv_plan_info* info) {
+  if (info != nullptr) std::memset(info, 0, sizeof(*info));
+  if (qo_indptr_h == nullptr || num_qo_heads < 1 || num_kv_heads < 1) return SKV_ERR_INVALID;
+  if (num_qo_heads % num_kv_heads != 0) return SKV_ERR_INVALID;
+  if (head_dim != 64 && head_dim != 128) return SKV_ERR_UNSUPPORTED;
+  std::vector<ReqShape> req;
+  skv_status st = check_table_h(batch, kv_indptr_h, kv_last_page_len_h, page_size, req);
+  if (st != SKV_OK) return st;
+  if (batch > 0 && qo_indptr_h[0] != 0) return SKV_ERR_INVALID;
+  for (int32_t r = 0; r < batch; ++r) {
+    req[r].q_start = qo_indptr_h[r];
+    req[r].q_len = qo_indptr_h[r + 1] - qo_indptr_h[r];
+    if (req[r].q_len < 0) return SKV_ERR_INVALID;
+  }
+  const int32_t g = num_qo_heads / num_kv_heads;
+  const int32_t kernel = KERNEL_GQA_SIMT;
+  const int32_t q_tile = std::max<int32_t>(1, 16 / g);
+  return plan_common(batch, req, q_tile, num_kv_heads, policy, param, split_indptr_h, split_bounds_h,
+                     kernel, plan_h, plan_capacity, info);
+}
+
+skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
+                        const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_heads,
+                        int32_t policy, int32_t param, const int32_t* split_indptr_h,
+                        const int32_t* split_bounds_h, int32_t* plan_h, int64_t plan_capacity,
+                        skv_plan_info* info) {
+  if (info != nullptr) std::memset(info, 0, sizeof(*info));
+  if (q_len < 1 || num_heads < 1) return SKV_ERR_INVALID;
+  std::vector<ReqShape> req;
+  skv_status st = check_table_h(batch, kv_indptr_h, kv_last_page_len_h, page_size, req);
+  if (st != SKV_OK) return st;
+  for (int32_t r = 0; r < batch; ++r) {
+    req[r].q_start = r * q_len;
+    req[r].q_len = q_len;
+  }
+  const int32_t fold = skv_mla_fold_ratio(num_heads, q_len, 128);
+  return plan_common(batch, req, fold, 1, policy, param, split_indptr_h, split_bounds_h, KERNEL_MLA_SIMT,
+                     plan_h, plan_capacity, info);
+}
+
+skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan_d,
+                              const skv_plan_info* info, skv_stream_t stream) {
+  if (p == nullptr) return SKV_ERR_INVALID;
+  skv_status st = check_plan(plan_d, info);
+  if (st != SKV_OK) return st;
+  if (p->batch < 0 || p->total_q < 0 || p->page_size < 1 || p->num_pages < 0) return SKV_ERR_INVALID;
+  if (p->num_qo_heads < 1 || p->num_kv_heads < 1 || p->num_qo_heads % p->num_kv_heads) return SKV_ERR_INVALID;
+  if (p->head_dim != 64 && p->head_dim != 128) return SKV_ERR_UNSUPPORTED;
+  if (p->o_dtype != SKV_F32 && p->o_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
+  if (info->num_work > 0) {
+    if (!p->q || !p->k_cache || !p->v_cache || !p->kv_indptr || !p->kv_indices || !p->kv_last_page_len || !p->o)
+      return SKV_ERR_INVALID;
+  }
+  for (int i = 0; i < 3; ++i) {
+    if (p->k_stride[i] < 0 || p->v_stride[i] < 0) return SKV_ERR_INVALID;
+    if ((p->k_stride[i] % 8) || (p->v_stride[i] % 8)) return SKV_ERR_ALIGNMENT;
+  }
+  if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
+    return SKV_ERR_ALIGNMENT;
+  if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
+  if (info->kernel != KERNEL_GQA_SIMT) return SKV_ERR_INVALID;
+  const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
+                       p->k_stride[2] == p->v_stride[2];
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
+  int e = launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
+  return cuda_status(e);
+}
+
+skv_status skv_merge_plan(const float* o_part, const float* lse_part, const int32_t* plan_d,
+                          const skv_plan_info* info, int32_t num_heads, int32_t head_dim, void* o,
+                          int32_t o_dtype, float* lse, skv_stream_t stream) {
+  skv_status st = check_plan(plan_d, info);
+  if (st != SKV_OK) return st;
+  if (info->num_merge_rows == 0) return SKV_OK;
+  if (plan_d == nullptr || o_part == nullptr || lse_part == nullptr || o == nullptr) return SKV_ERR_INVALID;
+  if (num_heads < 1 || num_heads > 256 || head_dim < 4 || head_dim % 4) return SKV_ERR_UNSUPPORTED;
+  if (o_dtype != SKV_F32 && o_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
+  const MergeItem* items = reinterpret_cast<const MergeItem*>(plan_d + 8LL * info->num_work);
+  return cuda_status(launch_merge(o_part, lse_part, nullptr, 0, items, info->num_merge_rows, num_heads, head_dim, o,
+                                  o_dtype, lse, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+skv_status skv_paged_attn_fwd(const skv_paged_params* p, const int32_t* plan_d,
+                              const skv_plan_info* info, skv_stream_t stream) {
+  skv_status st = skv_paged_attn_partial(p, plan_d, info, stream);
+  if (st != SKV_OK) return st;
+  return skv_merge_plan(p->o_part, p->lse_part, plan_d, info, p->num_qo_heads, p->head_dim, p->o, p->o_dtype,
+                        p->lse, stream);
+}
+
+skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d,
+                              const skv_plan_info* info, skv_stream_t stream) {
+  if (p == nullptr) return SKV_ERR_INVALID;
+  skv_status st = check_plan(plan_d, info);
+  if (st != SKV_OK) return st;
+  if (p->batch < 0 || p->q_len < 1 || p->num_heads < 1 || p->page_size < 1 || p->num_pages < 0)
+    return SKV_ERR_INVALID;
+  if (p->kv_dtype != SKV_BF16 && p->kv_dtype != SKV_E4M3) return SKV_ERR_UNSUPPORTED;
+  if (p->o_dtype != SKV_F32 && p->o_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
+  if (p->kv_dtype == SKV_E4M3 && !(p->kv_scale > 0.f && std::isfinite(p->kv_scale))) return SKV_ERR_INVALID;
+  if (info->num_work > 0) {
+    if (!p->q_nope || !p->q_pe || !p->ckv || !p->kpe || !p->kv_indptr || !p->kv_indices ||
+        !p->kv_last_page_len || !p->o)
+      return SKV_ERR_INVALID;
+  }
+  const int64_t esz = p->kv_dtype == SKV_E4M3 ? 1 : 2;
+  for (int i = 0; i < 2; ++i) {
+    if (p->ckv_stride[i] < 0 || p->kpe_stride[i] < 0) return SKV_ERR_INVALID;
+    if ((p->ckv_stride[i] * esz) % 16 || (p->kpe_stride[i] * esz) % 16) return SKV_ERR_ALIGNMENT;
+  }
+  if (!aligned16(p->q_nope) || !aligned16(p->q_pe) || !aligned16(p->ckv) || !aligned16(p->kpe) ||
+      !aligned16(p->o))
+    return SKV_ERR_ALIGNMENT;
+  if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
+  if (info->kernel != KERNEL_MLA_SIMT) return SKV_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
+  int e = launch_mla_simt(*p, work, info->num_work, info->q_tile, s);
+  return cuda_status(e);
+}
+
+skv_status skv_mla_decode_fwd(const skv_mla_params* p, const int32_t* plan_d,
+                              const skv_plan_info* info, skv_stream_t stream) {
+  skv_status st = skv_mla_decode_partial(p, plan_d, info, stream);
+  if (st != SKV_OK) return st;
+  return skv_merge_plan(p->o_part, p->lse_part, plan_d, info, p->num_heads, 512, p->o, p->o_dtype, p->lse,
+                        stream);
+}
+
+skv_status skv_merge_states(const float* o_states, const float* lse_states,
+                            const int32_t* state_indptr, int32_t num_states, int64_t num_rows,
+                            int32_t num_heads, int32_t head_dim, void* o_out, int32_t o_dtype,
+                            float* lse_out, skv_stream_t stream) {
+  if (num_rows < 0 || num_heads < 1 || head_dim < 1) return SKV_ERR_INVALID;
+  if (num_rows == 0) return SKV_OK;
+  if (o_states == nullptr || lse_states == nullptr || o_out == nullptr) return SKV_ERR_INVALID;
+  if (state_indptr == nullptr && num_states < 0) return SKV_ERR_INVALID;
+  if (num_rows > INT32_MAX) return SKV_ERR_UNSUPPORTED;
+  if (head_dim % 4 != 0 || num_heads > 256) return SKV_ERR_UNSUPPORTED;
+  if (o_dtype != SKV_F32 && o_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
+  if (!aligned16(o_states) || !aligned16(o_out)) return SKV_ERR_ALIGNMENT;
+  return cuda_status(launch_merge(o_states, lse_states, state_indptr, num_states, nullptr, num_rows, num_heads,
+                                  head_dim, o_out, o_dtype, lse_out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+skv_status skv_paged_kv_gather(const skv_paged_params* p, const int32_t* token_indptr,
+                               int64_t total_tokens, void* k_out, void* v_out, skv_stream_t stream) {
+  if (p == nullptr || total_tokens < 0) return SKV_ERR_INVALID;
+  if (total_tokens == 0) return SKV_OK;
+  if (!token_indptr || !k_out || !v_out || !p->k_cache || !p->v_cache || !p->kv_indptr || !p->kv_indices ||
+      !p->kv_last_page_len)
+    return SKV_ERR_INVALID;
+  if (p->batch < 1 || p->page_size < 1 || p->num_kv_heads < 1 || p->head_dim < 1) return SKV_ERR_INVALID;
+  if (total_tokens > INT32_MAX) return SKV_ERR_UNSUPPORTED;
+  const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
+                       p->k_stride[2] == p->v_stride[2];
+  return cuda_status(launch_gather(*p, token_indptr, total_tokens, k_out, v_out, same_kv,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,47 @@
+// Internal layout of plans and the launcher interface between the C ABI (api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/splitkv.h"
+
+namespace skv {
+
+// One work item = one CTA (per KV head for GQA): request r, query tokens
+// [q_start, q_start + q_count) (global rows of q), logical pages [page_begin, page_end) of the
+// request.  part_row < 0: write O/LSE directly; otherwise the partial of query token i (0-based
+// within the item) goes to row part_row + i * part_stride of o_part / lse_part.
+struct WorkItem {
+  int32_t r, q_start, q_count, page_begin, page_end, part_row, part_stride, split;
+};
+static_assert(sizeof(WorkItem) == 32, "work item is 8 int32 words");
+
+// One merge item = one output row combined from state_count consecutive partial rows.
+struct MergeItem {
+  int32_t out_row, state_begin, state_count, pad;
+};
+static_assert(sizeof(MergeItem) == 16, "merge item is 4 int32 words");
+
+enum KernelId : int32_t {
+  KERNEL_GQA_SIMT = 1,
+  KERNEL_MLA_SIMT = 11,
+};
+
+// Plan words: [work items (8 words each)] [merge items (4 words each)].
+inline int64_t plan_words(int32_t num_work, int32_t num_merge) {
+  return 8LL * num_work + 4LL * num_merge;
+}
+
+// Launchers (host functions defined next to their kernels).  Return cudaError_t as int.
+int launch_gqa_simt(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
+                    bool same_kv, cudaStream_t s);
+int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work, int q_tile,
+                    cudaStream_t s);
+int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,
+                 int32_t num_states, const MergeItem* items, int64_t num_rows, int32_t num_heads,
+                 int32_t head_dim, void* o_out, int32_t o_dtype, float* lse_out, cudaStream_t s);
+int launch_gather(const skv_paged_params& p, const int32_t* token_indptr, int64_t total_tokens,
+                  void* k_out, void* v_out, bool same_kv, cudaStream_t s);
+
+}  // namespace skv

@@ -1,0 +1,201 @@
+"""Host-side checks of the C ABI (no GPU): the library loads and exports every declared symbol,
+the planner lays out splits / partial rows / merges as documented, and argument validation
+returns its error codes before anything is launched."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import split_kv_merge_b200 as skv
+from workloads import even_split_pages, llama70b_decode_case, tiny_gqa_case
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"SKV_API\s+[\w\s\*]+?\b(skv_\w+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared_symbols()
+    assert len(declared) >= 9
+    lib = ctypes.CDLL(skv.library_path())
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(skv.SYMBOLS) <= declared
+
+
+def test_version_and_status_strings():
+    assert skv.version() >= 1
+    assert skv.status_str(0) == "ok"
+    for code in (1, 2, 3, 4, 5, 16, 17, 18):
+        assert skv.status_str(code) != "unknown status"
+
+
+@pytest.mark.parametrize("H,q_len,F", [(16, 1, 1), (16, 4, 4), (128, 1, 1), (128, 4, 1), (32, 4, 4),
+                                       (64, 4, 2), (48, 6, 2), (16, 16, 8), (1, 3, 3)])
+def test_mla_fold_ratio(H, q_len, F):
+    # largest divisor F of q_len with H * F <= 128
+    assert skv.mla_fold_ratio(H, q_len, 128) == F
+
+
+def _items(plan):
+    w = plan.words[: 8 * plan.info.num_work].reshape(-1, 8)
+    m = plan.words[8 * plan.info.num_work:].reshape(-1, 4)
+    return w, m
+
+
+def test_tiny_fixed_two_splits_layout():
+    c = tiny_gqa_case()
+    plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, 16, 8, 2, 64, "fixed", 2)
+    w, m = _items(plan)
+    info = plan.info
+    assert info.num_work == 8 and info.max_splits == 2 and info.total_splits == 8
+    assert info.num_partial_rows == 8 and info.num_merge_rows == 4
+    # splits (2,1), (4,4), (7,6), (8,8) pages, ceil first
+    by_req = {}
+    for r, qs, qc, pb, pe, prow, pstride, j in w:
+        by_req.setdefault(int(r), {})[int(j)] = (int(pb), int(pe), int(prow), int(pstride))
+    assert [by_req[r][0][1] - by_req[r][0][0] for r in range(4)] == [2, 4, 7, 8]
+    assert [by_req[r][1][1] - by_req[r][1][0] for r in range(4)] == [1, 4, 6, 8]
+    for r in range(4):
+        assert by_req[r][0][2] + 1 == by_req[r][1][2]   # partial rows part_base + j
+        assert by_req[r][0][3] == 2
+    # merge items: out_row r, states [2r, 2r+2)
+    assert sorted(map(tuple, m[:, :3].tolist())) == [(r, 2 * r, 2) for r in range(4)]
+    # equals the generator's ceil-first split
+    assert [[0, by_req[r][0][1], by_req[r][1][1]] for r in range(4)] == even_split_pages(c.kv_indptr, 2)
+
+
+def test_plan_explicit_and_empty_splits():
+    kv_indptr = np.array([0, 3, 3, 8], np.int32)
+    last = np.array([5, 0, 16], np.int32)
+    qo = np.array([0, 2, 3, 4], np.int32)
+    sps = [[0, 0, 2, 3], [0, 0], [0, 5]]
+    plan = skv.plan_paged(qo, kv_indptr, last, 16, 4, 2, 128, "explicit", 0, sps)
+    w, m = _items(plan)
+    assert plan.info.num_partial_rows == 2 * 3   # request 0: 2 query tokens x 3 splits
+    assert plan.info.num_merge_rows == 2
+    r0 = w[w[:, 0] == 0]
+    assert sorted(r0[:, 7].tolist()) == [0, 1, 2]
+    # query token i, split j -> row i*S + j
+    for row in r0:
+        assert row[5] == 0 * 3 + row[7] and row[6] == 3
+    # request with no pages still gets a work item (writes O=0, LSE=-inf)
+    r1 = w[w[:, 0] == 1]
+    assert len(r1) == 1 and r1[0, 3] == 0 and r1[0, 4] == 0 and r1[0, 5] == -1
+
+
+def test_plan_balanced_covers_every_page_once():
+    c = llama70b_decode_case(batch=64)
+    plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, 16, 64, 8, 128, "balanced", 148)
+    w, m = _items(plan)
+    n = np.diff(c.kv_indptr)
+    for r in range(64):
+        rows = w[w[:, 0] == r]
+        spans = sorted((int(a), int(b)) for a, b in rows[:, 3:5])
+        assert spans[0][0] == 0 and spans[-1][1] == n[r]
+        assert all(spans[i][1] == spans[i + 1][0] for i in range(len(spans) - 1))
+    sizes = (w[:, 4] - w[:, 3])
+    assert list(sizes) == sorted(sizes, reverse=True)       # longest first
+    assert plan.info.num_work * 8 >= 148                    # enough CTAs for every SM
+
+
+@pytest.mark.parametrize("bad", ["last_zero", "last_big", "hq_not_multiple", "head_dim", "indptr_decreasing",
+                                 "explicit_bad_end", "fixed_zero"])
+def test_plan_rejects_bad_input(bad):
+    kv_indptr = np.array([0, 2, 5], np.int32)
+    last = np.array([3, 16], np.int32)
+    qo = np.array([0, 1, 2], np.int32)
+    args = dict(hq=8, hk=2, d=64, policy="none", param=0, sps=None)
+    if bad == "last_zero":
+        last = np.array([0, 16], np.int32)
+    elif bad == "last_big":
+        last = np.array([17, 16], np.int32)
+    elif bad == "hq_not_multiple":
+        args["hq"] = 6; args["hk"] = 4
+    elif bad == "head_dim":
+        args["d"] = 96
+    elif bad == "indptr_decreasing":
+        kv_indptr = np.array([0, 2, 1], np.int32)
+    elif bad == "explicit_bad_end":
+        args["policy"] = "explicit"; args["sps"] = [[0, 1], [0, 2]]
+    elif bad == "fixed_zero":
+        args["policy"] = "fixed"
+    with pytest.raises(skv.SkvError) as e:
+        skv.plan_paged(qo, kv_indptr, last, 16, args["hq"], args["hk"], args["d"], args["policy"], args["param"],
+                       args["sps"])
+    assert e.value.code in (skv.ERR_INVALID, skv.ERR_UNSUPPORTED)
+
+
+def test_launch_validation_returns_before_launch():
+    """Invalid arguments come back as status codes without touching the GPU (the pointers here
+    are never dereferenced)."""
+    info = skv.PlanInfo()
+    info.num_work, info.q_tile, info.kernel = 1, 1, 1
+    p = skv.PagedParams()
+    fake = 1 << 20  # 16-byte aligned, never dereferenced
+    p.q = p.k_cache = p.v_cache = p.kv_indptr = p.kv_indices = p.kv_last_page_len = p.o = fake
+    for i in range(3):
+        p.k_stride[i] = p.v_stride[i] = [2048, 128, 64][i]
+    p.batch, p.total_q, p.num_pages, p.page_size = 1, 1, 4, 16
+    p.num_qo_heads, p.num_kv_heads, p.head_dim, p.sm_scale = 8, 2, 64, 0.125
+    fwd = skv._paged_fwd
+
+    def call(**kw):
+        q = skv.PagedParams.from_buffer_copy(p)
+        for k, v in kw.items():
+            setattr(q, k, v)
+        return fwd(ctypes.byref(q), fake, ctypes.byref(info), None)
+
+    assert call(head_dim=96) == skv.ERR_UNSUPPORTED
+    assert call(num_qo_heads=6, num_kv_heads=4) == skv.ERR_INVALID
+    assert call(o=None) == skv.ERR_INVALID
+    assert call(q=fake + 2) == skv.ERR_ALIGNMENT
+    assert call(o_dtype=7) == skv.ERR_UNSUPPORTED
+    bad = skv.PagedParams.from_buffer_copy(p)
+    bad.k_stride[1] = 100   # not a multiple of 8 elements
+    assert fwd(ctypes.byref(bad), fake, ctypes.byref(info), None) == skv.ERR_ALIGNMENT
+    info2 = skv.PlanInfo.from_buffer_copy(info)
+    info2.num_partial_rows = 4     # plan splits but no partial buffers given
+    assert fwd(ctypes.byref(p), fake, ctypes.byref(info2), None) == skv.ERR_WORKSPACE
+    assert fwd(None, fake, ctypes.byref(info), None) == skv.ERR_INVALID
+    assert fwd(ctypes.byref(p), None, ctypes.byref(info), None) == skv.ERR_INVALID
+    # merge_states validation
+    assert skv._merge(fake, fake, None, -1, 4, 8, 64, fake, 1, None, None) == skv.ERR_INVALID
+    assert skv._merge(fake, fake, None, 2, 4, 8, 62, fake, 1, None, None) == skv.ERR_UNSUPPORTED
+    assert skv._merge(fake, fake, None, 2, 4, 300, 64, fake, 1, None, None) == skv.ERR_UNSUPPORTED
+    assert skv._merge(fake, fake, None, 2, 0, 8, 64, fake, 1, None, None) == skv.OK   # nothing to do
+
+
+def test_mla_validation():
+    info = skv.PlanInfo()
+    info.num_work, info.q_tile, info.kernel = 1, 1, 11
+    p = skv.MlaParams()
+    fake = 1 << 20
+    p.q_nope = p.q_pe = p.ckv = p.kpe = p.kv_indptr = p.kv_indices = p.kv_last_page_len = p.o = fake
+    p.ckv_stride[0], p.ckv_stride[1] = 64 * 576, 576
+    p.kpe_stride[0], p.kpe_stride[1] = 64 * 576, 576
+    p.batch, p.q_len, p.num_heads, p.num_pages, p.page_size, p.sm_scale = 1, 1, 16, 4, 64, 0.07
+    fwd = skv._mla_fwd
+
+    def call(**kw):
+        q = skv.MlaParams.from_buffer_copy(p)
+        for k, v in kw.items():
+            setattr(q, k, v)
+        return fwd(ctypes.byref(q), fake, ctypes.byref(info), None)
+
+    assert call(kv_dtype=5) == skv.ERR_UNSUPPORTED
+    assert call(kv_dtype=skv.E4M3, kv_scale=0.0) == skv.ERR_INVALID
+    assert call(q_len=0) == skv.ERR_INVALID
+    assert call(kpe=fake + 8) == skv.ERR_ALIGNMENT
+    bad = skv.MlaParams.from_buffer_copy(p)
+    bad.ckv_stride[1] = 577
+    assert fwd(ctypes.byref(bad), fake, ctypes.byref(info), None) == skv.ERR_ALIGNMENT

@@ -316,6 +316,22 @@ def pin_bf16():
     np.testing.assert_array_equal(got[ok], ref[ok])
 
 
+def test_e4m3_encoder_is_nearest_even():
+    """The generator's fp8 encoder picks the nearest e4m3fn value, ties to the even code."""
+    pos = OA.e4m3_to_f64(np.arange(0x7F, dtype=np.uint8))
+    rng = np.random.Generator(np.random.PCG64(8))
+    x = np.concatenate([rng.standard_normal(20000) * 60, rng.standard_normal(2000) * 1e-3,
+                        (pos[1:] + pos[:-1]) / 2, -(pos[1:] + pos[:-1]) / 2, [500.0, -1e9, 0.0]])
+    got = OA.e4m3_to_f64(e4m3_encode(x))
+    a = np.minimum(np.abs(x), 448.0)
+    d = np.abs(pos[None, :] - a[:, None])
+    best = d.min(axis=1)
+    assert np.all(np.abs(np.abs(got) - a) == best)
+    ties = (d == best[:, None]).sum(axis=1) > 1
+    codes = e4m3_encode(x) & 0x7F
+    assert np.all(codes[ties] % 2 == 0)
+
+
 PINS = [pin_brute_force, pin_decimal, pin_sdpa_library, pin_closed_forms, pin_split_merge,
         pin_merge_special, pin_permutation, pin_broadcast, pin_mla, pin_e4m3, pin_bf16]
 

@@ -23,6 +23,7 @@ decode with seqlen_q folding) and the "Move the Query, Not the Cache" summary
 """
 from __future__ import annotations
 
+import functools
 import math
 from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
@@ -54,31 +55,28 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def _e4m3_positive_values() -> np.ndarray:
-    # codes 0x00..0x7E (0x7F is NaN): exponent field e (4 bits, bias 7), mantissa m (3 bits)
-    vals = []
-    for c in range(0x7F):
-        e, m = c >> 3, c & 7
-        vals.append((m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
-    return np.array(vals, dtype=np.float64)
-
-
-_E4M3_POS = _e4m3_positive_values()
-
-
-def e4m3_encode(x: np.ndarray) -> np.ndarray:
-    """Encode float values as OCP e4m3fn codes: round to nearest, ties to even mantissa,
-    saturating to +-448.  (Storage-format conversion for the synthetic fp8 cache.)"""
-    x = np.asarray(x, dtype=np.float64)
-    a = np.minimum(np.abs(x), 448.0)
-    hi = np.searchsorted(_E4M3_POS, a, side="left")  # first value >= a
-    hi = np.minimum(hi, len(_E4M3_POS) - 1)
-    lo = np.maximum(hi - 1, 0)
-    d_hi = _E4M3_POS[hi] - a
-    d_lo = a - _E4M3_POS[lo]
-    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ((hi & 1) == 0))
-    code = np.where(pick_hi, hi, lo).astype(np.uint8)
-    return code | np.where(np.signbit(x), np.uint8(0x80), np.uint8(0))
+def e4m3_encode(x: np.ndarray, chunk: int = 1 << 24) -> np.ndarray:
+    """Encode values as OCP e4m3fn codes: round to nearest, ties to even mantissa, saturating to
+    +-448.  Exponent from frexp, mantissa rounded with rint (half-to-even); everything below 2^-6
+    is on the subnormal grid m * 2^-9.  (Storage-format conversion for the synthetic fp8 cache.)"""
+    x = np.asarray(x)
+    flat = x.reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint8)
+    for lo in range(0, flat.size, chunk):
+        v = flat[lo:lo + chunk].astype(np.float64)
+        a = np.minimum(np.abs(v), 448.0)
+        sub = a < 2.0 ** -6
+        mant, ex = np.frexp(np.where(sub, 1.0, a))        # a = mant * 2^ex, mant in [0.5, 1)
+        e = ex - 1                                         # a = (2 mant) * 2^e, 2 mant in [1, 2)
+        m = np.rint((2.0 * mant - 1.0) * 8.0)
+        carry = m == 8.0
+        e = np.where(carry, e + 1, e)
+        m = np.where(carry, 0.0, m)
+        code_n = ((e + 7) << 3).astype(np.int64) | m.astype(np.int64)
+        code_s = np.rint(a * 2.0 ** 9).astype(np.int64)   # 0..8 (8 is the smallest normal, code 0x08)
+        code = np.minimum(np.where(sub, code_s, code_n), 0x7E).astype(np.uint8)
+        out[lo:lo + chunk] = code | np.where(np.signbit(v), np.uint8(0x80), np.uint8(0))
+    return out.reshape(x.shape)
 
 
 # ----------------------------------------------------------------------------- random draws
@@ -340,6 +338,22 @@ def shared_kv_prefill_case(replicated: bool = False, n_batches: int = 32, q_len:
                      1.0 / math.sqrt(d), num_pages, meta={"kv_len": kv_len, "q_len": q_len})
 
 
+@functools.lru_cache(maxsize=4)
+def _latent_cache(seed: int, num_pages: int, page_size: int, kv_dtype: str):
+    """[num_pages, P, 576] latent cache (read-only, shared between MLA sub-configurations)."""
+    raw = normal_f32(seed, 3, num_pages * page_size * 576).reshape(num_pages, page_size, 576)
+    if kv_dtype == "bf16":
+        cache, kv_scale = f32_to_bf16_bits(raw), 1.0
+    elif kv_dtype == "e4m3":
+        amax = float(np.max(np.abs(raw)))
+        kv_scale = float(np.float32(amax / 448.0))
+        cache = e4m3_encode(raw / np.float64(kv_scale))
+    else:
+        raise ValueError(kv_dtype)
+    cache.setflags(write=False)
+    return cache, kv_scale
+
+
 def mla_decode_case(num_heads: int = 16, q_len: int = 1, kv_dtype: str = "bf16", batch: int = 32,
                     seed: int = 4, len_range=(4096, 32768), page_size: int = 64,
                     poison: bool = False) -> MlaCase:
@@ -351,18 +365,9 @@ def mla_decode_case(num_heads: int = 16, q_len: int = 1, kv_dtype: str = "bf16",
     kv_indptr, kv_indices, last, num_pages = build_page_table(rng, lengths, page_size, 0)
     q_nope = normal_bf16(seed, 1 + 10 * num_heads + q_len, (batch, q_len, num_heads, 512))
     q_pe = normal_bf16(seed, 2 + 10 * num_heads + q_len, (batch, q_len, num_heads, 64))
-    raw = normal_f32(seed, 3, num_pages * page_size * 576).reshape(num_pages, page_size, 576)
-    if kv_dtype == "bf16":
-        cache = f32_to_bf16_bits(raw)
-        kv_scale = 1.0
-    elif kv_dtype == "e4m3":
-        amax = float(np.max(np.abs(raw)))
-        kv_scale = float(np.float32(amax / 448.0))
-        cache = e4m3_encode(raw / np.float64(kv_scale))
-    else:
-        raise ValueError(kv_dtype)
-    del raw
+    cache, kv_scale = _latent_cache(seed, num_pages, page_size, kv_dtype)
     if poison:
+        cache = cache.copy()
         used = np.zeros(num_pages, dtype=bool)
         used[kv_indices] = True
         nan = BF16_NAN if kv_dtype == "bf16" else E4M3_NAN
