@@ -211,8 +211,14 @@ skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32
     if (req[r].q_len < 0) return SKV_ERR_INVALID;
   }
   const int32_t g = num_qo_heads / num_kv_heads;
-  const int32_t kernel = KERNEL_GQA_SIMT;
-  const int32_t q_tile = std::max<int32_t>(1, 16 / g);
+  int32_t max_q = 1;
+  for (const auto& q : req) max_q = std::max(max_q, q.q_len);
+  // tensor-core decode when the shape fits its tiles (query rows of a work item <= 16), else the
+  // generic CUDA-core kernel
+  const int32_t tc_q_tile = std::max<int32_t>(1, std::min<int32_t>(16 / std::max<int32_t>(g, 1), max_q));
+  const bool tc = g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
+  const int32_t kernel = tc ? KERNEL_GQA_TC_DECODE : KERNEL_GQA_SIMT;
+  const int32_t q_tile = tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
   return plan_common(batch, req, q_tile, num_kv_heads, policy, param, split_indptr_h, split_bounds_h,
                      kernel, plan_h, plan_capacity, info);
 }
@@ -256,12 +262,13 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
   if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
     return SKV_ERR_ALIGNMENT;
   if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
-  if (info->kernel != KERNEL_GQA_SIMT) return SKV_ERR_INVALID;
+  if (info->kernel != KERNEL_GQA_SIMT && info->kernel != KERNEL_GQA_TC_DECODE) return SKV_ERR_INVALID;
   const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
                        p->k_stride[2] == p->v_stride[2];
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  int e = launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
+  int e = info->kernel == KERNEL_GQA_TC_DECODE ? launch_gqa_tc_decode(*p, work, info->num_work, info->q_tile, s)
+                                                : launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
   return cuda_status(e);
 }
 

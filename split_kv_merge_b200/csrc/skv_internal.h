@@ -25,6 +25,7 @@ static_assert(sizeof(MergeItem) == 16, "merge item is 4 int32 words");
 
 enum KernelId : int32_t {
   KERNEL_GQA_SIMT = 1,
+  KERNEL_GQA_TC_DECODE = 2,
   KERNEL_MLA_SIMT = 11,
 };
 
@@ -36,6 +37,9 @@ inline int64_t plan_words(int32_t num_work, int32_t num_merge) {
 // Launchers (host functions defined next to their kernels).  Return cudaError_t as int.
 int launch_gqa_simt(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
                     bool same_kv, cudaStream_t s);
+bool gqa_tc_decode_supported(int head_dim, int page_size, int group, int q_tile);
+int launch_gqa_tc_decode(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
+                         cudaStream_t s);
 int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work, int q_tile,
                     cudaStream_t s);
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,
