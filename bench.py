@@ -175,10 +175,11 @@ def _cpu_baseline(cases, budget_s=12.0):
                       f"{dt:.1f} s, {os.cpu_count()} host cores visible)"}
 
 
-def _make_cases(rank: int):
+def _make_cases(rank: int, batch: int = 64):
     from workloads import llama70b_decode_case
-    seed = 2 + 1000 * rank   # each rank holds its own batch of 64 requests (weak scaling)
-    return [llama70b_decode_case(independent_v=False, seed=seed), llama70b_decode_case(independent_v=True, seed=seed)]
+    seed = 2 + 1000 * rank   # each rank holds its own batch of requests (weak scaling)
+    return [llama70b_decode_case(independent_v=False, seed=seed, batch=batch),
+            llama70b_decode_case(independent_v=True, seed=seed, batch=batch)]
 
 
 def run_reference(args):
@@ -233,7 +234,7 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cases = _make_cases(rank)
+    cases = _make_cases(rank, args.batch)
     kv_bytes_step = sum(_kv_bytes(c) for c in cases)
     runs = []
     for c in cases:
@@ -409,6 +410,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--ref-budget", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=64, help="requests per GPU (64 = the benchmark workload; "
+                                                          "smaller only for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

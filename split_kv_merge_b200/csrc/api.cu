@@ -28,7 +28,7 @@ struct ReqShape {
 
 // Shared planner: work items over (request, query tile, split) and merge items for split rows.
 skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t q_tile,
-                       int64_t units_per_page, int32_t policy, int32_t param,
+                       int64_t units_per_page, int32_t units_per_sm, int32_t policy, int32_t param,
                        const int32_t* split_indptr_h, const int32_t* split_bounds_h,
                        int32_t kernel, int32_t* plan_h, int64_t plan_capacity,
                        skv_plan_info* info) {
@@ -51,9 +51,11 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t 
       const int64_t tiles = (q.q_len + q_tile - 1) / q_tile;
       total_units += tiles * q.n_pages * units_per_page;
     }
-    // aim for ~8 work items per SM-slot pair of waves; never below 8 pages per chunk
-    const int64_t target_items = (int64_t)sms * 8;
-    chunk = std::max<int64_t>(8, (total_units + target_items - 1) / std::max<int64_t>(1, target_items));
+    // chunk (pages per split) so that about `units_per_sm` CTA-units land on every SM: a work item
+    // of p pages becomes `units_per_page` CTA-units (one per KV head for GQA) of p pages each, so
+    // the total CTA-unit work is total_units page-units.  Never below 8 pages.
+    const int64_t target = std::max<int64_t>(1, (int64_t)sms * units_per_sm);
+    chunk = std::max<int64_t>(8, (total_units + target - 1) / target);
   } else if (policy == SKV_SPLIT_FIXED) {
     if (param < 1) return SKV_ERR_INVALID;
   } else if (policy == SKV_SPLIT_EXPLICIT) {
@@ -83,8 +85,7 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t 
     } else {
       if (policy == SKV_SPLIT_FIXED) S = param;
       if (policy == SKV_SPLIT_BALANCED) {
-        const int64_t units = (int64_t)q.n_pages * units_per_page;
-        S = (int32_t)std::max<int64_t>(1, (units + chunk - 1) / chunk);
+        S = (int32_t)std::max<int64_t>(1, ((int64_t)q.n_pages + chunk - 1) / chunk);
         S = std::min<int32_t>(S, std::max<int32_t>(1, q.n_pages));
       }
       bounds.push_back(0);
@@ -215,12 +216,18 @@ skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32
   for (const auto& q : req) max_q = std::max(max_q, q.q_len);
   // tensor-core decode when the shape fits its tiles (query rows of a work item <= 16), else the
   // generic CUDA-core kernel
+  // all-KV-heads tensor-core decode when every request's query rows per KV head fit its 8
+  // columns (whole pages stream contiguously); else the per-KV-head tensor-core decode; else the
+  // generic CUDA-core kernel
+  const bool wide = g <= 8 && 8 % g == 0 && max_q * g <= 8 &&
+                    gqa_tc_wide_supported(head_dim, page_size, num_kv_heads, g, 8 / g);
   const int32_t tc_q_tile = std::max<int32_t>(1, std::min<int32_t>(16 / std::max<int32_t>(g, 1), max_q));
-  const bool tc = g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
-  const int32_t kernel = tc ? KERNEL_GQA_TC_DECODE : KERNEL_GQA_SIMT;
-  const int32_t q_tile = tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
-  return plan_common(batch, req, q_tile, num_kv_heads, policy, param, split_indptr_h, split_bounds_h,
-                     kernel, plan_h, plan_capacity, info);
+  const bool tc = !wide && g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
+  const int32_t kernel = wide ? KERNEL_GQA_TC_WIDE : tc ? KERNEL_GQA_TC_DECODE : KERNEL_GQA_SIMT;
+  const int32_t q_tile = wide ? 8 / g : tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
+  // persistent tensor-core kernel: a few large units per SM; CUDA-core kernel: many small CTAs
+  return plan_common(batch, req, q_tile, wide ? 1 : num_kv_heads, (wide || tc) ? 6 : 64, policy, param,
+                     split_indptr_h, split_bounds_h, kernel, plan_h, plan_capacity, info);
 }
 
 skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
@@ -238,7 +245,7 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
     req[r].q_len = q_len;
   }
   const int32_t fold = skv_mla_fold_ratio(num_heads, q_len, 128);
-  return plan_common(batch, req, fold, 1, policy, param, split_indptr_h, split_bounds_h, KERNEL_MLA_SIMT,
+  return plan_common(batch, req, fold, 1, 8, policy, param, split_indptr_h, split_bounds_h, KERNEL_MLA_SIMT,
                      plan_h, plan_capacity, info);
 }
 
@@ -262,13 +269,15 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
   if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
     return SKV_ERR_ALIGNMENT;
   if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
-  if (info->kernel != KERNEL_GQA_SIMT && info->kernel != KERNEL_GQA_TC_DECODE) return SKV_ERR_INVALID;
+  if (info->kernel != KERNEL_GQA_SIMT && info->kernel != KERNEL_GQA_TC_DECODE && info->kernel != KERNEL_GQA_TC_WIDE)
+    return SKV_ERR_INVALID;
   const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
                        p->k_stride[2] == p->v_stride[2];
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  int e = info->kernel == KERNEL_GQA_TC_DECODE ? launch_gqa_tc_decode(*p, work, info->num_work, info->q_tile, s)
-                                                : launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
+  int e = info->kernel == KERNEL_GQA_TC_WIDE     ? launch_gqa_tc_wide(*p, work, info->num_work, info->q_tile, s)
+          : info->kernel == KERNEL_GQA_TC_DECODE ? launch_gqa_tc_decode(*p, work, info->num_work, info->q_tile, s)
+                                                 : launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
   return cuda_status(e);
 }
 
@@ -279,7 +288,7 @@ skv_status skv_merge_plan(const float* o_part, const float* lse_part, const int3
   if (st != SKV_OK) return st;
   if (info->num_merge_rows == 0) return SKV_OK;
   if (plan_d == nullptr || o_part == nullptr || lse_part == nullptr || o == nullptr) return SKV_ERR_INVALID;
-  if (num_heads < 1 || num_heads > 256 || head_dim < 4 || head_dim % 4) return SKV_ERR_UNSUPPORTED;
+  if (num_heads < 1 || num_heads > 65535 || head_dim < 4 || head_dim % 4) return SKV_ERR_UNSUPPORTED;
   if (o_dtype != SKV_F32 && o_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
   const MergeItem* items = reinterpret_cast<const MergeItem*>(plan_d + 8LL * info->num_work);
   return cuda_status(launch_merge(o_part, lse_part, nullptr, 0, items, info->num_merge_rows, num_heads, head_dim, o,
@@ -342,7 +351,7 @@ skv_status skv_merge_states(const float* o_states, const float* lse_states,
   if (o_states == nullptr || lse_states == nullptr || o_out == nullptr) return SKV_ERR_INVALID;
   if (state_indptr == nullptr && num_states < 0) return SKV_ERR_INVALID;
   if (num_rows > INT32_MAX) return SKV_ERR_UNSUPPORTED;
-  if (head_dim % 4 != 0 || num_heads > 256) return SKV_ERR_UNSUPPORTED;
+  if (head_dim % 4 != 0 || num_heads > 65535) return SKV_ERR_UNSUPPORTED;
   if (o_dtype != SKV_F32 && o_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
   if (!aligned16(o_states) || !aligned16(o_out)) return SKV_ERR_ALIGNMENT;
   return cuda_status(launch_merge(o_states, lse_states, state_indptr, num_states, nullptr, num_rows, num_heads,

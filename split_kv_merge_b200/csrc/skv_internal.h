@@ -26,6 +26,7 @@ static_assert(sizeof(MergeItem) == 16, "merge item is 4 int32 words");
 enum KernelId : int32_t {
   KERNEL_GQA_SIMT = 1,
   KERNEL_GQA_TC_DECODE = 2,
+  KERNEL_GQA_TC_WIDE = 3,
   KERNEL_MLA_SIMT = 11,
 };
 
@@ -40,6 +41,8 @@ int launch_gqa_simt(const skv_paged_params& p, const WorkItem* work, int num_wor
 bool gqa_tc_decode_supported(int head_dim, int page_size, int group, int q_tile);
 int launch_gqa_tc_decode(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
                          cudaStream_t s);
+bool gqa_tc_wide_supported(int head_dim, int page_size, int num_kv_heads, int group, int q_tile);
+int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile, cudaStream_t s);
 int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work, int q_tile,
                     cudaStream_t s);
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,

@@ -171,7 +171,7 @@ def test_launch_validation_returns_before_launch():
     # merge_states validation
     assert skv._merge(fake, fake, None, -1, 4, 8, 64, fake, 1, None, None) == skv.ERR_INVALID
     assert skv._merge(fake, fake, None, 2, 4, 8, 62, fake, 1, None, None) == skv.ERR_UNSUPPORTED
-    assert skv._merge(fake, fake, None, 2, 4, 300, 64, fake, 1, None, None) == skv.ERR_UNSUPPORTED
+    assert skv._merge(fake, fake, None, 2, 4, 70000, 64, fake, 1, None, None) == skv.ERR_UNSUPPORTED
     assert skv._merge(fake, fake, None, 2, 0, 8, 64, fake, 1, None, None) == skv.OK   # nothing to do
 
 

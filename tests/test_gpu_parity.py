@@ -307,3 +307,64 @@ def test_deterministic_bitwise():
     o1, l1, _, _ = _run_paged(c, "balanced", 148)
     o2, l2, _, _ = _run_paged(c, "balanced", 148)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ----------------------------------------------------------------------------- kernel coverage
+@pytest.mark.parametrize("page_size", [16, 64])
+@pytest.mark.parametrize("policy,param", [("none", 0), ("fixed", 3), ("balanced", 148)])
+def test_all_heads_decode_edges(page_size, policy, param):
+    """The all-KV-heads decode kernel (8 KV heads, 8 query rows each): empty requests, a request
+    with no query rows, lengths around page and tile boundaries, poisoned unused pages/tails."""
+    from workloads.gen import _make_paged
+    c = _make_paged("wide_edge", 21, [0, 16, 17, 1, 32, 300, 1000], 1, 64, 8, 128, page_size, True,
+                    extra_pages=3, poison=True, qo_lens=[1, 1, 0, 1, 1, 1, 1])
+    o, lse, ex, _ = _run_paged(c, policy, param)
+    assert ex["plan"].info.kernel == 3
+    O, LSE = _oracle_paged(c)
+    _cmp(_np(o), _np(lse), O, LSE, where=f"wide edge P{page_size} {policy}")
+
+
+def test_all_heads_decode_two_query_tokens():
+    """g = 4 with two query tokens per request also fills the 8 columns per KV head."""
+    from workloads.gen import _make_paged
+    c = _make_paged("wide_q2", 22, [700, 33, 2048], 2, 32, 8, 128, 16, False)
+    o, lse, ex, _ = _run_paged(c, "fixed", 2)
+    assert ex["plan"].info.kernel == 3 and ex["plan"].info.q_tile == 2
+    O, LSE = _oracle_paged(c)
+    _cmp(_np(o), _np(lse), O, LSE, where="wide q2")
+
+
+def test_per_head_tensor_core_decode():
+    """Shapes the all-heads kernel does not take (4 KV heads, 4 query rows each) run on the
+    per-KV-head tensor-core kernel."""
+    from workloads.gen import _make_paged
+    c = _make_paged("perhead", 23, [500, 64, 1500, 0], 1, 16, 4, 128, 32, True, poison=True)
+    o, lse, ex, _ = _run_paged(c, "fixed", 2)
+    assert ex["plan"].info.kernel == 2
+    O, LSE = _oracle_paged(c)
+    _cmp(_np(o), _np(lse), O, LSE, where="per-head tc")
+
+
+@pytest.mark.parametrize("policy,param", [("none", 0), ("fixed", 3)])
+def test_all_heads_decode_rising_scores(policy, param):
+    """Scores that keep growing along the sequence (K scaled up with the token position, and one
+    dominant key near the end) make the running maximum rise many times, exercising the rescale
+    of l and of O in tensor memory."""
+    from workloads.gen import _make_paged, bf16_bits_to_f32, f32_to_bf16_bits
+    import oracle.attention as OA_
+    c = _make_paged("rising", 24, [40, 333, 1200, 2047], 1, 64, 8, 128, 16, False)
+    k = bf16_bits_to_f32(c.k_store).copy()
+    for r in range(c.batch):
+        pages, slots = OA_.request_token_slots(c.kv_indptr, c.kv_indices, c.kv_last_page_len, 16, r)
+        L = len(pages)
+        ramp = (1.0 + 6.0 * np.arange(L) / max(1, L)).astype(np.float32)
+        k[pages, slots] *= ramp[:, None, None]
+        if L > 8:  # a dominant key near the end, aligned with query head 0 of each KV head
+            q0 = bf16_bits_to_f32(c.q[c.qo_indptr[r]]).reshape(8, 8, 128)[:, 0, :]
+            k[pages[L - 5], slots[L - 5]] = 30.0 * q0 / np.linalg.norm(q0, axis=1, keepdims=True)
+    c.k_store = f32_to_bf16_bits(k).reshape(c.k_store.shape)
+    c.k = c.k_store
+    o, lse, ex, _ = _run_paged(c, policy, param)
+    assert ex["plan"].info.kernel == 3
+    O, LSE = _oracle_paged(c)
+    _cmp(_np(o), _np(lse), O, LSE, where=f"rising {policy}")
