@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "paged decode attention: achieved KV GB/s (% of HBM peak), µs per decode step"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-KERNEL_SOURCES = ["split_kv_merge_b200/csrc/gqa_tc_decode.cu", "split_kv_merge_b200/csrc/gqa_simt.cu"]
+KERNEL_SOURCES = ["split_kv_merge_b200/csrc/gqa_tc_wide.cu", "split_kv_merge_b200/csrc/tc_ptx.cuh"]
 
 
 def _peaks():
@@ -316,7 +316,8 @@ def run_ours(args):
     attn_avg_ms = statistics.mean(attn_ms)
     per_launch_bytes = kv_bytes_step / len(runs)
     achieved = per_launch_bytes / (attn_avg_ms * 1e-3) / 1e9
-    kernel = "gqa_tc_decode" if runs[0]["plan"].info.kernel == 2 else "gqa_simt_kernel"
+    kernel = {1: "gqa_simt_kernel", 2: "gqa_tc_decode_kernel", 3: "gqa_tc_wide_kernel"}.get(
+        runs[0]["plan"].info.kernel, "unknown")
     src_hash = _kernel_hash(KERNEL_SOURCES)
     tr = _traffic_record(kernel, src_hash)
     line = {

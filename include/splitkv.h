@@ -76,8 +76,9 @@ typedef enum { SKV_BF16 = 0, SKV_F32 = 1, SKV_E4M3 = 2 } skv_dtype;
 typedef enum {
   SKV_SPLIT_NONE = 0,     /* one split per request                                           */
   SKV_SPLIT_FIXED = 1,    /* `param` splits per request (earlier splits take the extra page)  */
-  SKV_SPLIT_BALANCED = 2, /* chunk sizes chosen so all SMs stay busy; `param` = SM count       */
-                          /* (0 = query the current device)                                    */
+  SKV_SPLIT_BALANCED = 2, /* splits chosen so all SMs stay busy; `param` = SM count (0 = query */
+                          /* the current device).  For the persistent tensor-core kernels the  */
+                          /* KV of all requests is cut into `param` equal slices, one per CTA. */
   SKV_SPLIT_EXPLICIT = 3  /* boundaries given in split_indptr_h / split_bounds_h               */
 } skv_split_policy;
 
@@ -91,6 +92,9 @@ typedef struct {
   int32_t plan_words;       /* int32 words of the plan actually used                          */
   int32_t max_splits;       /* largest split count of any request                             */
   int32_t total_splits;     /* sum over requests of their split counts                        */
+  int32_t num_ctas;         /* persistent kernels: CTAs the plan was balanced for (else 0);  */
+                            /*   CTA c runs work items cta_indptr[c] .. cta_indptr[c+1]       */
+  int32_t cta_offset;       /* int32 word offset of cta_indptr [num_ctas+1] in the plan       */
 } skv_plan_info;
 
 /* -------------------------------------------------------------------------------------------

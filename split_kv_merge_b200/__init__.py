@@ -38,7 +38,8 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("num_work", ctypes.c_int32), ("num_partial_rows", ctypes.c_int32),
                 ("num_merge_rows", ctypes.c_int32), ("kernel", ctypes.c_int32),
                 ("q_tile", ctypes.c_int32), ("plan_words", ctypes.c_int32),
-                ("max_splits", ctypes.c_int32), ("total_splits", ctypes.c_int32)]
+                ("max_splits", ctypes.c_int32), ("total_splits", ctypes.c_int32),
+                ("num_ctas", ctypes.c_int32), ("cta_offset", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {k: getattr(self, k) for k, _ in self._fields_}

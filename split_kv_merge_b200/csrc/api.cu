@@ -26,74 +26,153 @@ struct ReqShape {
   int32_t q_start, q_len, n_pages;
 };
 
+int device_sms(int param) {
+  int sms = param;
+  if (sms <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+    cudaGetLastError();
+  }
+  return sms;
+}
+
+// Persistent-kernel options of the planner: the CTA count the work is balanced over and the
+// tokens one kernel tile covers.  flat_ctas == 0: not persistent (one CTA per work item).
+struct PersistOpts {
+  int32_t flat_ctas = 0;
+  int32_t tile_tokens = 128;
+  int32_t page_size = 1;
+};
+
+// Tiles of logical pages [a, b) of a request of length L (pages of `page_size` tokens).
+int64_t range_tiles(int64_t a, int64_t b, int64_t L, int32_t P, int32_t tile) {
+  const int64_t t0 = a * P, t1 = std::min<int64_t>(b * P, L);
+  return t1 > t0 ? (t1 - t0 + tile - 1) / tile : 0;
+}
+
 // Shared planner: work items over (request, query tile, split) and merge items for split rows.
-skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t q_tile,
-                       int64_t units_per_page, int32_t units_per_sm, int32_t policy, int32_t param,
-                       const int32_t* split_indptr_h, const int32_t* split_bounds_h,
-                       int32_t kernel, int32_t* plan_h, int64_t plan_capacity,
-                       skv_plan_info* info) {
+// BALANCED with a persistent kernel cuts the concatenated KV of all requests into flat_ctas
+// slices of equal tile count (cuts at page boundaries, no piece below a few tiles), so every CTA
+// streams the same amount and requests are split only where a slice boundary falls; the other
+// policies hand whole work items to the persistent CTAs longest-first (greedy least-loaded).
+skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const std::vector<int64_t>& kv_len,
+                       int32_t q_tile, int64_t units_per_page, int32_t units_per_sm, int32_t policy, int32_t param,
+                       const int32_t* split_indptr_h, const int32_t* split_bounds_h, int32_t kernel,
+                       const PersistOpts& po, int32_t* plan_h, int64_t plan_capacity, skv_plan_info* info) {
   if (info == nullptr) return SKV_ERR_INVALID;
   std::memset(info, 0, sizeof(*info));
   if (q_tile < 1) return SKV_ERR_INVALID;
-  // per-request split counts
+  if (policy == SKV_SPLIT_FIXED) {
+    if (param < 1) return SKV_ERR_INVALID;
+  } else if (policy == SKV_SPLIT_EXPLICIT) {
+    if (split_indptr_h == nullptr || split_bounds_h == nullptr) return SKV_ERR_INVALID;
+    if (split_indptr_h[0] != 0) return SKV_ERR_INVALID;
+  } else if (policy != SKV_SPLIT_NONE && policy != SKV_SPLIT_BALANCED) {
+    return SKV_ERR_INVALID;
+  }
+  const bool persistent = po.flat_ctas > 0;
+  const bool flat = persistent && policy == SKV_SPLIT_BALANCED;
+  const int P = po.page_size, T = po.tile_tokens;
+
+  // ---- per-request split boundaries (and, for the flat cut, the CTA of every piece)
+  std::vector<std::vector<int32_t>> bounds(batch);
+  std::vector<std::vector<int32_t>> piece_cta(batch);
   int64_t chunk = 0;
-  if (policy == SKV_SPLIT_BALANCED) {
-    int sms = param;
-    if (sms <= 0) {
-      int dev = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        sms = 148;
-      cudaGetLastError();
-    }
+  if (policy == SKV_SPLIT_BALANCED && !flat) {
+    const int sms = device_sms(param);
     int64_t total_units = 0;
     for (const auto& q : req) {
       const int64_t tiles = (q.q_len + q_tile - 1) / q_tile;
       total_units += tiles * q.n_pages * units_per_page;
     }
-    // chunk (pages per split) so that about `units_per_sm` CTA-units land on every SM: a work item
-    // of p pages becomes `units_per_page` CTA-units (one per KV head for GQA) of p pages each, so
-    // the total CTA-unit work is total_units page-units.  Never below 8 pages.
+    // pages per split so that about `units_per_sm` CTA-units land on every SM: a work item of p
+    // pages becomes `units_per_page` CTA-units (one per KV head for GQA); never below 8 pages.
     const int64_t target = std::max<int64_t>(1, (int64_t)sms * units_per_sm);
     chunk = std::max<int64_t>(8, (total_units + target - 1) / target);
-  } else if (policy == SKV_SPLIT_FIXED) {
-    if (param < 1) return SKV_ERR_INVALID;
-  } else if (policy == SKV_SPLIT_EXPLICIT) {
-    if (split_indptr_h == nullptr || split_bounds_h == nullptr) return SKV_ERR_INVALID;
-    if (split_indptr_h[0] != 0) return SKV_ERR_INVALID;
-  } else if (policy != SKV_SPLIT_NONE) {
-    return SKV_ERR_INVALID;
   }
-
-  std::vector<WorkItem> work;
-  std::vector<MergeItem> merges;
-  int32_t part_base = 0, max_splits = 0, total_splits = 0;
-  std::vector<int32_t> bounds;
-  for (int32_t r = 0; r < batch; ++r) {
-    const ReqShape& q = req[r];
-    int32_t S = 1;
-    bounds.clear();
-    if (policy == SKV_SPLIT_EXPLICIT) {
-      S = split_indptr_h[r + 1] - split_indptr_h[r];
-      if (S < 1) return SKV_ERR_INVALID;
-      const int32_t* b = split_bounds_h + split_indptr_h[r] + r;
-      if (b[0] != 0 || b[S] != q.n_pages) return SKV_ERR_INVALID;
-      for (int j = 0; j <= S; ++j) {
-        if (j > 0 && b[j] < b[j - 1]) return SKV_ERR_INVALID;
-        bounds.push_back(b[j]);
+  if (flat) {
+    const int G = po.flat_ctas;
+    std::vector<int64_t> w(batch, 0);
+    double total = 0;
+    for (int32_t r = 0; r < batch; ++r) {
+      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile;
+      w[r] = qt * range_tiles(0, req[r].n_pages, kv_len[r], P, T);
+      total += (double)w[r];
+    }
+    const double target = total / G;
+    const int64_t min_piece = std::max<int64_t>(1, std::min<int64_t>(4, (int64_t)target));
+    int cta = 0;
+    double cum = 0;
+    for (int32_t r = 0; r < batch; ++r) {
+      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile;
+      const int32_t n = req[r].n_pages;
+      bounds[r].push_back(0);
+      if (n == 0 || qt == 0) {  // nothing to stream: one (empty) piece on the current CTA
+        bounds[r].push_back(n);
+        piece_cta[r].push_back(cta);
+        continue;
       }
-    } else {
-      if (policy == SKV_SPLIT_FIXED) S = param;
-      if (policy == SKV_SPLIT_BALANCED) {
-        S = (int32_t)std::max<int64_t>(1, ((int64_t)q.n_pages + chunk - 1) / chunk);
-        S = std::min<int32_t>(S, std::max<int32_t>(1, q.n_pages));
-      }
-      bounds.push_back(0);
-      for (int j = 0; j < S; ++j) {
-        const int32_t rem = q.n_pages - bounds.back();
-        bounds.push_back(bounds.back() + (rem + (S - j) - 1) / (S - j));  // ceil first
+      int32_t a = 0;
+      while (a < n) {
+        double room = (cta + 1) * target - cum;
+        if (room < (double)min_piece && cta < G - 1) {
+          ++cta;
+          room = (cta + 1) * target - cum;
+        }
+        // largest b with work(a, b) <= room (at least one page), or the whole rest
+        int32_t b = a + 1;
+        if (cta == G - 1) {
+          b = n;
+        } else {
+          while (b < n && (double)(qt * range_tiles(a, b + 1, kv_len[r], P, T)) <= room) ++b;
+          if (qt * range_tiles(b, n, kv_len[r], P, T) < min_piece) b = n;  // no tiny remainder
+        }
+        const int64_t wt = qt * range_tiles(a, b, kv_len[r], P, T);
+        bounds[r].push_back(b);
+        piece_cta[r].push_back(cta);
+        cum += (double)wt;
+        a = b;
+        if (cum >= (cta + 1) * target - 0.5 && cta < G - 1) ++cta;
       }
     }
+  } else {
+    for (int32_t r = 0; r < batch; ++r) {
+      const ReqShape& q = req[r];
+      int32_t S = 1;
+      if (policy == SKV_SPLIT_EXPLICIT) {
+        S = split_indptr_h[r + 1] - split_indptr_h[r];
+        if (S < 1) return SKV_ERR_INVALID;
+        const int32_t* b = split_bounds_h + split_indptr_h[r] + r;
+        if (b[0] != 0 || b[S] != q.n_pages) return SKV_ERR_INVALID;
+        for (int j = 0; j <= S; ++j) {
+          if (j > 0 && b[j] < b[j - 1]) return SKV_ERR_INVALID;
+          bounds[r].push_back(b[j]);
+        }
+      } else {
+        if (policy == SKV_SPLIT_FIXED) S = param;
+        if (policy == SKV_SPLIT_BALANCED) {
+          S = (int32_t)std::max<int64_t>(1, ((int64_t)q.n_pages + chunk - 1) / chunk);
+          S = std::min<int32_t>(S, std::max<int32_t>(1, q.n_pages));
+        }
+        bounds[r].push_back(0);
+        for (int j = 0; j < S; ++j) {
+          const int32_t rem = q.n_pages - bounds[r].back();
+          bounds[r].push_back(bounds[r].back() + (rem + (S - j) - 1) / (S - j));  // ceil first
+        }
+      }
+    }
+  }
+
+  // ---- work items, merge items
+  std::vector<WorkItem> work;
+  std::vector<int32_t> work_cta;
+  std::vector<MergeItem> merges;
+  int32_t part_base = 0, max_splits = 0, total_splits = 0;
+  for (int32_t r = 0; r < batch; ++r) {
+    const ReqShape& q = req[r];
+    const int32_t S = (int32_t)bounds[r].size() - 1;
     max_splits = std::max(max_splits, S);
     total_splits += S;
     if (q.q_len == 0) continue;
@@ -104,12 +183,13 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t 
         w.r = r;
         w.q_start = q.q_start + q0;
         w.q_count = qc;
-        w.page_begin = bounds[j];
-        w.page_end = bounds[j + 1];
+        w.page_begin = bounds[r][j];
+        w.page_end = bounds[r][j + 1];
         w.part_row = S > 1 ? part_base + q0 * S + j : -1;
         w.part_stride = S;
         w.split = j;
         work.push_back(w);
+        work_cta.push_back(flat ? piece_cta[r][j] : 0);
       }
     }
     if (S > 1) {
@@ -117,10 +197,43 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t 
       part_base += q.q_len * S;
     }
   }
-  // longest items first: the hardware hands out CTAs roughly in index order
-  std::stable_sort(work.begin(), work.end(), [](const WorkItem& a, const WorkItem& b) {
-    return (a.page_end - a.page_begin) * a.q_count > (b.page_end - b.page_begin) * b.q_count;
-  });
+  auto item_tiles = [&](const WorkItem& w) {
+    return (int64_t)w.q_count * (1 + range_tiles(w.page_begin, w.page_end, kv_len[w.r], P, T));
+  };
+  std::vector<int32_t> cta_indptr;
+  int32_t num_ctas = 0;
+  if (persistent) {
+    std::vector<int32_t> order(work.size());
+    for (size_t i = 0; i < work.size(); ++i) order[i] = (int32_t)i;
+    if (!flat) {
+      // longest first onto the least-loaded CTA
+      const int G = std::max<int32_t>(1, std::min<int32_t>(po.flat_ctas, (int32_t)work.size()));
+      std::stable_sort(order.begin(), order.end(),
+                       [&](int32_t x, int32_t y) { return item_tiles(work[x]) > item_tiles(work[y]); });
+      std::vector<int64_t> load(G, 0);
+      for (int32_t i : order) {
+        const int c = (int)(std::min_element(load.begin(), load.end()) - load.begin());
+        work_cta[i] = c;
+        load[c] += item_tiles(work[i]);
+      }
+    }
+    for (int32_t c : work_cta) num_ctas = std::max(num_ctas, c + 1);
+    std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return work_cta[x] < work_cta[y]; });
+    std::vector<WorkItem> sorted;
+    sorted.reserve(work.size());
+    cta_indptr.assign(num_ctas + 1, 0);
+    for (int32_t i : order) {
+      sorted.push_back(work[i]);
+      ++cta_indptr[work_cta[i] + 1];
+    }
+    for (int c = 0; c < num_ctas; ++c) cta_indptr[c + 1] += cta_indptr[c];
+    work.swap(sorted);
+  } else {
+    // longest items first: the hardware hands out CTAs roughly in index order
+    std::stable_sort(work.begin(), work.end(), [](const WorkItem& a, const WorkItem& b) {
+      return (a.page_end - a.page_begin) * a.q_count > (b.page_end - b.page_begin) * b.q_count;
+    });
+  }
   info->num_work = (int32_t)work.size();
   info->num_partial_rows = part_base;
   info->num_merge_rows = (int32_t)merges.size();
@@ -128,13 +241,17 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, int32_t 
   info->q_tile = q_tile;
   info->max_splits = max_splits;
   info->total_splits = total_splits;
-  const int64_t words = plan_words(info->num_work, info->num_merge_rows);
+  info->num_ctas = num_ctas;
+  const int64_t base_words = plan_words(info->num_work, info->num_merge_rows);
+  info->cta_offset = persistent ? (int32_t)base_words : 0;
+  const int64_t words = base_words + (persistent ? num_ctas + 1 : 0);
   if (words > INT32_MAX) return SKV_ERR_INVALID;
   info->plan_words = (int32_t)words;
   if (plan_h == nullptr || plan_capacity < words) return SKV_ERR_WORKSPACE;
   if (!work.empty()) std::memcpy(plan_h, work.data(), work.size() * sizeof(WorkItem));
   if (!merges.empty())
     std::memcpy(plan_h + 8 * work.size(), merges.data(), merges.size() * sizeof(MergeItem));
+  if (persistent) std::memcpy(plan_h + base_words, cta_indptr.data(), (num_ctas + 1) * sizeof(int32_t));
   return SKV_OK;
 }
 
@@ -225,9 +342,19 @@ skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32
   const bool tc = !wide && g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
   const int32_t kernel = wide ? KERNEL_GQA_TC_WIDE : tc ? KERNEL_GQA_TC_DECODE : KERNEL_GQA_SIMT;
   const int32_t q_tile = wide ? 8 / g : tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
-  // persistent tensor-core kernel: a few large units per SM; CUDA-core kernel: many small CTAs
-  return plan_common(batch, req, q_tile, wide ? 1 : num_kv_heads, (wide || tc) ? 6 : 64, policy, param,
-                     split_indptr_h, split_bounds_h, kernel, plan_h, plan_capacity, info);
+  std::vector<int64_t> kv_len(batch);
+  for (int32_t r = 0; r < batch; ++r)
+    kv_len[r] = req[r].n_pages == 0 ? 0
+                                    : (int64_t)(req[r].n_pages - 1) * page_size + kv_last_page_len_h[r];
+  PersistOpts po;
+  po.page_size = page_size;
+  if (wide) {  // persistent all-heads kernel: 16-token tiles, one CTA per SM
+    po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
+    po.tile_tokens = 16;
+  }
+  // per-KV-head tensor-core kernel: a few large units per SM; CUDA-core kernel: many small CTAs
+  return plan_common(batch, req, kv_len, q_tile, wide ? 1 : num_kv_heads, tc ? 6 : 64, policy, param,
+                     split_indptr_h, split_bounds_h, kernel, po, plan_h, plan_capacity, info);
 }
 
 skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
@@ -245,8 +372,14 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
     req[r].q_len = q_len;
   }
   const int32_t fold = skv_mla_fold_ratio(num_heads, q_len, 128);
-  return plan_common(batch, req, fold, 1, 8, policy, param, split_indptr_h, split_bounds_h, KERNEL_MLA_SIMT,
-                     plan_h, plan_capacity, info);
+  std::vector<int64_t> kv_len(batch);
+  for (int32_t r = 0; r < batch; ++r)
+    kv_len[r] = req[r].n_pages == 0 ? 0
+                                    : (int64_t)(req[r].n_pages - 1) * page_size + kv_last_page_len_h[r];
+  PersistOpts po;
+  po.page_size = page_size;
+  return plan_common(batch, req, kv_len, fold, 1, 8, policy, param, split_indptr_h, split_bounds_h,
+                     KERNEL_MLA_SIMT, po, plan_h, plan_capacity, info);
 }
 
 skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan_d,
@@ -275,7 +408,11 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
                        p->k_stride[2] == p->v_stride[2];
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  int e = info->kernel == KERNEL_GQA_TC_WIDE     ? launch_gqa_tc_wide(*p, work, info->num_work, info->q_tile, s)
+  if (info->kernel == KERNEL_GQA_TC_WIDE &&
+      (info->num_ctas < 1 || info->cta_offset < 8LL * info->num_work + 4LL * info->num_merge_rows))
+    return SKV_ERR_INVALID;
+  int e = info->kernel == KERNEL_GQA_TC_WIDE
+              ? launch_gqa_tc_wide(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile, s)
           : info->kernel == KERNEL_GQA_TC_DECODE ? launch_gqa_tc_decode(*p, work, info->num_work, info->q_tile, s)
                                                  : launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
   return cuda_status(e);

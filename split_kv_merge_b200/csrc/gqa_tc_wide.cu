@@ -77,7 +77,8 @@ struct WArgs {
   const int32_t* kv_indptr;
   const int32_t* kv_indices;
   const int32_t* last;
-  int num_pages, page_size, hq, q_tile, num_units;
+  int num_pages, page_size, hq, q_tile, num_ctas;
+  const int32_t* cta_indptr;  // CTA c runs work items cta_indptr[c] .. cta_indptr[c+1]
   float scale_log2;
   void* o;
   float* lse;
@@ -186,7 +187,7 @@ gqa_tc_wide_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   const uint32_t tmem = *tmem_holder;
   const uint32_t tm_s = tmem, tm_o = tmem + 2 * kN;
 
-  const int G_ = gridDim.x;
+  const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
   if (warp == 4) {
     // ======================================================================= TMA producer
     // The whole warp walks the units: lanes hold the page ids of the next 32 tiles (one per lane)
@@ -210,7 +211,7 @@ gqa_tc_wide_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       q_pending = false;
       return true;
     };
-    for (int u = blockIdx.x; u < a.num_units && ok; u += G_) {
+    for (int u = u_begin; u < u_end && ok; ++u) {
       const WUnit x = load_wunit(a, work, u);
       if (x.ntiles == 0) continue;
       const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
@@ -309,7 +310,7 @@ gqa_tc_wide_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         tc::mma_commit(empty_bar(st));
         return true;
       };
-      for (int u = blockIdx.x; u < a.num_units && ok; u += G_) {
+      for (int u = u_begin; u < u_end && ok; ++u) {
         const WUnit x = load_wunit(a, work, u);
         if (x.ntiles == 0) continue;
         const int ob = n_unit & 1;
@@ -361,7 +362,7 @@ gqa_tc_wide_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         ok = tc::mbar_wait(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
       tc::tc_fence_after();
     };
-    for (int u = blockIdx.x; u < a.num_units && ok; u += G_) {
+    for (int u = u_begin; u < u_end && ok; ++u) {
       const WUnit x = load_wunit(a, work, u);
       const int rows = x.q_count * G;      // valid columns per KV head
       if (x.ntiles == 0) {
@@ -566,16 +567,6 @@ bool make_map_w(CUtensorMap* m, const void* base, int rank, const cuuint64_t* di
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int num_sms_w() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int G, typename OutT>
 int launch_w(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm, const WArgs& a,
              const WorkItem* work, cudaStream_t s) {
@@ -587,8 +578,7 @@ int launch_w(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  const int grid = std::min(a.num_units, num_sms_w());
-  gqa_tc_wide_kernel<G, OutT><<<grid, kThreads, smem, s>>>(km, vm, qm, a, work);
+  gqa_tc_wide_kernel<G, OutT><<<a.num_ctas, kThreads, smem, s>>>(km, vm, qm, a, work);
   return (int)cudaGetLastError();
 }
 
@@ -611,8 +601,9 @@ bool gqa_tc_wide_supported(int head_dim, int page_size, int num_kv_heads, int gr
          page_size <= 256 && page_size % kTok == 0;
 }
 
-int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile, cudaStream_t s) {
-  if (num_work == 0) return 0;
+int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
+                       int q_tile, cudaStream_t s) {
+  if (num_ctas == 0) return 0;
   const int g = p.num_qo_heads / p.num_kv_heads;
   if (!gqa_tc_wide_supported(p.head_dim, p.page_size, p.num_kv_heads, g, q_tile)) return (int)cudaErrorInvalidValue;
   CUtensorMap km, vm, qm;
@@ -644,7 +635,8 @@ int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, int num_
   a.page_size = p.page_size;
   a.hq = p.num_qo_heads;
   a.q_tile = q_tile;
-  a.num_units = num_work;
+  a.num_ctas = num_ctas;
+  a.cta_indptr = cta_indptr;
   a.scale_log2 = p.sm_scale * kLog2e;
   a.o = p.o;
   a.lse = p.lse;

@@ -42,7 +42,8 @@ bool gqa_tc_decode_supported(int head_dim, int page_size, int group, int q_tile)
 int launch_gqa_tc_decode(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
                          cudaStream_t s);
 bool gqa_tc_wide_supported(int head_dim, int page_size, int num_kv_heads, int group, int q_tile);
-int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile, cudaStream_t s);
+int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
+                       int q_tile, cudaStream_t s);
 int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work, int q_tile,
                     cudaStream_t s);
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,

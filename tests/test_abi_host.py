@@ -47,8 +47,9 @@ def test_mla_fold_ratio(H, q_len, F):
 
 
 def _items(plan):
-    w = plan.words[: 8 * plan.info.num_work].reshape(-1, 8)
-    m = plan.words[8 * plan.info.num_work:].reshape(-1, 4)
+    nw, nm = plan.info.num_work, plan.info.num_merge_rows
+    w = plan.words[: 8 * nw].reshape(-1, 8)
+    m = plan.words[8 * nw: 8 * nw + 4 * nm].reshape(-1, 4)
     return w, m
 
 
@@ -94,8 +95,11 @@ def test_plan_explicit_and_empty_splits():
 
 
 def test_plan_balanced_covers_every_page_once():
+    """Balanced plan for the persistent all-heads decode kernel: every page of every request is in
+    exactly one work item, and the CTAs' shares of 16-token tiles are equal up to one small piece."""
     c = llama70b_decode_case(batch=64)
     plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, 16, 64, 8, 128, "balanced", 148)
+    info = plan.info
     w, m = _items(plan)
     n = np.diff(c.kv_indptr)
     for r in range(64):
@@ -103,9 +107,24 @@ def test_plan_balanced_covers_every_page_once():
         spans = sorted((int(a), int(b)) for a, b in rows[:, 3:5])
         assert spans[0][0] == 0 and spans[-1][1] == n[r]
         assert all(spans[i][1] == spans[i + 1][0] for i in range(len(spans) - 1))
-    sizes = (w[:, 4] - w[:, 3])
-    assert list(sizes) == sorted(sizes, reverse=True)       # longest first
-    assert plan.info.num_work * 8 >= 148                    # enough CTAs for every SM
+    assert info.num_ctas == 148 and info.cta_offset == 8 * info.num_work + 4 * info.num_merge_rows
+    cta = plan.words[info.cta_offset: info.cta_offset + info.num_ctas + 1]
+    assert cta[0] == 0 and cta[-1] == info.num_work and np.all(np.diff(cta) >= 1)
+    L = c.kv_lengths()
+    tiles = np.array([sum(-(-(min(b * 16, L[r]) - a * 16) // 16) for r, _, _, a, b, *_ in w[cta[i]:cta[i + 1]])
+                      for i in range(info.num_ctas)])
+    assert tiles.sum() == np.sum(-(-L // 16))
+    assert tiles.max() <= tiles.mean() + 5 and tiles.min() >= tiles.mean() - 5
+    assert info.total_splits < 64 + 2 * 148       # each CTA boundary cuts at most one request
+
+
+def test_plan_persistent_fixed_assigns_longest_first():
+    c = llama70b_decode_case(batch=16)
+    plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, 16, 64, 8, 128, "fixed", 3)
+    info = plan.info
+    assert info.num_ctas == min(148, info.num_work)
+    cta = plan.words[info.cta_offset: info.cta_offset + info.num_ctas + 1]
+    assert cta[-1] == info.num_work
 
 
 @pytest.mark.parametrize("bad", ["last_zero", "last_big", "hq_not_multiple", "head_dim", "indptr_decreasing",
