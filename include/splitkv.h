@@ -168,6 +168,24 @@ SKV_API skv_status skv_merge_plan(const float* o_part, const float* lse_part, co
                                   void* o, int32_t o_dtype, float* lse, skv_stream_t stream);
 
 /* -------------------------------------------------------------------------------------------
+ * skv_paged_attn_fwd_static_scratch -- skv_paged_attn_fwd without caller-provided split partials.
+ *   No counterpart on the pages this library follows: it exists for callers that cannot
+ *   allocate device memory -- a serving engine that gives nearly all device memory to its KV
+ *   cache at start-up and keeps no allocator on the decode path, or a plain-C / foreign-runtime
+ *   caller with no device allocator of its own (cudaMalloc would also synchronize the device).
+ *   Same arguments and results as skv_paged_attn_fwd; p->o_part / p->lse_part are ignored.  The
+ *   partials go to one file-scope device array of 32 MiB that every GPU loading this library
+ *   holds until the process exits; plans whose partials (num_partial_rows * Hq * (D + 1) floats,
+ *   each part rounded up to 256 B) exceed it return SKV_ERR_WORKSPACE with nothing launched.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *   that device current); make that first call before any stream capture.  Allocates nothing.
+ *   All calls share the array and it keeps the last call's contents (every partial is written
+ *   before it is read, so nothing needs clearing); calls that overlap on the GPU race.
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_paged_attn_fwd_static_scratch(const skv_paged_params* p, const int32_t* plan_d,
+                                                     const skv_plan_info* info, skv_stream_t stream);
+
+/* -------------------------------------------------------------------------------------------
  * skv_plan_mla -- host-side planner for skv_mla_decode_fwd (same split policies).  The fold
  *   ratio F (seqlen_q tokens folded into the head/row dimension) is skv_mla_fold_ratio(H,
  *   q_len, 128) and is reported in info->q_tile.

@@ -89,6 +89,8 @@ _paged_partial = _proto("skv_paged_attn_partial", ctypes.c_int, [ctypes.POINTER(
                                                                   ctypes.POINTER(PlanInfo), _vp])
 _mla_partial = _proto("skv_mla_decode_partial", ctypes.c_int, [ctypes.POINTER(MlaParams), _vp,
                                                                 ctypes.POINTER(PlanInfo), _vp])
+_paged_static = _proto("skv_paged_attn_fwd_static_scratch", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp,
+                                                                          ctypes.POINTER(PlanInfo), _vp])
 _merge_plan = _proto("skv_merge_plan", ctypes.c_int, [_vp, _vp, _vp, ctypes.POINTER(PlanInfo), ctypes.c_int32,
                                                        ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp])
 _merge = _proto("skv_merge_states", ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
@@ -101,7 +103,7 @@ _version = _proto("skv_version", ctypes.c_int32, [])
 
 SYMBOLS = ["skv_plan_paged", "skv_paged_attn_fwd", "skv_paged_attn_partial", "skv_merge_plan", "skv_plan_mla",
            "skv_mla_decode_fwd", "skv_mla_decode_partial", "skv_merge_states", "skv_paged_kv_gather",
-           "skv_mla_fold_ratio", "skv_status_str", "skv_version"]
+           "skv_mla_fold_ratio", "skv_status_str", "skv_version", "skv_paged_attn_fwd_static_scratch"]
 
 
 class SkvError(RuntimeError):
@@ -252,6 +254,17 @@ def paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len,
     fn = {"all": _paged_fwd, "partial": _paged_partial}[phase]
     _check(fn(ctypes.byref(p), _dptr(plan.device), ctypes.byref(plan.info), _stream_ptr(stream)),
            "skv_paged_attn_fwd" if phase == "all" else "skv_paged_attn_partial")
+
+
+def paged_attn_fwd_static_scratch(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan: Plan, o,
+                                  lse=None, status=None, sm_scale: Optional[float] = None,
+                                  num_pages: Optional[int] = None, stream=None) -> None:
+    """skv_paged_attn_fwd_static_scratch: paged_attn_fwd with the split partials kept in the
+    library's own fixed 32 MiB device array, for callers that cannot allocate device memory."""
+    p = _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, o, lse, None, None,
+                      status, sm_scale, num_pages)
+    _check(_paged_static(ctypes.byref(p), _dptr(plan.device), ctypes.byref(plan.info), _stream_ptr(stream)),
+           "skv_paged_attn_fwd_static_scratch")
 
 
 def mla_decode_fwd(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len, plan: Plan, o, lse=None,
