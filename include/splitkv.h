@@ -186,13 +186,16 @@ SKV_API skv_status skv_paged_attn_fwd_static_scratch(const skv_paged_params* p, 
                                                      const skv_plan_info* info, skv_stream_t stream);
 
 /* -------------------------------------------------------------------------------------------
- * skv_plan_mla -- host-side planner for skv_mla_decode_fwd (same split policies).  The fold
- *   ratio F (seqlen_q tokens folded into the head/row dimension) is skv_mla_fold_ratio(H,
- *   q_len, 128) and is reported in info->q_tile.
+ * skv_plan_mla -- host-side planner for skv_mla_decode_fwd (same split policies); kv_dtype is
+ *   the cache type (SKV_BF16 or SKV_E4M3) the plan will run on.  The fold ratio F (seqlen_q
+ *   tokens folded into the query-row dimension of a work item) is reported in info->q_tile:
+ *   F = skv_mla_fold_ratio(H, q_len, R) with R the rows the chosen kernel puts on one tile
+ *   (16 or 32 for the tensor-core kernel, which splits H > R heads into groups of R; 128 for
+ *   the CUDA-core kernel).
  * ----------------------------------------------------------------------------------------- */
 SKV_API skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
                         const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_heads,
-                        int32_t policy, int32_t param, const int32_t* split_indptr_h,
+                        int32_t kv_dtype, int32_t policy, int32_t param, const int32_t* split_indptr_h,
                         const int32_t* split_bounds_h, int32_t* plan_h, int64_t plan_capacity,
                         skv_plan_info* info);
 

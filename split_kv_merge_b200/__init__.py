@@ -79,8 +79,8 @@ _plan_paged = _proto("skv_plan_paged", ctypes.c_int, [ctypes.c_int32, _i32p, _i3
                                                        ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, _i32p,
                                                        ctypes.c_int64, ctypes.POINTER(PlanInfo)])
 _plan_mla = _proto("skv_plan_mla", ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32,
-                                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _i32p, _i32p,
-                                                   _i32p, ctypes.c_int64, ctypes.POINTER(PlanInfo)])
+                                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                   _i32p, _i32p, _i32p, ctypes.c_int64, ctypes.POINTER(PlanInfo)])
 _paged_fwd = _proto("skv_paged_attn_fwd", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp,
                                                           ctypes.POINTER(PlanInfo), _vp])
 _mla_fwd = _proto("skv_mla_decode_fwd", ctypes.c_int, [ctypes.POINTER(MlaParams), _vp,
@@ -208,12 +208,14 @@ def plan_paged(qo_indptr, kv_indptr, kv_last_page_len, page_size: int, num_qo_he
 
 def plan_mla(batch_q_len: int, kv_indptr, kv_last_page_len, page_size: int, num_heads: int,
              policy="balanced", param: int = 0,
-             split_page_start: Optional[Sequence[Sequence[int]]] = None) -> Plan:
-    """Host planner (skv_plan_mla).  ``batch_q_len`` is the query length of every request."""
+             split_page_start: Optional[Sequence[Sequence[int]]] = None, kv_dtype="bf16") -> Plan:
+    """Host planner (skv_plan_mla).  ``batch_q_len`` is the query length of every request;
+    ``kv_dtype`` the latent cache type ("bf16" / "e4m3") the plan will run on."""
     ki, la = _i32(kv_indptr), _i32(kv_last_page_len)
     b = len(ki) - 1
-    return _plan(_plan_mla, lambda pol: (b, batch_q_len, _ptr_i32(ki), _ptr_i32(la), page_size, num_heads, pol,
-                                         param),
+    kd = {"bf16": BF16, "e4m3": E4M3}[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    return _plan(_plan_mla, lambda pol: (b, batch_q_len, _ptr_i32(ki), _ptr_i32(la), page_size, num_heads, kd,
+                                         pol, param),
                  policy, split_page_start, "skv_plan_mla")
 
 

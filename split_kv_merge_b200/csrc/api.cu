@@ -39,7 +39,9 @@ int device_sms(int param) {
 }
 
 // Persistent-kernel options of the planner: the CTA count the work is balanced over and the
-// tokens one kernel tile covers.  flat_ctas == 0: not persistent (one CTA per work item).
+// tokens one kernel tile covers.  flat_ctas == 0: not persistent (one CTA per work item).  For
+// persistent kernels `units_per_page` counts how many times a CTA streams each page of a work
+// item (MLA head groups), so the slices are balanced in streamed tiles.
 struct PersistOpts {
   int32_t flat_ctas = 0;
   int32_t tile_tokens = 128;
@@ -97,7 +99,7 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
     std::vector<int64_t> w(batch, 0);
     double total = 0;
     for (int32_t r = 0; r < batch; ++r) {
-      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile;
+      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile * units_per_page;
       w[r] = qt * range_tiles(0, req[r].n_pages, kv_len[r], P, T);
       total += (double)w[r];
     }
@@ -106,7 +108,7 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
     int cta = 0;
     double cum = 0;
     for (int32_t r = 0; r < batch; ++r) {
-      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile;
+      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile * units_per_page;
       const int32_t n = req[r].n_pages;
       bounds[r].push_back(0);
       if (n == 0 || qt == 0) {  // nothing to stream: one (empty) piece on the current CTA
@@ -359,11 +361,12 @@ skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32
 
 skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
                         const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_heads,
-                        int32_t policy, int32_t param, const int32_t* split_indptr_h,
+                        int32_t kv_dtype, int32_t policy, int32_t param, const int32_t* split_indptr_h,
                         const int32_t* split_bounds_h, int32_t* plan_h, int64_t plan_capacity,
                         skv_plan_info* info) {
   if (info != nullptr) std::memset(info, 0, sizeof(*info));
   if (q_len < 1 || num_heads < 1) return SKV_ERR_INVALID;
+  if (kv_dtype != SKV_BF16 && kv_dtype != SKV_E4M3) return SKV_ERR_UNSUPPORTED;
   std::vector<ReqShape> req;
   skv_status st = check_table_h(batch, kv_indptr_h, kv_last_page_len_h, page_size, req);
   if (st != SKV_OK) return st;
@@ -371,15 +374,27 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
     req[r].q_start = r * q_len;
     req[r].q_len = q_len;
   }
-  const int32_t fold = skv_mla_fold_ratio(num_heads, q_len, 128);
   std::vector<int64_t> kv_len(batch);
   for (int32_t r = 0; r < batch; ++r)
     kv_len[r] = req[r].n_pages == 0 ? 0
                                     : (int64_t)(req[r].n_pages - 1) * page_size + kv_last_page_len_h[r];
+  // tensor-core kernel: 16 query rows per tile when all of a request's rows fit, else 32 (heads
+  // beyond 32 in groups of 32); the fold puts as many query tokens as fit into those rows
+  const int32_t nr = (int64_t)num_heads * q_len <= 16 ? 16 : 32;
+  const bool tc = mla_tc_supported(kv_dtype, page_size, num_heads, nr);
   PersistOpts po;
   po.page_size = page_size;
-  return plan_common(batch, req, kv_len, fold, 1, 8, policy, param, split_indptr_h, split_bounds_h,
-                     KERNEL_MLA_SIMT, po, plan_h, plan_capacity, info);
+  int32_t kernel = KERNEL_MLA_SIMT, fold = skv_mla_fold_ratio(num_heads, q_len, 128);
+  int64_t head_groups = 1;
+  if (tc) {
+    kernel = nr == 16 ? KERNEL_MLA_TC16 : KERNEL_MLA_TC32;
+    fold = num_heads <= nr ? skv_mla_fold_ratio(num_heads, q_len, nr) : 1;
+    head_groups = num_heads <= nr ? 1 : num_heads / nr;
+    po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
+    po.tile_tokens = 128;
+  }
+  return plan_common(batch, req, kv_len, fold, head_groups, 8, policy, param, split_indptr_h, split_bounds_h,
+                     kernel, po, plan_h, plan_capacity, info);
 }
 
 skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan_d,
@@ -464,10 +479,15 @@ skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d
       !aligned16(p->o))
     return SKV_ERR_ALIGNMENT;
   if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
-  if (info->kernel != KERNEL_MLA_SIMT) return SKV_ERR_INVALID;
+  const bool tc = info->kernel == KERNEL_MLA_TC16 || info->kernel == KERNEL_MLA_TC32;
+  if (info->kernel != KERNEL_MLA_SIMT && !tc) return SKV_ERR_INVALID;
+  if (tc && (info->num_ctas < 1 || info->cta_offset < 8LL * info->num_work + 4LL * info->num_merge_rows))
+    return SKV_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  int e = launch_mla_simt(*p, work, info->num_work, info->q_tile, s);
+  int e = tc ? launch_mla_tc(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile,
+                             info->kernel == KERNEL_MLA_TC16 ? 16 : 32, s)
+             : launch_mla_simt(*p, work, info->num_work, info->q_tile, s);
   return cuda_status(e);
 }
 

@@ -1,0 +1,637 @@
+// MLA latent decode on the tensor cores (tcgen05 + TMEM), bf16 latent cache, TMA page staging.
+//
+// What it computes (FlashInfer PR #3309 page, MLA decode): every head reads one latent row per
+// token -- a 512-d compressed KV (ckv) and a 64-d rope key (kpe); s = scale (q_nope . ckv +
+// q_pe . kpe), V = ckv.  seqlen_q is folded into the row dimension: a work item's rows are
+// (query token, head) pairs, n = qi * Hc + h, with Hc = min(H, NR) heads per unit and the fold
+// ratio F = q_tile tokens chosen by the planner so rows = F * Hc <= NR.  When H > NR the heads
+// are split into H / NR unit groups that run one after another on the same CTA and slice of KV.
+//
+// B200 design.  A 128-token tile of latent rows is 144 KB (bf16), too big to hold through
+// QK -> softmax -> PV while the next tiles stream in.  So:
+//   * S^T[128 tokens, NR] = C[128, 576] . Q^T[576, NR] with tokens as M (the 16-32 query rows
+//     are far too few for M); C streams through a ring of 32 KB slots (128 tokens x 128 latent
+//     dims, two 64-column swizzled halves) and each slot is released as soon as its MMAs are done.
+//   * O^T[512, NR] += V^T . P^T runs one tile later from a second pass over the same 512 ckv
+//     dims (four 32 KB slots, one 128-dim M block each), re-read while it is still in L2; only
+//     the HBM read of each tile counts against the KV bytes, the second pass costs L2 bandwidth.
+//   * Slot order: K(0), then per tile t: K(t+1), V(t) -- the V slots of t wait only for the
+//     softmax of t while K(t+1) is multiplied.
+//   * Online softmax with a lazily raised maximum (only when a score passes the running max by
+//     more than 2^8): the column max over 128 token lanes is a shuffle + 4-warp exchange paid only
+//     on a raise; O^T lives in TMEM and is rescaled there by all four softmax warps when needed.
+//   * Tokens past the end of the unit get s = -inf by selection; their V rows in the second-pass
+//     slots are zeroed before the PV that reads them.
+// Roles: warp 4 TMA producer, warp 5 TMEM allocation + MMA issue, warps 0-3 softmax / epilogue.
+// All waits are bounded (SKV_DEV_TIMEOUT); roles leave together; TMEM is always released.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tc_ptx.cuh"
+
+namespace skv {
+
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kSlotBytes = 32768;      // 128 tokens x 128 dims bf16 (two 16 KB swizzled halves)
+constexpr int kHalf = 16384;
+constexpr int kThreads = 192;
+constexpr int kKSlots = 5;             // ckv 0..511 in four slots + kpe
+constexpr int kVSlots = 4;
+constexpr float kRaise = 8.f;
+
+template <int NR>
+struct MlaCfg {
+  static constexpr int kStages = NR == 16 ? 6 : 5;
+  static constexpr int kQRegion = NR * 128;             // one 64-column region of Q
+  static constexpr int kQBytes = 9 * kQRegion;          // q_nope (8 regions) + q_pe
+  static constexpr int kPBytes = 2 * NR * 128;          // NR rows x 128 tokens bf16 (2 regions)
+  static constexpr int ring = 0;
+  static constexpr int q = ring + kStages * kSlotBytes;
+  static constexpr int p = q + kQBytes;
+  static constexpr int red = p + 2 * kPBytes;           // [4][NR] float
+  static constexpr int alpha = red + 4 * NR * 4;        // [NR]
+  static constexpr int inv = alpha + NR * 4;            // [NR]
+  static constexpr int lse = inv + NR * 4;              // [NR]
+  static constexpr int bars = lse + NR * 4;
+  static constexpr int nbars = 2 * kStages + 2 + 2 * 4 + 1;  // ring, Q, S, P, O full x2, O free
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int total = misc + 16;
+  static constexpr int tmem_cols = 256;                 // S 2 x NR, O 4 x NR
+};
+
+struct MArgs {
+  const int32_t* kv_indptr;
+  const int32_t* kv_indices;
+  const int32_t* last;
+  const int32_t* cta_indptr;
+  int num_pages, page_size, heads, hc, hg, q_tile;
+  float scale_log2;
+  void* o;
+  float* lse;
+  float* o_part;
+  float* lse_part;
+  int32_t* status;
+};
+
+struct MUnit {
+  int r, q_start, q_count, page_begin, page_end, part_row, part_stride;
+  int t0, t1, ntiles;
+};
+
+__device__ __forceinline__ MUnit load_munit(const MArgs& a, const WorkItem* work, int u) {
+  MUnit x;
+  const WorkItem w = work[u];
+  x.r = w.r;
+  x.q_start = w.q_start;
+  x.q_count = w.q_count;
+  x.page_begin = w.page_begin;
+  x.page_end = w.page_end;
+  x.part_row = w.part_row;
+  x.part_stride = w.part_stride;
+  const int L = request_len(a.kv_indptr, a.last, w.r, a.page_size);
+  x.t0 = w.page_begin * a.page_size;
+  x.t1 = min(w.page_end * a.page_size, L);
+  x.ntiles = x.t1 > x.t0 ? (x.t1 - x.t0 + kTile - 1) / kTile : 0;
+  return x;
+}
+
+__device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// position (within the unit's slot sequence K(0), [K(t+1), V(t)]...) of V(t)'s first slot
+__device__ __forceinline__ int vpos(int t, int T) { return kKSlots * min(t + 2, T) + kVSlots * t; }
+
+template <int NR, typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant__ CUtensorMap kpe_map,
+              const __grid_constant__ CUtensorMap qn_map, const __grid_constant__ CUtensorMap qp_map, MArgs a,
+              const WorkItem* __restrict__ work) {
+  using C = MlaCfg<NR>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = tc::smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::misc + 4);
+  const uint32_t bar0 = sbase + C::bars;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
+  auto qfull_bar = [&]() { return bar0 + 8u * (2 * NS); };
+  auto qempty_bar = [&]() { return bar0 + 8u * (2 * NS + 1); };
+  auto sfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 2 + b); };
+  auto sempty_bar = [&](int b) { return bar0 + 8u * (2 * NS + 4 + b); };
+  auto pfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 6 + b); };
+  auto ofull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 8 + b); };
+  auto ofree_bar = [&]() { return bar0 + 8u * (2 * NS + 10); };
+  static_assert(C::nbars == 2 * NS + 11, "barrier count");
+  static_assert(C::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(full_bar(s), 1);
+      tc::mbar_init(empty_bar(s), 1);
+    }
+    tc::mbar_init(qfull_bar(), 1);
+    tc::mbar_init(qempty_bar(), 1);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(sfull_bar(b), 1);
+      tc::mbar_init(sempty_bar(b), 4);
+      tc::mbar_init(pfull_bar(b), 4);
+      tc::mbar_init(ofull_bar(b), 1);
+    }
+    tc::mbar_init(ofree_bar(), 4);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tc::prefetch_tmap(&ckv_map);
+    tc::prefetch_tmap(&kpe_map);
+    tc::prefetch_tmap(&qn_map);
+    tc::prefetch_tmap(&qp_map);
+  }
+  // ring slots start as zeros: rows of a partial tile that no page fills must be finite
+  for (int i = tid; i < NS * kSlotBytes / 16; i += kThreads)
+    reinterpret_cast<uint4*>(smem + C::ring)[i] = make_uint4(0, 0, 0, 0);
+  tc::fence_proxy_async_smem();
+  if (warp == 5) tc::tmem_alloc(tc::smem_u32(tmem_holder), C::tmem_cols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tm_s = tmem, tm_o = tmem + 2 * NR;
+
+  const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
+  const int P = a.page_size;
+  const int box_rows = min(P, kTile);
+
+  if (warp == 4) {
+    // ======================================================================= TMA producer
+    int g = 0, n_unit = 0;  // slot-load sequence counter, units with tiles
+    bool ok = true;
+    for (int u = u_begin; u < u_end && ok; ++u) {
+      const MUnit x = load_munit(a, work, u);
+      if (x.ntiles == 0) continue;
+      const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
+      const int npages = x.page_end - x.page_begin;
+      for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+        // Q of this unit once the previous unit's last S MMA is done
+        if (lane == 0) {
+          if (n_unit >= 1) ok = tc::mbar_wait(qempty_bar(), (n_unit + 1) & 1, abort_flag, a.status);
+          if (ok) {
+            const int rows = a.hc * a.q_tile;
+            tc::mbar_arrive_expect_tx(qfull_bar(), (uint32_t)(9 * rows * 128));
+            for (int rg = 0; rg < 8; ++rg)
+              tma3(sbase + C::q + rg * C::kQRegion, &qn_map, qfull_bar(), rg * 64, hgi * a.hc, x.q_start);
+            tma3(sbase + C::q + 8 * C::kQRegion, &qp_map, qfull_bar(), 0, hgi * a.hc, x.q_start);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        int win = -1000000, pid = 0;  // lanes hold the ids of pages [win, win + 32) of the unit
+        const int T = x.ntiles;
+        auto load_tile = [&](int t, bool kphase) -> bool {
+          const int pi0 = (t * kTile) / P;
+          const int npg = P >= kTile ? 1 : min(kTile / P, npages - pi0);
+          const int slot0 = P >= kTile ? (t * kTile) % P : 0;
+          if (pi0 < win || pi0 + npg > win + 32) {  // keep the previous tile's pages (V pass) in view
+            win = max(0, pi0 - (P >= kTile ? 1 : kTile / P));
+            pid = (lane < 32 && win + lane < npages) ? __ldg(ids + win + lane) : 0;
+          }
+          const int nsl = kphase ? kKSlots : kVSlots;
+          for (int sl = 0; sl < nsl; ++sl, ++g) {
+            const int st = g % NS;
+            bool okl = true;
+            if (lane == 0) {
+              if (g >= NS) okl = tc::mbar_wait(empty_bar(st), ((g / NS) + 1) & 1, abort_flag, a.status);
+              if (okl) {
+                const bool kpe = kphase && sl == kKSlots - 1;
+                const int halves = kpe ? 1 : 2;
+                tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(halves * npg * box_rows * 128));
+              }
+            }
+            okl = __shfl_sync(0xffffffffu, okl ? 1 : 0, 0) != 0;
+            if (!okl) return false;
+            const uint32_t dst = sbase + C::ring + st * kSlotBytes;
+            for (int i = 0; i < npg; ++i) {
+              const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
+              if (lane == 0) {
+                if ((unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
+                const uint32_t row_off = (uint32_t)(i * box_rows * 128);
+                if (kphase && sl == kKSlots - 1) {
+                  tma3(dst + row_off, &kpe_map, full_bar(st), 0, slot0, page);
+                } else {
+                  tma3(dst + row_off, &ckv_map, full_bar(st), sl * 128, slot0, page);
+                  tma3(dst + kHalf + row_off, &ckv_map, full_bar(st), sl * 128 + 64, slot0, page);
+                }
+              }
+            }
+          }
+          return true;
+        };
+        ok = load_tile(0, true);
+        for (int t = 0; t < T && ok; ++t) {
+          if (t + 1 < T) ok = load_tile(t + 1, true);
+          if (ok) ok = load_tile(t, false);
+        }
+        ++n_unit;
+      }
+    }
+    if (!ok && lane == 0) {  // drain issued copies (bounded) before the CTA can exit
+      for (int q = max(0, g - NS); q < g; ++q) {
+        const uint64_t t_start = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(full_bar(q % NS), (q / NS) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ======================================================================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, NR, false, false);
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, NR, true, false);
+      int g = 0, n_unit = 0, n_tile = 0;
+      bool ok = true;
+      for (int u = u_begin; u < u_end && ok; ++u) {
+        const MUnit x = load_munit(a, work, u);
+        if (x.ntiles == 0) continue;
+        for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+          const int T = x.ntiles;
+          ok = tc::mbar_wait(qfull_bar(), n_unit & 1, abort_flag, a.status);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t qs = sbase + C::q;
+          auto issue_s = [&](int t) -> bool {  // consumes the 5 K-phase slots of tile t
+            const int tt = n_tile + t, sb = tt & 1;
+            if (tt >= 2 && !tc::mbar_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1, abort_flag, a.status)) return false;
+            for (int sl = 0; sl < kKSlots; ++sl, ++g) {
+              const int st = g % NS;
+              if (!tc::mbar_wait(full_bar(st), (g / NS) & 1, abort_flag, a.status)) return false;
+              tc::tc_fence_after();
+              const uint32_t base = sbase + C::ring + st * kSlotBytes;
+              const int nk = sl == kKSlots - 1 ? 4 : 8;
+              for (int k = 0; k < nk; ++k) {
+                const int qreg = sl == kKSlots - 1 ? 8 : 2 * sl + (k >> 2);
+                const uint64_t ad = tc::sdesc_sw128(base + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
+                const uint64_t bd = tc::sdesc_sw128(qs + qreg * C::kQRegion + (k & 3) * 32, 16, 1024);
+                tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, (sl > 0 || k > 0) ? 1u : 0u);
+              }
+              tc::mma_commit(empty_bar(st));
+            }
+            tc::mma_commit(sfull_bar(sb));
+            return true;
+          };
+          auto issue_pv = [&](int t) -> bool {  // consumes the 4 V-phase slots of tile t
+            const int tt = n_tile + t, pb = tt & 1;
+            if (!tc::mbar_wait(pfull_bar(pb), (tt >> 1) & 1, abort_flag, a.status)) return false;
+            // the single O^T buffer was read by the previous unit's epilogue
+            if (t == 0 && n_unit >= 1 && !tc::mbar_wait(ofree_bar(), (n_unit + 1) & 1, abort_flag, a.status))
+              return false;
+            tc::tc_fence_after();
+            const uint32_t ps = sbase + C::p + pb * C::kPBytes;
+            for (int b = 0; b < kVSlots; ++b, ++g) {
+              const int st = g % NS;
+              if (!tc::mbar_wait(full_bar(st), (g / NS) & 1, abort_flag, a.status)) return false;
+              tc::tc_fence_after();
+              const uint32_t vs = sbase + C::ring + st * kSlotBytes;
+              for (int k = 0; k < kTile / 16; ++k) {
+                const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
+                const uint64_t bd = tc::sdesc_sw128(ps + (k >> 2) * (NR * 128) + (k & 3) * 32, 16, 1024);
+                tc::mma_bf16(tm_o + b * NR, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+              }
+              tc::mma_commit(empty_bar(st));
+            }
+            tc::mma_commit(ofull_bar(pb));
+            return true;
+          };
+          ok = issue_s(0);
+          for (int t = 0; t < T && ok; ++t) {
+            if (t + 1 < T) ok = issue_s(t + 1);
+            if (ok && t + 1 == T) tc::mma_commit(qempty_bar());  // Q free after the last S
+            if (ok) ok = issue_pv(t);
+          }
+          n_tile += T;
+          ++n_unit;
+        }
+      }
+    }
+  } else {
+    // ======================================================================= softmax / epilogue
+    float* red = reinterpret_cast<float*>(smem + C::red);
+    float* alpha_s = reinterpret_cast<float*>(smem + C::alpha);
+    float* inv_s = reinterpret_cast<float*>(smem + C::inv);
+    float* lse_s = reinterpret_cast<float*>(smem + C::lse);
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    int g = 0, n_unit = 0, n_tile = 0, pv_seen = 0;
+    bool ok = true;
+    auto consume_pv = [&](int upto) {
+      for (; pv_seen <= upto; ++pv_seen)
+        ok = tc::mbar_wait(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
+      tc::tc_fence_after();
+    };
+    for (int u = u_begin; u < u_end && ok; ++u) {
+      const MUnit x = load_munit(a, work, u);
+      const int rows = x.q_count * a.hc;
+      for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+        const int h0 = hgi * a.hc;
+        if (x.ntiles == 0) {  // no tokens: O = 0, LSE = -inf
+          for (int n = 0; n < rows; ++n) {
+            const int qi = n / a.hc, h = h0 + n % a.hc;
+            for (int d = tid; d < 512; d += 128) {
+              if (x.part_row < 0)
+                store_out(reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.heads + h) * 512 + d, 0.f);
+              else
+                a.o_part[(((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h) * 512 + d] = 0.f;
+            }
+            if (tid == 0) {
+              if (x.part_row < 0) {
+                if (a.lse != nullptr) a.lse[(int64_t)(x.q_start + qi) * a.heads + h] = -INFINITY;
+              } else {
+                a.lse_part[((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h] = -INFINITY;
+              }
+            }
+          }
+          continue;
+        }
+        const int T = x.ntiles;
+        float m[NR], l[NR];
+#pragma unroll
+        for (int n = 0; n < NR; ++n) {
+          m[n] = -INFINITY;
+          l[n] = 0.f;
+        }
+        bool failed = false;
+        for (int t = 0; t < T; ++t) {
+          const int tt = n_tile + t, sb = tt & 1;
+          ok = tc::mbar_wait(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
+          tc::tc_fence_after();
+          float s[NR];
+#pragma unroll
+          for (int c = 0; c < NR; c += 16) {
+            float v16[16];
+            tc::tmem_ld_x16(tm_s + lane_base + sb * NR + c, v16);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) s[c + i] = v16[i];
+          }
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(sempty_bar(sb));
+          const bool valid = x.t0 + t * kTile + tid < x.t1;
+          bool raise = false;
+#pragma unroll
+          for (int n = 0; n < NR; ++n) {
+            s[n] = (valid && n < rows) ? s[n] * a.scale_log2 : -INFINITY;
+            raise |= s[n] > m[n] + kRaise;
+          }
+          if (tc::bar_or(1, 128, raise || !ok || t == 0)) {
+            if (!tc::bar_and(1, 128, ok)) {
+              failed = true;
+              break;
+            }
+            float* rr = red;  // one exchange buffer, guarded by the barriers around its use
+#pragma unroll
+            for (int n = 0; n < NR; ++n) {
+              const float v = warp_max(s[n]);
+              if (lane == 0) rr[warp * NR + n] = v;
+            }
+            tc::named_bar_sync(1, 128);
+            float al[NR];
+#pragma unroll
+            for (int n = 0; n < NR; ++n) {
+              const float mx = fmaxf(fmaxf(rr[n], rr[NR + n]), fmaxf(rr[2 * NR + n], rr[3 * NR + n]));
+              const float mn = fmaxf(m[n], mx);
+              al[n] = (mn == -INFINITY || m[n] == mn) ? 1.f : exp2f(m[n] - mn);
+              l[n] *= al[n];
+              m[n] = mn;
+            }
+            if (t > 0) {  // rescale O^T in TMEM (every thread owns lane `tid` of the 4 blocks)
+              if (tid < NR) alpha_s[tid] = al[tid];
+              tc::named_bar_sync(1, 128);
+              consume_pv(tt - 1);
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+#pragma unroll
+                for (int c = 0; c < NR; c += 16) {
+                  float ov[16];
+                  tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, ov);
+                  tc::tmem_wait_ld();
+#pragma unroll
+                  for (int i = 0; i < 16; ++i) ov[i] *= alpha_s[c + i];
+                  tc::tmem_st_x16(tm_o + lane_base + b * NR + c, ov);
+                }
+              }
+              tc::tmem_wait_st();
+              tc::tc_fence_before();
+            }
+            tc::named_bar_sync(1, 128);  // red / alpha_s reads done before any later rewrite
+          }
+          // a partial tile: zero this token's V rows in the 4 second-pass slots (once they land)
+          if (!valid) {
+            const int gv = g + vpos(t, T);
+            for (int b = 0; b < kVSlots; ++b) {
+              const int q = gv + b, st = q % NS;
+              ok = tc::mbar_wait(full_bar(st), (q / NS) & 1, abort_flag, a.status) && ok;
+              uint8_t* row = smem + C::ring + st * kSlotBytes + tid * 128;
+#pragma unroll
+              for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) reinterpret_cast<uint4*>(row + hf * kHalf)[i] = make_uint4(0, 0, 0, 0);
+            }
+          }
+          if (tt >= 2 && pv_seen <= tt - 2) consume_pv(tt - 2);  // P(t) reuses PV(t-2)'s buffer
+          uint8_t* pb = smem + C::p + (tt & 1) * C::kPBytes + (tid >> 6) * (NR * 128);
+#pragma unroll
+          for (int n = 0; n < NR; ++n) {
+            const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - m[n]);
+            l[n] += p;
+            *reinterpret_cast<__nv_bfloat16*>(pb + tc::sw128_offset(n, tid & 63)) = __float2bfloat16_rn(p);
+          }
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(pfull_bar(tt & 1));
+        }
+        if (failed) {
+          ok = false;
+          break;
+        }
+        g += (kKSlots + kVSlots) * T;
+        n_tile += T;
+        ++n_unit;
+        consume_pv(n_tile - 1);
+        // column sums over the 128 token lanes
+#pragma unroll
+        for (int n = 0; n < NR; ++n) {
+          const float v = warp_sum(l[n]);
+          if (lane == 0) red[warp * NR + n] = v;
+        }
+        if (!tc::bar_and(1, 128, ok)) {
+          ok = false;
+          break;
+        }
+        if (tid < NR) {
+          const float lt = red[tid] + red[NR + tid] + red[2 * NR + tid] + red[3 * NR + tid];
+          inv_s[tid] = lt > 0.f ? 1.f / lt : 0.f;
+          lse_s[tid] = lt > 0.f ? (m[tid] + log2f(lt)) * kLn2 : -INFINITY;
+        }
+        float ov[4][NR];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int c = 0; c < NR; c += 16) {
+            float v16[16];
+            tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, v16);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ov[b][c + i] = v16[i];
+          }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(ofree_bar());
+        tc::named_bar_sync(1, 128);
+#pragma unroll
+        for (int n = 0; n < NR; ++n) {
+          if (n >= rows) break;
+          const int qi = n / a.hc, h = h0 + n % a.hc;
+          const float iv = inv_s[n];
+          if (x.part_row < 0) {
+            OutT* dst = reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.heads + h) * 512 + tid;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) store_out(dst + b * 128, ov[b][n] * iv);
+          } else {
+            float* dst = a.o_part + (((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h) * 512 + tid;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) dst[b * 128] = ov[b][n] * iv;
+          }
+        }
+        if (tid < rows) {
+          const int qi = tid / a.hc, h = h0 + tid % a.hc;
+          if (x.part_row < 0) {
+            if (a.lse != nullptr) a.lse[(int64_t)(x.q_start + qi) * a.heads + h] = lse_s[tid];
+          } else {
+            a.lse_part[((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h] = lse_s[tid];
+          }
+        }
+        tc::named_bar_sync(1, 128);  // inv_s / lse_s / red reads done before the next unit
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, MlaCfg<NR>::tmem_cols);
+  }
+}
+
+// ------------------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_m() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map_m(CUtensorMap* m, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+                const cuuint32_t* box) {
+  auto fn = encode_fn_m();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides_bytes, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NR, typename OutT>
+int launch_m(const CUtensorMap* maps, const MArgs& a, int num_ctas, const WorkItem* work, cudaStream_t s) {
+  const int smem = MlaCfg<NR>::total + 1024;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel<NR, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return (int)e;
+    attr_set = true;
+  }
+  mla_tc_kernel<NR, OutT><<<num_ctas, kThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a, work);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit) {
+  const bool page_ok = page_size >= 8 && (page_size <= kTile ? kTile % page_size == 0 : page_size % kTile == 0);
+  return kv_dtype == SKV_BF16 && page_ok && (rows_per_unit == 16 || rows_per_unit == 32) &&
+         (num_heads <= rows_per_unit || num_heads % rows_per_unit == 0);
+}
+
+int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
+                  int q_tile, int rows_per_unit, cudaStream_t s) {
+  if (num_ctas == 0) return 0;
+  const int NR = rows_per_unit;
+  if (!mla_tc_supported(p.kv_dtype, p.page_size, p.num_heads, NR)) return (int)cudaErrorInvalidValue;
+  const int hc = std::min(p.num_heads, NR);
+  if (hc * q_tile > NR) return (int)cudaErrorInvalidValue;
+  const int box_rows = std::min(p.page_size, kTile);
+  const int total_q = p.batch * p.q_len;
+  CUtensorMap maps[4];
+  {
+    const cuuint64_t dims[3] = {512, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t st[2] = {(cuuint64_t)p.ckv_stride[1] * 2, (cuuint64_t)p.ckv_stride[0] * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    if (!make_map_m(&maps[0], p.ckv, dims, st, box)) return (int)cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t st[2] = {(cuuint64_t)p.kpe_stride[1] * 2, (cuuint64_t)p.kpe_stride[0] * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    if (!make_map_m(&maps[1], p.kpe, dims, st, box)) return (int)cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {512, (cuuint64_t)p.num_heads, (cuuint64_t)std::max(1, total_q)};
+    const cuuint64_t st[2] = {512 * 2, (cuuint64_t)p.num_heads * 512 * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)hc, (cuuint32_t)q_tile};
+    if (!make_map_m(&maps[2], p.q_nope, dims, st, box)) return (int)cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)p.num_heads, (cuuint64_t)std::max(1, total_q)};
+    const cuuint64_t st[2] = {64 * 2, (cuuint64_t)p.num_heads * 64 * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)hc, (cuuint32_t)q_tile};
+    if (!make_map_m(&maps[3], p.q_pe, dims, st, box)) return (int)cudaErrorInvalidValue;
+  }
+  MArgs a;
+  a.kv_indptr = p.kv_indptr;
+  a.kv_indices = p.kv_indices;
+  a.last = p.kv_last_page_len;
+  a.cta_indptr = cta_indptr;
+  a.num_pages = p.num_pages;
+  a.page_size = p.page_size;
+  a.heads = p.num_heads;
+  a.hc = hc;
+  a.hg = p.num_heads / hc;
+  a.q_tile = q_tile;
+  a.scale_log2 = p.sm_scale * kLog2e;
+  a.o = p.o;
+  a.lse = p.lse;
+  a.o_part = p.o_part;
+  a.lse_part = p.lse_part;
+  a.status = p.status;
+  const bool bf = p.o_dtype == SKV_BF16;
+  if (NR == 16)
+    return bf ? launch_m<16, __nv_bfloat16>(maps, a, num_ctas, work, s) : launch_m<16, float>(maps, a, num_ctas, work, s);
+  return bf ? launch_m<32, __nv_bfloat16>(maps, a, num_ctas, work, s) : launch_m<32, float>(maps, a, num_ctas, work, s);
+}
+
+}  // namespace skv

@@ -28,6 +28,8 @@ enum KernelId : int32_t {
   KERNEL_GQA_TC_DECODE = 2,
   KERNEL_GQA_TC_WIDE = 3,
   KERNEL_MLA_SIMT = 11,
+  KERNEL_MLA_TC16 = 12,  // tensor-core MLA, 16 query rows per unit
+  KERNEL_MLA_TC32 = 13,  // tensor-core MLA, 32 query rows per unit
 };
 
 // Plan words: [work items (8 words each)] [merge items (4 words each)].
@@ -46,6 +48,9 @@ int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, const in
                        int q_tile, cudaStream_t s);
 int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work, int q_tile,
                     cudaStream_t s);
+bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit);
+int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
+                  int q_tile, int rows_per_unit, cudaStream_t s);
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,
                  int32_t num_states, const MergeItem* items, int64_t num_rows, int32_t num_heads,
                  int32_t head_dim, void* o_out, int32_t o_dtype, float* lse_out, cudaStream_t s);

@@ -57,7 +57,8 @@ def mla_decode(q_nope, q_pe, ckv, kpe, kv_indptr_h, kv_indices, kv_last_page_len
     dev = q_nope.device
     B, q_len, H = q_nope.shape[:3]
     if plan is None:
-        plan = plan_mla(q_len, kv_indptr_h, kv_last_page_len_h, ckv.shape[1], H, policy, param, split_page_start)
+        kd = "bf16" if ckv.dtype == torch.bfloat16 else "e4m3"
+        plan = plan_mla(q_len, kv_indptr_h, kv_last_page_len_h, ckv.shape[1], H, policy, param, split_page_start, kd)
     if plan.device is None:
         plan.to(dev)
     kv_indptr = _dev_i32(kv_indptr_h, dev) if kv_indptr is None else kv_indptr
