@@ -142,6 +142,20 @@ def _dist():
     return ws, rank, local
 
 
+def aggregate_over_ranks(local_ms: float, local_bytes: int, device=None):
+    """Whole-job numbers: the slowest rank's device time and the bytes all ranks processed
+    (all-reduce MAX / SUM over the default process group; identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(local_ms), int(local_bytes)
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    b = torch.tensor([int(local_bytes)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(b.item())
+
+
 def _kv_bytes(case):
     L = case.kv_lengths()
     return int(L.sum()) * case.num_kv_heads * case.head_dim * 2 * 2
@@ -294,12 +308,7 @@ def run_ours(args):
     total_ms = start.elapsed_time(end)
     attn_ms = [ev_a[j].elapsed_time(ev_b[j]) for j in range(n_ev)]
     merge_ms = [ev_b[j].elapsed_time(ev_c[j]) for j in range(n_ev)]
-    if ws > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    total_bytes = kv_bytes_step * args.steps * ws
+    total_ms, total_bytes = aggregate_over_ranks(total_ms, kv_bytes_step * args.steps, dev)
     value = total_bytes / (total_ms * 1e-3) / 1e9
     ms_per_step = total_ms / args.steps
 
@@ -402,6 +411,103 @@ def _e2e(args, runs, dev, stream, skv, torch):
             "ms_per_step": round(dt / steps * 1e3, 4)}
 
 
+# ----------------------------------------------------------------------------- other configurations
+def _time_device(step, steps, warmup, torch, stream):
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_workload(args):
+    """One timed JSON line per configuration other than the Llama-70B decode (device time, inputs
+    resident; KV working sets above L2 except the tiny and shared-KV cases, which are noted)."""
+    import torch
+    import split_kv_merge_b200 as skv
+    from workloads import mla_decode_case, route_case, shared_kv_prefill_case, tiny_gqa_case
+    from workloads.device import mla_to_device, paged_to_device, route_to_device
+    peaks, src = _peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]))
+    tf = float(peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]))
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    names = args.workload.split(",")
+    if names == ["all"]:
+        names = ["tiny", "shared_kv"] + [f"mla_h{h}_q{q}_{d}" for h in (16, 128) for q in (1, 4)
+                                         for d in ("bf16", "e4m3")] + ["route"]
+    for name in names:
+        line = {"workload": name, "peaks": src}
+        if name in ("tiny", "shared_kv"):
+            c = tiny_gqa_case() if name == "tiny" else shared_kv_prefill_case()
+            d = paged_to_device(c, dev)
+            pol, par = ("fixed", 2) if name == "tiny" else ("none", 0)
+            plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, c.page_size, c.num_qo_heads,
+                                  c.num_kv_heads, c.head_dim, pol, par).to(dev)
+            n = max(1, plan.info.num_partial_rows)
+            o = torch.empty(c.q.shape[0], c.num_qo_heads, c.head_dim, device=dev)
+            lse = torch.empty(c.q.shape[0], c.num_qo_heads, device=dev)
+            op = torch.empty(n, c.num_qo_heads, c.head_dim, device=dev)
+            lp = torch.empty(n, c.num_qo_heads, device=dev)
+            step = lambda: skv.paged_attn_fwd(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"],
+                                              d["kv_last_page_len"], plan, o, lse, op, lp, None, c.sm_scale,
+                                              c.num_pages, stream)
+            L = c.kv_lengths()
+            q_rows = np.diff(c.qo_indptr)
+            kv_bytes = int(L.sum()) * c.num_kv_heads * c.head_dim * 4
+            flops = float(np.sum(q_rows * L)) * c.num_qo_heads * 4 * c.head_dim
+            if name == "shared_kv":   # the one shared KV is read once
+                kv_bytes = int(L[0]) * c.num_kv_heads * c.head_dim * 4
+            line["kernel"] = plan.info.kernel
+        elif name.startswith("mla_"):
+            _, hs, qs, dt = name.split("_")
+            H, q = int(hs[1:]), int(qs[1:])
+            c = mla_decode_case(H, q, dt)
+            d = mla_to_device(c, dev)
+            plan = skv.plan_mla(q, c.kv_indptr, c.kv_last_page_len, c.page_size, H, "balanced", 0,
+                                kv_dtype=dt).to(dev)
+            n = max(1, plan.info.num_partial_rows)
+            o = torch.empty(c.batch, q, H, 512, device=dev)
+            lse = torch.empty(c.batch, q, H, device=dev)
+            op = torch.empty(n, H, 512, device=dev)
+            lp = torch.empty(n, H, device=dev)
+            step = lambda: skv.mla_decode_fwd(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], d["kv_indptr"],
+                                              d["kv_indices"], d["kv_last_page_len"], plan, o, lse, op, lp, None,
+                                              c.sm_scale, c.kv_scale, c.num_pages, stream)
+            L = c.kv_lengths()
+            kv_bytes = int(L.sum()) * (1152 if dt == "bf16" else 576)
+            flops = float(L.sum()) * H * q * 2 * (576 + 512)
+            line["kernel"] = plan.info.kernel
+        elif name == "route":
+            c = route_case()
+            d = route_to_device(c, dev)
+            rm = skv.RouteMerge(c.sel, c.num_heads, dev)
+            out_o = torch.empty(c.sel.shape[0], c.num_heads, 512, device=dev)
+            out_l = torch.empty(c.sel.shape[0], c.num_heads, device=dev)
+            step = lambda: rm(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], d["sel_cqk"], sm_scale=c.sm_scale,
+                              stream=stream, o=out_o, lse=out_l)
+            kv_bytes = int(c.sel.size) * 1152              # gathered rows
+            flops = float(c.sel.size) * c.num_heads * 2 * (576 + 512)
+            line["kernel"] = rm.plan.info.kernel
+        else:
+            raise SystemExit(f"unknown workload {name}")
+        ms = _time_device(step, args.steps, args.warmup, torch, stream)
+        t_mem, t_tc = kv_bytes / (hbm * 1e9), flops / (tf * 1e12)
+        line.update({"us": round(ms * 1e3, 2), "kv_bytes": kv_bytes, "flops": flops,
+                     "GBps": round(kv_bytes / (ms * 1e-3) / 1e9, 1), "TFLOPs": round(flops / (ms * 1e-3) / 1e12, 2),
+                     "bound": "hbm" if t_mem >= t_tc else "tensor",
+                     "roofline_frac": round(max(t_mem, t_tc) / (ms * 1e-3), 4),
+                     "pct_hbm_measured": round(100 * kv_bytes / (ms * 1e-3) / 1e9 / hbm, 1),
+                     "pct_tensor_burst": round(100 * flops / (ms * 1e-3) / 1e12 / tf, 1)})
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -413,11 +519,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=64, help="requests per GPU (64 = the benchmark workload; "
                                                           "smaller only for profiler captures)")
+    ap.add_argument("--workload", default="llama70b",
+                    help="llama70b (the benchmark line) | tiny | shared_kv | mla_h{16,128}_q{1,4}_{bf16,e4m3} | "
+                         "route | all (one line per configuration)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != "llama70b":
+        return run_workload(args)
     return run_ours(args)
 
 

@@ -262,6 +262,14 @@ SKV_API skv_status skv_paged_kv_gather(const skv_paged_params* p, const int32_t*
                                int64_t total_tokens, void* k_out, void* v_out,
                                skv_stream_t stream);
 
+/* -------------------------------------------------------------------------------------------
+ * skv_test_wait_timeout -- test hook for device-side failure detection: one CTA waits on an
+ *   mbarrier that is never arrived on, with the bounded wait every tensor-core kernel uses, and
+ *   gives up after limit_ns (<= 10 s) writing SKV_DEV_TIMEOUT to the device status word.  The
+ *   context stays usable (nothing traps or hangs).
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_test_wait_timeout(int32_t* status, int64_t limit_ns, skv_stream_t stream);
+
 /* Fold ratio used by the MLA kernels: the largest divisor F of q_len with num_heads * F <=
  * tile_m (F >= 1).  Rows per work item = num_heads * F; work items per request = q_len / F. */
 SKV_API int32_t skv_mla_fold_ratio(int32_t num_heads, int32_t q_len, int32_t tile_m);

@@ -97,13 +97,15 @@ _merge = _proto("skv_merge_states", ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int32
                                                     ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp])
 _gather = _proto("skv_paged_kv_gather", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp, ctypes.c_int64, _vp,
                                                         _vp, _vp])
+_wait_timeout = _proto("skv_test_wait_timeout", ctypes.c_int, [_vp, ctypes.c_int64, _vp])
 _fold = _proto("skv_mla_fold_ratio", ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32])
 _status_str = _proto("skv_status_str", ctypes.c_char_p, [ctypes.c_int32])
 _version = _proto("skv_version", ctypes.c_int32, [])
 
 SYMBOLS = ["skv_plan_paged", "skv_paged_attn_fwd", "skv_paged_attn_partial", "skv_merge_plan", "skv_plan_mla",
            "skv_mla_decode_fwd", "skv_mla_decode_partial", "skv_merge_states", "skv_paged_kv_gather",
-           "skv_mla_fold_ratio", "skv_status_str", "skv_version", "skv_paged_attn_fwd_static_scratch"]
+           "skv_mla_fold_ratio", "skv_status_str", "skv_version", "skv_paged_attn_fwd_static_scratch",
+           "skv_test_wait_timeout"]
 
 
 class SkvError(RuntimeError):
@@ -324,6 +326,11 @@ def paged_kv_gather(k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, t
                       status, None, num_pages)
     _check(_gather(ctypes.byref(p), _dptr(token_indptr), total_tokens, _dptr(k_out), _dptr(v_out),
                    _stream_ptr(stream)), "skv_paged_kv_gather")
+
+
+def test_wait_timeout(status, limit_ns: int, stream=None) -> None:
+    """skv_test_wait_timeout (failure-detection test hook)."""
+    _check(_wait_timeout(_dptr(status), int(limit_ns), _stream_ptr(stream)), "skv_test_wait_timeout")
 
 
 def library_path() -> str:

@@ -515,6 +515,11 @@ skv_status skv_merge_states(const float* o_states, const float* lse_states,
                                   head_dim, o_out, o_dtype, lse_out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+skv_status skv_test_wait_timeout(int32_t* status, int64_t limit_ns, skv_stream_t stream) {
+  if (status == nullptr || limit_ns < 0 || limit_ns > 10000000000LL) return SKV_ERR_INVALID;
+  return cuda_status(launch_wait_timeout(status, (uint64_t)limit_ns, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 skv_status skv_paged_kv_gather(const skv_paged_params* p, const int32_t* token_indptr,
                                int64_t total_tokens, void* k_out, void* v_out, skv_stream_t stream) {
   if (p == nullptr || total_tokens < 0) return SKV_ERR_INVALID;

@@ -6,7 +6,7 @@
 // 16-byte loads; per-(state, head) weights are computed once into shared memory.
 #include <algorithm>
 
-#include "skv_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace skv {
 
@@ -97,7 +97,36 @@ merge_kernel(const float* __restrict__ o_states, const float* __restrict__ lse_s
   }
 }
 
+// Test hook for failure detection: waits on an mbarrier that nothing ever arrives on, with the
+// same bounded wait the tensor-core kernels use (limit `limit_ns`), and must come back with
+// SKV_DEV_TIMEOUT in the status word instead of hanging.
+__global__ void wait_timeout_kernel(int32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = tc::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    tc::mbar_init(b, 1);
+    abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = tc::globaltimer_ns();
+    while (!tc::mbar_try_wait(b, 0)) {
+      if (tc::globaltimer_ns() - t0 > limit_ns) {
+        report(status, SKV_DEV_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
 }  // namespace
+
+int launch_wait_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s) {
+  wait_timeout_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return (int)cudaGetLastError();
+}
 
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,
                  int32_t num_states, const MergeItem* items, int64_t num_rows, int32_t num_heads,

@@ -51,6 +51,7 @@ int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work,
 bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit);
 int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                   int q_tile, int rows_per_unit, cudaStream_t s);
+int launch_wait_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,
                  int32_t num_states, const MergeItem* items, int64_t num_rows, int32_t num_heads,
                  int32_t head_dim, void* o_out, int32_t o_dtype, float* lse_out, cudaStream_t s);

@@ -370,3 +370,20 @@ def test_all_heads_decode_rising_scores(policy, param):
     assert ex["plan"].info.kernel == 3
     O, LSE = _oracle_paged(c)
     _cmp(_np(o), _np(lse), O, LSE, where=f"rising {policy}")
+
+
+# ----------------------------------------------------------------------------- failure detection
+def test_bounded_wait_reports_timeout_and_context_stays_usable():
+    """A wait on a barrier nothing arrives on gives up after its limit and reports SKV_DEV_TIMEOUT;
+    the context keeps working afterwards (no trap, no hang)."""
+    import time
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    t0 = time.perf_counter()
+    skv.test_wait_timeout(status, 50_000_000)   # 50 ms
+    torch.cuda.synchronize()
+    assert int(status.item()) == skv.DEV_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    c = tiny_gqa_case()
+    o, lse, _, _ = _run_paged(c, "fixed", 2)
+    O, LSE = _oracle_paged(c)
+    _cmp(_np(o), _np(lse), O, LSE, where="after timeout")
