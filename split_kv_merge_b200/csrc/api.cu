@@ -391,7 +391,7 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
     fold = num_heads <= nr ? skv_mla_fold_ratio(num_heads, q_len, nr) : 1;
     head_groups = num_heads <= nr ? 1 : num_heads / nr;
     po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
-    po.tile_tokens = 128;
+    po.tile_tokens = mla_tc_tile_tokens();
   }
   return plan_common(batch, req, kv_len, fold, head_groups, 8, policy, param, split_indptr_h, split_bounds_h,
                      kernel, po, plan_h, plan_capacity, info);

@@ -7,22 +7,22 @@
 // ratio F = q_tile tokens chosen by the planner so rows = F * Hc <= NR.  When H > NR the heads
 // are split into H / NR unit groups that run one after another on the same CTA and slice of KV.
 //
-// B200 design.  A 128-token tile of latent rows is 144 KB (bf16), too big to hold through
-// QK -> softmax -> PV while the next tiles stream in.  So:
-//   * S^T[128 tokens, NR] = C[128, 576] . Q^T[576, NR] with tokens as M (the 16-32 query rows
-//     are far too few for M); C streams through a ring of 32 KB slots (128 tokens x 128 latent
-//     dims, two 64-column swizzled halves) and each slot is released as soon as its MMAs are done.
-//   * O^T[512, NR] += V^T . P^T runs one tile later from a second pass over the same 512 ckv
-//     dims (four 32 KB slots, one 128-dim M block each), re-read while it is still in L2; only
-//     the HBM read of each tile counts against the KV bytes, the second pass costs L2 bandwidth.
-//   * Slot order: K(0), then per tile t: K(t+1), V(t) -- the V slots of t wait only for the
-//     softmax of t while K(t+1) is multiplied.
+// B200 design.  A latent row is 1152 B, so a tile is 64 tokens (72 KB) and is held in shared
+// memory from QK to PV while the next tiles stream in:
+//   * S^T[64 tokens, NR] = C[64, 576] . Q^T[576, NR]  (M = 64 tokens: TMEM rows land in lanes
+//     0-15 of each warp quarter; the 16-32 query rows are far too few for M);
+//   * O^T[512, NR] += V^T[512, 64] . P^T[64, NR]  in four M = 128 blocks of head dims, V read
+//     MN-major from the same shared tiles, O^T accumulated in TMEM across the tiles of a unit.
+//   * Two TMA rings: ckv in 16 KB slots, each one 128-dim V block of a tile (two 64-column
+//     swizzled halves), released after that block's PV; kpe in 8 KB slots released after QK.
 //   * Online softmax with a lazily raised maximum (only when a score passes the running max by
-//     more than 2^8): the column max over 128 token lanes is a shuffle + 4-warp exchange paid only
-//     on a raise; O^T lives in TMEM and is rescaled there by all four softmax warps when needed.
-//   * Tokens past the end of the unit get s = -inf by selection; their V rows in the second-pass
-//     slots are zeroed before the PV that reads them.
-// Roles: warp 4 TMA producer, warp 5 TMEM allocation + MMA issue, warps 0-3 softmax / epilogue.
+//     more than 2^8): the column max over the 64 token lanes is a 16-lane shuffle + 4-warp
+//     exchange paid only on a raise; O^T is rescaled in TMEM by all four softmax warps then.
+//   * Tokens past the end of the unit get s = -inf by selection and their V rows are zeroed in
+//     the held tile before the PV that reads them.
+// Roles: warp 4 TMA producer, warp 5 TMEM allocation + QK MMA issue, warp 6 PV MMA issue (a
+// separate thread, so PV(t) is issued as soon as P(t) is ready instead of behind QK(t+1), which
+// releases tile t's slots earlier), warps 0-3 softmax / epilogue.
 // All waits are bounded (SKV_DEV_TIMEOUT); roles leave together; TMEM is always released.
 #include <cudaTypedefs.h>
 
@@ -34,32 +34,34 @@ namespace skv {
 
 namespace {
 
-constexpr int kTile = 128;
-constexpr int kSlotBytes = 32768;      // 128 tokens x 128 dims bf16 (two 16 KB swizzled halves)
-constexpr int kHalf = 16384;
-constexpr int kThreads = 192;
-constexpr int kKSlots = 5;             // ckv 0..511 in four slots + kpe
-constexpr int kVSlots = 4;
+constexpr int kTile = 64;              // tokens per tile
+constexpr int kHalf = kTile * 128;     // one 64-column swizzled region of a tile: 8 KB
+constexpr int kCSlot = 2 * kHalf;      // ckv slot: one 128-dim block (16 KB)
+constexpr int kKSlot = kHalf;          // kpe slot (8 KB)
+constexpr int kThreads = 224;        // 4 softmax warps, TMA warp, QK-MMA warp, PV-MMA warp
+constexpr int kBlocks = 4;             // 512 ckv dims = 4 blocks of 128
 constexpr float kRaise = 8.f;
 
 template <int NR>
 struct MlaCfg {
-  static constexpr int kStages = NR == 16 ? 6 : 5;
+  static constexpr int kCStages = NR == 16 ? 10 : 9;
+  static constexpr int kKStages = 4;
   static constexpr int kQRegion = NR * 128;             // one 64-column region of Q
   static constexpr int kQBytes = 9 * kQRegion;          // q_nope (8 regions) + q_pe
-  static constexpr int kPBytes = 2 * NR * 128;          // NR rows x 128 tokens bf16 (2 regions)
-  static constexpr int ring = 0;
-  static constexpr int q = ring + kStages * kSlotBytes;
+  static constexpr int kPBytes = NR * 128;              // NR rows x 64 tokens bf16 (1 region)
+  static constexpr int cring = 0;
+  static constexpr int kring = cring + kCStages * kCSlot;
+  static constexpr int q = kring + kKStages * kKSlot;
   static constexpr int p = q + kQBytes;
   static constexpr int red = p + 2 * kPBytes;           // [4][NR] float
   static constexpr int alpha = red + 4 * NR * 4;        // [NR]
   static constexpr int inv = alpha + NR * 4;            // [NR]
   static constexpr int lse = inv + NR * 4;              // [NR]
   static constexpr int bars = lse + NR * 4;
-  static constexpr int nbars = 2 * kStages + 2 + 2 * 4 + 1;  // ring, Q, S, P, O full x2, O free
+  static constexpr int nbars = 2 * kCStages + 2 * kKStages + 11;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
-  static constexpr int tmem_cols = 256;                 // S 2 x NR, O 4 x NR
+  static constexpr int tmem_cols = 256;                 // S 2 x NR (M=64 lanes), O 4 x NR
 };
 
 struct MArgs {
@@ -106,16 +108,13 @@ __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint3
       : "memory");
 }
 
-// position (within the unit's slot sequence K(0), [K(t+1), V(t)]...) of V(t)'s first slot
-__device__ __forceinline__ int vpos(int t, int T) { return kKSlots * min(t + 2, T) + kVSlots * t; }
-
 template <int NR, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
 mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant__ CUtensorMap kpe_map,
               const __grid_constant__ CUtensorMap qn_map, const __grid_constant__ CUtensorMap qp_map, MArgs a,
               const WorkItem* __restrict__ work) {
   using C = MlaCfg<NR>;
-  constexpr int NS = C::kStages;
+  constexpr int NC = C::kCStages, NK = C::kKStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = tc::smem_u32(smem);
@@ -124,22 +123,28 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::misc + 4);
   const uint32_t bar0 = sbase + C::bars;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
-  auto qfull_bar = [&]() { return bar0 + 8u * (2 * NS); };
-  auto qempty_bar = [&]() { return bar0 + 8u * (2 * NS + 1); };
-  auto sfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 2 + b); };
-  auto sempty_bar = [&](int b) { return bar0 + 8u * (2 * NS + 4 + b); };
-  auto pfull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 6 + b); };
-  auto ofull_bar = [&](int b) { return bar0 + 8u * (2 * NS + 8 + b); };
-  auto ofree_bar = [&]() { return bar0 + 8u * (2 * NS + 10); };
-  static_assert(C::nbars == 2 * NS + 11, "barrier count");
+  auto cfull_bar = [&](int s) { return bar0 + 8u * s; };
+  auto cempty_bar = [&](int s) { return bar0 + 8u * (NC + s); };
+  auto kfull_bar = [&](int s) { return bar0 + 8u * (2 * NC + s); };
+  auto kempty_bar = [&](int s) { return bar0 + 8u * (2 * NC + NK + s); };
+  const uint32_t bar1 = bar0 + 8u * (2 * NC + 2 * NK);
+  auto qfull_bar = [&]() { return bar1; };
+  auto qempty_bar = [&]() { return bar1 + 8u; };
+  auto sfull_bar = [&](int b) { return bar1 + 8u * (2 + b); };
+  auto sempty_bar = [&](int b) { return bar1 + 8u * (4 + b); };
+  auto pfull_bar = [&](int b) { return bar1 + 8u * (6 + b); };
+  auto ofull_bar = [&](int b) { return bar1 + 8u * (8 + b); };
+  auto ofree_bar = [&]() { return bar1 + 8u * 10; };
   static_assert(C::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
 
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      tc::mbar_init(full_bar(s), 1);
-      tc::mbar_init(empty_bar(s), 1);
+    for (int s = 0; s < NC; ++s) {
+      tc::mbar_init(cfull_bar(s), 1);
+      tc::mbar_init(cempty_bar(s), 1);
+    }
+    for (int s = 0; s < NK; ++s) {
+      tc::mbar_init(kfull_bar(s), 1);
+      tc::mbar_init(kempty_bar(s), 1);
     }
     tc::mbar_init(qfull_bar(), 1);
     tc::mbar_init(qempty_bar(), 1);
@@ -159,9 +164,9 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     tc::prefetch_tmap(&qn_map);
     tc::prefetch_tmap(&qp_map);
   }
-  // ring slots start as zeros: rows of a partial tile that no page fills must be finite
-  for (int i = tid; i < NS * kSlotBytes / 16; i += kThreads)
-    reinterpret_cast<uint4*>(smem + C::ring)[i] = make_uint4(0, 0, 0, 0);
+  // ckv slots start as zeros: rows of a partial tile that no page fills must be finite
+  for (int i = tid; i < NC * kCSlot / 16; i += kThreads)
+    reinterpret_cast<uint4*>(smem + C::cring)[i] = make_uint4(0, 0, 0, 0);
   tc::fence_proxy_async_smem();
   if (warp == 5) tc::tmem_alloc(tc::smem_u32(tmem_holder), C::tmem_cols);
   tc::tc_fence_before();
@@ -176,7 +181,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
 
   if (warp == 4) {
     // ======================================================================= TMA producer
-    int g = 0, n_unit = 0;  // slot-load sequence counter, units with tiles
+    int gc = 0, gk = 0, n_unit = 0;
     bool ok = true;
     for (int u = u_begin; u < u_end && ok; ++u) {
       const MUnit x = load_munit(a, work, u);
@@ -184,8 +189,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
       const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
       const int npages = x.page_end - x.page_begin;
       for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
-        // Q of this unit once the previous unit's last S MMA is done
-        if (lane == 0) {
+        if (lane == 0) {  // Q of this unit once the previous unit's last S MMA is done
           if (n_unit >= 1) ok = tc::mbar_wait(qempty_bar(), (n_unit + 1) & 1, abort_flag, a.status);
           if (ok) {
             const int rows = a.hc * a.q_tile;
@@ -197,67 +201,66 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         int win = -1000000, pid = 0;  // lanes hold the ids of pages [win, win + 32) of the unit
-        const int T = x.ntiles;
-        auto load_tile = [&](int t, bool kphase) -> bool {
+        for (int t = 0; t < x.ntiles && ok; ++t) {
           const int pi0 = (t * kTile) / P;
           const int npg = P >= kTile ? 1 : min(kTile / P, npages - pi0);
           const int slot0 = P >= kTile ? (t * kTile) % P : 0;
-          if (pi0 < win || pi0 + npg > win + 32) {  // keep the previous tile's pages (V pass) in view
-            win = max(0, pi0 - (P >= kTile ? 1 : kTile / P));
-            pid = (lane < 32 && win + lane < npages) ? __ldg(ids + win + lane) : 0;
+          if (pi0 < win || pi0 + npg > win + 32) {
+            win = pi0;
+            pid = (win + lane < npages) ? __ldg(ids + win + lane) : 0;
           }
-          const int nsl = kphase ? kKSlots : kVSlots;
-          for (int sl = 0; sl < nsl; ++sl, ++g) {
-            const int st = g % NS;
-            bool okl = true;
-            if (lane == 0) {
-              if (g >= NS) okl = tc::mbar_wait(empty_bar(st), ((g / NS) + 1) & 1, abort_flag, a.status);
-              if (okl) {
-                const bool kpe = kphase && sl == kKSlots - 1;
-                const int halves = kpe ? 1 : 2;
-                tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(halves * npg * box_rows * 128));
-              }
-            }
-            okl = __shfl_sync(0xffffffffu, okl ? 1 : 0, 0) != 0;
-            if (!okl) return false;
-            const uint32_t dst = sbase + C::ring + st * kSlotBytes;
-            for (int i = 0; i < npg; ++i) {
-              const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
-              if (lane == 0) {
-                if ((unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
-                const uint32_t row_off = (uint32_t)(i * box_rows * 128);
-                if (kphase && sl == kKSlots - 1) {
-                  tma3(dst + row_off, &kpe_map, full_bar(st), 0, slot0, page);
-                } else {
-                  tma3(dst + row_off, &ckv_map, full_bar(st), sl * 128, slot0, page);
-                  tma3(dst + kHalf + row_off, &ckv_map, full_bar(st), sl * 128 + 64, slot0, page);
-                }
-              }
+          // lane 0 claims the tile's kpe slot and its four ckv slots (waits + expected bytes); then
+          // nine lanes issue the nine TMA boxes at once (a single issuing thread serialises them)
+          const int sk = gk % NK;
+          int sc[kBlocks];
+#pragma unroll
+          for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
+          if (lane == 0) {
+            if (gk >= NK) ok = tc::mbar_wait(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
+            if (ok) tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(npg * box_rows * 128));
+            for (int b = 0; b < kBlocks && ok; ++b) {
+              const int g = gc + b;
+              if (g >= NC) ok = tc::mbar_wait(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
+              if (ok) tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * npg * box_rows * 128));
             }
           }
-          return true;
-        };
-        ok = load_tile(0, true);
-        for (int t = 0; t < T && ok; ++t) {
-          if (t + 1 < T) ok = load_tile(t + 1, true);
-          if (ok) ok = load_tile(t, false);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          for (int i = 0; i < npg; ++i) {
+            const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
+            if (lane == 0 && (unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
+            const uint32_t row_off = (uint32_t)(i * box_rows * 128);
+            if (lane == 8) {
+              tma3(sbase + C::kring + sk * kKSlot + row_off, &kpe_map, kfull_bar(sk), 0, slot0, page);
+            } else if (lane < 8) {
+              const int b = lane >> 1, hf = lane & 1;
+              tma3(sbase + C::cring + sc[b] * kCSlot + hf * kHalf + row_off, &ckv_map, cfull_bar(sc[b]),
+                   b * 128 + hf * 64, slot0, page);
+            }
+          }
+          ++gk;
+          gc += kBlocks;
         }
         ++n_unit;
       }
     }
     if (!ok && lane == 0) {  // drain issued copies (bounded) before the CTA can exit
-      for (int q = max(0, g - NS); q < g; ++q) {
+      for (int q = max(0, gc - NC); q < gc; ++q) {
         const uint64_t t_start = tc::globaltimer_ns();
-        while (!tc::mbar_try_wait(full_bar(q % NS), (q / NS) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
+        while (!tc::mbar_try_wait(cfull_bar(q % NC), (q / NC) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
+        }
+      }
+      for (int q = max(0, gk - NK); q < gk; ++q) {
+        const uint64_t t_start = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(kfull_bar(q % NK), (q / NK) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
         }
       }
     }
   } else if (warp == 5) {
-    // ======================================================================= MMA issuer
+    // ======================================================================= QK MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, NR, false, false);
-      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, NR, true, false);
-      int g = 0, n_unit = 0, n_tile = 0;
+      constexpr uint32_t idesc_s = tc::idesc_bf16_f32(64, NR, false, false);
+      int gc = 0, gk = 0, n_unit = 0, n_tile = 0;
       bool ok = true;
       for (int u = u_begin; u < u_end && ok; ++u) {
         const MUnit x = load_munit(a, work, u);
@@ -268,68 +271,88 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           if (!ok) break;
           tc::tc_fence_after();
           const uint32_t qs = sbase + C::q;
-          auto issue_s = [&](int t) -> bool {  // consumes the 5 K-phase slots of tile t
+          for (int t = 0; t < T && ok; ++t) {  // kpe slot (released) + the 4 ckv blocks (kept for PV)
             const int tt = n_tile + t, sb = tt & 1;
-            if (tt >= 2 && !tc::mbar_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1, abort_flag, a.status)) return false;
-            for (int sl = 0; sl < kKSlots; ++sl, ++g) {
-              const int st = g % NS;
-              if (!tc::mbar_wait(full_bar(st), (g / NS) & 1, abort_flag, a.status)) return false;
-              tc::tc_fence_after();
-              const uint32_t base = sbase + C::ring + st * kSlotBytes;
-              const int nk = sl == kKSlots - 1 ? 4 : 8;
-              for (int k = 0; k < nk; ++k) {
-                const int qreg = sl == kKSlots - 1 ? 8 : 2 * sl + (k >> 2);
-                const uint64_t ad = tc::sdesc_sw128(base + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
-                const uint64_t bd = tc::sdesc_sw128(qs + qreg * C::kQRegion + (k & 3) * 32, 16, 1024);
-                tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, (sl > 0 || k > 0) ? 1u : 0u);
-              }
-              tc::mma_commit(empty_bar(st));
-            }
-            tc::mma_commit(sfull_bar(sb));
-            return true;
-          };
-          auto issue_pv = [&](int t) -> bool {  // consumes the 4 V-phase slots of tile t
-            const int tt = n_tile + t, pb = tt & 1;
-            if (!tc::mbar_wait(pfull_bar(pb), (tt >> 1) & 1, abort_flag, a.status)) return false;
-            // the single O^T buffer was read by the previous unit's epilogue
-            if (t == 0 && n_unit >= 1 && !tc::mbar_wait(ofree_bar(), (n_unit + 1) & 1, abort_flag, a.status))
-              return false;
+            if (tt >= 2) ok = tc::mbar_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1, abort_flag, a.status);
+            const int sk = gk % NK;
+            if (ok) ok = tc::mbar_wait(kfull_bar(sk), (gk / NK) & 1, abort_flag, a.status);
+            if (!ok) break;
             tc::tc_fence_after();
-            const uint32_t ps = sbase + C::p + pb * C::kPBytes;
-            for (int b = 0; b < kVSlots; ++b, ++g) {
-              const int st = g % NS;
-              if (!tc::mbar_wait(full_bar(st), (g / NS) & 1, abort_flag, a.status)) return false;
-              tc::tc_fence_after();
-              const uint32_t vs = sbase + C::ring + st * kSlotBytes;
-              for (int k = 0; k < kTile / 16; ++k) {
-                const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
-                const uint64_t bd = tc::sdesc_sw128(ps + (k >> 2) * (NR * 128) + (k & 3) * 32, 16, 1024);
-                tc::mma_bf16(tm_o + b * NR, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
-              }
-              tc::mma_commit(empty_bar(st));
+            const uint32_t kb = sbase + C::kring + sk * kKSlot;
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = tc::sdesc_sw128(kb + k * 32, 16, 1024);
+              const uint64_t bd = tc::sdesc_sw128(qs + 8 * C::kQRegion + k * 32, 16, 1024);
+              tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, k > 0 ? 1u : 0u);
             }
-            tc::mma_commit(ofull_bar(pb));
-            return true;
-          };
-          ok = issue_s(0);
-          for (int t = 0; t < T && ok; ++t) {
-            if (t + 1 < T) ok = issue_s(t + 1);
-            if (ok && t + 1 == T) tc::mma_commit(qempty_bar());  // Q free after the last S
-            if (ok) ok = issue_pv(t);
+            tc::mma_commit(kempty_bar(sk));
+            ++gk;
+            for (int b = 0; b < kBlocks && ok; ++b, ++gc) {
+              const int st = gc % NC;
+              ok = tc::mbar_wait(cfull_bar(st), (gc / NC) & 1, abort_flag, a.status);
+              if (!ok) break;
+              tc::tc_fence_after();
+              const uint32_t cb = sbase + C::cring + st * kCSlot;
+              for (int k = 0; k < 8; ++k) {
+                const uint64_t ad = tc::sdesc_sw128(cb + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
+                const uint64_t bd = tc::sdesc_sw128(qs + (2 * b + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
+                tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, 1u);
+              }
+            }
+            if (!ok) break;
+            tc::mma_commit(sfull_bar(sb));
+            if (t + 1 == T) tc::mma_commit(qempty_bar());  // Q free after the unit's last QK
           }
           n_tile += T;
           ++n_unit;
         }
       }
     }
-  } else {
+  } else if (warp == 6) {
+    // ======================================================================= PV MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, NR, true, false);
+      int gc = 0, n_unit = 0, n_tile = 0;
+      bool ok = true;
+      for (int u = u_begin; u < u_end && ok; ++u) {
+        const MUnit x = load_munit(a, work, u);
+        if (x.ntiles == 0) continue;
+        for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+          const int T = x.ntiles;
+          for (int t = 0; t < T && ok; ++t) {  // the 4 ckv blocks of tile t, released afterwards
+            const int tt = n_tile + t, pb = tt & 1;
+            ok = tc::mbar_wait(pfull_bar(pb), (tt >> 1) & 1, abort_flag, a.status);
+            // the single O^T buffer was read by the previous unit's epilogue
+            if (ok && t == 0 && n_unit >= 1) ok = tc::mbar_wait(ofree_bar(), (n_unit + 1) & 1, abort_flag, a.status);
+            if (!ok) break;
+            tc::tc_fence_after();
+            const uint32_t ps = sbase + C::p + pb * C::kPBytes;
+            for (int b = 0; b < kBlocks; ++b, ++gc) {
+              const int st = gc % NC;
+              const uint32_t vs = sbase + C::cring + st * kCSlot;
+              for (int k = 0; k < kTile / 16; ++k) {
+                const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
+                const uint64_t bd = tc::sdesc_sw128(ps + k * 32, 16, 1024);
+                tc::mma_bf16(tm_o + b * NR, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+              }
+              tc::mma_commit(cempty_bar(st));
+            }
+            tc::mma_commit(ofull_bar(pb));
+          }
+          n_tile += T;
+          ++n_unit;
+        }
+      }
+    }
+  } else if (warp < 4) {
     // ======================================================================= softmax / epilogue
     float* red = reinterpret_cast<float*>(smem + C::red);
     float* alpha_s = reinterpret_cast<float*>(smem + C::alpha);
     float* inv_s = reinterpret_cast<float*>(smem + C::inv);
     float* lse_s = reinterpret_cast<float*>(smem + C::lse);
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    int g = 0, n_unit = 0, n_tile = 0, pv_seen = 0;
+    const bool srow = lane < 16;              // this lane holds an S^T row (M = 64 layout)
+    const int tok_in_tile = 16 * warp + (lane & 15);
+    int gc = 0, n_unit = 0, n_tile = 0, pv_seen = 0;
     bool ok = true;
     auto consume_pv = [&](int upto) {
       for (; pv_seen <= upto; ++pv_seen)
@@ -361,6 +384,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           continue;
         }
         const int T = x.ntiles;
+        const int gc0 = gc;
         float m[NR], l[NR];
 #pragma unroll
         for (int n = 0; n < NR; ++n) {
@@ -384,7 +408,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           tc::tc_fence_before();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(sempty_bar(sb));
-          const bool valid = x.t0 + t * kTile + tid < x.t1;
+          const bool valid = srow && x.t0 + t * kTile + tok_in_tile < x.t1;
           bool raise = false;
 #pragma unroll
           for (int n = 0; n < NR; ++n) {
@@ -396,28 +420,32 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
               failed = true;
               break;
             }
-            float* rr = red;  // one exchange buffer, guarded by the barriers around its use
 #pragma unroll
             for (int n = 0; n < NR; ++n) {
-              const float v = warp_max(s[n]);
-              if (lane == 0) rr[warp * NR + n] = v;
+              float v = s[n];
+#pragma unroll
+              for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+              if (lane == 0) red[warp * NR + n] = v;
             }
             tc::named_bar_sync(1, 128);
             float al[NR];
 #pragma unroll
             for (int n = 0; n < NR; ++n) {
-              const float mx = fmaxf(fmaxf(rr[n], rr[NR + n]), fmaxf(rr[2 * NR + n], rr[3 * NR + n]));
+              const float mx = fmaxf(fmaxf(red[n], red[NR + n]), fmaxf(red[2 * NR + n], red[3 * NR + n]));
               const float mn = fmaxf(m[n], mx);
               al[n] = (mn == -INFINITY || m[n] == mn) ? 1.f : exp2f(m[n] - mn);
               l[n] *= al[n];
               m[n] = mn;
             }
             if (t > 0) {  // rescale O^T in TMEM (every thread owns lane `tid` of the 4 blocks)
-              if (tid < NR) alpha_s[tid] = al[tid];
+              if (tid == 0) {
+#pragma unroll
+                for (int n = 0; n < NR; ++n) alpha_s[n] = al[n];
+              }
               tc::named_bar_sync(1, 128);
               consume_pv(tt - 1);
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
+              for (int b = 0; b < kBlocks; ++b) {
 #pragma unroll
                 for (int c = 0; c < NR; c += 16) {
                   float ov[16];
@@ -433,13 +461,11 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             }
             tc::named_bar_sync(1, 128);  // red / alpha_s reads done before any later rewrite
           }
-          // a partial tile: zero this token's V rows in the 4 second-pass slots (once they land)
-          if (!valid) {
-            const int gv = g + vpos(t, T);
-            for (int b = 0; b < kVSlots; ++b) {
-              const int q = gv + b, st = q % NS;
-              ok = tc::mbar_wait(full_bar(st), (q / NS) & 1, abort_flag, a.status) && ok;
-              uint8_t* row = smem + C::ring + st * kSlotBytes + tid * 128;
+          if (srow && !valid) {  // zero this token's V row in the tile's four held ckv blocks
+#pragma unroll 1
+            for (int b = 0; b < kBlocks; ++b) {
+              const int st = (gc0 + kBlocks * t + b) % NC;
+              uint8_t* row = smem + C::cring + st * kCSlot + tok_in_tile * 128;
 #pragma unroll
               for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
@@ -447,12 +473,15 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             }
           }
           if (tt >= 2 && pv_seen <= tt - 2) consume_pv(tt - 2);  // P(t) reuses PV(t-2)'s buffer
-          uint8_t* pb = smem + C::p + (tt & 1) * C::kPBytes + (tid >> 6) * (NR * 128);
+          if (srow) {
+            uint8_t* pb = smem + C::p + (tt & 1) * C::kPBytes;
 #pragma unroll
-          for (int n = 0; n < NR; ++n) {
-            const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - m[n]);
-            l[n] += p;
-            *reinterpret_cast<__nv_bfloat16*>(pb + tc::sw128_offset(n, tid & 63)) = __float2bfloat16_rn(p);
+            for (int n = 0; n < NR; ++n) {
+              const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - m[n]);
+              l[n] += p;
+              if (n < rows)
+                *reinterpret_cast<__nv_bfloat16*>(pb + tc::sw128_offset(n, tok_in_tile)) = __float2bfloat16_rn(p);
+            }
           }
           tc::fence_proxy_async_smem();
           __syncwarp();
@@ -462,11 +491,11 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           ok = false;
           break;
         }
-        g += (kKSlots + kVSlots) * T;
+        gc = gc0 + kBlocks * T;
         n_tile += T;
         ++n_unit;
         consume_pv(n_tile - 1);
-        // column sums over the 128 token lanes
+        // column sums over the 64 token lanes (lanes 16-31 of each warp hold zeros)
 #pragma unroll
         for (int n = 0; n < NR; ++n) {
           const float v = warp_sum(l[n]);
@@ -476,14 +505,17 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           ok = false;
           break;
         }
-        if (tid < NR) {
-          const float lt = red[tid] + red[NR + tid] + red[2 * NR + tid] + red[3 * NR + tid];
-          inv_s[tid] = lt > 0.f ? 1.f / lt : 0.f;
-          lse_s[tid] = lt > 0.f ? (m[tid] + log2f(lt)) * kLn2 : -INFINITY;
-        }
-        float ov[4][NR];
+        if (tid == 0) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+          for (int n = 0; n < NR; ++n) {
+            const float lt = red[n] + red[NR + n] + red[2 * NR + n] + red[3 * NR + n];
+            inv_s[n] = lt > 0.f ? 1.f / lt : 0.f;
+            lse_s[n] = lt > 0.f ? (m[n] + log2f(lt)) * kLn2 : -INFINITY;
+          }
+        }
+        float ov[kBlocks][NR];
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b)
 #pragma unroll
           for (int c = 0; c < NR; c += 16) {
             float v16[16];
@@ -504,11 +536,11 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           if (x.part_row < 0) {
             OutT* dst = reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.heads + h) * 512 + tid;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) store_out(dst + b * 128, ov[b][n] * iv);
+            for (int b = 0; b < kBlocks; ++b) store_out(dst + b * 128, ov[b][n] * iv);
           } else {
             float* dst = a.o_part + (((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h) * 512 + tid;
 #pragma unroll
-            for (int b = 0; b < 4; ++b) dst[b * 128] = ov[b][n] * iv;
+            for (int b = 0; b < kBlocks; ++b) dst[b * 128] = ov[b][n] * iv;
           }
         }
         if (tid < rows) {
@@ -576,6 +608,8 @@ bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_u
   return kv_dtype == SKV_BF16 && page_ok && (rows_per_unit == 16 || rows_per_unit == 32) &&
          (num_heads <= rows_per_unit || num_heads % rows_per_unit == 0);
 }
+
+int mla_tc_tile_tokens() { return kTile; }
 
 int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                   int q_tile, int rows_per_unit, cudaStream_t s) {

@@ -49,6 +49,7 @@ int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, const in
 int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work, int q_tile,
                     cudaStream_t s);
 bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit);
+int mla_tc_tile_tokens();
 int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                   int q_tile, int rows_per_unit, cudaStream_t s);
 int launch_wait_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
