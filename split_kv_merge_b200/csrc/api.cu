@@ -333,17 +333,20 @@ skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32
   const int32_t g = num_qo_heads / num_kv_heads;
   int32_t max_q = 1;
   for (const auto& q : req) max_q = std::max(max_q, q.q_len);
-  // tensor-core decode when the shape fits its tiles (query rows of a work item <= 16), else the
-  // generic CUDA-core kernel
   // all-KV-heads tensor-core decode when every request's query rows per KV head fit its 8
   // columns (whole pages stream contiguously); else the per-KV-head tensor-core decode; else the
   // generic CUDA-core kernel
   const bool wide = g <= 8 && 8 % g == 0 && max_q * g <= 8 &&
                     gqa_tc_wide_supported(head_dim, page_size, num_kv_heads, g, 8 / g);
+  // more query rows per KV head than one 16-column decode tile holds: 128-row prefill tiles
+  const bool prefill = !wide && (int64_t)max_q * g > 16 && gqa_tc_prefill_supported(head_dim, page_size, g);
   const int32_t tc_q_tile = std::max<int32_t>(1, std::min<int32_t>(16 / std::max<int32_t>(g, 1), max_q));
-  const bool tc = !wide && g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
-  const int32_t kernel = wide ? KERNEL_GQA_TC_WIDE : tc ? KERNEL_GQA_TC_DECODE : KERNEL_GQA_SIMT;
-  const int32_t q_tile = wide ? 8 / g : tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
+  const bool tc = !wide && !prefill && g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
+  const int32_t kernel = wide      ? KERNEL_GQA_TC_WIDE
+                         : prefill ? KERNEL_GQA_TC_PREFILL
+                         : tc      ? KERNEL_GQA_TC_DECODE
+                                   : KERNEL_GQA_SIMT;
+  const int32_t q_tile = wide ? 8 / g : prefill ? 128 / g : tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
   std::vector<int64_t> kv_len(batch);
   for (int32_t r = 0; r < batch; ++r)
     kv_len[r] = req[r].n_pages == 0 ? 0
@@ -355,7 +358,7 @@ skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32
     po.tile_tokens = 16;
   }
   // per-KV-head tensor-core kernel: a few large units per SM; CUDA-core kernel: many small CTAs
-  return plan_common(batch, req, kv_len, q_tile, wide ? 1 : num_kv_heads, tc ? 6 : 64, policy, param,
+  return plan_common(batch, req, kv_len, q_tile, wide ? 1 : num_kv_heads, prefill ? 2 : tc ? 6 : 64, policy, param,
                      split_indptr_h, split_bounds_h, kernel, po, plan_h, plan_capacity, info);
 }
 
@@ -417,7 +420,8 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
   if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
     return SKV_ERR_ALIGNMENT;
   if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
-  if (info->kernel != KERNEL_GQA_SIMT && info->kernel != KERNEL_GQA_TC_DECODE && info->kernel != KERNEL_GQA_TC_WIDE)
+  if (info->kernel != KERNEL_GQA_SIMT && info->kernel != KERNEL_GQA_TC_DECODE && info->kernel != KERNEL_GQA_TC_WIDE &&
+      info->kernel != KERNEL_GQA_TC_PREFILL)
     return SKV_ERR_INVALID;
   const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
                        p->k_stride[2] == p->v_stride[2];
@@ -428,6 +432,7 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
     return SKV_ERR_INVALID;
   int e = info->kernel == KERNEL_GQA_TC_WIDE
               ? launch_gqa_tc_wide(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile, s)
+          : info->kernel == KERNEL_GQA_TC_PREFILL ? launch_gqa_tc_prefill(*p, work, info->num_work, info->q_tile, s)
           : info->kernel == KERNEL_GQA_TC_DECODE ? launch_gqa_tc_decode(*p, work, info->num_work, info->q_tile, s)
                                                  : launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
   return cuda_status(e);

@@ -27,6 +27,7 @@ enum KernelId : int32_t {
   KERNEL_GQA_SIMT = 1,
   KERNEL_GQA_TC_DECODE = 2,
   KERNEL_GQA_TC_WIDE = 3,
+  KERNEL_GQA_TC_PREFILL = 4,  // tensor-core, 128 query rows (tokens x group heads) per unit
   KERNEL_MLA_SIMT = 11,
   KERNEL_MLA_TC16 = 12,  // tensor-core MLA, 16 query rows per unit
   KERNEL_MLA_TC32 = 13,  // tensor-core MLA, 32 query rows per unit
@@ -46,6 +47,9 @@ int launch_gqa_tc_decode(const skv_paged_params& p, const WorkItem* work, int nu
 bool gqa_tc_wide_supported(int head_dim, int page_size, int num_kv_heads, int group, int q_tile);
 int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                        int q_tile, cudaStream_t s);
+bool gqa_tc_prefill_supported(int head_dim, int page_size, int group);
+int launch_gqa_tc_prefill(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
+                          cudaStream_t s);
 int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work, int q_tile,
                     cudaStream_t s);
 bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit);

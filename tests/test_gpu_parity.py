@@ -372,6 +372,57 @@ def test_all_heads_decode_rising_scores(policy, param):
     _cmp(_np(o), _np(lse), O, LSE, where=f"rising {policy}")
 
 
+PREFILL_SHAPES = {
+    # name: (hq, hk, page_size, kv lengths, query lengths, independent V)
+    "g4_p64": (32, 8, 64, [0, 1, 63, 64, 65, 1000, 3000], [5, 0, 40, 33, 1, 128, 70], False),
+    "g1_p128": (4, 4, 128, [129, 1, 700, 384], [130, 17, 1, 64], True),
+    "g1_p256": (2, 2, 256, [1000, 255, 256, 3], [20, 200, 9, 33], False),
+    "g8_p16": (64, 8, 16, [17, 300, 2049], [3, 16, 40], True),
+    "g16_p32": (32, 2, 32, [500, 31, 1025], [8, 2, 9], False),
+}
+
+
+@pytest.mark.parametrize("shape", sorted(PREFILL_SHAPES))
+@pytest.mark.parametrize("policy,param", [("none", 0), ("fixed", 3), ("balanced", 148)])
+def test_prefill_tensor_core(shape, policy, param):
+    """Shapes with more query rows per KV head than a decode tile holds run on the 128-row
+    prefill kernel: group sizes 1 to 16, page sizes 16 to 256 (several pages per 128-key tile and
+    several tiles per page), empty requests and requests with no query rows, ragged key tails,
+    poisoned unused slots, independent V strides, whole and split KV."""
+    from workloads.gen import _make_paged
+    hq, hk, P, lens, qlens, indep = PREFILL_SHAPES[shape]
+    c = _make_paged("prefill_" + shape, 31, lens, 1, hq, hk, 128, P, indep, extra_pages=2, poison=True,
+                    qo_lens=qlens)
+    o, lse, ex, _ = _run_paged(c, policy, param)
+    assert ex["plan"].info.kernel == 4 and ex["plan"].info.q_tile == 128 // (hq // hk)
+    O, LSE = _oracle_paged(c)
+    _cmp(_np(o), _np(lse), O, LSE, where=f"prefill {shape} {policy}")
+
+
+def test_prefill_tensor_core_rising_scores_fp32_and_bf16_out():
+    """fp32 and bf16 output, with keys scaled up along the sequence so the running maximum of every row keeps
+    rising (the rescale of l and of the row of O in tensor memory)."""
+    from workloads.gen import _make_paged, bf16_bits_to_f32, f32_to_bf16_bits
+    c = _make_paged("prefill_rising", 32, [3000, 700, 129], 1, 32, 8, 128, 64, False, qo_lens=[50, 9, 128])
+    k = bf16_bits_to_f32(c.k_store).copy()
+    for r in range(c.batch):
+        pages, slots = OA.request_token_slots(c.kv_indptr, c.kv_indices, c.kv_last_page_len, 64, r)
+        L = len(pages)
+        k[pages, slots] *= (1.0 + 9.0 * np.arange(L) / max(1, L)).astype(np.float32)[:, None, None]
+    c.k_store = f32_to_bf16_bits(k).reshape(c.k_store.shape)
+    c.k = c.k_store
+    O, LSE = _oracle_paged(c)
+    o, lse, ex, _ = _run_paged(c, "fixed", 2)
+    assert ex["plan"].info.kernel == 4
+    _cmp(_np(o), _np(lse), O, LSE, where="prefill rising")
+    # bf16 output: the final rounding adds up to half a bf16 ulp (|O| * 2^-8 bounds it) on top of
+    # the fp32 result's error; rows here are close to single V rows, so |O| reaches a few units
+    ob, lb, _, _ = _run_paged(c, "fixed", 2, o_dtype=torch.bfloat16)
+    err = np.abs(_np(ob) - O) - np.abs(O) * 2.0 ** -8
+    assert float(err.max()) <= O_TOL, f"prefill rising bf16: {float(err.max())}"
+    assert float(np.max(np.abs(_np(lb) - LSE))) <= LSE_TOL
+
+
 # ----------------------------------------------------------------------------- failure detection
 def test_bounded_wait_reports_timeout_and_context_stays_usable():
     """A wait on a barrier nothing arrives on gives up after its limit and reports SKV_DEV_TIMEOUT;
