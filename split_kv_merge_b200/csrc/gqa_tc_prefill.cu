@@ -52,6 +52,36 @@ struct Smem {
 };
 static_assert(Smem::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
 
+// packed f32 pairs (sm_100 f32x2 arithmetic), 3-input max, hardware exp2
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 struct PArgs {
   const int32_t* kv_indptr;
   const int32_t* kv_indices;
@@ -242,22 +272,32 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       tc::tc_fence_after();
       float s[kTile];
 #pragma unroll
-      for (int c = 0; c < kTile; c += 16) {
+      for (int c = 0; c < kTile; c += 16) {  // all loads in flight, one wait
         float v16[16];
         tc::tmem_ld_x16(tm_s + lane_base + sb * kTile + c, v16);
-        tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i) s[c + i] = v16[i];
       }
+      tc::tmem_wait_ld();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(sempty_bar(sb));
       const int nvalid = t1 - (t0 + t * kTile);   // keys of this tile that exist (>= 1)
-      float mx = -INFINITY;
+      if (nvalid < kTile) {                       // the item's last tile only
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        s[c] = c < nvalid ? s[c] * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kTile; ++c) s[c] = c < nvalid ? s[c] : -INFINITY;
+      }
+      float mx;
+      {  // raw row maximum in 8 independent chains (the scale is positive: scale after)
+        float q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float v = fmax3(s[16 * j], s[16 * j + 1], s[16 * j + 2]);
+#pragma unroll
+          for (int i = 3; i < 15; i += 2) v = fmax3(v, s[16 * j + i], s[16 * j + i + 1]);
+          q[j] = fmaxf(v, s[16 * j + 15]);
+        }
+        mx = fmax3(fmax3(q[0], q[1], q[2]), fmax3(q[3], q[4], q[5]), fmaxf(q[6], q[7])) * a.scale_log2;
       }
       const bool raise = mx > m + kRaise;
       if (__any_sync(0xffffffffu, raise)) {  // warp-uniform: TMEM access below is warp-collective
@@ -294,25 +334,34 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       }
       if (t >= 2 && pv_seen <= t - 2) consume_pv(t - 2);  // P(t) reuses the buffer PV(t-2) read
       uint8_t* prow = smem + Smem::p + (t & 1) * kKBytes;
-      float lsum = 0.f, lrsum = 0.f;
+      // p = 2^(s * scale - m) (ex2 of -inf is +0); sums of the exact and of the rounded weights in
+      // packed pairs, two chains each
+      const uint64_t sc2 = pk2(a.scale_log2, a.scale_log2), nm2 = pk2(-m, -m);
+      uint64_t la[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)}, lb[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < kTile; c += 8) {
         uint32_t pk[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float p0 = s[c + 2 * i] == -INFINITY ? 0.f : exp2f(s[c + 2 * i] - m);
-          const float p1 = s[c + 2 * i + 1] == -INFINITY ? 0.f : exp2f(s[c + 2 * i + 1] - m);
+          float x0, x1;
+          upk2(fma2(pk2(s[c + 2 * i], s[c + 2 * i + 1]), sc2, nm2), x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
           __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          lsum += p0 + p1;
-          lrsum += __low2float(h2) + __high2float(h2);
           pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          la[i & 1] = add2(la[i & 1], pk2(p0, p1));
+          lb[i & 1] = add2(lb[i & 1], pk2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u)));
         }
         // row r, keys c..c+7: region c/64, 16-byte chunk (c%64)/8 swizzled by r%8
         const uint32_t off = (uint32_t)((c >> 6) * kRegion + r * 128 + (((((c & 63) >> 3) ^ (r & 7)) & 7) << 4));
         *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      l += lsum;
-      lr += lrsum;
+      {
+        float a0, a1, b0, b1;
+        upk2(add2(la[0], la[1]), a0, a1);
+        upk2(add2(lb[0], lb[1]), b0, b1);
+        l += a0 + a1;
+        lr += b0 + b1;
+      }
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(pfull_bar(t & 1));
