@@ -384,7 +384,8 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
   // tensor-core kernel: 16 query rows per tile when all of a request's rows fit, else 32 (heads
   // beyond 32 in groups of 32); the fold puts as many query tokens as fit into those rows
   const int32_t nr = (int64_t)num_heads * q_len <= 16 ? 16 : 32;
-  const bool tc = mla_tc_supported(kv_dtype, page_size, num_heads, nr);
+  const bool tc = kv_dtype == SKV_E4M3 ? mla_tc_fp8_supported(page_size, num_heads, nr)
+                                       : mla_tc_supported(kv_dtype, page_size, num_heads, nr);
   PersistOpts po;
   po.page_size = page_size;
   int32_t kernel = KERNEL_MLA_SIMT, fold = skv_mla_fold_ratio(num_heads, q_len, 128);
@@ -490,9 +491,12 @@ skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d
     return SKV_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  int e = tc ? launch_mla_tc(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile,
-                             info->kernel == KERNEL_MLA_TC16 ? 16 : 32, s)
-             : launch_mla_simt(*p, work, info->num_work, info->q_tile, s);
+  const int rows = info->kernel == KERNEL_MLA_TC16 ? 16 : 32;
+  int e = !tc                         ? launch_mla_simt(*p, work, info->num_work, info->q_tile, s)
+          : p->kv_dtype == SKV_E4M3 ? launch_mla_tc_fp8(*p, work, plan_d + info->cta_offset, info->num_ctas,
+                                                        info->q_tile, rows, s)
+                                      : launch_mla_tc(*p, work, plan_d + info->cta_offset, info->num_ctas,
+                                                      info->q_tile, rows, s);
   return cuda_status(e);
 }
 

@@ -29,8 +29,8 @@ enum KernelId : int32_t {
   KERNEL_GQA_TC_WIDE = 3,
   KERNEL_GQA_TC_PREFILL = 4,  // tensor-core, 128 query rows (tokens x group heads) per unit
   KERNEL_MLA_SIMT = 11,
-  KERNEL_MLA_TC16 = 12,  // tensor-core MLA, 16 query rows per unit
-  KERNEL_MLA_TC32 = 13,  // tensor-core MLA, 32 query rows per unit
+  KERNEL_MLA_TC16 = 12,  // tensor-core MLA, 16 query rows per unit (bf16 or e4m3 cache)
+  KERNEL_MLA_TC32 = 13,  // tensor-core MLA, 32 query rows per unit (bf16 or e4m3 cache)
 };
 
 // Plan words: [work items (8 words each)] [merge items (4 words each)].
@@ -56,6 +56,9 @@ bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_u
 int mla_tc_tile_tokens();
 int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                   int q_tile, int rows_per_unit, cudaStream_t s);
+bool mla_tc_fp8_supported(int page_size, int num_heads, int rows_per_unit);
+int launch_mla_tc_fp8(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
+                      int q_tile, int rows_per_unit, cudaStream_t s);
 int launch_wait_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,
                  int32_t num_states, const MergeItem* items, int64_t num_rows, int32_t num_heads,
