@@ -20,9 +20,10 @@
 //     exchange paid only on a raise; O^T is rescaled in TMEM by all four softmax warps then.
 //   * Tokens past the end of the unit get s = -inf by selection and their V rows are zeroed in
 //     the held tile before the PV that reads them.
-// Roles: warp 4 TMA producer, warp 5 TMEM allocation + QK MMA issue, warp 6 PV MMA issue (a
-// separate thread, so PV(t) is issued as soon as P(t) is ready instead of behind QK(t+1), which
-// releases tile t's slots earlier), warps 0-3 softmax / epilogue.
+// Roles: warp 4 TMA producer; warps 5-8 MMA issue, one per SM sub-partition (an MMA whose operands
+// stream from shared memory holds its issuing thread for ~80 cycles, and issuers on different
+// sub-partitions overlap): issuer w computes QK quarter w into its own partial S^T accumulator and
+// PV block w; warp 5 also allocates TMEM; warps 0-3 softmax / epilogue.
 // All waits are bounded (SKV_DEV_TIMEOUT); roles leave together; TMEM is always released.
 #include <cudaTypedefs.h>
 
@@ -38,7 +39,8 @@ constexpr int kTile = 64;              // tokens per tile
 constexpr int kHalf = kTile * 128;     // one 64-column swizzled region of a tile: 8 KB
 constexpr int kCSlot = 2 * kHalf;      // ckv slot: one 128-dim block (16 KB)
 constexpr int kKSlot = kHalf;          // kpe slot (8 KB)
-constexpr int kThreads = 224;        // 4 softmax warps, TMA warp, QK-MMA warp, PV-MMA warp
+constexpr int kIssuers = 4;          // MMA issuing warps 5-8, one per SM sub-partition
+constexpr int kThreads = (5 + kIssuers) * 32;  // 4 softmax warps, TMA warp, 4 MMA-issuing warps
 constexpr int kBlocks = 4;             // 512 ckv dims = 4 blocks of 128
 constexpr float kRaise = 8.f;
 
@@ -57,11 +59,14 @@ struct MlaCfg {
   static constexpr int alpha = red + 4 * NR * 4;        // [NR]
   static constexpr int inv = alpha + NR * 4;            // [NR]
   static constexpr int lse = inv + NR * 4;              // [NR]
-  static constexpr int bars = lse + NR * 4;
+  static constexpr int mrow = lse + NR * 4;             // [NR] running maximum of every row
+  static constexpr int bars = mrow + NR * 4;
   static constexpr int nbars = 2 * kCStages + 2 * kKStages + 11;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
-  static constexpr int tmem_cols = 256;                 // S 2 x NR (M=64 lanes), O 4 x NR
+  // S: 2 buffers x 4 partial accumulators (one per issuer) x NR (M=64 lanes); O^T: 4 blocks x NR
+  static constexpr int s_cols = 2 * kIssuers * NR;
+  static constexpr int tmem_cols = s_cols + 4 * NR <= 256 ? 256 : 512;
 };
 
 struct MArgs {
@@ -98,6 +103,13 @@ __device__ __forceinline__ MUnit load_munit(const MArgs& a, const WorkItem* work
   x.t1 = min(w.page_end * a.page_size, L);
   x.ntiles = x.t1 > x.t0 ? (x.t1 - x.t0 + kTile - 1) / kTile : 0;
   return x;
+}
+
+// maximum over the warp (sm_100 redux on f32)
+__device__ __forceinline__ float redux_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 
 __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2) {
@@ -144,15 +156,15 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     }
     for (int s = 0; s < NK; ++s) {
       tc::mbar_init(kfull_bar(s), 1);
-      tc::mbar_init(kempty_bar(s), 1);
+      tc::mbar_init(kempty_bar(s), kIssuers);
     }
     tc::mbar_init(qfull_bar(), 1);
-    tc::mbar_init(qempty_bar(), 1);
+    tc::mbar_init(qempty_bar(), kIssuers);
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(sfull_bar(b), 1);
+      tc::mbar_init(sfull_bar(b), kIssuers);
       tc::mbar_init(sempty_bar(b), 4);
       tc::mbar_init(pfull_bar(b), 4);
-      tc::mbar_init(ofull_bar(b), 1);
+      tc::mbar_init(ofull_bar(b), kIssuers);
     }
     tc::mbar_init(ofree_bar(), 4);
     *abort_flag = 0;
@@ -173,7 +185,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tm_s = tmem, tm_o = tmem + 2 * NR;
+  const uint32_t tm_s = tmem, tm_o = tmem + C::s_cols;
 
   const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
   const int P = a.page_size;
@@ -190,7 +202,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
       const int npages = x.page_end - x.page_begin;
       for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
         if (lane == 0) {  // Q of this unit once the previous unit's last S MMA is done
-          if (n_unit >= 1) ok = tc::mbar_wait(qempty_bar(), (n_unit + 1) & 1, abort_flag, a.status);
+          if (n_unit >= 1) ok = tc::mbar_wait_sleep(qempty_bar(), (n_unit + 1) & 1, abort_flag, a.status);
           if (ok) {
             const int rows = a.hc * a.q_tile;
             tc::mbar_arrive_expect_tx(qfull_bar(), (uint32_t)(9 * rows * 128));
@@ -216,11 +228,11 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
 #pragma unroll
           for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
           if (lane == 0) {
-            if (gk >= NK) ok = tc::mbar_wait(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
+            if (gk >= NK) ok = tc::mbar_wait_sleep(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
             if (ok) tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(npg * box_rows * 128));
             for (int b = 0; b < kBlocks && ok; ++b) {
               const int g = gc + b;
-              if (g >= NC) ok = tc::mbar_wait(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
+              if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
               if (ok) tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * npg * box_rows * 128));
             }
           }
@@ -256,88 +268,79 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         }
       }
     }
-  } else if (warp == 5) {
-    // ======================================================================= QK MMA issuer
+  } else if (warp >= 5) {
+    // ======================================================================= MMA issuers
+    // Issuer w: QK quarter w of every tile (rope k-step w + ckv block w: 9 MMAs) into its own
+    // partial S^T accumulator, and PV block w (4 MMAs) into O^T block w: four issuing threads on
+    // four sub-partitions keep several MMAs' operand fetches in flight.  Per tile the order is
+    // QK(t) then PV(t - 1).  Only issuer w reads ckv block w of a tile, so it alone frees it.
     if (lane == 0) {
+      const int w = warp - 5;
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(64, NR, false, false);
-      int gc = 0, gk = 0, n_unit = 0, n_tile = 0;
-      bool ok = true;
-      for (int u = u_begin; u < u_end && ok; ++u) {
-        const MUnit x = load_munit(a, work, u);
-        if (x.ntiles == 0) continue;
-        for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
-          const int T = x.ntiles;
-          ok = tc::mbar_wait(qfull_bar(), n_unit & 1, abort_flag, a.status);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint32_t qs = sbase + C::q;
-          for (int t = 0; t < T && ok; ++t) {  // kpe slot (released) + the 4 ckv blocks (kept for PV)
-            const int tt = n_tile + t, sb = tt & 1;
-            if (tt >= 2) ok = tc::mbar_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1, abort_flag, a.status);
-            const int sk = gk % NK;
-            if (ok) ok = tc::mbar_wait(kfull_bar(sk), (gk / NK) & 1, abort_flag, a.status);
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint32_t kb = sbase + C::kring + sk * kKSlot;
-            for (int k = 0; k < 4; ++k) {
-              const uint64_t ad = tc::sdesc_sw128(kb + k * 32, 16, 1024);
-              const uint64_t bd = tc::sdesc_sw128(qs + 8 * C::kQRegion + k * 32, 16, 1024);
-              tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, k > 0 ? 1u : 0u);
-            }
-            tc::mma_commit(kempty_bar(sk));
-            ++gk;
-            for (int b = 0; b < kBlocks && ok; ++b, ++gc) {
-              const int st = gc % NC;
-              ok = tc::mbar_wait(cfull_bar(st), (gc / NC) & 1, abort_flag, a.status);
-              if (!ok) break;
-              tc::tc_fence_after();
-              const uint32_t cb = sbase + C::cring + st * kCSlot;
-              for (int k = 0; k < 8; ++k) {
-                const uint64_t ad = tc::sdesc_sw128(cb + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
-                const uint64_t bd = tc::sdesc_sw128(qs + (2 * b + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
-                tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, 1u);
-              }
-            }
-            if (!ok) break;
-            tc::mma_commit(sfull_bar(sb));
-            if (t + 1 == T) tc::mma_commit(qempty_bar());  // Q free after the unit's last QK
-          }
-          n_tile += T;
-          ++n_unit;
-        }
-      }
-    }
-  } else if (warp == 6) {
-    // ======================================================================= PV MMA issuer
-    if (lane == 0) {
       constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, NR, true, false);
-      int gc = 0, n_unit = 0, n_tile = 0;
+      int g = 0, n_unit = 0, n_tile = 0;
       bool ok = true;
+      const uint32_t qs = sbase + C::q;
       for (int u = u_begin; u < u_end && ok; ++u) {
         const MUnit x = load_munit(a, work, u);
         if (x.ntiles == 0) continue;
         for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
           const int T = x.ntiles;
-          for (int t = 0; t < T && ok; ++t) {  // the 4 ckv blocks of tile t, released afterwards
-            const int tt = n_tile + t, pb = tt & 1;
-            ok = tc::mbar_wait(pfull_bar(pb), (tt >> 1) & 1, abort_flag, a.status);
-            // the single O^T buffer was read by the previous unit's epilogue
-            if (ok && t == 0 && n_unit >= 1) ok = tc::mbar_wait(ofree_bar(), (n_unit + 1) & 1, abort_flag, a.status);
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint32_t ps = sbase + C::p + pb * C::kPBytes;
-            for (int b = 0; b < kBlocks; ++b, ++gc) {
-              const int st = gc % NC;
-              const uint32_t vs = sbase + C::cring + st * kCSlot;
-              for (int k = 0; k < kTile / 16; ++k) {
-                const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
-                const uint64_t bd = tc::sdesc_sw128(ps + k * 32, 16, 1024);
-                tc::mma_bf16(tm_o + b * NR, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+          ok = tc::mbar_wait_sleep(qfull_bar(), n_unit & 1, abort_flag, a.status);
+          if (ok) tc::tc_fence_after();
+          // issue whichever is ready: PV(pv) (frees the tile's ckv blocks: first) or QK(qk)
+          int qk = 0, pv = 0;
+          tc::PollClock clk;
+          while (ok && pv < T) {
+            bool did = false;
+            if (pv < qk) {  // ---- PV(pv), block w
+              const int tp = n_tile + pv, pb = tp & 1;
+              const int cb = kBlocks * (g + pv) + w, st = cb % NC;
+              // the single O^T buffer was read by the previous unit's epilogue
+              if (tc::mbar_test_wait(pfull_bar(pb), (tp >> 1) & 1) &&
+                  (pv > 0 || n_unit == 0 || tc::mbar_test_wait(ofree_bar(), (n_unit + 1) & 1))) {
+                tc::tc_fence_after();
+                const uint32_t ps = sbase + C::p + pb * C::kPBytes;
+                const uint32_t vs = sbase + C::cring + st * kCSlot;
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k) {
+                  const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
+                  const uint64_t bd = tc::sdesc_sw128(ps + k * 32, 16, 1024);
+                  tc::mma_bf16(tm_o + w * NR, ad, bd, idesc_o, (pv > 0 || k > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(cempty_bar(st));
+                tc::mma_commit(ofull_bar(pb));
+                ++pv;
+                did = true;
               }
-              tc::mma_commit(cempty_bar(st));
             }
-            tc::mma_commit(ofull_bar(pb));
+            if (!did && qk < T) {  // ---- QK(qk), quarter w
+              const int tt = n_tile + qk, sb = tt & 1, gk = g + qk, sk = gk % NK;
+              const int cb = kBlocks * (g + qk) + w, st = cb % NC;
+              if ((tt < 2 || tc::mbar_test_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1)) &&
+                  tc::mbar_test_wait(kfull_bar(sk), (gk / NK) & 1) && tc::mbar_test_wait(cfull_bar(st), (cb / NC) & 1)) {
+                tc::tc_fence_after();
+                const uint32_t d = tm_s + (sb * kIssuers + w) * NR;
+                tc::mma_bf16(d, tc::sdesc_sw128(sbase + C::kring + sk * kKSlot + w * 32, 16, 1024),
+                             tc::sdesc_sw128(qs + 8 * C::kQRegion + w * 32, 16, 1024), idesc_s, 0u);
+                tc::mma_commit(kempty_bar(sk));
+                const uint32_t cbase = sbase + C::cring + st * kCSlot;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const uint64_t ad = tc::sdesc_sw128(cbase + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
+                  const uint64_t bd =
+                      tc::sdesc_sw128(qs + (2 * w + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
+                  tc::mma_bf16(d, ad, bd, idesc_s, 1u);
+                }
+                tc::mma_commit(sfull_bar(sb));
+                if (qk + 1 == T) tc::mma_commit(qempty_bar());  // Q free after the unit's last QK
+                ++qk;
+                did = true;
+              }
+            }
+            ok = clk.step(did, abort_flag, a.status);
           }
+          g += T;
           n_tile += T;
           ++n_unit;
         }
@@ -349,6 +352,8 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     float* alpha_s = reinterpret_cast<float*>(smem + C::alpha);
     float* inv_s = reinterpret_cast<float*>(smem + C::inv);
     float* lse_s = reinterpret_cast<float*>(smem + C::lse);
+    // the running maxima are the same in every thread: they live in shared memory
+    float* m_s = reinterpret_cast<float*>(smem + C::mrow);
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const bool srow = lane < 16;              // this lane holds an S^T row (M = 64 layout)
     const int tok_in_tile = 16 * warp + (lane & 15);
@@ -356,7 +361,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     bool ok = true;
     auto consume_pv = [&](int upto) {
       for (; pv_seen <= upto; ++pv_seen)
-        ok = tc::mbar_wait(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
+        ok = tc::mbar_wait_sleep(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
       tc::tc_fence_after();
     };
     for (int u = u_begin; u < u_end && ok; ++u) {
@@ -385,25 +390,30 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         }
         const int T = x.ntiles;
         const int gc0 = gc;
-        float m[NR], l[NR];
+        float l[NR];
 #pragma unroll
-        for (int n = 0; n < NR; ++n) {
-          m[n] = -INFINITY;
-          l[n] = 0.f;
-        }
+        for (int n = 0; n < NR; ++n) l[n] = 0.f;
+        if (tid < NR) m_s[tid] = -INFINITY;
+        tc::named_bar_sync(1, 128);
         bool failed = false;
         for (int t = 0; t < T; ++t) {
           const int tt = n_tile + t, sb = tt & 1;
-          ok = tc::mbar_wait(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
+          ok = tc::mbar_wait_sleep(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
           tc::tc_fence_after();
           float s[NR];
 #pragma unroll
-          for (int c = 0; c < NR; c += 16) {
-            float v16[16];
-            tc::tmem_ld_x16(tm_s + lane_base + sb * NR + c, v16);
-            tc::tmem_wait_ld();
+          for (int w = 0; w < kIssuers; ++w) {  // sum of the four partial accumulators
+            float v[NR];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) s[c + i] = v16[i];
+            for (int c = 0; c < NR; c += 16) {
+              float v16[16];
+              tc::tmem_ld_x16(tm_s + lane_base + (sb * kIssuers + w) * NR + c, v16);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[c + i] = v16[i];
+            }
+            tc::tmem_wait_ld();  // registers of a TMEM load are read only after the wait
+#pragma unroll
+            for (int n = 0; n < NR; ++n) s[n] = w == 0 ? v[n] : s[n] + v[n];
           }
           tc::tc_fence_before();
           __syncwarp();
@@ -413,7 +423,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
 #pragma unroll
           for (int n = 0; n < NR; ++n) {
             s[n] = (valid && n < rows) ? s[n] * a.scale_log2 : -INFINITY;
-            raise |= s[n] > m[n] + kRaise;
+            raise |= s[n] > m_s[n] + kRaise;
           }
           if (tc::bar_or(1, 128, raise || !ok || t == 0)) {
             if (!tc::bar_and(1, 128, ok)) {
@@ -421,38 +431,35 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
               break;
             }
 #pragma unroll
-            for (int n = 0; n < NR; ++n) {
-              float v = s[n];
-#pragma unroll
-              for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            for (int n = 0; n < NR; ++n) {  // column max over the warp's 16 token lanes (others -inf)
+              const float v = redux_max(s[n]);
               if (lane == 0) red[warp * NR + n] = v;
             }
             tc::named_bar_sync(1, 128);
-            float al[NR];
-#pragma unroll
-            for (int n = 0; n < NR; ++n) {
+            if (tid < NR) {  // one thread per row: new maximum and the factor for l and O
+              const int n = tid;
               const float mx = fmaxf(fmaxf(red[n], red[NR + n]), fmaxf(red[2 * NR + n], red[3 * NR + n]));
-              const float mn = fmaxf(m[n], mx);
-              al[n] = (mn == -INFINITY || m[n] == mn) ? 1.f : exp2f(m[n] - mn);
-              l[n] *= al[n];
-              m[n] = mn;
+              const float mo = m_s[n], mn = fmaxf(mo, mx);
+              alpha_s[n] = (mn == -INFINITY || mo == mn) ? 1.f : exp2f(mo - mn);
+              m_s[n] = mn;
             }
+            tc::named_bar_sync(1, 128);
+#pragma unroll
+            for (int n = 0; n < NR; ++n) l[n] *= alpha_s[n];
             if (t > 0) {  // rescale O^T in TMEM (every thread owns lane `tid` of the 4 blocks)
-              if (tid == 0) {
-#pragma unroll
-                for (int n = 0; n < NR; ++n) alpha_s[n] = al[n];
-              }
-              tc::named_bar_sync(1, 128);
               consume_pv(tt - 1);
+#pragma unroll 1
+              for (int c = 0; c < NR; c += 16) {  // 16 columns at a time: few registers held
+                float al[16];
 #pragma unroll
-              for (int b = 0; b < kBlocks; ++b) {
-#pragma unroll
-                for (int c = 0; c < NR; c += 16) {
+                for (int i = 0; i < 16; ++i) al[i] = alpha_s[c + i];
+#pragma unroll 1
+                for (int b = 0; b < kBlocks; ++b) {
                   float ov[16];
                   tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, ov);
                   tc::tmem_wait_ld();
 #pragma unroll
-                  for (int i = 0; i < 16; ++i) ov[i] *= alpha_s[c + i];
+                  for (int i = 0; i < 16; ++i) ov[i] *= al[i];
                   tc::tmem_st_x16(tm_o + lane_base + b * NR + c, ov);
                 }
               }
@@ -475,9 +482,12 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           if (tt >= 2 && pv_seen <= tt - 2) consume_pv(tt - 2);  // P(t) reuses PV(t-2)'s buffer
           if (srow) {
             uint8_t* pb = smem + C::p + (tt & 1) * C::kPBytes;
+            float mloc[NR];  // read the maxima before the stores below (they may alias for the compiler)
+#pragma unroll
+            for (int n = 0; n < NR; ++n) mloc[n] = m_s[n];
 #pragma unroll
             for (int n = 0; n < NR; ++n) {
-              const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - m[n]);
+              const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - mloc[n]);
               l[n] += p;
               if (n < rows)
                 *reinterpret_cast<__nv_bfloat16*>(pb + tc::sw128_offset(n, tok_in_tile)) = __float2bfloat16_rn(p);
@@ -510,7 +520,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           for (int n = 0; n < NR; ++n) {
             const float lt = red[n] + red[NR + n] + red[2 * NR + n] + red[3 * NR + n];
             inv_s[n] = lt > 0.f ? 1.f / lt : 0.f;
-            lse_s[n] = lt > 0.f ? (m[n] + log2f(lt)) * kLn2 : -INFINITY;
+            lse_s[n] = lt > 0.f ? (m_s[n] + log2f(lt)) * kLn2 : -INFINITY;
           }
         }
         float ov[kBlocks][NR];

@@ -44,7 +44,8 @@ constexpr int kTileBytes = 4 * kCSlot + kHalf;  // ckv blocks + kpe block: 72 KB
 constexpr int kSlots = 2;
 constexpr int kBlocks = 4;
 constexpr int kConvWarps = 8;
-constexpr int kFirstConv = 7;
+constexpr int kIssuers = 4;                     // MMA issuing warps 4-7, one per SM sub-partition
+constexpr int kFirstConv = 4 + kIssuers;
 constexpr int kThreads = (kFirstConv + kConvWarps) * 32;
 constexpr float kRaise = 8.f;
 constexpr int kNoRows = INT_MIN;                // page id placeholder: the warp has no rows in the tile
@@ -64,10 +65,12 @@ struct Cfg8 {
   static constexpr int qmax = lse + NR * 4;     // [4] float
   static constexpr int mrow = qmax + 16;        // [NR] float: running maximum of every row
   static constexpr int bars = mrow + NR * 4;
-  static constexpr int nbars = 2 * kSlots + 12;
+  static constexpr int nbars = 2 * kSlots + 11;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
-  static constexpr int tmem_cols = 256;         // S 2 x NR, O 4 x NR
+  // S: 2 buffers x 4 partial accumulators (one per issuer) x NR; O^T: 4 blocks x NR
+  static constexpr int s_cols = 2 * kIssuers * NR;
+  static constexpr int tmem_cols = s_cols + 4 * NR <= 256 ? 256 : 512;
 };
 
 struct M8Args {
@@ -168,6 +171,13 @@ __device__ __forceinline__ void cvt16(const uint4& v, uint4& lo, uint4& hi) {
   hi.w = e4m3x2_to_f16x2(v.w >> 16);
 }
 
+// maximum over the warp (sm_100 redux on f32)
+__device__ __forceinline__ float redux_max(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 // kind::f16 instruction descriptor with f16 A and B, f32 D
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
@@ -192,33 +202,31 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
   const uint32_t bar1 = bar0 + 8u * (2 * kSlots);
   auto qfull_bar = [&]() { return bar1; };
   auto qready_bar = [&]() { return bar1 + 8u; };
-  auto qempty_bar = [&]() { return bar1 + 16u; };
-  auto sfull_bar = [&](int b) { return bar1 + 8u * (3 + b); };
-  auto sempty_bar = [&](int b) { return bar1 + 8u * (5 + b); };
-  auto pfull_bar = [&](int b) { return bar1 + 8u * (7 + b); };
-  auto ofull_bar = [&](int b) { return bar1 + 8u * (9 + b); };
-  auto ofree_bar = [&]() { return bar1 + 8u * 11; };
+  auto sfull_bar = [&](int b) { return bar1 + 8u * (2 + b); };
+  auto sempty_bar = [&](int b) { return bar1 + 8u * (4 + b); };
+  auto pfull_bar = [&](int b) { return bar1 + 8u * (6 + b); };
+  auto ofull_bar = [&](int b) { return bar1 + 8u * (8 + b); };
+  auto ofree_bar = [&]() { return bar1 + 8u * 10; };
   static_assert(C::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
 
   if (tid == 0) {
     for (int s = 0; s < kSlots; ++s) {
       tc::mbar_init(tfull_bar(s), kConvWarps);
-      tc::mbar_init(tempty_bar(s), 1);
+      tc::mbar_init(tempty_bar(s), kIssuers);
     }
     tc::mbar_init(qfull_bar(), 1);
     tc::mbar_init(qready_bar(), 4);
-    tc::mbar_init(qempty_bar(), 1);
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(sfull_bar(b), 1);
+      tc::mbar_init(sfull_bar(b), kIssuers);
       tc::mbar_init(sempty_bar(b), 4);
       tc::mbar_init(pfull_bar(b), 4);
-      tc::mbar_init(ofull_bar(b), 1);
+      tc::mbar_init(ofull_bar(b), kIssuers);
     }
     tc::mbar_init(ofree_bar(), 4);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (tid == 0) {
     tc::prefetch_tmap(&qn_map);
     tc::prefetch_tmap(&qp_map);
   }
@@ -227,7 +235,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tm_s = tmem, tm_o = tmem + 2 * NR;
+  const uint32_t tm_s = tmem, tm_o = tmem + C::s_cols;
 
   const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
 
@@ -297,7 +305,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
       if (!v || !ok) return false;
       const int slot = gt % kSlots;
       if (gt >= kSlots) {
-        if (lane == 0) ok = tc::mbar_wait(tempty_bar(slot), ((gt / kSlots) + 1) & 1, abort_flag, a.status);
+        if (lane == 0) ok = tc::mbar_wait_sleep(tempty_bar(slot), ((gt / kSlots) + 1) & 1, abort_flag, a.status);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (!ok) return false;
       }
@@ -311,104 +319,74 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
     };
     while (step(DA, va) && step(DB, vb)) {
     }
-  } else if (warp == 4) {
-    // ======================================================================= query TMA
+  } else if (warp >= 4) {
+    // ======================================================================= MMA issuers
+    // Issuer w: QK quarter w of every tile (rope k-step w + ckv block w: 9 MMAs) into its own
+    // partial S^T accumulator, and PV block w (4 MMAs) into O^T block w.  Per tile the order is
+    // QK(t) then PV(t - 1), so S(t) is in flight while the softmax finishes P(t - 1).
     if (lane == 0) {
-      int n_unit = 0;
-      bool ok = true;
-      for (int u = u_begin; u < u_end && ok; ++u) {
-        const MUnit8 x = load_unit8(a, work, u);
-        if (x.ntiles == 0) continue;
-        for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
-          if (n_unit >= 1) ok = tc::mbar_wait(qempty_bar(), (n_unit + 1) & 1, abort_flag, a.status);
-          if (!ok) break;
-          const int rows = a.hc * a.q_tile;
-          tc::mbar_arrive_expect_tx(qfull_bar(), (uint32_t)(9 * rows * 128));
-          for (int rg = 0; rg < 8; ++rg)
-            tc::tma_load_3d(sbase + C::q + rg * C::kQRegion, &qn_map, qfull_bar(), rg * 64, hgi * a.hc, x.q_start);
-          tc::tma_load_3d(sbase + C::q + 8 * C::kQRegion, &qp_map, qfull_bar(), 0, hgi * a.hc, x.q_start);
-          ++n_unit;
-        }
-      }
-      if (!ok && n_unit >= 1) {  // the last query copy may still be landing (bounded)
-        const uint64_t t_start = tc::globaltimer_ns();
-        while (!tc::mbar_try_wait(qfull_bar(), (n_unit - 1) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
-        }
-      }
-    }
-  } else if (warp == 5) {
-    // ======================================================================= QK MMA issuer
-    if (lane == 0) {
+      const int w = warp - 4;
       constexpr uint32_t idesc_s = idesc_f16_f32(64, NR, false, false);
-      int gt = 0, n_unit = 0, n_tile = 0;
-      bool ok = true;
-      for (int u = u_begin; u < u_end && ok; ++u) {
-        const MUnit8 x = load_unit8(a, work, u);
-        if (x.ntiles == 0) continue;
-        for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
-          const int T = x.ntiles;
-          ok = tc::mbar_wait(qready_bar(), n_unit & 1, abort_flag, a.status);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint32_t qs = sbase + C::q;
-          for (int t = 0; t < T && ok; ++t, ++gt) {
-            const int tt = n_tile + t, sb = tt & 1, slot = gt % kSlots;
-            if (tt >= 2) ok = tc::mbar_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1, abort_flag, a.status);
-            if (ok) ok = tc::mbar_wait(tfull_bar(slot), (gt / kSlots) & 1, abort_flag, a.status);
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint32_t tb = sbase + C::tiles + slot * kTileBytes;
-            for (int k = 0; k < 4; ++k) {  // rope part: 64 dims
-              const uint64_t ad = tc::sdesc_sw128(tb + 4 * kCSlot + k * 32, 16, 1024);
-              const uint64_t bd = tc::sdesc_sw128(qs + 8 * C::kQRegion + k * 32, 16, 1024);
-              tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, k > 0 ? 1u : 0u);
-            }
-            for (int b = 0; b < kBlocks; ++b) {
-              for (int k = 0; k < 8; ++k) {
-                const uint64_t ad = tc::sdesc_sw128(tb + b * kCSlot + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
-                const uint64_t bd = tc::sdesc_sw128(qs + (2 * b + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
-                tc::mma_bf16(tm_s + sb * NR, ad, bd, idesc_s, 1u);
-              }
-            }
-            tc::mma_commit(sfull_bar(sb));
-            if (t + 1 == T) tc::mma_commit(qempty_bar());  // Q free after the unit's last QK
-          }
-          n_tile += T;
-          ++n_unit;
-        }
-      }
-    }
-  } else if (warp == 6) {
-    // ======================================================================= PV MMA issuer
-    if (lane == 0) {
       constexpr uint32_t idesc_o = idesc_f16_f32(128, NR, true, false);
       int gt = 0, n_unit = 0, n_tile = 0;
       bool ok = true;
+      const uint32_t qs = sbase + C::q;
       for (int u = u_begin; u < u_end && ok; ++u) {
         const MUnit8 x = load_unit8(a, work, u);
         if (x.ntiles == 0) continue;
         for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
           const int T = x.ntiles;
-          for (int t = 0; t < T && ok; ++t, ++gt) {
-            const int tt = n_tile + t, pb = tt & 1, slot = gt % kSlots;
-            ok = tc::mbar_wait(pfull_bar(pb), (tt >> 1) & 1, abort_flag, a.status);
-            // the single O^T buffer was read by the previous unit's epilogue
-            if (ok && t == 0 && n_unit >= 1) ok = tc::mbar_wait(ofree_bar(), (n_unit + 1) & 1, abort_flag, a.status);
-            if (!ok) break;
-            tc::tc_fence_after();
-            const uint32_t ps = sbase + C::p + pb * C::kPBytes;
-            const uint32_t tb = sbase + C::tiles + slot * kTileBytes;
-            for (int b = 0; b < kBlocks; ++b) {
-              const uint32_t vs = tb + b * kCSlot;
-              for (int k = 0; k < kTile / 16; ++k) {
-                const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
-                const uint64_t bd = tc::sdesc_sw128(ps + k * 32, 16, 1024);
-                tc::mma_bf16(tm_o + b * NR, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+          ok = tc::mbar_wait_sleep(qready_bar(), n_unit & 1, abort_flag, a.status);
+          if (ok) tc::tc_fence_after();
+          // issue whichever is ready: PV(pv) (frees the tile slot: first) or QK(qk)
+          int qk = 0, pv = 0;
+          tc::PollClock clk;
+          while (ok && pv < T) {
+            bool did = false;
+            if (pv < qk) {  // ---- PV(pv), block w
+              const int tp = n_tile + pv, pb = tp & 1, g = gt + pv, slot = g % kSlots;
+              // the single O^T buffer was read by the previous unit's epilogue
+              if (tc::mbar_test_wait(pfull_bar(pb), (tp >> 1) & 1) &&
+                  (pv > 0 || n_unit == 0 || tc::mbar_test_wait(ofree_bar(), (n_unit + 1) & 1))) {
+                tc::tc_fence_after();
+                const uint32_t ps = sbase + C::p + pb * C::kPBytes;
+                const uint32_t vs = sbase + C::tiles + slot * kTileBytes + w * kCSlot;
+#pragma unroll
+                for (int k = 0; k < kTile / 16; ++k) {
+                  const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
+                  const uint64_t bd = tc::sdesc_sw128(ps + k * 32, 16, 1024);
+                  tc::mma_bf16(tm_o + w * NR, ad, bd, idesc_o, (pv > 0 || k > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(tempty_bar(slot));
+                tc::mma_commit(ofull_bar(pb));
+                ++pv;
+                did = true;
               }
             }
-            tc::mma_commit(tempty_bar(slot));
-            tc::mma_commit(ofull_bar(pb));
+            if (!did && qk < T) {  // ---- QK(qk), quarter w
+              const int tt = n_tile + qk, sb = tt & 1, g = gt + qk, slot = g % kSlots;
+              if ((tt < 2 || tc::mbar_test_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1)) &&
+                  tc::mbar_test_wait(tfull_bar(slot), (g / kSlots) & 1)) {
+                tc::tc_fence_after();
+                const uint32_t tb = sbase + C::tiles + slot * kTileBytes;
+                const uint32_t d = tm_s + (sb * kIssuers + w) * NR;
+                tc::mma_bf16(d, tc::sdesc_sw128(tb + 4 * kCSlot + w * 32, 16, 1024),
+                             tc::sdesc_sw128(qs + 8 * C::kQRegion + w * 32, 16, 1024), idesc_s, 0u);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const uint64_t ad = tc::sdesc_sw128(tb + w * kCSlot + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
+                  const uint64_t bd =
+                      tc::sdesc_sw128(qs + (2 * w + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
+                  tc::mma_bf16(d, ad, bd, idesc_s, 1u);
+                }
+                tc::mma_commit(sfull_bar(sb));
+                ++qk;
+                did = true;
+              }
+            }
+            ok = clk.step(did, abort_flag, a.status);
           }
+          gt += T;
           n_tile += T;
           ++n_unit;
         }
@@ -427,11 +405,11 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const bool srow = lane < 16;              // this lane holds an S^T row (M = 64 layout)
     const int tok_in_tile = 16 * warp + (lane & 15);
-    int n_unit = 0, n_tile = 0, pv_seen = 0;
+    int n_unit = 0, n_tile = 0, pv_seen = 0, q_issued = 0, q_landed = 0;
     bool ok = true;
     auto consume_pv = [&](int upto) {
       for (; pv_seen <= upto; ++pv_seen)
-        ok = tc::mbar_wait(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
+        ok = tc::mbar_wait_sleep(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
       tc::tc_fence_after();
     };
     for (int u = u_begin; u < u_end && ok; ++u) {
@@ -458,9 +436,18 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
           }
           continue;
         }
-        // ---- queries of this unit: bf16 (TMA) -> f16 in place, shifted by 2^-k
-        ok = tc::mbar_wait(qfull_bar(), n_unit & 1, abort_flag, a.status) && ok;
-        const int qrows = a.hc * a.q_tile;     // rows the query copy filled
+        // ---- queries of this unit: bf16 (TMA) -> f16 in place, shifted by 2^-k.  The buffer is
+        // free: every QK of the previous unit completed before its last S was consumed here.
+        const int qrows = a.hc * a.q_tile;     // rows the query copy fills
+        if (tid == 0) {
+          tc::mbar_arrive_expect_tx(qfull_bar(), (uint32_t)(9 * qrows * 128));
+          for (int rg = 0; rg < 8; ++rg)
+            tc::tma_load_3d(sbase + C::q + rg * C::kQRegion, &qn_map, qfull_bar(), rg * 64, h0, x.q_start);
+          tc::tma_load_3d(sbase + C::q + 8 * C::kQRegion, &qp_map, qfull_bar(), 0, h0, x.q_start);
+        }
+        q_issued = n_unit + 1;
+        ok = tc::mbar_wait_sleep(qfull_bar(), n_unit & 1, abort_flag, a.status) && ok;
+        if (ok) q_landed = n_unit + 1;
         constexpr int kChunks = 9 * NR * 8;     // 16-byte chunks of the query block
         float qm = 0.f;
         for (int ci = tid; ci < kChunks; ci += 128) {
@@ -505,17 +492,23 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
         bool failed = false;
         for (int t = 0; t < T; ++t) {
           const int tt = n_tile + t, sb = tt & 1;
-          ok = tc::mbar_wait(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
+          ok = tc::mbar_wait_sleep(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
           tc::tc_fence_after();
           float s[NR];
 #pragma unroll
-          for (int c = 0; c < NR; c += 16) {
-            float v16[16];
-            tc::tmem_ld_x16(tm_s + lane_base + sb * NR + c, v16);
+          for (int w = 0; w < kIssuers; ++w) {  // sum of the four partial accumulators
+            float v[NR];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) s[c + i] = v16[i];
+            for (int c = 0; c < NR; c += 16) {
+              float v16[16];
+              tc::tmem_ld_x16(tm_s + lane_base + (sb * kIssuers + w) * NR + c, v16);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[c + i] = v16[i];
+            }
+            tc::tmem_wait_ld();  // registers of a TMEM load are read only after the wait
+#pragma unroll
+            for (int n = 0; n < NR; ++n) s[n] = w == 0 ? v[n] : s[n] + v[n];
           }
-          tc::tmem_wait_ld();
           tc::tc_fence_before();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(sempty_bar(sb));
@@ -532,37 +525,35 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
               break;
             }
 #pragma unroll
-            for (int n = 0; n < NR; ++n) {
-              float v = s[n];
-#pragma unroll
-              for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            for (int n = 0; n < NR; ++n) {  // column max over the warp's 16 token lanes (others -inf)
+              const float v = redux_max(s[n]);
               if (lane == 0) red[warp * NR + n] = v;
             }
             tc::named_bar_sync(1, 128);
-#pragma unroll
-            for (int n = 0; n < NR; ++n) {
+            if (tid < NR) {  // one thread per row: new maximum and the factor for l and O
+              const int n = tid;
               const float mx = fmaxf(fmaxf(red[n], red[NR + n]), fmaxf(red[2 * NR + n], red[3 * NR + n]));
               const float mo = m_s[n], mn = fmaxf(mo, mx);
-              const float al = (mn == -INFINITY || mo == mn) ? 1.f : exp2f(mo - mn);
-              l[n] *= al;
-              if (tid == 0) alpha_s[n] = al;
+              alpha_s[n] = (mn == -INFINITY || mo == mn) ? 1.f : exp2f(mo - mn);
+              m_s[n] = mn;
             }
-            tc::named_bar_sync(1, 128);  // every thread has read the old maxima
-            if (tid < NR) {
-              const int n = tid;
-              m_s[n] = fmaxf(m_s[n], fmaxf(fmaxf(red[n], red[NR + n]), fmaxf(red[2 * NR + n], red[3 * NR + n])));
-            }
+            tc::named_bar_sync(1, 128);
+#pragma unroll
+            for (int n = 0; n < NR; ++n) l[n] *= alpha_s[n];
             if (t > 0) {  // rescale O^T in TMEM (every thread owns lane `tid` of the 4 blocks)
               consume_pv(tt - 1);
+#pragma unroll 1
+              for (int c = 0; c < NR; c += 16) {  // 16 columns at a time: few registers held
+                float al[16];
 #pragma unroll
-              for (int b = 0; b < kBlocks; ++b) {
-#pragma unroll
-                for (int c = 0; c < NR; c += 16) {
+                for (int i = 0; i < 16; ++i) al[i] = alpha_s[c + i];
+#pragma unroll 1
+                for (int b = 0; b < kBlocks; ++b) {
                   float ov[16];
                   tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, ov);
                   tc::tmem_wait_ld();
 #pragma unroll
-                  for (int i = 0; i < 16; ++i) ov[i] *= alpha_s[c + i];
+                  for (int i = 0; i < 16; ++i) ov[i] *= al[i];
                   tc::tmem_st_x16(tm_o + lane_base + b * NR + c, ov);
                 }
               }
@@ -574,9 +565,12 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
           if (tt >= 2 && pv_seen <= tt - 2) consume_pv(tt - 2);  // P(t) reuses PV(t-2)'s buffer
           if (srow) {
             uint8_t* pb = smem + C::p + (tt & 1) * C::kPBytes;
+            float mloc[NR];  // read the maxima before the stores below (they may alias for the compiler)
+#pragma unroll
+            for (int n = 0; n < NR; ++n) mloc[n] = m_s[n];
 #pragma unroll
             for (int n = 0; n < NR; ++n) {
-              const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - m_s[n]);
+              const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - mloc[n]);
               l[n] += p;
               if (n < rows) *reinterpret_cast<__half*>(pb + tc::sw128_offset(n, tok_in_tile)) = __float2half_rn(p);
             }
@@ -647,6 +641,11 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
           }
         }
         tc::named_bar_sync(1, 128);  // inv_s / lse_s / red reads done before the next unit
+      }
+    }
+    if (tid == 0 && q_issued > q_landed) {  // a query copy may still be landing (bounded wait)
+      const uint64_t t_start = tc::globaltimer_ns();
+      while (!tc::mbar_try_wait(qfull_bar(), (q_issued - 1) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
       }
     }
   }

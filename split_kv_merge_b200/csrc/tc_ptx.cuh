@@ -101,6 +101,71 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Non-blocking test of a phase (for threads that poll several barriers).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bookkeeping for a polling loop: call with progressed = whether anything was issued this round.
+// Returns false (after setting the abort flag and the status) once nothing has progressed for
+// kWaitLimitNs, or when another role has aborted.
+struct PollClock {
+  uint64_t last = 0;
+  __device__ __forceinline__ bool step(bool progressed, volatile int* abort_flag, int32_t* status) {
+    if (progressed) {
+      last = 0;
+      return true;
+    }
+    const uint64_t now = globaltimer_ns();
+    if (last == 0) last = now;
+    if (*abort_flag) return false;
+    if (now - last > kWaitLimitNs) {
+      *abort_flag = 1;
+      report(status, SKV_DEV_TIMEOUT);
+      return false;
+    }
+    __nanosleep(32);
+    return true;
+  }
+};
+
+// try_wait that lets the hardware suspend the thread (up to hint_ns) until the phase completes:
+// a waiting warp stops taking issue slots from the warps that share its sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait like mbar_wait, suspending between checks instead of spinning.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      report(status, SKV_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------ TMA (no multicast)
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
                                             int c2) {
