@@ -1,34 +1,33 @@
-// MLA latent decode on the tensor cores for an fp8 (e4m3) latent cache.
+// MLA latent decode on the tensor cores for an fp8 (e4m3) latent cache, in native fp8 MMAs.
 //
 // What it computes (FlashInfer PR #3309 page, MLA decode; the e4m3 cache of the same page):
 // every head reads one latent row per token, a 512-d compressed KV (ckv) and a 64-d rope key
 // (kpe), both stored as e4m3 with one per-tensor scale; s = sm_scale * kv_scale *
-// (q_nope . ckv + q_pe . kpe), V = kv_scale * ckv.  The e4m3 values are decoded exactly.
-// seqlen_q is folded into the row dimension as in the bf16 kernel: rows n = qi * Hc + h of a
-// unit, Hc = min(H, NR), F = q_tile tokens with F * Hc <= NR; H > NR runs H / NR head groups.
+// (q_nope . ckv + q_pe . kpe), V = kv_scale * ckv.  seqlen_q is folded into the row dimension as
+// in the bf16 kernel: rows n = qi * Hc + h of a unit, Hc = min(H, NR), F = q_tile tokens with
+// F * Hc <= NR; H > NR runs H / NR head groups.
 //
-// B200 design.  The MMAs run in kind::f16 with f16 operands: every e4m3 value is an f16
-// normal (or zero), so cvt.rn.f16x2.e4m3x2 is exact and no scale touches the cache.  Queries
-// are converted to f16 once per unit after a power-of-two shift 2^-k chosen from the unit's
-// largest |q| (k = 0 unless |q| >= 2^15), and 2^k goes back into the softmax scale: exact for
-// every query value of f16 normal magnitude.  P is written as f16.
-//   * Converter warps (8) stream the cache with coalesced 16-byte loads (one 512-byte ckv row
-//     per warp instruction), two tiles ahead in registers, convert and store f16 straight into
-//     the swizzled K-major layout the MMAs read: no raw fp8 staging in shared memory, so the
-//     per-tile shared-memory traffic stays at the converted tile plus the MMA operand reads.
-//     Rows past the end of the unit are stored as zeros (finite V rows, masked scores).
-//   * Converted tiles (64 tokens: four 16 KB ckv blocks + one 8 KB kpe block) sit in two slots,
-//     held from QK to PV; PV's completion frees the slot.
-//   * S^T[64 tokens, NR] = C . Q^T (M = 64: TMEM rows in lanes 0-15 of each warp quarter) and
-//     O^T[512, NR] += V^T . P^T (four M = 128 blocks), online softmax with a lazily raised
-//     maximum and O^T rescaled in TMEM on a raise -- as in the bf16 kernel.
-// Roles: warps 0-3 softmax / query conversion / epilogue, warp 4 query TMA, warp 5 TMEM + QK
-// MMA issue, warp 6 PV MMA issue, warps 7-14 cache conversion.  All waits are bounded.
+// B200 design: tcgen05.mma kind::f8f6f4 straight on the e4m3 cache tiles, so the cache is never
+// converted and a 64-token tile is 36 KB of shared memory (four or three of them in flight).
+//   * Both other operands are split into two e4m3 terms, hi = rn(x) and lo = rn(x - hi), stacked
+//     as 2 NR columns of N: queries (bf16, 8 significant bits) after a power-of-two scaling that
+//     puts the unit's largest |q| in [128, 256) -- exact for every |q| above 2^-10 of that maximum
+//     -- and the softmax weights p in [0, 2^8] (bf16-like precision, 8 significant bits).  The
+//     scaling goes back into the softmax scale; S and O sum their hi and lo columns.
+//   * S^T[64 tokens, 2 NR] = C . [Q_hi; Q_lo]^T, K = 32 per MMA: 16 ckv k-steps (128-byte
+//     swizzled rows) + 2 rope k-steps (64-byte swizzled rows); M = 64, so TMEM rows sit in lanes
+//     0-15 of each warp quarter.  The k-steps are split over 4 (NR = 16) or 2 (NR = 32) issuers
+//     into partial accumulators that the softmax adds.
+//   * O^T[512, 2 NR] += V^T . [P_hi; P_lo]^T in four M = 128 blocks (V read MN-major from the same
+//     tile), one block per issuer.
+//   * Online softmax with a lazily raised maximum (only when a score passes it by more than 2^8),
+//     O^T rescaled in TMEM on a raise; tokens past the end of the unit get s = -inf by selection
+//     and their V rows are zeroed in the tile before the PV that reads them.
+// Roles: warps 0-3 softmax / query split / epilogue, warp 4 TMA, warps 5-8 MMA issue (one per SM
+// sub-partition; each polls for whichever of PV(t) and QK(t') is ready).  All waits are bounded.
 #include <cudaTypedefs.h>
-#include <cuda_fp16.h>
 
 #include <algorithm>
-#include <climits>
 #include <mutex>
 
 #include "tc_ptx.cuh"
@@ -37,46 +36,42 @@ namespace skv {
 
 namespace {
 
-constexpr int kTile = 64;                       // tokens per tile
-constexpr int kHalf = kTile * 128;              // one 64-column swizzled region: 8 KB
-constexpr int kCSlot = 2 * kHalf;               // one 128-dim ckv block of a tile: 16 KB
-constexpr int kTileBytes = 4 * kCSlot + kHalf;  // ckv blocks + kpe block: 72 KB
-constexpr int kSlots = 2;
+constexpr int kTile = 64;                        // tokens per tile
+constexpr int kCRegion = kTile * 128;            // 128 ckv dims (bytes) x 64 tokens: 8 KB
+constexpr int kKRegion = kTile * 64;             // 64 rope dims x 64 tokens: 4 KB (64-byte rows)
+constexpr int kTileBytes = 4 * kCRegion + kKRegion;
 constexpr int kBlocks = 4;
-constexpr int kConvWarps = 8;
-constexpr int kIssuers = 4;                     // MMA issuing warps 4-7, one per SM sub-partition
-constexpr int kFirstConv = 4 + kIssuers;
-constexpr int kThreads = (kFirstConv + kConvWarps) * 32;
+constexpr int kIssuers = 4;
+constexpr int kThreads = (5 + kIssuers) * 32;
 constexpr float kRaise = 8.f;
-constexpr int kNoRows = INT_MIN;                // page id placeholder: the warp has no rows in the tile
 
 template <int NR>
 struct Cfg8 {
+  static constexpr int kQParts = NR == 16 ? 4 : 2;     // QK partial accumulators (issuers 0..)
+  static constexpr int kStages = NR == 16 ? 4 : 3;     // tiles in flight
+  static constexpr int kQStage = NR * 128;             // one 64-column bf16 region of the query copy
+  static constexpr int kQOps = 2 * NR * 128;           // one 128-dim region of [Q_hi; Q_lo] (e4m3)
+  static constexpr int kPBytes = 2 * NR * 128;         // [P_hi; P_lo], 64 tokens used of 128 bytes
   static constexpr int tiles = 0;
-  static constexpr int kQRegion = NR * 128;
-  static constexpr int kQBytes = 9 * kQRegion;
-  static constexpr int kPBytes = NR * 128;
-  static constexpr int q = tiles + kSlots * kTileBytes;
-  static constexpr int p = q + kQBytes;
-  static constexpr int red = p + 2 * kPBytes;   // [4][NR] float
+  static constexpr int qstage = tiles + kStages * kTileBytes;
+  static constexpr int qops = qstage + 9 * kQStage;
+  static constexpr int p = qops + 5 * kQOps;
+  static constexpr int red = p + 2 * kPBytes;           // [4][NR] float
   static constexpr int alpha = red + 4 * NR * 4;
   static constexpr int inv = alpha + NR * 4;
   static constexpr int lse = inv + NR * 4;
-  static constexpr int qmax = lse + NR * 4;     // [4] float
-  static constexpr int mrow = qmax + 16;        // [NR] float: running maximum of every row
-  static constexpr int bars = mrow + NR * 4;
-  static constexpr int nbars = 2 * kSlots + 11;
+  static constexpr int mrow = lse + NR * 4;             // [NR] running maxima
+  static constexpr int qmax = mrow + NR * 4;            // [4] float
+  static constexpr int bars = qmax + 16;
+  static constexpr int nbars = 2 * kStages + 11;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
-  // S: 2 buffers x 4 partial accumulators (one per issuer) x NR; O^T: 4 blocks x NR
-  static constexpr int s_cols = 2 * kIssuers * NR;
-  static constexpr int tmem_cols = s_cols + 4 * NR <= 256 ? 256 : 512;
+  static constexpr int s_cols = 2 * kQParts * 2 * NR;  // 2 buffers x parts x [hi | lo]
+  static constexpr int tmem_cols = 512;                 // S + O^T (4 blocks x 2 NR) <= 512
+  static_assert(s_cols + 4 * 2 * NR <= 512, "TMEM");
 };
 
 struct M8Args {
-  const uint8_t* ckv;
-  const uint8_t* kpe;
-  int64_t cs0, cs1, ks0, ks1;                   // strides in bytes
   const int32_t* kv_indptr;
   const int32_t* kv_indices;
   const int32_t* last;
@@ -113,82 +108,57 @@ __device__ __forceinline__ MUnit8 load_unit8(const M8Args& a, const WorkItem* wo
   return x;
 }
 
-// Position in the CTA's sequence of tiles: unit u, head group hgi, tile t (units without
-// tokens are skipped; every head group streams the unit's tiles again).
-struct Cursor {
-  int u, hgi, t, T, t0, t1;
-  const int32_t* ids;
-  bool done;
-};
-
-__device__ __forceinline__ void cursor_seek(Cursor& c, const M8Args& a, const WorkItem* work, int u_end) {
-  for (; c.u < u_end; ++c.u) {
-    const MUnit8 x = load_unit8(a, work, c.u);
-    if (x.ntiles > 0) {
-      c.T = x.ntiles;
-      c.t0 = x.t0;
-      c.t1 = x.t1;
-      c.ids = a.kv_indices + a.kv_indptr[x.r];
-      return;
-    }
-  }
-  c.done = true;
+// shared-memory matrix descriptor (sm_100): layout 2 = 128-byte swizzle, 4 = 64-byte swizzle
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)layout << 61;
+  return d;
 }
-__device__ __forceinline__ void cursor_next(Cursor& c, const M8Args& a, const WorkItem* work, int u_end) {
-  if (c.done) return;
-  if (++c.t < c.T) return;
-  c.t = 0;
-  if (++c.hgi < a.hg) return;
-  c.hgi = 0;
-  ++c.u;
-  cursor_seek(c, a, work, u_end);
+__device__ __forceinline__ uint64_t sw128(uint32_t saddr) { return sdesc(saddr, 16, 1024, 2); }
+
+// D[tmem] (+)= A . B, kind::f8f6f4 (the e4m3 formats come from the instruction descriptor)
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// instruction descriptor: e4m3 A and B (format code 0), f32 D
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
-  uint32_t r;
-  const uint16_t v = (uint16_t)two_bytes;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+// two floats -> two e4m3 bytes (round to nearest even, saturating), low byte = a
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
   return r;
 }
-
-// 16 e4m3 values (bytes in memory order) -> 16 f16 in two 16-byte chunks (dims 0-7, 8-15)
-__device__ __forceinline__ void cvt16(const uint4& v, uint4& lo, uint4& hi) {
-  lo.x = e4m3x2_to_f16x2(v.x & 0xffffu);
-  lo.y = e4m3x2_to_f16x2(v.x >> 16);
-  lo.z = e4m3x2_to_f16x2(v.y & 0xffffu);
-  lo.w = e4m3x2_to_f16x2(v.y >> 16);
-  hi.x = e4m3x2_to_f16x2(v.z & 0xffffu);
-  hi.y = e4m3x2_to_f16x2(v.z >> 16);
-  hi.z = e4m3x2_to_f16x2(v.w & 0xffffu);
-  hi.w = e4m3x2_to_f16x2(v.w >> 16);
+// e4m3 byte -> float (exact)
+__device__ __forceinline__ float e4m3_val(uint32_t byte) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)byte));
+  return __half2float(__ushort_as_half((unsigned short)(h & 0xffffu)));
 }
 
-// maximum over the warp (sm_100 redux on f32)
 __device__ __forceinline__ float redux_max(float v) {
   float r;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
 }
 
-// kind::f16 instruction descriptor with f16 A and B, f32 D
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
 template <int NR, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
-mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_constant__ CUtensorMap qp_map, M8Args a,
+mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant__ CUtensorMap kpe_map,
+                  const __grid_constant__ CUtensorMap qn_map, const __grid_constant__ CUtensorMap qp_map, M8Args a,
                   const WorkItem* __restrict__ work) {
   using C = Cfg8<NR>;
+  constexpr int NS = C::kStages, NQ = C::kQParts;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = tc::smem_u32(smem);
@@ -197,9 +167,9 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::misc + 4);
   const uint32_t bar0 = sbase + C::bars;
-  auto tfull_bar = [&](int s) { return bar0 + 8u * s; };
-  auto tempty_bar = [&](int s) { return bar0 + 8u * (kSlots + s); };
-  const uint32_t bar1 = bar0 + 8u * (2 * kSlots);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (NS + s); };
+  const uint32_t bar1 = bar0 + 8u * (2 * NS);
   auto qfull_bar = [&]() { return bar1; };
   auto qready_bar = [&]() { return bar1 + 8u; };
   auto sfull_bar = [&](int b) { return bar1 + 8u * (2 + b); };
@@ -210,14 +180,14 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
   static_assert(C::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
 
   if (tid == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      tc::mbar_init(tfull_bar(s), kConvWarps);
-      tc::mbar_init(tempty_bar(s), kIssuers);
+    for (int s = 0; s < NS; ++s) {
+      tc::mbar_init(full_bar(s), 1);
+      tc::mbar_init(empty_bar(s), kIssuers);
     }
     tc::mbar_init(qfull_bar(), 1);
     tc::mbar_init(qready_bar(), 4);
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(sfull_bar(b), kIssuers);
+      tc::mbar_init(sfull_bar(b), NQ);
       tc::mbar_init(sempty_bar(b), 4);
       tc::mbar_init(pfull_bar(b), 4);
       tc::mbar_init(ofull_bar(b), kIssuers);
@@ -226,7 +196,9 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (tid == 0) {
+  if (warp == 4 && lane == 0) {
+    tc::prefetch_tmap(&ckv_map);
+    tc::prefetch_tmap(&kpe_map);
     tc::prefetch_tmap(&qn_map);
     tc::prefetch_tmap(&qp_map);
   }
@@ -238,99 +210,85 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
   const uint32_t tm_s = tmem, tm_o = tmem + C::s_cols;
 
   const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
+  const int P = a.page_size;
+  const int box_rows = min(P, kTile);
 
-  if (warp >= kFirstConv) {
-    // ======================================================================= cache conversion
-    const int cw = warp - kFirstConv;  // this warp's rows of every tile: tokens 8cw .. 8cw + 7
-    const int P = a.page_size;
+  if (warp == 4) {
+    // ======================================================================= TMA producer
+    int g = 0, n_unit = 0;
     bool ok = true;
-    Cursor cf{u_begin, 0, 0, 0, 0, 0, nullptr, false};  // the next tile to fetch
-    cursor_seek(cf, a, work, u_end);
-    // page id of this warp's 8 rows of a tile (8 | P and tiles start on page starts: one page)
-    auto load_id = [&](const Cursor& c) -> int {
-      if (c.done) return kNoRows;
-      const int tok = c.t0 + c.t * kTile + 8 * cw;
-      return tok < c.t1 ? __ldg(c.ids + tok / P) : kNoRows;
-    };
-    // issue the loads of tile cf into D (zeros for rows past the unit's end), then advance cf
-    // and start the page-id load of the tile after it
-    int idf = load_id(cf);
-    auto fetch = [&](uint4 (&D)[9]) -> bool {
-      if (cf.done) return false;
-      const int page = idf;
-      const int tok = cf.t0 + cf.t * kTile + 8 * cw;
-      const int n = page == kNoRows ? 0 : min(8, cf.t1 - tok);
-      const bool oob = n > 0 && (unsigned)page >= (unsigned)a.num_pages;
-      if (oob && lane == 0) report(a.status, SKV_DEV_PAGE_OOB);
-      const int nv = oob ? 0 : n;
-      const int slot = nv > 0 ? tok % P : 0;
-      const uint8_t* cb = a.ckv + (int64_t)(nv > 0 ? page : 0) * a.cs0 + (int64_t)slot * a.cs1 + lane * 16;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) D[j] = j < nv ? ldg_stream(cb + (int64_t)j * a.cs1) : make_uint4(0, 0, 0, 0);
-      const int jk = lane >> 2;
-      D[8] = jk < nv ? ldg_stream(a.kpe + (int64_t)page * a.ks0 + (int64_t)(slot + jk) * a.ks1 + (lane & 3) * 16)
-                     : make_uint4(0, 0, 0, 0);
-      cursor_next(cf, a, work, u_end);
-      idf = load_id(cf);
-      return true;
-    };
-    // store one tile's rows of this warp as f16 in the K-major 128-byte-swizzled layout
-    auto convert = [&](const uint4 (&D)[9], uint8_t* tile) {
-      const int b = lane >> 3, hf = (lane >> 2) & 1, ch = (lane & 3) * 2, sw = (lane >> 2) & 1;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int ti = 8 * cw + j, x = ti & 7;
-        uint4 lo, hi;
-        cvt16(D[j], lo, hi);
-        uint8_t* row = tile + b * kCSlot + hf * kHalf + ti * 128;
-        // alternate which chunk goes first between neighbouring lane quads: 4-way banks per store
-        *reinterpret_cast<uint4*>(row + (((ch + sw) ^ x) << 4)) = sw ? hi : lo;
-        *reinterpret_cast<uint4*>(row + (((ch + 1 - sw) ^ x) << 4)) = sw ? lo : hi;
-      }
-      {
-        const int ti = 8 * cw + (lane >> 2), x = ti & 7, kc = (lane & 3) * 2;
-        uint4 lo, hi;
-        cvt16(D[8], lo, hi);
-        uint8_t* row = tile + 4 * kCSlot + ti * 128;
-        *reinterpret_cast<uint4*>(row + ((kc ^ x) << 4)) = lo;
-        *reinterpret_cast<uint4*>(row + (((kc + 1) ^ x) << 4)) = hi;
-      }
-    };
-    uint4 DA[9], DB[9];
-    bool va = fetch(DA);
-    bool vb = fetch(DB);
-    int gt = 0;
-    // one step: convert the oldest fetched tile (in D), refill D with the next tile
-    auto step = [&](uint4 (&D)[9], bool& v) -> bool {
-      if (!v || !ok) return false;
-      const int slot = gt % kSlots;
-      if (gt >= kSlots) {
-        if (lane == 0) ok = tc::mbar_wait_sleep(tempty_bar(slot), ((gt / kSlots) + 1) & 1, abort_flag, a.status);
+    for (int u = u_begin; u < u_end && ok; ++u) {
+      const MUnit8 x = load_unit8(a, work, u);
+      if (x.ntiles == 0) continue;
+      const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
+      const int npages = x.page_end - x.page_begin;
+      for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+        if (lane == 0) {  // queries of this unit once the previous unit's copy has been split
+          if (n_unit >= 1) ok = tc::mbar_wait_sleep(qready_bar(), (n_unit - 1) & 1, abort_flag, a.status);
+          if (ok) {
+            const int rows = a.hc * a.q_tile;
+            tc::mbar_arrive_expect_tx(qfull_bar(), (uint32_t)(9 * rows * 128));
+            for (int rg = 0; rg < 8; ++rg)
+              tc::tma_load_3d(sbase + C::qstage + rg * C::kQStage, &qn_map, qfull_bar(), rg * 64, hgi * a.hc,
+                              x.q_start);
+            tc::tma_load_3d(sbase + C::qstage + 8 * C::kQStage, &qp_map, qfull_bar(), 0, hgi * a.hc, x.q_start);
+          }
+        }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) return false;
+        int win = -1000000, pid = 0;  // lanes hold the ids of pages [win, win + 32) of the unit
+        for (int t = 0; t < x.ntiles && ok; ++t, ++g) {
+          const int pi0 = (t * kTile) / P;
+          const int npg = P >= kTile ? 1 : min(kTile / P, npages - pi0);
+          const int slot0 = P >= kTile ? (t * kTile) % P : 0;
+          if (pi0 < win || pi0 + npg > win + 32) {
+            win = pi0;
+            pid = (win + lane < npages) ? __ldg(ids + win + lane) : 0;
+          }
+          const int st = g % NS;
+          if (lane == 0) {
+            if (g >= NS) ok = tc::mbar_wait_sleep(empty_bar(st), ((g / NS) + 1) & 1, abort_flag, a.status);
+            if (ok) tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(npg * box_rows * (4 * 128 + 64)));
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          const uint32_t tb = sbase + C::tiles + st * kTileBytes;
+          for (int i = 0; i < npg; ++i) {  // five boxes per page, issued by five lanes at once
+            const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
+            if (lane == 0 && (unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
+            if (lane < 4)
+              tc::tma_load_3d(tb + lane * kCRegion + i * box_rows * 128, &ckv_map, full_bar(st), lane * 128, slot0,
+                              page);
+            else if (lane == 4)
+              tc::tma_load_3d(tb + 4 * kCRegion + i * box_rows * 64, &kpe_map, full_bar(st), 0, slot0, page);
+          }
+        }
+        ++n_unit;
       }
-      convert(D, smem + C::tiles + slot * kTileBytes);
-      tc::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(tfull_bar(slot));
-      ++gt;
-      v = fetch(D);
-      return true;
-    };
-    while (step(DA, va) && step(DB, vb)) {
     }
-  } else if (warp >= 4) {
+    if (!ok && lane == 0) {  // drain issued copies (bounded) before the CTA can exit
+      for (int q = max(0, g - NS); q < g; ++q) {
+        const uint64_t t_start = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(full_bar(q % NS), (q / NS) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
+        }
+      }
+      if (n_unit >= 1) {
+        const uint64_t t_start = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(qfull_bar(), (n_unit - 1) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
+        }
+      }
+    }
+  } else if (warp >= 5) {
     // ======================================================================= MMA issuers
-    // Issuer w: QK quarter w of every tile (rope k-step w + ckv block w: 9 MMAs) into its own
-    // partial S^T accumulator, and PV block w (4 MMAs) into O^T block w.  Per tile the order is
-    // QK(t) then PV(t - 1), so S(t) is in flight while the softmax finishes P(t - 1).
+    // Issuer w: PV block w (two k-steps of 32 tokens) and, for w < NQ, QK part w (its share of the
+    // 16 ckv k-steps; parts 0 and 1 also take rope k-steps 0 and 1).  PV first when both are ready.
     if (lane == 0) {
-      const int w = warp - 4;
-      constexpr uint32_t idesc_s = idesc_f16_f32(64, NR, false, false);
-      constexpr uint32_t idesc_o = idesc_f16_f32(128, NR, true, false);
-      int gt = 0, n_unit = 0, n_tile = 0;
+      const int w = warp - 5;
+      constexpr uint32_t idesc_s = idesc_e4m3(64, 2 * NR, false);
+      constexpr uint32_t idesc_o = idesc_e4m3(128, 2 * NR, true);
+      constexpr int kRegionsPerPart = 4 / NQ;
+      int g = 0, n_unit = 0, n_tile = 0;
       bool ok = true;
-      const uint32_t qs = sbase + C::q;
+      const uint32_t qo = sbase + C::qops;
       for (int u = u_begin; u < u_end && ok; ++u) {
         const MUnit8 x = load_unit8(a, work, u);
         if (x.ntiles == 0) continue;
@@ -338,47 +296,45 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
           const int T = x.ntiles;
           ok = tc::mbar_wait_sleep(qready_bar(), n_unit & 1, abort_flag, a.status);
           if (ok) tc::tc_fence_after();
-          // issue whichever is ready: PV(pv) (frees the tile slot: first) or QK(qk)
-          int qk = 0, pv = 0;
+          int qk = w < NQ ? 0 : T, pv = 0;  // issuers without a QK part only run PV
           tc::PollClock clk;
           while (ok && pv < T) {
             bool did = false;
-            if (pv < qk) {  // ---- PV(pv), block w
-              const int tp = n_tile + pv, pb = tp & 1, g = gt + pv, slot = g % kSlots;
-              // the single O^T buffer was read by the previous unit's epilogue
-              if (tc::mbar_test_wait(pfull_bar(pb), (tp >> 1) & 1) &&
+            {  // ---- PV(pv), block w: needs P(pv), which implies every QK part of the tile is done
+              const int tp = n_tile + pv, pb = tp & 1, gg = g + pv, st = gg % NS;
+              if (pv < T && tc::mbar_test_wait(pfull_bar(pb), (tp >> 1) & 1) &&
                   (pv > 0 || n_unit == 0 || tc::mbar_test_wait(ofree_bar(), (n_unit + 1) & 1))) {
                 tc::tc_fence_after();
+                const uint32_t vs = sbase + C::tiles + st * kTileBytes + w * kCRegion;
                 const uint32_t ps = sbase + C::p + pb * C::kPBytes;
-                const uint32_t vs = sbase + C::tiles + slot * kTileBytes + w * kCSlot;
 #pragma unroll
-                for (int k = 0; k < kTile / 16; ++k) {
-                  const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
-                  const uint64_t bd = tc::sdesc_sw128(ps + k * 32, 16, 1024);
-                  tc::mma_bf16(tm_o + w * NR, ad, bd, idesc_o, (pv > 0 || k > 0) ? 1u : 0u);
-                }
-                tc::mma_commit(tempty_bar(slot));
+                for (int k = 0; k < 2; ++k)
+                  mma_f8(tm_o + w * 2 * NR, sdesc(vs + k * 4096, 8192, 1024, 2), sw128(ps + k * 32), idesc_o,
+                         (pv > 0 || k > 0) ? 1u : 0u);
+                tc::mma_commit(empty_bar(st));
                 tc::mma_commit(ofull_bar(pb));
                 ++pv;
                 did = true;
               }
             }
-            if (!did && qk < T) {  // ---- QK(qk), quarter w
-              const int tt = n_tile + qk, sb = tt & 1, g = gt + qk, slot = g % kSlots;
+            if (!did && qk < T) {  // ---- QK(qk), part w
+              const int tt = n_tile + qk, sb = tt & 1, gg = g + qk, st = gg % NS;
               if ((tt < 2 || tc::mbar_test_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1)) &&
-                  tc::mbar_test_wait(tfull_bar(slot), (g / kSlots) & 1)) {
+                  tc::mbar_test_wait(full_bar(st), (gg / NS) & 1)) {
                 tc::tc_fence_after();
-                const uint32_t tb = sbase + C::tiles + slot * kTileBytes;
-                const uint32_t d = tm_s + (sb * kIssuers + w) * NR;
-                tc::mma_bf16(d, tc::sdesc_sw128(tb + 4 * kCSlot + w * 32, 16, 1024),
-                             tc::sdesc_sw128(qs + 8 * C::kQRegion + w * 32, 16, 1024), idesc_s, 0u);
+                const uint32_t tb = sbase + C::tiles + st * kTileBytes;
+                const uint32_t d = tm_s + (sb * NQ + w) * 2 * NR;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  const uint64_t ad = tc::sdesc_sw128(tb + w * kCSlot + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
-                  const uint64_t bd =
-                      tc::sdesc_sw128(qs + (2 * w + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
-                  tc::mma_bf16(d, ad, bd, idesc_s, 1u);
+                for (int rr = 0; rr < kRegionsPerPart; ++rr) {
+                  const int r = w * kRegionsPerPart + rr;
+#pragma unroll
+                  for (int k = 0; k < 4; ++k)
+                    mma_f8(d, sw128(tb + r * kCRegion + k * 32), sw128(qo + r * C::kQOps + k * 32), idesc_s,
+                           (rr > 0 || k > 0) ? 1u : 0u);
                 }
+                if (w < 2)  // rope k-step w (64-byte swizzled rows)
+                  mma_f8(d, sdesc(tb + 4 * kCRegion + w * 32, 16, 512, 4), sw128(qo + 4 * C::kQOps + w * 32),
+                         idesc_s, 1u);
                 tc::mma_commit(sfull_bar(sb));
                 ++qk;
                 did = true;
@@ -386,7 +342,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
             }
             ok = clk.step(did, abort_flag, a.status);
           }
-          gt += T;
+          g += T;
           n_tile += T;
           ++n_unit;
         }
@@ -398,14 +354,12 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
     float* alpha_s = reinterpret_cast<float*>(smem + C::alpha);
     float* inv_s = reinterpret_cast<float*>(smem + C::inv);
     float* lse_s = reinterpret_cast<float*>(smem + C::lse);
+    float* m_s = reinterpret_cast<float*>(smem + C::mrow);  // the same in every thread
     float* qmax_s = reinterpret_cast<float*>(smem + C::qmax);
-    // the running maxima are the same in every thread: they live in shared memory (registers
-    // are scarce with 480 threads)
-    float* m_s = reinterpret_cast<float*>(smem + C::mrow);
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const bool srow = lane < 16;              // this lane holds an S^T row (M = 64 layout)
     const int tok_in_tile = 16 * warp + (lane & 15);
-    int n_unit = 0, n_tile = 0, pv_seen = 0, q_issued = 0, q_landed = 0;
+    int g = 0, n_unit = 0, n_tile = 0, pv_seen = 0;
     bool ok = true;
     auto consume_pv = [&](int upto) {
       for (; pv_seen <= upto; ++pv_seen)
@@ -436,54 +390,58 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
           }
           continue;
         }
-        // ---- queries of this unit: bf16 (TMA) -> f16 in place, shifted by 2^-k.  The buffer is
-        // free: every QK of the previous unit completed before its last S was consumed here.
-        const int qrows = a.hc * a.q_tile;     // rows the query copy fills
-        if (tid == 0) {
-          tc::mbar_arrive_expect_tx(qfull_bar(), (uint32_t)(9 * qrows * 128));
-          for (int rg = 0; rg < 8; ++rg)
-            tc::tma_load_3d(sbase + C::q + rg * C::kQRegion, &qn_map, qfull_bar(), rg * 64, h0, x.q_start);
-          tc::tma_load_3d(sbase + C::q + 8 * C::kQRegion, &qp_map, qfull_bar(), 0, h0, x.q_start);
-        }
-        q_issued = n_unit + 1;
+        // ---- queries: bf16 copy -> [Q_hi; Q_lo] e4m3 terms of q * 2^e, 2^e putting max |q| in [128, 256)
         ok = tc::mbar_wait_sleep(qfull_bar(), n_unit & 1, abort_flag, a.status) && ok;
-        if (ok) q_landed = n_unit + 1;
-        constexpr int kChunks = 9 * NR * 8;     // 16-byte chunks of the query block
+        const int qrows = a.hc * a.q_tile;     // rows the query copy filled
         float qm = 0.f;
-        for (int ci = tid; ci < kChunks; ci += 128) {
+        for (int ci = tid; ci < 9 * NR * 8; ci += 128) {
           if ((ci % (NR * 8)) / 8 >= qrows) continue;
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + C::q + ci * 16);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + C::qstage + ci * 16);
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            qm = fmaxf(qm, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xffff0000u))));
+            qm = fmaxf(qm, fmaxf(fabsf(__uint_as_float(wv[i] << 16)), fabsf(__uint_as_float(wv[i] & 0xffff0000u))));
         }
         qm = warp_max(qm);
         if (lane == 0) qmax_s[warp] = qm;
         if (tid < NR) m_s[tid] = -INFINITY;
         tc::named_bar_sync(1, 128);
         qm = fmaxf(fmaxf(qmax_s[0], qmax_s[1]), fmaxf(qmax_s[2], qmax_s[3]));
-        int k_shift = 0;
-        if (qm >= 32768.f) k_shift = (qm == qm && qm < INFINITY) ? min(ilogbf(qm) - 14, 200) : 200;
-        const float qs_mul = ldexpf(1.f, -k_shift);
-        for (int ci = tid; ci < kChunks; ci += 128) {
-          if ((ci % (NR * 8)) / 8 >= qrows) continue;
-          uint4* pv = reinterpret_cast<uint4*>(smem + C::q + ci * 16);
-          const uint4 v = *pv;
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o4[4];
+        const int e = (qm > 0.f && qm < INFINITY) ? 7 - ilogbf(qm) : 0;
+        const float qmul = ldexpf(1.f, e);
+        // staging chunk ci: region rg (64 dims), row n, 16-byte chunk c (8 dims); it becomes 8
+        // bytes of Q_hi (row n) and of Q_lo (row NR + n); rows past the copy are zeros
+        for (int ci = tid; ci < 9 * NR * 8; ci += 128) {
+          const int rg = ci / (NR * 8), n = (ci % (NR * 8)) / 8, c = ci % 8;
+          uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
+          if (n < qrows) {
+            const int cs = (c ^ (n & 7)) & 7;  // the copy is 128-byte swizzled
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + C::qstage + rg * C::kQStage + n * 128 + cs * 16);
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __half2 h2 = __floats2half2_rn(__uint_as_float(w[i] << 16) * qs_mul,
-                                           __uint_as_float(w[i] & 0xffff0000u) * qs_mul);
-            o4[i] = *reinterpret_cast<uint32_t*>(&h2);
+            for (int i = 0; i < 4; ++i) {
+              const float x0 = __uint_as_float(wv[i] << 16) * qmul;
+              const float x1 = __uint_as_float(wv[i] & 0xffff0000u) * qmul;
+              const uint32_t h2 = e4m3x2(x0, x1);
+              const uint32_t l2 = e4m3x2(x0 - e4m3_val(h2 & 0xff), x1 - e4m3_val(h2 >> 8));
+              hi[i >> 1] |= h2 << (16 * (i & 1));
+              lo[i >> 1] |= l2 << (16 * (i & 1));
+            }
           }
-          *pv = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          // dims d0 .. d0 + 7: region d0 / 128 (region 4 = rope), byte b0 within the 128-byte row
+          const int d0 = rg < 8 ? rg * 64 + c * 8 : 512 + c * 8;
+          const int r = d0 >> 7, b0 = d0 & 127;
+          const int rh = n, rl = NR + n;
+          uint8_t* base = smem + C::qops + r * C::kQOps;
+          *reinterpret_cast<uint2*>(base + rh * 128 + ((((b0 >> 4) ^ (rh & 7)) & 7) << 4) + (b0 & 15)) =
+              make_uint2(hi[0], hi[1]);
+          *reinterpret_cast<uint2*>(base + rl * 128 + ((((b0 >> 4) ^ (rl & 7)) & 7) << 4) + (b0 & 15)) =
+              make_uint2(lo[0], lo[1]);
         }
         tc::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(qready_bar());
-        const float sl2 = ldexpf(a.scale_log2, k_shift);
+        const float sl2 = ldexpf(a.scale_log2, -e);
 
         const int T = x.ntiles;
         float l[NR];
@@ -491,23 +449,23 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
         for (int n = 0; n < NR; ++n) l[n] = 0.f;
         bool failed = false;
         for (int t = 0; t < T; ++t) {
-          const int tt = n_tile + t, sb = tt & 1;
+          const int tt = n_tile + t, sb = tt & 1, gg = g + t, st = gg % NS;
           ok = tc::mbar_wait_sleep(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
           tc::tc_fence_after();
           float s[NR];
 #pragma unroll
-          for (int w = 0; w < kIssuers; ++w) {  // sum of the four partial accumulators
-            float v[NR];
+          for (int pp = 0; pp < NQ; ++pp) {  // partial accumulators, hi + lo columns
+            float v[2 * NR];
 #pragma unroll
-            for (int c = 0; c < NR; c += 16) {
+            for (int c = 0; c < 2 * NR; c += 16) {
               float v16[16];
-              tc::tmem_ld_x16(tm_s + lane_base + (sb * kIssuers + w) * NR + c, v16);
+              tc::tmem_ld_x16(tm_s + lane_base + (sb * NQ + pp) * 2 * NR + c, v16);
 #pragma unroll
               for (int i = 0; i < 16; ++i) v[c + i] = v16[i];
             }
             tc::tmem_wait_ld();  // registers of a TMEM load are read only after the wait
 #pragma unroll
-            for (int n = 0; n < NR; ++n) s[n] = w == 0 ? v[n] : s[n] + v[n];
+            for (int n = 0; n < NR; ++n) s[n] = pp == 0 ? v[n] + v[NR + n] : s[n] + (v[n] + v[NR + n]);
           }
           tc::tc_fence_before();
           __syncwarp();
@@ -540,21 +498,21 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
             tc::named_bar_sync(1, 128);
 #pragma unroll
             for (int n = 0; n < NR; ++n) l[n] *= alpha_s[n];
-            if (t > 0) {  // rescale O^T in TMEM (every thread owns lane `tid` of the 4 blocks)
+            if (t > 0) {  // rescale O^T (hi and lo columns) in TMEM; thread tid owns lane tid of each block
               consume_pv(tt - 1);
 #pragma unroll 1
-              for (int c = 0; c < NR; c += 16) {  // 16 columns at a time: few registers held
+              for (int c = 0; c < 2 * NR; c += 16) {
                 float al[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) al[i] = alpha_s[c + i];
+                for (int i = 0; i < 16; ++i) al[i] = alpha_s[(c + i) % NR];
 #pragma unroll 1
                 for (int b = 0; b < kBlocks; ++b) {
                   float ov[16];
-                  tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, ov);
+                  tc::tmem_ld_x16(tm_o + lane_base + b * 2 * NR + c, ov);
                   tc::tmem_wait_ld();
 #pragma unroll
                   for (int i = 0; i < 16; ++i) ov[i] *= al[i];
-                  tc::tmem_st_x16(tm_o + lane_base + b * NR + c, ov);
+                  tc::tmem_st_x16(tm_o + lane_base + b * 2 * NR + c, ov);
                 }
               }
               tc::tmem_wait_st();
@@ -562,17 +520,36 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
             }
             tc::named_bar_sync(1, 128);  // red / alpha_s reads done before any later rewrite
           }
+          if (srow && !valid) {  // zero this token's V row in the tile (the copy landed before QK)
+            ok = tc::mbar_wait_sleep(full_bar(st), (gg / NS) & 1, abort_flag, a.status) && ok;
+            uint8_t* row = smem + C::tiles + st * kTileBytes + tok_in_tile * 128;
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) reinterpret_cast<uint4*>(row + b * kCRegion)[i] = make_uint4(0, 0, 0, 0);
+          }
           if (tt >= 2 && pv_seen <= tt - 2) consume_pv(tt - 2);  // P(t) reuses PV(t-2)'s buffer
           if (srow) {
-            uint8_t* pb = smem + C::p + (tt & 1) * C::kPBytes;
+            uint8_t* pbuf = smem + C::p + (tt & 1) * C::kPBytes;
             float mloc[NR];  // read the maxima before the stores below (they may alias for the compiler)
 #pragma unroll
             for (int n = 0; n < NR; ++n) mloc[n] = m_s[n];
+            const int tk = tok_in_tile;
 #pragma unroll
-            for (int n = 0; n < NR; ++n) {
-              const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - mloc[n]);
-              l[n] += p;
-              if (n < rows) *reinterpret_cast<__half*>(pb + tc::sw128_offset(n, tok_in_tile)) = __float2half_rn(p);
+            for (int n = 0; n < NR; n += 2) {
+              const float p0 = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - mloc[n]);
+              const float p1 = (s[n + 1] == -INFINITY) ? 0.f : exp2f(s[n + 1] - mloc[n + 1]);
+              l[n] += p0;
+              l[n + 1] += p1;
+              if (n < rows) {  // rows n, n + 1 of P_hi and of P_lo, column tk (byte stores)
+                const uint32_t h2 = e4m3x2(p0, p1);
+                const uint32_t l2 = e4m3x2(p0 - e4m3_val(h2 & 0xff), p1 - e4m3_val(h2 >> 8));
+                const int r0 = n, r1 = n + 1, q0 = NR + n, q1 = NR + n + 1;
+                pbuf[r0 * 128 + ((((tk >> 4) ^ (r0 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(h2 & 0xff);
+                pbuf[r1 * 128 + ((((tk >> 4) ^ (r1 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(h2 >> 8);
+                pbuf[q0 * 128 + ((((tk >> 4) ^ (q0 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(l2 & 0xff);
+                pbuf[q1 * 128 + ((((tk >> 4) ^ (q1 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(l2 >> 8);
+              }
             }
           }
           tc::fence_proxy_async_smem();
@@ -583,6 +560,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
           ok = false;
           break;
         }
+        g += T;
         n_tile += T;
         ++n_unit;
         consume_pv(n_tile - 1);
@@ -596,27 +574,31 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
           ok = false;
           break;
         }
-        if (tid == 0) {
-#pragma unroll
-          for (int n = 0; n < NR; ++n) {
-            const float lt = red[n] + red[NR + n] + red[2 * NR + n] + red[3 * NR + n];
-            inv_s[n] = lt > 0.f ? a.kv_scale / lt : 0.f;
-            lse_s[n] = lt > 0.f ? (m_s[n] + log2f(lt)) * kLn2 : -INFINITY;
-          }
+        if (tid < NR) {
+          const int n = tid;
+          const float lt = red[n] + red[NR + n] + red[2 * NR + n] + red[3 * NR + n];
+          inv_s[n] = lt > 0.f ? a.kv_scale / lt : 0.f;
+          lse_s[n] = lt > 0.f ? (m_s[n] + log2f(lt)) * kLn2 : -INFINITY;
         }
         tc::named_bar_sync(1, 128);
-        // O^T block by block: thread tid holds head dim b * 128 + tid of every row
+        // O^T block by block: thread tid holds head dim b * 128 + tid of every row (hi + lo)
 #pragma unroll 1
         for (int b = 0; b < kBlocks; ++b) {
           float ov[NR];
 #pragma unroll
-          for (int c = 0; c < NR; c += 16) {
-            float v16[16];
-            tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, v16);
+          for (int hl = 0; hl < 2; ++hl) {
+            float vv[NR];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) ov[c + i] = v16[i];
+            for (int c = 0; c < NR; c += 16) {
+              float v16[16];
+              tc::tmem_ld_x16(tm_o + lane_base + b * 2 * NR + hl * NR + c, v16);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) vv[c + i] = v16[i];
+            }
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int n = 0; n < NR; ++n) ov[n] = hl == 0 ? vv[n] : ov[n] + vv[n];
           }
-          tc::tmem_wait_ld();
 #pragma unroll
           for (int n = 0; n < NR; ++n) {
             if (n >= rows) break;
@@ -643,11 +625,6 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap qn_map, const __grid_const
         tc::named_bar_sync(1, 128);  // inv_s / lse_s / red reads done before the next unit
       }
     }
-    if (tid == 0 && q_issued > q_landed) {  // a query copy may still be landing (bounded wait)
-      const uint64_t t_start = tc::globaltimer_ns();
-      while (!tc::mbar_try_wait(qfull_bar(), (q_issued - 1) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
-      }
-    }
   }
 
   tc::tc_fence_before();
@@ -672,14 +649,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_m8() {
   return fn;
 }
 
-bool make_qmap(CUtensorMap* m, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
-               const cuuint32_t* box) {
+bool make_map8(CUtensorMap* m, CUtensorMapDataType type, CUtensorMapSwizzle swz, const void* base,
+               const cuuint64_t* dims, const cuuint64_t* strides_bytes, const cuuint32_t* box) {
   auto fn = encode_fn_m8();
   if (fn == nullptr) return false;
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides_bytes, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, type, 3, const_cast<void*>(base), dims, strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int NR, typename OutT>
@@ -692,14 +668,15 @@ int launch_m8(const CUtensorMap* maps, const M8Args& a, int num_ctas, const Work
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  mla_tc_fp8_kernel<NR, OutT><<<num_ctas, kThreads, smem, s>>>(maps[0], maps[1], a, work);
+  mla_tc_fp8_kernel<NR, OutT><<<num_ctas, kThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a, work);
   return (int)cudaGetLastError();
 }
 
 }  // namespace
 
 bool mla_tc_fp8_supported(int page_size, int num_heads, int rows_per_unit) {
-  return page_size >= 8 && page_size % 8 == 0 && (rows_per_unit == 16 || rows_per_unit == 32) &&
+  const bool page_ok = page_size >= 8 && (page_size <= kTile ? kTile % page_size == 0 : page_size % kTile == 0);
+  return page_ok && (rows_per_unit == 16 || rows_per_unit == 32) &&
          (num_heads <= rows_per_unit || num_heads % rows_per_unit == 0);
 }
 
@@ -712,26 +689,37 @@ int launch_mla_tc_fp8(const skv_mla_params& p, const WorkItem* work, const int32
   const int hc = std::min(p.num_heads, NR);
   if (hc * q_tile > NR) return (int)cudaErrorInvalidValue;
   const int total_q = p.batch * p.q_len;
-  CUtensorMap maps[2];
+  const int box_rows = std::min(p.page_size, kTile);
+  CUtensorMap maps[4];
+  {
+    const cuuint64_t dims[3] = {512, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t st[2] = {(cuuint64_t)p.ckv_stride[1], (cuuint64_t)p.ckv_stride[0]};
+    const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+    if (!make_map8(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B, p.ckv, dims, st, box))
+      return (int)cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t st[2] = {(cuuint64_t)p.kpe_stride[1], (cuuint64_t)p.kpe_stride[0]};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    if (!make_map8(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_64B, p.kpe, dims, st, box))
+      return (int)cudaErrorInvalidValue;
+  }
   {
     const cuuint64_t dims[3] = {512, (cuuint64_t)p.num_heads, (cuuint64_t)std::max(1, total_q)};
     const cuuint64_t st[2] = {512 * 2, (cuuint64_t)p.num_heads * 512 * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)hc, (cuuint32_t)q_tile};
-    if (!make_qmap(&maps[0], p.q_nope, dims, st, box)) return (int)cudaErrorInvalidValue;
+    if (!make_map8(&maps[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, p.q_nope, dims, st, box))
+      return (int)cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[3] = {64, (cuuint64_t)p.num_heads, (cuuint64_t)std::max(1, total_q)};
     const cuuint64_t st[2] = {64 * 2, (cuuint64_t)p.num_heads * 64 * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)hc, (cuuint32_t)q_tile};
-    if (!make_qmap(&maps[1], p.q_pe, dims, st, box)) return (int)cudaErrorInvalidValue;
+    if (!make_map8(&maps[3], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, p.q_pe, dims, st, box))
+      return (int)cudaErrorInvalidValue;
   }
   M8Args a;
-  a.ckv = static_cast<const uint8_t*>(p.ckv);
-  a.kpe = static_cast<const uint8_t*>(p.kpe);
-  a.cs0 = p.ckv_stride[0];
-  a.cs1 = p.ckv_stride[1];
-  a.ks0 = p.kpe_stride[0];
-  a.ks1 = p.kpe_stride[1];
   a.kv_indptr = p.kv_indptr;
   a.kv_indices = p.kv_indices;
   a.last = p.kv_last_page_len;
