@@ -51,19 +51,20 @@ struct Cfg8 {
   static constexpr int kStages = NR == 16 ? 4 : 3;     // tiles in flight
   static constexpr int kQStage = NR * 128;             // one 64-column bf16 region of the query copy
   static constexpr int kQOps = 2 * NR * 128;           // one 128-dim region of [Q_hi; Q_lo] (e4m3)
-  static constexpr int kPBytes = 2 * NR * 128;         // [P_hi; P_lo], 64 tokens used of 128 bytes
+  static constexpr int kPBytes = kTile * 128;          // P^T MN-major: token rows of [P_hi | P_lo] bytes
   static constexpr int tiles = 0;
   static constexpr int qstage = tiles + kStages * kTileBytes;
   static constexpr int qops = qstage + 9 * kQStage;
   static constexpr int p = qops + 5 * kQOps;
-  static constexpr int red = p + 2 * kPBytes;           // [4][NR] float
+  static constexpr int kPBufs = 3;                      // P(t) reuses the buffer of PV(t - 3)
+  static constexpr int red = p + kPBufs * kPBytes;      // [4][NR] float
   static constexpr int alpha = red + 4 * NR * 4;
   static constexpr int inv = alpha + NR * 4;
   static constexpr int lse = inv + NR * 4;
   static constexpr int mrow = lse + NR * 4;             // [NR] running maxima
   static constexpr int qmax = mrow + NR * 4;            // [4] float
   static constexpr int bars = qmax + 16;
-  static constexpr int nbars = 2 * kStages + 11;
+  static constexpr int nbars = 2 * kStages + 14;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
   static constexpr int s_cols = 2 * kQParts * 2 * NR;  // 2 buffers x parts x [hi | lo]
@@ -139,11 +140,22 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
   return r;
 }
-// e4m3 byte -> float (exact)
-__device__ __forceinline__ float e4m3_val(uint32_t byte) {
+// two e4m3 bytes (low byte first) -> the two floats (exact)
+__device__ __forceinline__ float2 e4m3x2_val(uint32_t two) {
   uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)byte));
-  return __half2float(__ushort_as_half((unsigned short)(h & 0xffffu)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)two));
+  return __half22float2(*reinterpret_cast<__half2*>(&h));
+}
+// [hi | lo] e4m3 split of two floats: hi = rn(x), lo = rn(x - hi), as two packed byte pairs
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = e4m3x2(x0, x1);
+  const float2 hv = e4m3x2_val(hi);
+  lo = e4m3x2(x0 - hv.x, x1 - hv.y);
+}
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 __device__ __forceinline__ float redux_max(float v) {
@@ -174,9 +186,9 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
   auto qready_bar = [&]() { return bar1 + 8u; };
   auto sfull_bar = [&](int b) { return bar1 + 8u * (2 + b); };
   auto sempty_bar = [&](int b) { return bar1 + 8u * (4 + b); };
-  auto pfull_bar = [&](int b) { return bar1 + 8u * (6 + b); };
-  auto ofull_bar = [&](int b) { return bar1 + 8u * (8 + b); };
-  auto ofree_bar = [&]() { return bar1 + 8u * 10; };
+  auto pfull_bar = [&](int b) { return bar1 + 8u * (6 + b); };   // one per P buffer
+  auto ofull_bar = [&](int b) { return bar1 + 8u * (9 + b); };   // four: PV(t) on t & 3
+  auto ofree_bar = [&]() { return bar1 + 8u * 13; };
   static_assert(C::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
 
   if (tid == 0) {
@@ -189,9 +201,9 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(sfull_bar(b), NQ);
       tc::mbar_init(sempty_bar(b), 4);
-      tc::mbar_init(pfull_bar(b), 4);
-      tc::mbar_init(ofull_bar(b), kIssuers);
     }
+    for (int b = 0; b < C::kPBufs; ++b) tc::mbar_init(pfull_bar(b), 4);
+    for (int b = 0; b < 4; ++b) tc::mbar_init(ofull_bar(b), kIssuers);
     tc::mbar_init(ofree_bar(), 4);
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -284,7 +296,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
     if (lane == 0) {
       const int w = warp - 5;
       constexpr uint32_t idesc_s = idesc_e4m3(64, 2 * NR, false);
-      constexpr uint32_t idesc_o = idesc_e4m3(128, 2 * NR, true);
+      constexpr uint32_t idesc_o = idesc_e4m3(128, 2 * NR, true) | (1u << 16);  // P^T MN-major too
       constexpr int kRegionsPerPart = 4 / NQ;
       int g = 0, n_unit = 0, n_tile = 0;
       bool ok = true;
@@ -301,18 +313,18 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
           while (ok && pv < T) {
             bool did = false;
             {  // ---- PV(pv), block w: needs P(pv), which implies every QK part of the tile is done
-              const int tp = n_tile + pv, pb = tp & 1, gg = g + pv, st = gg % NS;
-              if (pv < T && tc::mbar_test_wait(pfull_bar(pb), (tp >> 1) & 1) &&
+              const int tp = n_tile + pv, pb = tp % C::kPBufs, gg = g + pv, st = gg % NS;
+              if (pv < T && tc::mbar_test_wait(pfull_bar(pb), (tp / C::kPBufs) & 1) &&
                   (pv > 0 || n_unit == 0 || tc::mbar_test_wait(ofree_bar(), (n_unit + 1) & 1))) {
                 tc::tc_fence_after();
                 const uint32_t vs = sbase + C::tiles + st * kTileBytes + w * kCRegion;
                 const uint32_t ps = sbase + C::p + pb * C::kPBytes;
 #pragma unroll
                 for (int k = 0; k < 2; ++k)
-                  mma_f8(tm_o + w * 2 * NR, sdesc(vs + k * 4096, 8192, 1024, 2), sw128(ps + k * 32), idesc_o,
-                         (pv > 0 || k > 0) ? 1u : 0u);
+                  mma_f8(tm_o + w * 2 * NR, sdesc(vs + k * 4096, 8192, 1024, 2), sdesc(ps + k * 4096, 8192, 1024, 2),
+                         idesc_o, (pv > 0 || k > 0) ? 1u : 0u);
                 tc::mma_commit(empty_bar(st));
-                tc::mma_commit(ofull_bar(pb));
+                tc::mma_commit(ofull_bar(tp & 3));
                 ++pv;
                 did = true;
               }
@@ -363,7 +375,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
     bool ok = true;
     auto consume_pv = [&](int upto) {
       for (; pv_seen <= upto; ++pv_seen)
-        ok = tc::mbar_wait_sleep(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
+        ok = tc::mbar_wait_sleep(ofull_bar(pv_seen & 3), (pv_seen >> 2) & 1, abort_flag, a.status) && ok;
       tc::tc_fence_after();
     };
     for (int u = u_begin; u < u_end && ok; ++u) {
@@ -422,8 +434,8 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
             for (int i = 0; i < 4; ++i) {
               const float x0 = __uint_as_float(wv[i] << 16) * qmul;
               const float x1 = __uint_as_float(wv[i] & 0xffff0000u) * qmul;
-              const uint32_t h2 = e4m3x2(x0, x1);
-              const uint32_t l2 = e4m3x2(x0 - e4m3_val(h2 & 0xff), x1 - e4m3_val(h2 >> 8));
+              uint32_t h2, l2;
+              split2(x0, x1, h2, l2);
               hi[i >> 1] |= h2 << (16 * (i & 1));
               lo[i >> 1] |= l2 << (16 * (i & 1));
             }
@@ -444,28 +456,38 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
         const float sl2 = ldexpf(a.scale_log2, -e);
 
         const int T = x.ntiles;
-        float l[NR];
+        // P phase: lanes 0-15 take rows [0, NR/2) of their token, lanes 16-31 rows [NR/2, NR) of the
+        // token of lane - 16; l[j] is the partial sum of row half * NR/2 + j
+        constexpr int NH = NR / 2;
+        const int half = lane >> 4;
+        float l[NH];
 #pragma unroll
-        for (int n = 0; n < NR; ++n) l[n] = 0.f;
+        for (int j = 0; j < NH; ++j) l[j] = 0.f;
         bool failed = false;
         for (int t = 0; t < T; ++t) {
           const int tt = n_tile + t, sb = tt & 1, gg = g + t, st = gg % NS;
           ok = tc::mbar_wait_sleep(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
           tc::tc_fence_after();
           float s[NR];
+          constexpr int kGrp = NR == 16 ? 2 : 1;  // partial accumulators loaded per TMEM wait
 #pragma unroll
-          for (int pp = 0; pp < NQ; ++pp) {  // partial accumulators, hi + lo columns
-            float v[2 * NR];
+          for (int pp = 0; pp < NQ; pp += kGrp) {  // partial accumulators, hi + lo columns
+            float v[kGrp][2 * NR];
 #pragma unroll
-            for (int c = 0; c < 2 * NR; c += 16) {
-              float v16[16];
-              tc::tmem_ld_x16(tm_s + lane_base + (sb * NQ + pp) * 2 * NR + c, v16);
+            for (int q = 0; q < kGrp; ++q)
 #pragma unroll
-              for (int i = 0; i < 16; ++i) v[c + i] = v16[i];
-            }
+              for (int c = 0; c < 2 * NR; c += 16) {
+                float v16[16];
+                tc::tmem_ld_x16(tm_s + lane_base + (sb * NQ + pp + q) * 2 * NR + c, v16);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[q][c + i] = v16[i];
+              }
             tc::tmem_wait_ld();  // registers of a TMEM load are read only after the wait
 #pragma unroll
-            for (int n = 0; n < NR; ++n) s[n] = pp == 0 ? v[n] + v[NR + n] : s[n] + (v[n] + v[NR + n]);
+            for (int q = 0; q < kGrp; ++q)
+#pragma unroll
+              for (int n = 0; n < NR; ++n)
+                s[n] = (pp == 0 && q == 0) ? v[q][n] + v[q][NR + n] : s[n] + (v[q][n] + v[q][NR + n]);
           }
           tc::tc_fence_before();
           __syncwarp();
@@ -497,7 +519,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
             }
             tc::named_bar_sync(1, 128);
 #pragma unroll
-            for (int n = 0; n < NR; ++n) l[n] *= alpha_s[n];
+            for (int j = 0; j < NH; ++j) l[j] *= alpha_s[half * NH + j];
             if (t > 0) {  // rescale O^T (hi and lo columns) in TMEM; thread tid owns lane tid of each block
               consume_pv(tt - 1);
 #pragma unroll 1
@@ -528,33 +550,48 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
 #pragma unroll
               for (int i = 0; i < 8; ++i) reinterpret_cast<uint4*>(row + b * kCRegion)[i] = make_uint4(0, 0, 0, 0);
           }
-          if (tt >= 2 && pv_seen <= tt - 2) consume_pv(tt - 2);  // P(t) reuses PV(t-2)'s buffer
-          if (srow) {
-            uint8_t* pbuf = smem + C::p + (tt & 1) * C::kPBytes;
-            float mloc[NR];  // read the maxima before the stores below (they may alias for the compiler)
+          if (tt >= C::kPBufs && pv_seen <= tt - C::kPBufs) consume_pv(tt - C::kPBufs);  // P(t)'s buffer was PV's
+          {
+            float sv[NH], mloc[NH];
 #pragma unroll
-            for (int n = 0; n < NR; ++n) mloc[n] = m_s[n];
-            const int tk = tok_in_tile;
+            for (int jj = 0; jj < NH; ++jj) {  // upper rows move from lane l to lane l + 16
+              const float up = __shfl_sync(0xffffffffu, s[NH + jj], lane & 15);
+              sv[jj] = half ? up : s[jj];
+              mloc[jj] = m_s[half * NH + jj];
+            }
+            // token row of P^T (MN-major, 128-byte swizzle): bytes [0, NR) = P_hi, [NR, 2 NR) = P_lo
+            uint8_t* prow = smem + C::p + (tt % C::kPBufs) * C::kPBytes + tok_in_tile * 128;
+            uint32_t hw[NH / 4], lw[NH / 4];
 #pragma unroll
-            for (int n = 0; n < NR; n += 2) {
-              const float p0 = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - mloc[n]);
-              const float p1 = (s[n + 1] == -INFINITY) ? 0.f : exp2f(s[n + 1] - mloc[n + 1]);
-              l[n] += p0;
-              l[n + 1] += p1;
-              if (n < rows) {  // rows n, n + 1 of P_hi and of P_lo, column tk (byte stores)
-                const uint32_t h2 = e4m3x2(p0, p1);
-                const uint32_t l2 = e4m3x2(p0 - e4m3_val(h2 & 0xff), p1 - e4m3_val(h2 >> 8));
-                const int r0 = n, r1 = n + 1, q0 = NR + n, q1 = NR + n + 1;
-                pbuf[r0 * 128 + ((((tk >> 4) ^ (r0 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(h2 & 0xff);
-                pbuf[r1 * 128 + ((((tk >> 4) ^ (r1 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(h2 >> 8);
-                pbuf[q0 * 128 + ((((tk >> 4) ^ (q0 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(l2 & 0xff);
-                pbuf[q1 * 128 + ((((tk >> 4) ^ (q1 & 7)) & 7) << 4) + (tk & 15)] = (uint8_t)(l2 >> 8);
+            for (int jj = 0; jj < NH; jj += 2) {
+              // masked scores give 0 (rows past the unit's rows have no finite maximum)
+              const float p0 = sv[jj] == -INFINITY ? 0.f : ex2(sv[jj] - mloc[jj]);
+              const float p1 = sv[jj + 1] == -INFINITY ? 0.f : ex2(sv[jj + 1] - mloc[jj + 1]);
+              l[jj] += p0;
+              l[jj + 1] += p1;
+              uint32_t h2, l2;
+              split2(p0, p1, h2, l2);
+              if ((jj & 2) == 0) {
+                hw[jj >> 2] = h2;
+                lw[jj >> 2] = l2;
+              } else {
+                hw[jj >> 2] |= h2 << 16;
+                lw[jj >> 2] |= l2 << 16;
               }
+            }
+            const int x7 = tok_in_tile & 7;
+            const int bh = half * NH, bl = NR + half * NH;  // first byte of this lane's hi / lo rows
+            if constexpr (NH == 8) {
+              *reinterpret_cast<uint2*>(prow + ((((bh >> 4) ^ x7) & 7) << 4) + (bh & 15)) = make_uint2(hw[0], hw[1]);
+              *reinterpret_cast<uint2*>(prow + ((((bl >> 4) ^ x7) & 7) << 4) + (bl & 15)) = make_uint2(lw[0], lw[1]);
+            } else {
+              *reinterpret_cast<uint4*>(prow + ((((bh >> 4) ^ x7) & 7) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4*>(prow + ((((bl >> 4) ^ x7) & 7) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
           }
           tc::fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) tc::mbar_arrive(pfull_bar(tt & 1));
+          if (lane == 0) tc::mbar_arrive(pfull_bar(tt % C::kPBufs));
         }
         if (failed) {
           ok = false;
@@ -564,11 +601,13 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
         n_tile += T;
         ++n_unit;
         consume_pv(n_tile - 1);
-        // column sums over the 64 token lanes (lanes 16-31 of each warp hold zeros)
+        // row sums over the 64 tokens: each 16-lane half of a warp holds half of the rows
 #pragma unroll
-        for (int n = 0; n < NR; ++n) {
-          const float v = warp_sum(l[n]);
-          if (lane == 0) red[warp * NR + n] = v;
+        for (int j = 0; j < NH; ++j) {
+          float v = l[j];
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if ((lane & 15) == 0) red[warp * NR + half * NH + j] = v;
         }
         if (!tc::bar_and(1, 128, ok)) {
           ok = false;
