@@ -2,8 +2,8 @@
 //   M = max_j LSE_j,  LSE = M + ln sum_j exp(LSE_j - M),  O = sum_j exp(LSE_j - LSE) O_j
 // (the merge "via online softmax" of the route primitive, "Move the Query, Not the Cache",
 // Methodology; the in-CTA partial + row-statistics merge of the FlashInfer PR #5597 page,
-// section 3).  HBM-bound: one CTA per output row streams its S x H x D partial floats with
-// 16-byte loads; per-(state, head) weights are computed once into shared memory.
+// section 3).  HBM-bound: a CTA per output row and group of heads streams its S x H x D partial
+// floats with 16-byte loads.
 #include <algorithm>
 
 #include "tc_ptx.cuh"
@@ -13,19 +13,19 @@ namespace skv {
 namespace {
 
 constexpr int kMergeThreads = 128;
-constexpr int kStateChunk = 32;
+constexpr int kStateChunk = 8;
 constexpr int kMaxHeadsPerBlock = 8;
 
-// One CTA per (output row, group of hg heads): hg * D = 512 floats, one float4 per thread per
-// state.  Pass 1 (one warp per head): M and LSE over the row's states.  Pass 2: per state chunk,
-// the weights exp(LSE_j - LSE) go to shared memory and every thread accumulates its float4.
+// One CTA per (output row, group of hg heads): hg * D = 512 floats, one float4 per thread.  A
+// thread issues the LSE and the O float4 of up to kStateChunk states at once (one memory round
+// trip for the usual few splits) and combines them with a running maximum:
+//   M' = max(M, max_j LSE_j),  l' = l e^(M - M') + sum_j e^(LSE_j - M'),  acc likewise with O_j,
+// so after the last chunk LSE = M + ln l and O = acc / l -- the same sums as the two-pass form.
 template <typename OutT>
 __global__ void __launch_bounds__(kMergeThreads)
 merge_kernel(const float* __restrict__ o_states, const float* __restrict__ lse_states,
              const int32_t* __restrict__ state_indptr, int num_states, const MergeItem* __restrict__ items,
              int64_t num_rows, int H, int D, int hg, OutT* __restrict__ o_out, float* __restrict__ lse_out) {
-  __shared__ float lse_s[kMaxHeadsPerBlock];
-  __shared__ float w_s[kStateChunk][kMaxHeadsPerBlock];
   const int64_t row = blockIdx.x;
   const int h0 = blockIdx.y * hg;
   const int nh = min(hg, H - h0);
@@ -39,61 +39,55 @@ merge_kernel(const float* __restrict__ o_states, const float* __restrict__ lse_s
   } else {
     out_row = row; base = row; S = num_states; jstride = num_rows;
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int hh = warp; hh < nh; hh += kMergeThreads / 32) {
-    const int h = h0 + hh;
-    float M = -INFINITY;
-    for (int j = lane; j < S; j += 32) M = fmaxf(M, lse_states[(base + j * jstride) * H + h]);
-    M = warp_max(M);
-    float tot = 0.f;
-    if (M != -INFINITY)
-      for (int j = lane; j < S; j += 32) {
-        const float lj = lse_states[(base + j * jstride) * H + h];
-        tot += (lj == -INFINITY) ? 0.f : exp2f((lj - M) * kLog2e);
-      }
-    tot = warp_sum(tot);
-    const float lse = (M == -INFINITY) ? -INFINITY : M + log2f(tot) * kLn2;
-    if (lane == 0) {
-      lse_s[hh] = lse;
-      if (lse_out != nullptr) lse_out[out_row * H + h] = lse;
-    }
-  }
-  __syncthreads();
   const int n4 = nh * D / 4;  // float4 of this block
-  for (int e0 = 0; e0 < n4; e0 += kMergeThreads) {
-    const int e = e0 + threadIdx.x;
+  for (int e = threadIdx.x; e < n4; e += kMergeThreads) {
+    const int h = h0 + (e * 4) / D;
+    float M = -INFINITY, l = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int hh = (e * 4) / D;
     for (int j0 = 0; j0 < S; j0 += kStateChunk) {
       const int nj = min(kStateChunk, S - j0);
-      __syncthreads();
-      for (int idx = threadIdx.x; idx < nj * nh; idx += kMergeThreads) {
-        const int j = idx / nh, k = idx % nh;
-        const float lj = lse_states[(base + (j0 + j) * jstride) * H + h0 + k];
-        const float L = lse_s[k];
-        w_s[j][k] = (lj == -INFINITY || L == -INFINITY) ? 0.f : exp2f((lj - L) * kLog2e);
-      }
-      __syncthreads();
-      if (e < n4) {
-        for (int j = 0; j < nj; ++j) {
-          const float4* src = reinterpret_cast<const float4*>(
-              o_states + ((base + (j0 + j) * jstride) * (int64_t)H + h0) * D);
-          const float wt = w_s[j][hh];
-          const float4 x = __ldg(src + e);
-          acc.x = fmaf(wt, x.x, acc.x);
-          acc.y = fmaf(wt, x.y, acc.y);
-          acc.z = fmaf(wt, x.z, acc.z);
-          acc.w = fmaf(wt, x.w, acc.w);
+      float lj[kStateChunk];
+      float4 x[kStateChunk];
+#pragma unroll
+      for (int j = 0; j < kStateChunk; ++j) {  // all loads of the chunk in flight together
+        if (j < nj) {
+          const int64_t st = base + (int64_t)(j0 + j) * jstride;
+          lj[j] = __ldg(lse_states + st * H + h);
+          x[j] = __ldg(reinterpret_cast<const float4*>(o_states + (st * H + h0) * (int64_t)D) + e);
+        } else {
+          lj[j] = -INFINITY;
+          x[j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+      float mc = M;
+#pragma unroll
+      for (int j = 0; j < kStateChunk; ++j) mc = fmaxf(mc, lj[j]);
+      if (mc == -INFINITY) continue;  // every state so far is empty
+      const float sc = M == -INFINITY ? 0.f : exp2f((M - mc) * kLog2e);
+      l *= sc;
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+#pragma unroll
+      for (int j = 0; j < kStateChunk; ++j) {
+        const float wt = lj[j] == -INFINITY ? 0.f : exp2f((lj[j] - mc) * kLog2e);
+        l += wt;
+        acc.x = fmaf(wt, x[j].x, acc.x);
+        acc.y = fmaf(wt, x[j].y, acc.y);
+        acc.z = fmaf(wt, x[j].z, acc.z);
+        acc.w = fmaf(wt, x[j].w, acc.w);
+      }
+      M = mc;
     }
-    if (e < n4) {
-      OutT* dst = o_out + (out_row * (int64_t)H + h0) * D + (int64_t)e * 4;
-      store_out(dst + 0, acc.x);
-      store_out(dst + 1, acc.y);
-      store_out(dst + 2, acc.z);
-      store_out(dst + 3, acc.w);
-    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    OutT* dst = o_out + (out_row * (int64_t)H + h0) * D + (int64_t)e * 4;
+    store_out(dst + 0, acc.x * inv);
+    store_out(dst + 1, acc.y * inv);
+    store_out(dst + 2, acc.z * inv);
+    store_out(dst + 3, acc.w * inv);
+    if (lse_out != nullptr && (e * 4) % D == 0)
+      lse_out[out_row * H + h] = l > 0.f ? M + log2f(l) * kLn2 : -INFINITY;
   }
 }
 
