@@ -75,6 +75,7 @@ struct MArgs {
   const int32_t* last;
   const int32_t* cta_indptr;
   int num_pages, page_size, heads, hc, hg, q_tile;
+  int gather;  // page size 1: token rows fetched with tile::gather4 from 2-D maps
   float scale_log2;
   void* o;
   float* lse;
@@ -110,6 +111,16 @@ __device__ __forceinline__ float redux_max(float v) {
   float r;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
+}
+
+// four rows (ids y0..y3) x one 64-column box of a 2-D tensor map, into four consecutive 128-byte rows
+__device__ __forceinline__ void gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y0, int y1,
+                                        int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2) {
@@ -212,6 +223,57 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           }
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (a.gather) {
+          // page size 1 (a page id is a token row): lane l fetches rows 4g .. 4g + 3 (g = l % 16)
+          // of the tile for regions l / 16, l / 16 + 2, ... (8 ckv halves + the rope block), one
+          // gather4 each; its four row ids are loaded a tile ahead.  Rows past the unit repeat
+          // the unit's first row (masked, and their V rows zeroed, downstream).
+          const int grp = lane & 15;
+          auto load_ids = [&](int t, int (&v)[4]) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int k = t * kTile + 4 * grp + i;
+              v[i] = (t < x.ntiles && k < npages) ? __ldg(ids + k) : (t < x.ntiles ? __ldg(ids) : 0);
+            }
+          };
+          int cur[4];
+          load_ids(0, cur);
+          for (int t = 0; t < x.ntiles && ok; ++t) {
+            const int sk = gk % NK;
+            int sc[kBlocks];
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
+            if (lane == 0) {
+              if (gk >= NK) ok = tc::mbar_wait_sleep(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
+              if (ok) tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(kTile * 128));
+              for (int b = 0; b < kBlocks && ok; ++b) {
+                const int g = gc + b;
+                if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
+                if (ok) tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * kTile * 128));
+              }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if ((unsigned)cur[i] >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);  // reads zeros
+            for (int r = lane >> 4; r < 9; r += 2) {
+              if (r < 8) {
+                const int b = r >> 1, hf = r & 1;
+                gather4(sbase + C::cring + sc[b] * kCSlot + hf * kHalf + grp * 4 * 128, &ckv_map, cfull_bar(sc[b]),
+                        b * 128 + hf * 64, cur[0], cur[1], cur[2], cur[3]);
+              } else {
+                gather4(sbase + C::kring + sk * kKSlot + grp * 4 * 128, &kpe_map, kfull_bar(sk), 0, cur[0], cur[1],
+                        cur[2], cur[3]);
+              }
+            }
+            load_ids(t + 1, cur);
+            ++gk;
+            gc += kBlocks;
+          }
+          ++n_unit;
+          continue;
+        }
         int win = -1000000, pid = 0;  // lanes hold the ids of pages [win, win + 32) of the unit
         for (int t = 0; t < x.ntiles && ok; ++t) {
           const int pi0 = (t * kTile) / P;
@@ -589,11 +651,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_m() {
 }
 
 bool make_map_m(CUtensorMap* m, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
-                const cuuint32_t* box) {
+                const cuuint32_t* box, int rank = 3) {
   auto fn = encode_fn_m();
   if (fn == nullptr) return false;
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides_bytes, box, estr,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -614,7 +676,8 @@ int launch_m(const CUtensorMap* maps, const MArgs& a, int num_ctas, const WorkIt
 }  // namespace
 
 bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit) {
-  const bool page_ok = page_size >= 8 && (page_size <= kTile ? kTile % page_size == 0 : page_size % kTile == 0);
+  const bool page_ok = page_size == 1 ||
+                       (page_size >= 8 && (page_size <= kTile ? kTile % page_size == 0 : page_size % kTile == 0));
   return kv_dtype == SKV_BF16 && page_ok && (rows_per_unit == 16 || rows_per_unit == 32) &&
          (num_heads <= rows_per_unit || num_heads % rows_per_unit == 0);
 }
@@ -631,13 +694,23 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
   const int box_rows = std::min(p.page_size, kTile);
   const int total_q = p.batch * p.q_len;
   CUtensorMap maps[4];
-  {
+  const bool gather = p.page_size == 1;
+  if (gather) {  // token rows: 2-D maps (dims, row = page id), boxes one row high for tile::gather4
+    const cuuint64_t cd[2] = {512, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t cs[1] = {(cuuint64_t)p.ckv_stride[0] * 2};
+    const cuuint64_t kd[2] = {64, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t ks[1] = {(cuuint64_t)p.kpe_stride[0] * 2};
+    const cuuint32_t box[2] = {64, 1};
+    if (!make_map_m(&maps[0], p.ckv, cd, cs, box, 2) || !make_map_m(&maps[1], p.kpe, kd, ks, box, 2))
+      return (int)cudaErrorInvalidValue;
+  }
+  if (!gather) {
     const cuuint64_t dims[3] = {512, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
     const cuuint64_t st[2] = {(cuuint64_t)p.ckv_stride[1] * 2, (cuuint64_t)p.ckv_stride[0] * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     if (!make_map_m(&maps[0], p.ckv, dims, st, box)) return (int)cudaErrorInvalidValue;
   }
-  {
+  if (!gather) {
     const cuuint64_t dims[3] = {64, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
     const cuuint64_t st[2] = {(cuuint64_t)p.kpe_stride[1] * 2, (cuuint64_t)p.kpe_stride[0] * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
@@ -666,6 +739,7 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
   a.hc = hc;
   a.hg = p.num_heads / hc;
   a.q_tile = q_tile;
+  a.gather = gather ? 1 : 0;
   a.scale_log2 = p.sm_scale * kLog2e;
   a.o = p.o;
   a.lse = p.lse;
