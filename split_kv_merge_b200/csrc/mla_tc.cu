@@ -46,22 +46,23 @@ constexpr float kRaise = 8.f;
 
 template <int NR>
 struct MlaCfg {
-  static constexpr int kCStages = NR == 16 ? 10 : 9;
+  static constexpr int kCStages = NR == 16 ? 9 : 8;
   static constexpr int kKStages = 4;
   static constexpr int kQRegion = NR * 128;             // one 64-column region of Q
   static constexpr int kQBytes = 9 * kQRegion;          // q_nope (8 regions) + q_pe
-  static constexpr int kPBytes = NR * 128;              // NR rows x 64 tokens bf16 (1 region)
+  static constexpr int kPBytes = kTile * 128;           // P^T MN-major: one 128-byte row per token
+  static constexpr int kPBufs = 3;                      // P(t) reuses the buffer of PV(t - 3)
   static constexpr int cring = 0;
   static constexpr int kring = cring + kCStages * kCSlot;
   static constexpr int q = kring + kKStages * kKSlot;
   static constexpr int p = q + kQBytes;
-  static constexpr int red = p + 2 * kPBytes;           // [4][NR] float
+  static constexpr int red = p + kPBufs * kPBytes;      // [4][NR] float
   static constexpr int alpha = red + 4 * NR * 4;        // [NR]
   static constexpr int inv = alpha + NR * 4;            // [NR]
   static constexpr int lse = inv + NR * 4;              // [NR]
   static constexpr int mrow = lse + NR * 4;             // [NR] running maximum of every row
   static constexpr int bars = mrow + NR * 4;
-  static constexpr int nbars = 2 * kCStages + 2 * kKStages + 11;
+  static constexpr int nbars = 2 * kCStages + 2 * kKStages + 14;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
   // S: 2 buffers x 4 partial accumulators (one per issuer) x NR (M=64 lanes); O^T: 4 blocks x NR
@@ -104,6 +105,12 @@ __device__ __forceinline__ MUnit load_munit(const MArgs& a, const WorkItem* work
   x.t1 = min(w.page_end * a.page_size, L);
   x.ntiles = x.t1 > x.t0 ? (x.t1 - x.t0 + kTile - 1) / kTile : 0;
   return x;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 // maximum over the warp (sm_100 redux on f32)
@@ -155,9 +162,9 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
   auto qempty_bar = [&]() { return bar1 + 8u; };
   auto sfull_bar = [&](int b) { return bar1 + 8u * (2 + b); };
   auto sempty_bar = [&](int b) { return bar1 + 8u * (4 + b); };
-  auto pfull_bar = [&](int b) { return bar1 + 8u * (6 + b); };
-  auto ofull_bar = [&](int b) { return bar1 + 8u * (8 + b); };
-  auto ofree_bar = [&]() { return bar1 + 8u * 10; };
+  auto pfull_bar = [&](int b) { return bar1 + 8u * (6 + b); };   // one per P buffer
+  auto ofull_bar = [&](int b) { return bar1 + 8u * (9 + b); };   // four: PV(t) on t & 3
+  auto ofree_bar = [&]() { return bar1 + 8u * 13; };
   static_assert(C::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
 
   if (tid == 0) {
@@ -174,9 +181,9 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(sfull_bar(b), kIssuers);
       tc::mbar_init(sempty_bar(b), 4);
-      tc::mbar_init(pfull_bar(b), 4);
-      tc::mbar_init(ofull_bar(b), kIssuers);
     }
+    for (int b = 0; b < C::kPBufs; ++b) tc::mbar_init(pfull_bar(b), 4);
+    for (int b = 0; b < 4; ++b) tc::mbar_init(ofull_bar(b), kIssuers);
     tc::mbar_init(ofree_bar(), 4);
     *abort_flag = 0;
     tc::fence_mbar_init();
@@ -339,7 +346,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     if (lane == 0) {
       const int w = warp - 5;
       constexpr uint32_t idesc_s = tc::idesc_bf16_f32(64, NR, false, false);
-      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, NR, true, false);
+      constexpr uint32_t idesc_o = tc::idesc_bf16_f32(128, NR, true, true);  // V^T and P^T MN-major
       int g = 0, n_unit = 0, n_tile = 0;
       bool ok = true;
       const uint32_t qs = sbase + C::q;
@@ -356,10 +363,10 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           while (ok && pv < T) {
             bool did = false;
             if (pv < qk) {  // ---- PV(pv), block w
-              const int tp = n_tile + pv, pb = tp & 1;
+              const int tp = n_tile + pv, pb = tp % C::kPBufs;
               const int cb = kBlocks * (g + pv) + w, st = cb % NC;
               // the single O^T buffer was read by the previous unit's epilogue
-              if (tc::mbar_test_wait(pfull_bar(pb), (tp >> 1) & 1) &&
+              if (tc::mbar_test_wait(pfull_bar(pb), (tp / C::kPBufs) & 1) &&
                   (pv > 0 || n_unit == 0 || tc::mbar_test_wait(ofree_bar(), (n_unit + 1) & 1))) {
                 tc::tc_fence_after();
                 const uint32_t ps = sbase + C::p + pb * C::kPBytes;
@@ -367,11 +374,11 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
 #pragma unroll
                 for (int k = 0; k < kTile / 16; ++k) {
                   const uint64_t ad = tc::sdesc_sw128(vs + k * 2048, kHalf, 1024);
-                  const uint64_t bd = tc::sdesc_sw128(ps + k * 32, 16, 1024);
+                  const uint64_t bd = tc::sdesc_sw128(ps + k * 2048, 8192, 1024);
                   tc::mma_bf16(tm_o + w * NR, ad, bd, idesc_o, (pv > 0 || k > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(cempty_bar(st));
-                tc::mma_commit(ofull_bar(pb));
+                tc::mma_commit(ofull_bar(tp & 3));
                 ++pv;
                 did = true;
               }
@@ -423,7 +430,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     bool ok = true;
     auto consume_pv = [&](int upto) {
       for (; pv_seen <= upto; ++pv_seen)
-        ok = tc::mbar_wait_sleep(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
+        ok = tc::mbar_wait_sleep(ofull_bar(pv_seen & 3), (pv_seen >> 2) & 1, abort_flag, a.status) && ok;
       tc::tc_fence_after();
     };
     for (int u = u_begin; u < u_end && ok; ++u) {
@@ -452,9 +459,13 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         }
         const int T = x.ntiles;
         const int gc0 = gc;
-        float l[NR];
+        // P phase: lanes 0-15 take rows [0, NR/2) of their token, lanes 16-31 rows [NR/2, NR) of the
+        // token of lane - 16; l[j] is the partial sum of row half * NR/2 + j
+        constexpr int NH = NR / 2;
+        const int half = lane >> 4;
+        float l[NH];
 #pragma unroll
-        for (int n = 0; n < NR; ++n) l[n] = 0.f;
+        for (int j = 0; j < NH; ++j) l[j] = 0.f;
         if (tid < NR) m_s[tid] = -INFINITY;
         tc::named_bar_sync(1, 128);
         bool failed = false;
@@ -507,7 +518,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             }
             tc::named_bar_sync(1, 128);
 #pragma unroll
-            for (int n = 0; n < NR; ++n) l[n] *= alpha_s[n];
+            for (int j = 0; j < NH; ++j) l[j] *= alpha_s[half * NH + j];
             if (t > 0) {  // rescale O^T in TMEM (every thread owns lane `tid` of the 4 blocks)
               consume_pv(tt - 1);
 #pragma unroll 1
@@ -541,23 +552,39 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
                 for (int i = 0; i < 8; ++i) reinterpret_cast<uint4*>(row + hf * kHalf)[i] = make_uint4(0, 0, 0, 0);
             }
           }
-          if (tt >= 2 && pv_seen <= tt - 2) consume_pv(tt - 2);  // P(t) reuses PV(t-2)'s buffer
-          if (srow) {
-            uint8_t* pb = smem + C::p + (tt & 1) * C::kPBytes;
-            float mloc[NR];  // read the maxima before the stores below (they may alias for the compiler)
+          if (tt >= C::kPBufs && pv_seen <= tt - C::kPBufs) consume_pv(tt - C::kPBufs);  // P(t)'s buffer was PV's
+          {
+            float sv[NH], mloc[NH];
 #pragma unroll
-            for (int n = 0; n < NR; ++n) mloc[n] = m_s[n];
+            for (int jj = 0; jj < NH; ++jj) {  // upper rows move from lane l to lane l + 16
+              const float up = __shfl_sync(0xffffffffu, s[NH + jj], lane & 15);
+              sv[jj] = half ? up : s[jj];
+              mloc[jj] = m_s[half * NH + jj];
+            }
+            // token row of P^T (MN-major, 128-byte swizzle): bf16 of rows 0 .. NR-1
+            uint8_t* prow = smem + C::p + (tt % C::kPBufs) * C::kPBytes + tok_in_tile * 128;
+            uint32_t pw[NH / 2];
 #pragma unroll
-            for (int n = 0; n < NR; ++n) {
-              const float p = (s[n] == -INFINITY) ? 0.f : exp2f(s[n] - mloc[n]);
-              l[n] += p;
-              if (n < rows)
-                *reinterpret_cast<__nv_bfloat16*>(pb + tc::sw128_offset(n, tok_in_tile)) = __float2bfloat16_rn(p);
+            for (int jj = 0; jj < NH; jj += 2) {
+              // masked scores give 0 (rows past the unit's rows have no finite maximum)
+              const float p0 = sv[jj] == -INFINITY ? 0.f : ex2(sv[jj] - mloc[jj]);
+              const float p1 = sv[jj + 1] == -INFINITY ? 0.f : ex2(sv[jj + 1] - mloc[jj + 1]);
+              l[jj] += p0;
+              l[jj + 1] += p1;
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+              pw[jj >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            const int x7 = tok_in_tile & 7;
+#pragma unroll
+            for (int c = 0; c < NH / 8; ++c) {  // 16-byte chunk (half * NH / 8 + c) of the row
+              const int ch = half * (NH / 8) + c;
+              *reinterpret_cast<uint4*>(prow + (((ch ^ x7) & 7) << 4)) =
+                  make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             }
           }
           tc::fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) tc::mbar_arrive(pfull_bar(tt & 1));
+          if (lane == 0) tc::mbar_arrive(pfull_bar(tt % C::kPBufs));
         }
         if (failed) {
           ok = false;
@@ -567,11 +594,13 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         n_tile += T;
         ++n_unit;
         consume_pv(n_tile - 1);
-        // column sums over the 64 token lanes (lanes 16-31 of each warp hold zeros)
+        // row sums over the 64 tokens: each 16-lane half of a warp holds half of the rows
 #pragma unroll
-        for (int n = 0; n < NR; ++n) {
-          const float v = warp_sum(l[n]);
-          if (lane == 0) red[warp * NR + n] = v;
+        for (int j = 0; j < NH; ++j) {
+          float v = l[j];
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if ((lane & 15) == 0) red[warp * NR + half * NH + j] = v;
         }
         if (!tc::bar_and(1, 128, ok)) {
           ok = false;
