@@ -218,3 +218,43 @@ def test_mla_validation():
     bad = skv.MlaParams.from_buffer_copy(p)
     bad.ckv_stride[1] = 577
     assert fwd(ctypes.byref(bad), fake, ctypes.byref(info), None) == skv.ERR_ALIGNMENT
+
+
+# ----------------------------------------------------------------------------- kernel choice
+@pytest.mark.parametrize("hq,hk,q_len,page_size,kernel,q_tile", [
+    (64, 8, 1, 16, 3, 1),     # Llama decode: all-KV-heads decode kernel
+    (16, 4, 1, 32, 2, 1),     # 4 KV heads: per-head decode kernel (one token per unit)
+    (32, 8, 128, 64, 4, 32),  # shared-KV prefill: 128-row prefill kernel, 128 / g tokens per unit
+    (8, 8, 40, 128, 4, 128),  # g = 1 prefill with pages larger than a tile
+    (32, 2, 9, 32, 4, 8),     # g = 16: 9 tokens x 16 heads > one decode tile
+    (32, 8, 128, 4, 1, 4),    # page size 4 is below every tensor-core kernel: CUDA-core kernel
+])
+def test_paged_planner_kernel_choice(hq, hk, q_len, page_size, kernel, q_tile):
+    """The planner's dispatch: which kernel a shape runs on and how many query tokens a unit holds."""
+    n_req = 3
+    qo = (np.arange(n_req + 1) * q_len).astype(np.int32)
+    pages = np.array([5, 1, 9], np.int32)
+    kv_indptr = np.concatenate([[0], np.cumsum(pages)]).astype(np.int32)
+    last = np.full(n_req, page_size, np.int32)
+    plan = skv.plan_paged(qo, kv_indptr, last, page_size, hq, hk, 128, "none", 0)
+    assert plan.info.kernel == kernel and plan.info.q_tile == q_tile
+    w, _ = _items(plan)
+    assert np.all(w[:, 2] <= q_tile)                                    # q_count within the tile
+    assert sorted(set(map(tuple, w[:, [0, 1]].tolist()))) == sorted(
+        (r, int(qo[r]) + q0) for r in range(n_req) for q0 in range(0, q_len, q_tile))
+
+
+@pytest.mark.parametrize("H,q_len,kv_dtype,page_size,kernel", [
+    (16, 1, "bf16", 64, 12), (16, 4, "bf16", 64, 13), (128, 1, "bf16", 64, 13),
+    (16, 1, "e4m3", 64, 12), (128, 4, "e4m3", 64, 13),   # native fp8 tensor-core kernel
+    (16, 1, "bf16", 1, 12),                              # page size 1: row gather on the tensor cores
+    (16, 1, "e4m3", 1, 11),                              # e4m3 with page size 1: CUDA-core kernel
+    (16, 1, "bf16", 4, 11),
+])
+def test_mla_planner_kernel_choice(H, q_len, kv_dtype, page_size, kernel):
+    kv_indptr = np.array([0, 7, 7, 20], np.int32)
+    last = np.array([page_size, 1, max(1, page_size // 2)], np.int32)
+    plan = skv.plan_mla(q_len, kv_indptr, last, page_size, H, "balanced", 148, kv_dtype=kv_dtype)
+    assert plan.info.kernel == kernel
+    rows = {12: 16, 13: 32}.get(kernel, 128)
+    assert plan.info.q_tile == (skv.mla_fold_ratio(H, q_len, rows) if H <= rows else 1)
