@@ -46,6 +46,7 @@ struct PersistOpts {
   int32_t flat_ctas = 0;
   int32_t tile_tokens = 128;
   int32_t page_size = 1;
+  int32_t piece_cost = 0;  // fixed cost of a work item (query load, pipeline refill, epilogue), in tiles
 };
 
 // Tiles of logical pages [a, b) of a request of length L (pages of `page_size` tokens).
@@ -97,12 +98,20 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
   if (flat) {
     const int G = po.flat_ctas;
     std::vector<int64_t> w(batch, 0);
-    double total = 0;
+    double total = 0, piece_total = 0;
+    int64_t nonempty = 0;
     for (int32_t r = 0; r < batch; ++r) {
       const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile * units_per_page;
       w[r] = qt * range_tiles(0, req[r].n_pages, kv_len[r], P, T);
       total += (double)w[r];
+      if (w[r] > 0) {
+        ++nonempty;
+        piece_total += (double)po.piece_cost * (double)qt;
+      }
     }
+    // every piece of request r also costs po.piece_cost tiles per query unit of r: about one
+    // piece per request plus one per CTA boundary (charged at the mean)
+    if (nonempty > 0) total += piece_total + (double)(G - 1) * piece_total / (double)nonempty;
     const double target = total / G;
     const int64_t min_piece = std::max<int64_t>(1, std::min<int64_t>(4, (int64_t)target));
     int cta = 0;
@@ -117,11 +126,12 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
         continue;
       }
       int32_t a = 0;
+      const double pc = (double)po.piece_cost * (double)qt;
       while (a < n) {
-        double room = (cta + 1) * target - cum;
+        double room = (cta + 1) * target - cum - pc;
         if (room < (double)min_piece && cta < G - 1) {
           ++cta;
-          room = (cta + 1) * target - cum;
+          room = (cta + 1) * target - cum - pc;
         }
         // largest b with work(a, b) <= room (at least one page), or the whole rest
         int32_t b = a + 1;
@@ -134,7 +144,7 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
         const int64_t wt = qt * range_tiles(a, b, kv_len[r], P, T);
         bounds[r].push_back(b);
         piece_cta[r].push_back(cta);
-        cum += (double)wt;
+        cum += (double)wt + pc;
         a = b;
         if (cum >= (cta + 1) * target - 0.5 && cta < G - 1) ++cta;
       }
@@ -396,6 +406,7 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
     head_groups = num_heads <= nr ? 1 : num_heads / nr;
     po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
     po.tile_tokens = mla_tc_tile_tokens();
+    po.piece_cost = 4;  // measured: a work item's start and end cost about four 64-token tiles
   }
   return plan_common(batch, req, kv_len, fold, head_groups, 8, policy, param, split_indptr_h, split_bounds_h,
                      kernel, po, plan_h, plan_capacity, info);
