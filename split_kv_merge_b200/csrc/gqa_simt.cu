@@ -51,6 +51,7 @@ __device__ __forceinline__ float dot_row(const float* qs, const __nv_bfloat16* k
 
 template <int D, bool SAME_KV, typename OutT>
 __global__ void __launch_bounds__(128) gqa_simt_kernel(GqaArgs a, const WorkItem* __restrict__ work) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the merge pass may be scheduled
   constexpr int PER_LANE = D / 32;  // V dims per lane
   __shared__ __align__(16) float q_s[4][D];
   const WorkItem w = work[blockIdx.x];

@@ -103,6 +103,7 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = tc::smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  tc::grid_launch_dependents();  // the merge pass may be scheduled; it waits for this grid
 
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Smem::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);

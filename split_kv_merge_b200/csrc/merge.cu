@@ -29,6 +29,7 @@ merge_kernel(const float* __restrict__ o_states, const float* __restrict__ lse_s
   const int64_t row = blockIdx.x;
   const int h0 = blockIdx.y * hg;
   const int nh = min(hg, H - h0);
+  tc::grid_dependency_wait();  // the partials of the preceding attention grid are complete
   int64_t out_row, base, jstride;
   int S;
   if (items != nullptr) {
@@ -128,16 +129,26 @@ int launch_merge(const float* o_states, const float* lse_states, const int32_t* 
   if (num_rows == 0) return 0;
   if (head_dim % 4 != 0) return (int)cudaErrorInvalidValue;
   const int hg = std::max(1, std::min(kMaxHeadsPerBlock, 512 / head_dim));
-  dim3 grid((unsigned)num_rows, (unsigned)((num_heads + hg - 1) / hg));
+  // programmatic stream serialization: the merge may launch while the attention grid that wrote
+  // the partials is finishing; merge_kernel waits for that grid before its first read
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)num_rows, (unsigned)((num_heads + hg - 1) / hg));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (o_dtype == SKV_BF16)
-    merge_kernel<__nv_bfloat16><<<grid, kMergeThreads, 0, s>>>(o_states, lse_states, state_indptr, num_states, items,
-                                                              num_rows, num_heads, head_dim, hg,
-                                                              static_cast<__nv_bfloat16*>(o_out), lse_out);
+    e = cudaLaunchKernelEx(&cfg, merge_kernel<__nv_bfloat16>, o_states, lse_states, state_indptr, num_states, items,
+                           num_rows, num_heads, head_dim, hg, static_cast<__nv_bfloat16*>(o_out), lse_out);
   else
-    merge_kernel<float><<<grid, kMergeThreads, 0, s>>>(o_states, lse_states, state_indptr, num_states, items,
-                                                      num_rows, num_heads, head_dim, hg, static_cast<float*>(o_out),
-                                                      lse_out);
-  return (int)cudaGetLastError();
+    e = cudaLaunchKernelEx(&cfg, merge_kernel<float>, o_states, lse_states, state_indptr, num_states, items, num_rows,
+                           num_heads, head_dim, hg, static_cast<float*>(o_out), lse_out);
+  return (int)e;
 }
 
 }  // namespace skv

@@ -69,6 +69,7 @@ __device__ __forceinline__ float dot_span(const float* qs, const uint8_t* base, 
 
 template <bool E4M3, typename OutT>
 __global__ void __launch_bounds__(128) mla_simt_kernel(MlaArgs a, const WorkItem* __restrict__ work) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the merge pass may be scheduled
   constexpr int DV = 512, DR = 64, PER_LANE = DV / 32;
   __shared__ __align__(16) float q_s[4][DV + DR];
   const WorkItem w = work[blockIdx.x];
