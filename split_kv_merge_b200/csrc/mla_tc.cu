@@ -40,7 +40,8 @@ constexpr int kHalf = kTile * 128;     // one 64-column swizzled region of a til
 constexpr int kCSlot = 2 * kHalf;      // ckv slot: one 128-dim block (16 KB)
 constexpr int kKSlot = kHalf;          // kpe slot (8 KB)
 constexpr int kIssuers = 4;          // MMA issuing warps 5-8, one per SM sub-partition
-constexpr int kThreads = (5 + kIssuers) * 32;  // 4 softmax warps, TMA warp, 4 MMA-issuing warps
+constexpr int kGatherWarps = 4;      // page size 1: warp 4 and warps 9-11 fetch rows with cp.async
+constexpr int kThreads = (5 + kIssuers + kGatherWarps - 1) * 32;  // softmax, TMA, MMA, gather warps
 constexpr int kBlocks = 4;             // 512 ckv dims = 4 blocks of 128
 constexpr float kRaise = 8.f;
 
@@ -76,7 +77,10 @@ struct MArgs {
   const int32_t* last;
   const int32_t* cta_indptr;
   int num_pages, page_size, heads, hc, hg, q_tile;
-  int gather;  // page size 1: token rows fetched with tile::gather4 from 2-D maps
+  int gather;  // page size 1: token rows fetched with 16-byte cp.async by four warps
+  const uint8_t* ckv_rows;  // page size 1: row id i starts at ckv_rows + i * ckv_row_bytes
+  const uint8_t* kpe_rows;
+  int64_t ckv_row_bytes, kpe_row_bytes;
   float scale_log2;
   void* o;
   float* lse;
@@ -120,16 +124,6 @@ __device__ __forceinline__ float redux_max(float v) {
   return r;
 }
 
-// four rows (ids y0..y3) x one 64-column box of a 2-D tensor map, into four consecutive 128-byte rows
-__device__ __forceinline__ void gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y0, int y1,
-                                        int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], "
-      "[%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
@@ -170,11 +164,11 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
 
   if (tid == 0) {
     for (int s = 0; s < NC; ++s) {
-      tc::mbar_init(cfull_bar(s), 1);
+      tc::mbar_init(cfull_bar(s), a.gather ? kGatherWarps * 32 : 1);
       tc::mbar_init(cempty_bar(s), 1);
     }
     for (int s = 0; s < NK; ++s) {
-      tc::mbar_init(kfull_bar(s), 1);
+      tc::mbar_init(kfull_bar(s), a.gather ? kGatherWarps * 32 : 1);
       tc::mbar_init(kempty_bar(s), kIssuers);
     }
     tc::mbar_init(qfull_bar(), 1);
@@ -190,13 +184,15 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     tc::fence_mbar_init();
   }
   if (warp == 4 && lane == 0) {
-    tc::prefetch_tmap(&ckv_map);
-    tc::prefetch_tmap(&kpe_map);
+    if (!a.gather) {
+      tc::prefetch_tmap(&ckv_map);
+      tc::prefetch_tmap(&kpe_map);
+    }
     tc::prefetch_tmap(&qn_map);
     tc::prefetch_tmap(&qp_map);
   }
   // ckv slots start as zeros: rows of a partial tile that no page fills must be finite
-  for (int i = tid; i < NC * kCSlot / 16; i += kThreads)
+  for (int i = tid; i < NC * kCSlot / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + C::cring)[i] = make_uint4(0, 0, 0, 0);
   tc::fence_proxy_async_smem();
   if (warp == 5) tc::tmem_alloc(tc::smem_u32(tmem_holder), C::tmem_cols);
@@ -210,7 +206,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
   const int P = a.page_size;
   const int box_rows = min(P, kTile);
 
-  if (warp == 4) {
+  if (warp == 4 || (warp >= 5 + kIssuers && a.gather)) {
     // ======================================================================= TMA producer
     int gc = 0, gk = 0, n_unit = 0;
     bool ok = true;
@@ -220,7 +216,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
       const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
       const int npages = x.page_end - x.page_begin;
       for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
-        if (lane == 0) {  // Q of this unit once the previous unit's last S MMA is done
+        if (warp == 4 && lane == 0) {  // Q of this unit once the previous unit's last S MMA is done
           if (n_unit >= 1) ok = tc::mbar_wait_sleep(qempty_bar(), (n_unit + 1) & 1, abort_flag, a.status);
           if (ok) {
             const int rows = a.hc * a.q_tile;
@@ -232,53 +228,106 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         if (a.gather) {
-          // page size 1 (a page id is a token row): lane l fetches rows 4g .. 4g + 3 (g = l % 16)
-          // of the tile for regions l / 16, l / 16 + 2, ... (8 ckv halves + the rope block), one
-          // gather4 each; its four row ids are loaded a tile ahead.  Rows past the unit repeat
-          // the unit's first row (masked, and their V rows zeroed, downstream).
-          const int grp = lane & 15;
-          auto load_ids = [&](int t, int (&v)[4]) {
+          // page size 1 (a page id is a token row): 128 threads of four warps fetch the tile's 64
+          // rows with 16-byte cp.async, thread p taking half (p & 1) of row p >> 1 (36 chunks),
+          // straight into the swizzled slots; its row id is loaded a tile ahead.  Rows past the
+          // unit repeat the unit's first row (masked, and their V rows zeroed, downstream); an
+          // out-of-range id reads zeros.  A tile's barriers get one arrival per thread once its
+          // copies have landed (cp.async group wait + proxy fence), with the next tile in flight.
+          const int pidx = (warp == 4 ? 0 : warp - (5 + kIssuers) + 1) * 32 + lane;
+          // lane group of 8 per 128-byte row segment: thread (rg = pidx / 8, sub = pidx % 8) copies
+          // chunk sub of segment seg (0-7: ckv block seg / 2, half seg % 2; 8: rope) of rows
+          // pass * 16 + rg, so one warp instruction moves four rows x 128 contiguous bytes
+          const int rg = pidx >> 3, sub = pidx & 7;
+          const int gk0 = gk, gc0 = gc, T = x.ntiles;
+          auto row_ids = [&](int t, int (&v)[4]) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int k = t * kTile + 4 * grp + i;
-              v[i] = (t < x.ntiles && k < npages) ? __ldg(ids + k) : (t < x.ntiles ? __ldg(ids) : 0);
+            for (int ps = 0; ps < 4; ++ps) {
+              const int k = t * kTile + ps * 16 + rg;
+              v[ps] = (t < T && k < npages) ? __ldg(ids + k) : (t < T ? __ldg(ids) : 0);
             }
           };
-          int cur[4];
-          load_ids(0, cur);
-          for (int t = 0; t < x.ntiles && ok; ++t) {
-            const int sk = gk % NK;
-            int sc[kBlocks];
-#pragma unroll
-            for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
+          // slots of tile t are free (blocking wait, or a non-blocking test); warp-uniform result
+          auto claim = [&](int t, bool blocking) -> bool {
+            bool free = true;
             if (lane == 0) {
-              if (gk >= NK) ok = tc::mbar_wait_sleep(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
-              if (ok) tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(kTile * 128));
-              for (int b = 0; b < kBlocks && ok; ++b) {
-                const int g = gc + b;
-                if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
-                if (ok) tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * kTile * 128));
+              const int g = gk0 + t;
+              if (g >= NK) {
+                const uint32_t par = ((g / NK) + 1) & 1;
+                free = blocking ? tc::mbar_wait_sleep(kempty_bar(g % NK), par, abort_flag, a.status)
+                                : tc::mbar_test_wait(kempty_bar(g % NK), par);
+              }
+              for (int b = 0; b < kBlocks && free; ++b) {
+                const int gb = gc0 + kBlocks * t + b;
+                if (gb >= NC) {
+                  const uint32_t par = ((gb / NC) + 1) & 1;
+                  free = blocking ? tc::mbar_wait_sleep(cempty_bar(gb % NC), par, abort_flag, a.status)
+                                  : tc::mbar_test_wait(cempty_bar(gb % NC), par);
+                }
               }
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
+            return __shfl_sync(0xffffffffu, free ? 1 : 0, 0) != 0;
+          };
+          int id_next[4];
+          row_ids(0, id_next);
+          auto issue = [&](int t) {  // this thread's 36 chunks of tile t, one commit group
+            int idv[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if ((unsigned)cur[i] >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);  // reads zeros
-            for (int r = lane >> 4; r < 9; r += 2) {
-              if (r < 8) {
-                const int b = r >> 1, hf = r & 1;
-                gather4(sbase + C::cring + sc[b] * kCSlot + hf * kHalf + grp * 4 * 128, &ckv_map, cfull_bar(sc[b]),
-                        b * 128 + hf * 64, cur[0], cur[1], cur[2], cur[3]);
-              } else {
-                gather4(sbase + C::kring + sk * kKSlot + grp * 4 * 128, &kpe_map, kfull_bar(sk), 0, cur[0], cur[1],
-                        cur[2], cur[3]);
+            for (int ps = 0; ps < 4; ++ps) idv[ps] = id_next[ps];
+            row_ids(t + 1, id_next);
+            uint32_t seg_base[9];
+#pragma unroll
+            for (int sg = 0; sg < 8; ++sg)
+              seg_base[sg] = sbase + C::cring + ((gc0 + kBlocks * t + (sg >> 1)) % NC) * kCSlot + (sg & 1) * kHalf;
+            seg_base[8] = sbase + C::kring + ((gk0 + t) % NK) * kKSlot;
+#pragma unroll
+            for (int ps = 0; ps < 4; ++ps) {
+              const int row = ps * 16 + rg;
+              const bool in_range = (unsigned)idv[ps] < (unsigned)a.num_pages;
+              if (!in_range) report(a.status, SKV_DEV_PAGE_OOB);
+              const uint8_t* crow = a.ckv_rows + (int64_t)(in_range ? idv[ps] : 0) * a.ckv_row_bytes + sub * 16;
+              const uint8_t* krow = a.kpe_rows + (int64_t)(in_range ? idv[ps] : 0) * a.kpe_row_bytes + sub * 16;
+              const uint32_t nbytes = in_range ? 16u : 0u;
+              const uint32_t off = (uint32_t)row * 128u + ((((uint32_t)sub) ^ ((uint32_t)row & 7u)) << 4);
+#pragma unroll
+              for (int sg = 0; sg < 9; ++sg) {
+                const uint8_t* src = sg < 8 ? crow + sg * 128 : krow;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(seg_base[sg] + off), "l"(src),
+                             "r"(nbytes)
+                             : "memory");
               }
             }
-            load_ids(t + 1, cur);
-            ++gk;
-            gc += kBlocks;
+            asm volatile("cp.async.commit_group;" ::: "memory");
+          };
+          auto release = [&](int t) {  // this thread's copies of tile t have landed
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(kfull_bar((gk0 + t) % NK));
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) tc::mbar_arrive(cfull_bar((gc0 + kBlocks * t + b) % NC));
+          };
+          if (T > 0) {
+            ok = claim(0, true);
+            if (ok) issue(0);
           }
+          // keep the next tile in flight when its slots are already free; never hold tile t's
+          // release behind a wait for tile t + 1's slots
+          for (int t = 0; t < T && ok; ++t) {
+            const bool ahead = t + 1 < T && claim(t + 1, false);
+            if (ahead) {
+              issue(t + 1);
+              asm volatile("cp.async.wait_group 1;" ::: "memory");
+            } else {
+              asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
+            release(t);
+            if (t + 1 < T && !ahead) {
+              ok = claim(t + 1, true);
+              if (ok) issue(t + 1);
+            }
+          }
+          asm volatile("cp.async.wait_group 0;" ::: "memory");
+          gk = gk0 + T;
+          gc = gc0 + kBlocks * T;
           ++n_unit;
           continue;
         }
@@ -326,7 +375,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         ++n_unit;
       }
     }
-    if (!ok && lane == 0) {  // drain issued copies (bounded) before the CTA can exit
+    if (!ok && lane == 0 && !a.gather) {  // drain issued TMA copies (bounded) before the CTA can exit
       for (int q = max(0, gc - NC); q < gc; ++q) {
         const uint64_t t_start = tc::globaltimer_ns();
         while (!tc::mbar_try_wait(cfull_bar(q % NC), (q / NC) & 1) && tc::globaltimer_ns() - t_start < 50000000ull) {
@@ -338,7 +387,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
         }
       }
     }
-  } else if (warp >= 5) {
+  } else if (warp >= 5 && warp < 5 + kIssuers) {
     // ======================================================================= MMA issuers
     // Issuer w: QK quarter w of every tile (rope k-step w + ckv block w: 9 MMAs) into its own
     // partial S^T accumulator, and PV block w (4 MMAs) into O^T block w: four issuing threads on
@@ -699,7 +748,9 @@ int launch_m(const CUtensorMap* maps, const MArgs& a, int num_ctas, const WorkIt
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  mla_tc_kernel<NR, OutT><<<num_ctas, kThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a, work);
+  // the three extra gather warps exist only in row-gather mode
+  const int threads = a.gather ? kThreads : kThreads - (kGatherWarps - 1) * 32;
+  mla_tc_kernel<NR, OutT><<<num_ctas, threads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a, work);
   return (int)cudaGetLastError();
 }
 
@@ -725,14 +776,9 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
   const int total_q = p.batch * p.q_len;
   CUtensorMap maps[4];
   const bool gather = p.page_size == 1;
-  if (gather) {  // token rows: 2-D maps (dims, row = page id), boxes one row high for tile::gather4
-    const cuuint64_t cd[2] = {512, (cuuint64_t)std::max(1, p.num_pages)};
-    const cuuint64_t cs[1] = {(cuuint64_t)p.ckv_stride[0] * 2};
-    const cuuint64_t kd[2] = {64, (cuuint64_t)std::max(1, p.num_pages)};
-    const cuuint64_t ks[1] = {(cuuint64_t)p.kpe_stride[0] * 2};
-    const cuuint32_t box[2] = {64, 1};
-    if (!make_map_m(&maps[0], p.ckv, cd, cs, box, 2) || !make_map_m(&maps[1], p.kpe, kd, ks, box, 2))
-      return (int)cudaErrorInvalidValue;
+  if (gather) {  // rows are fetched by cp.async; the maps are unused but must be valid objects
+    maps[0] = CUtensorMap{};
+    maps[1] = CUtensorMap{};
   }
   if (!gather) {
     const cuuint64_t dims[3] = {512, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
@@ -770,6 +816,10 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
   a.hg = p.num_heads / hc;
   a.q_tile = q_tile;
   a.gather = gather ? 1 : 0;
+  a.ckv_rows = static_cast<const uint8_t*>(p.ckv);
+  a.kpe_rows = static_cast<const uint8_t*>(p.kpe);
+  a.ckv_row_bytes = p.ckv_stride[0] * 2;
+  a.kpe_row_bytes = p.kpe_stride[0] * 2;
   a.scale_log2 = p.sm_scale * kLog2e;
   a.o = p.o;
   a.lse = p.lse;

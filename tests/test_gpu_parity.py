@@ -210,6 +210,52 @@ def test_mla_full_sampled(H, q_len, kv_dtype):
          where=f"mla full {H} {q_len} {kv_dtype}")
 
 
+def _empty_request(c, j):
+    """Remove request j's pages from the page table (an empty KV: O = 0, LSE = -inf)."""
+    a, b = int(c.kv_indptr[j]), int(c.kv_indptr[j + 1])
+    c.kv_indices = np.concatenate([c.kv_indices[:a], c.kv_indices[b:]]).astype(np.int32)
+    c.kv_indptr = c.kv_indptr.copy()
+    c.kv_indptr[j + 1:] -= b - a
+    return c
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("page_size", [16, 128])
+@pytest.mark.parametrize("policy,param", [("none", 0), ("balanced", 148)])
+def test_mla_tensor_core_page_sizes_and_edges(kv_dtype, page_size, policy, param):
+    """Both MLA tensor-core kernels at other page sizes (several pages per 64-token tile, several
+    tiles per page): ragged lengths around tile and page boundaries, an empty request, poisoned
+    unused pages and tails (NaN rope, huge V), split or whole KV."""
+    c = mla_decode_case(16, 1, kv_dtype, batch=5, len_range=(1, 700), page_size=page_size, poison=True, seed=9)
+    c = _empty_request(c, 2)
+    o, lse, ex = _run_mla(c, policy, param)
+    assert ex["plan"].info.kernel == 12
+    O, LSE = _oracle_mla(c)
+    _cmp(_np(o), _np(lse), O, LSE, O_TOL_FP8 if kv_dtype == "e4m3" else O_TOL,
+         where=f"mla edges {kv_dtype} P{page_size} {policy}")
+
+
+@pytest.mark.parametrize("H,q_len", [(16, 1), (16, 2), (128, 1)])
+def test_mla_page_size_one_gather(H, q_len):
+    """Page size 1 (a page id is a token row) on the bf16 tensor-core kernel, rows fetched with
+    tile::gather4: permuted rows, lengths not a multiple of the 64-token tile, an empty request,
+    explicit uneven splits."""
+    c = mla_decode_case(H, q_len, "bf16", batch=4, len_range=(1, 300), page_size=1, poison=True, seed=11)
+    c = _empty_request(c, 1)
+    n = np.diff(c.kv_indptr)
+    sps = [[0] + ([int(n[r]) // 3] if n[r] > 3 else []) + [int(n[r])] for r in range(c.batch)]
+    o, lse, ex = _run_mla(c, "none", 0)
+    assert ex["plan"].info.kernel in (12, 13)
+    O, LSE = _oracle_mla(c)
+    _cmp(_np(o), _np(lse), O, LSE, where=f"mla P1 H{H} q{q_len}")
+    d = mla_to_device(c, DEV)
+    o2, lse2, ex2 = skv.mla_decode(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], c.kv_indptr, d["kv_indices"],
+                                   c.kv_last_page_len, sm_scale=c.sm_scale, kv_scale=c.kv_scale, policy="explicit",
+                                   split_page_start=sps, num_pages=c.num_pages)
+    torch.cuda.synchronize()
+    _cmp(_np(o2), _np(lse2), O, LSE, where=f"mla P1 H{H} q{q_len} explicit splits")
+
+
 # ----------------------------------------------------------------------------- route + merge
 def _route(c):
     d = route_to_device(c, DEV)
