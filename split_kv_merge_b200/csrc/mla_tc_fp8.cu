@@ -16,8 +16,8 @@
 //     scaling goes back into the softmax scale; S and O sum their hi and lo columns.
 //   * S^T[64 tokens, 2 NR] = C . [Q_hi; Q_lo]^T, K = 32 per MMA: 16 ckv k-steps (128-byte
 //     swizzled rows) + 2 rope k-steps (64-byte swizzled rows); M = 64, so TMEM rows sit in lanes
-//     0-15 of each warp quarter.  The k-steps are split over 4 (NR = 16) or 2 (NR = 32) issuers
-//     into partial accumulators that the softmax adds.
+//     0-15 of each warp quarter.  The k-steps are split over two issuers into two partial
+//     accumulators that the softmax adds.
 //   * O^T[512, 2 NR] += V^T . [P_hi; P_lo]^T in four M = 128 blocks (V read MN-major from the same
 //     tile), one block per issuer.
 //   * Online softmax with a lazily raised maximum (only when a score passes it by more than 2^8),
@@ -47,7 +47,7 @@ constexpr float kRaise = 8.f;
 
 template <int NR>
 struct Cfg8 {
-  static constexpr int kQParts = NR == 16 ? 4 : 2;     // QK partial accumulators (issuers 0..)
+  static constexpr int kQParts = 2;                     // QK partial accumulators (issuers 0, 1)
   static constexpr int kStages = NR == 16 ? 4 : 3;     // tiles in flight
   static constexpr int kQStage = NR * 128;             // one 64-column bf16 region of the query copy
   static constexpr int kQOps = 2 * NR * 128;           // one 128-dim region of [Q_hi; Q_lo] (e4m3)
@@ -470,7 +470,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
           ok = tc::mbar_wait_sleep(sfull_bar(sb), (tt >> 1) & 1, abort_flag, a.status) && ok;
           tc::tc_fence_after();
           float s[NR];
-          constexpr int kGrp = NR == 16 ? 2 : 1;  // partial accumulators loaded per TMEM wait
+          constexpr int kGrp = NR == 16 ? 2 : 1;  // partial accumulators loaded per TMEM wait (one wait at 16 rows)
 #pragma unroll
           for (int pp = 0; pp < NQ; pp += kGrp) {  // partial accumulators, hi + lo columns
             float v[kGrp][2 * NR];
