@@ -87,7 +87,11 @@ typedef struct {
   int32_t num_work;         /* work items (CTAs per KV head for GQA, per split for MLA)       */
   int32_t num_partial_rows; /* rows the o_part / lse_part buffers must hold (0: no split)     */
   int32_t num_merge_rows;   /* output rows combined from >1 split by the merge pass           */
-  int32_t kernel;           /* kernel variant the dispatcher picked (informational)           */
+  int32_t kernel;           /* kernel variant the dispatcher picked (informational): 1 GQA on  */
+                            /*   CUDA cores, 2 GQA tensor-core decode per KV head, 3 GQA      */
+                            /*   tensor-core decode over all KV heads, 4 GQA tensor-core      */
+                            /*   prefill (128 query rows), 11 MLA on CUDA cores, 12 / 13 MLA  */
+                            /*   tensor cores with 16 / 32 query rows per tile                */
   int32_t q_tile;           /* query tokens per work item (MLA: the fold ratio F)             */
   int32_t plan_words;       /* int32 words of the plan actually used                          */
   int32_t max_splits;       /* largest split count of any request                             */
@@ -191,7 +195,9 @@ SKV_API skv_status skv_paged_attn_fwd_static_scratch(const skv_paged_params* p, 
  *   tokens folded into the query-row dimension of a work item) is reported in info->q_tile:
  *   F = skv_mla_fold_ratio(H, q_len, R) with R the rows the chosen kernel puts on one tile
  *   (16 or 32 for the tensor-core kernel, which splits H > R heads into groups of R; 128 for
- *   the CUDA-core kernel).
+ *   the CUDA-core kernel).  The tensor-core kernels take page sizes >= 8 that divide or are
+ *   multiples of 64, and (bf16 cache only) page size 1, where every page id is a token row; other
+ *   page sizes run on the CUDA-core kernel.  Run a plan on the kv_dtype it was made for.
  * ----------------------------------------------------------------------------------------- */
 SKV_API skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
                         const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_heads,
