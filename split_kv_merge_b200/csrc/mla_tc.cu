@@ -1,4 +1,5 @@
-// MLA latent decode on the tensor cores (tcgen05 + TMEM), bf16 latent cache, TMA page staging.
+// MLA latent decode on the tensor cores (tcgen05 + TMEM), bf16 latent cache: TMA page staging, or
+// for page size 1 (route: every page id is a token row) a cp.async row gather.
 //
 // What it computes (FlashInfer PR #3309 page, MLA decode): every head reads one latent row per
 // token -- a 512-d compressed KV (ckv) and a 64-d rope key (kpe); s = scale (q_nope . ckv +
@@ -13,17 +14,21 @@
 //     0-15 of each warp quarter; the 16-32 query rows are far too few for M);
 //   * O^T[512, NR] += V^T[512, 64] . P^T[64, NR]  in four M = 128 blocks of head dims, V read
 //     MN-major from the same shared tiles, O^T accumulated in TMEM across the tiles of a unit.
-//   * Two TMA rings: ckv in 16 KB slots, each one 128-dim V block of a tile (two 64-column
-//     swizzled halves), released after that block's PV; kpe in 8 KB slots released after QK.
+//   * Two rings: ckv in 16 KB slots, each one 128-dim V block of a tile (two 64-column swizzled
+//     halves), released after that block's PV; kpe in 8 KB slots released after QK.  Paged
+//     caches fill them with TMA boxes (page windows, issued from nine lanes); page size 1 fills
+//     them with 16-byte cp.async from four warps, eight lanes per 128-byte row segment.
 //   * Online softmax with a lazily raised maximum (only when a score passes the running max by
-//     more than 2^8): the column max over the 64 token lanes is a 16-lane shuffle + 4-warp
-//     exchange paid only on a raise; O^T is rescaled in TMEM by all four softmax warps then.
+//     more than 2^8): the column max is a warp redux + 4-warp exchange paid only on a raise; O^T
+//     is rescaled in TMEM by all four softmax warps then.  P^T goes to shared memory MN-major,
+//     the two 16-lane halves of a warp writing the two halves of each token's rows.
 //   * Tokens past the end of the unit get s = -inf by selection and their V rows are zeroed in
 //     the held tile before the PV that reads them.
-// Roles: warp 4 TMA producer; warps 5-8 MMA issue, one per SM sub-partition (an MMA whose operands
-// stream from shared memory holds its issuing thread for ~80 cycles, and issuers on different
-// sub-partitions overlap): issuer w computes QK quarter w into its own partial S^T accumulator and
-// PV block w; warp 5 also allocates TMEM; warps 0-3 softmax / epilogue.
+// Roles: warp 4 producer (with warps 9-11 in row-gather mode); warps 5-8 MMA issue, one per SM
+// sub-partition (an MMA whose operands stream from shared memory holds its issuing thread for ~80
+// cycles, and issuers on different sub-partitions overlap): issuer w computes QK quarter w into its
+// own partial S^T accumulator and PV block w; warp 5 also allocates TMEM; warps 0-3 softmax /
+// epilogue.
 // All waits are bounded (SKV_DEV_TIMEOUT); roles leave together; TMEM is always released.
 #include <cudaTypedefs.h>
 
