@@ -38,7 +38,7 @@ constexpr int kStages = 2;
 constexpr int kRegion = kTile * 128;            // 16 KB: one 64-column half of a 128 x 128 tile
 constexpr int kKBytes = 2 * kRegion;            // 32 KB
 constexpr int kStageBytes = 2 * kKBytes;        // K + V
-constexpr int kThreads = 224;
+constexpr int kThreads = 352;  // softmax warps 0-3 and 7-10, TMA warp 4, QK warp 5, PV warp 6
 constexpr float kRaise = 8.f;
 
 struct Smem {
@@ -47,7 +47,8 @@ struct Smem {
   static constexpr int p = q + kKBytes;                   // 163840
   static constexpr int bars = p + 2 * kKBytes;            // 229376
   static constexpr int nbars = 2 * kStages + 1 + 2 * 4;
-  static constexpr int misc = bars + nbars * 8;
+  static constexpr int xch = bars + nbars * 8;            // [2][128] float: per-row exchange between halves
+  static constexpr int misc = xch + 2 * 128 * 4;
   static constexpr int total = misc + 16;
 };
 static_assert(Smem::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
@@ -150,8 +151,8 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     tc::mbar_init(qfull_bar(), 1);
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(sfull_bar(b), 1);
-      tc::mbar_init(sempty_bar(b), 4);
-      tc::mbar_init(pfull_bar(b), 4);
+      tc::mbar_init(sempty_bar(b), 8);
+      tc::mbar_init(pfull_bar(b), 8);
       tc::mbar_init(ofull_bar(b), 1);
     }
     *abort_flag = 0;
@@ -253,10 +254,17 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         tc::mma_commit(empty_bar(st));
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 4 || warp >= 7) {
     // ======================================================================= softmax / epilogue
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int r = tid;                       // this thread's query row
+    // Each row is split over two warps on the same TMEM lane quarter (warp w and warp w + 8, or
+    // 3 and 7): half hf takes keys [64 hf, 64 hf + 64) of every tile and head dims [64 hf,
+    // 64 hf + 64) of O; the two threads of a row exchange row maxima and sums through shared
+    // memory with a 64-thread named barrier per pair.
+    const int quarter = warp & 3, hf = warp < 4 ? 0 : 1;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int r = quarter * 32 + lane;       // this thread's query row
+    float* xch = reinterpret_cast<float*>(smem + Smem::xch);
+    auto pair_sync = [&]() { tc::named_bar_sync(1 + quarter, 64); };
     // l: sum of the exact weights (for the LSE); lr: of the bf16-rounded weights PV multiplies (the
     // divisor of O, so that a row dominated by one key reproduces that key's V)
     float m = -INFINITY, l = 0.f, lr = 0.f;
@@ -271,11 +279,12 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       const int sb = t & 1, st = t % kStages;
       ok = tc::mbar_wait(sfull_bar(sb), (t >> 1) & 1, abort_flag, a.status) && ok;
       tc::tc_fence_after();
-      float s[kTile];
+      constexpr int kH = kTile / 2;           // keys of this half
+      float s[kH];
 #pragma unroll
-      for (int c = 0; c < kTile; c += 16) {  // all loads in flight, one wait
+      for (int c = 0; c < kH; c += 16) {  // all loads in flight, one wait
         float v16[16];
-        tc::tmem_ld_x16(tm_s + lane_base + sb * kTile + c, v16);
+        tc::tmem_ld_x16(tm_s + lane_base + sb * kTile + hf * kH + c, v16);
 #pragma unroll
         for (int i = 0; i < 16; ++i) s[c + i] = v16[i];
       }
@@ -283,22 +292,27 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(sempty_bar(sb));
-      const int nvalid = t1 - (t0 + t * kTile);   // keys of this tile that exist (>= 1)
-      if (nvalid < kTile) {                       // the item's last tile only
+      const int nvalid = t1 - (t0 + t * kTile) - hf * kH;  // keys of this half that exist (may be <= 0)
+      if (nvalid < kH) {                                    // the item's last tile only
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) s[c] = c < nvalid ? s[c] : -INFINITY;
+        for (int c = 0; c < kH; ++c) s[c] = c < nvalid ? s[c] : -INFINITY;
       }
       float mx;
-      {  // raw row maximum in 8 independent chains (the scale is positive: scale after)
-        float q[8];
+      {  // raw row maximum in 4 independent chains (the scale is positive: scale after), then the
+         // other half's through shared memory
+        float q[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           float v = fmax3(s[16 * j], s[16 * j + 1], s[16 * j + 2]);
 #pragma unroll
           for (int i = 3; i < 15; i += 2) v = fmax3(v, s[16 * j + i], s[16 * j + i + 1]);
           q[j] = fmaxf(v, s[16 * j + 15]);
         }
-        mx = fmax3(fmax3(q[0], q[1], q[2]), fmax3(q[3], q[4], q[5]), fmaxf(q[6], q[7])) * a.scale_log2;
+        mx = fmaxf(fmaxf(q[0], q[1]), fmaxf(q[2], q[3])) * a.scale_log2;
+        xch[hf * 128 + r] = mx;
+        pair_sync();
+        mx = fmaxf(mx, xch[(1 - hf) * 128 + r]);
+        pair_sync();  // both reads done before the next tile's writes
       }
       const bool raise = mx > m + kRaise;
       if (__any_sync(0xffffffffu, raise)) {  // warp-uniform: TMEM access below is warp-collective
@@ -310,23 +324,24 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         if (t > 0) {  // rescale this row of O once the previous PV is done
           consume_pv(t - 1);
 #pragma unroll
-          for (int c = 0; c < kD; c += 16) {
+          for (int c = 0; c < kD / 2; c += 16) {  // this half's head dims of the row
             float ov[16];
-            tc::tmem_ld_x16(tm_o + lane_base + c, ov);
+            tc::tmem_ld_x16(tm_o + lane_base + hf * (kD / 2) + c, ov);
             tc::tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) ov[i] *= al;
-            tc::tmem_st_x16(tm_o + lane_base + c, ov);
+            tc::tmem_st_x16(tm_o + lane_base + hf * (kD / 2) + c, ov);
           }
           tc::tmem_wait_st();
           tc::tc_fence_before();
         }
       }
-      if (nvalid < kTile) {  // zero V rows of missing keys (each thread its share of the rows)
+      const int nvalid_tile = t1 - (t0 + t * kTile);
+      if (nvalid_tile < kTile) {  // zero V rows of missing keys (each thread its share of the rows)
         // the tile's copies have landed (the QK that read them is done); make that visible here
         ok = tc::mbar_wait(full_bar(st), (t / kStages) & 1, abort_flag, a.status) && ok;
         uint8_t* vb = smem + Smem::kv + st * kStageBytes + kKBytes;
-        for (int row = nvalid + (tid & 127); row < kTile; row += 128)
+        for (int row = nvalid_tile + hf * 128 + r; row < kTile; row += 256)
 #pragma unroll
           for (int rgn = 0; rgn < 2; ++rgn)
 #pragma unroll
@@ -340,7 +355,7 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       const uint64_t sc2 = pk2(a.scale_log2, a.scale_log2), nm2 = pk2(-m, -m);
       uint64_t la[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)}, lb[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kTile; c += 8) {
+      for (int c = 0; c < kH; c += 8) {
         uint32_t pk[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -352,8 +367,8 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
           la[i & 1] = add2(la[i & 1], pk2(p0, p1));
           lb[i & 1] = add2(lb[i & 1], pk2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u)));
         }
-        // row r, keys c..c+7: region c/64, 16-byte chunk (c%64)/8 swizzled by r%8
-        const uint32_t off = (uint32_t)((c >> 6) * kRegion + r * 128 + (((((c & 63) >> 3) ^ (r & 7)) & 7) << 4));
+        // row r, keys 64 hf + c .. + 7: region hf, 16-byte chunk c / 8 swizzled by r % 8
+        const uint32_t off = (uint32_t)(hf * kRegion + r * 128 + ((((c >> 3) ^ (r & 7)) & 7) << 4));
         *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       {
@@ -368,6 +383,13 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       if (lane == 0) tc::mbar_arrive(pfull_bar(t & 1));
     }
     consume_pv(T - 1);
+    xch[hf * 128 + r] = l;  // row sums: exact weights, then rounded weights, over both halves
+    pair_sync();
+    l += xch[(1 - hf) * 128 + r];
+    pair_sync();
+    xch[hf * 128 + r] = lr;
+    pair_sync();
+    lr += xch[(1 - hf) * 128 + r];
     const bool live = r < rows;
     const int qi = r / a.g, h = kh * a.g + r % a.g;
     const float inv = lr > 0.f ? 1.f / lr : 0.f;
@@ -376,18 +398,18 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     if (live) {
       const float lse = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
       if (w.part_row < 0) {
-        oo = reinterpret_cast<OutT*>(a.o) + ((int64_t)(w.q_start + qi) * a.hq + h) * kD;
-        if (a.lse != nullptr) a.lse[(int64_t)(w.q_start + qi) * a.hq + h] = lse;
+        oo = reinterpret_cast<OutT*>(a.o) + ((int64_t)(w.q_start + qi) * a.hq + h) * kD + hf * (kD / 2);
+        if (a.lse != nullptr && hf == 0) a.lse[(int64_t)(w.q_start + qi) * a.hq + h] = lse;
       } else {
         const int64_t prow = (int64_t)w.part_row + (int64_t)qi * w.part_stride;
-        op = a.o_part + (prow * a.hq + h) * kD;
-        a.lse_part[prow * a.hq + h] = lse;
+        op = a.o_part + (prow * a.hq + h) * kD + hf * (kD / 2);
+        if (hf == 0) a.lse_part[prow * a.hq + h] = lse;
       }
     }
 #pragma unroll
-    for (int c = 0; c < kD; c += 16) {  // every lane loads (warp-collective); live rows store
+    for (int c = 0; c < kD / 2; c += 16) {  // every lane loads (warp-collective); live rows store
       float ov[16];
-      tc::tmem_ld_x16(tm_o + lane_base + c, ov);
+      tc::tmem_ld_x16(tm_o + lane_base + hf * (kD / 2) + c, ov);
       tc::tmem_wait_ld();
       if (op != nullptr) {
 #pragma unroll
