@@ -34,7 +34,7 @@ namespace {
 constexpr int kTile = 128;                      // keys per tile
 constexpr int kRows = 128;                      // query rows per CTA
 constexpr int kD = 128;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kRegion = kTile * 128;            // 16 KB: one 64-column half of a 128 x 128 tile
 constexpr int kKBytes = 2 * kRegion;            // 32 KB
 constexpr int kStageBytes = 2 * kKBytes;        // K + V
@@ -43,15 +43,26 @@ constexpr float kRaise = 8.f;
 
 struct Smem {
   static constexpr int kv = 0;
-  static constexpr int q = kv + kStages * kStageBytes;    // 131072
-  static constexpr int p = q + kKBytes;                   // 163840
-  static constexpr int bars = p + 2 * kKBytes;            // 229376
+  static constexpr int q = kv + kStages * kStageBytes;    // 196608
+  static constexpr int bars = q + kKBytes;                // 229376 (P lives in TMEM)
   static constexpr int nbars = 2 * kStages + 1 + 2 * 4;
   static constexpr int xch = bars + nbars * 8;            // [2][128] float: per-row exchange between halves
   static constexpr int misc = xch + 2 * 128 * 4;
   static constexpr int total = misc + 16;
 };
 static_assert(Smem::total + 1024 <= 232448, "fits the 227 KB opt-in shared memory");
+
+// D[tmem] (+)= A[tmem] . B[smem], kind::f16: A rows in TMEM lanes, two bf16 per 32-bit column
+// (the even k in the low half)
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 // packed f32 pairs (sm_100 f32x2 arithmetic), 3-input max, hardware exp2
 __device__ __forceinline__ uint64_t pk2(float a, float b) {
@@ -163,7 +174,8 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tm_s = tmem, tm_o = tmem + 2 * kTile;   // S0, S1 (128 cols each), O (128 cols)
+  // TMEM: S0, S1 (128 fp32 columns each), O (128), P0, P1 (64 columns each: 128 bf16 keys per row)
+  const uint32_t tm_s = tmem, tm_o = tmem + 2 * kTile, tm_p = tmem + 3 * kTile;
 
   if (warp == 4) {
     // ======================================================================= TMA producer
@@ -243,12 +255,10 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         if (!ok) break;
         tc::tc_fence_after();
         const uint32_t vs = sbase + Smem::kv + st * kStageBytes + kKBytes;
-        const uint32_t ps = sbase + Smem::p + pb * kKBytes;
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k) {
-          const uint64_t ad = tc::sdesc_sw128(ps + (k >> 2) * kRegion + (k & 3) * 32, 16, 1024);
+        for (int k = 0; k < kTile / 16; ++k) {  // A = P from TMEM: 16 keys = 8 packed columns
           const uint64_t bd = tc::sdesc_sw128(vs + k * 2048, kRegion, 1024);
-          tc::mma_bf16(tm_o, ad, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+          mma_bf16_ts(tm_o, tm_p + pb * (kTile / 2) + k * 8, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
         }
         tc::mma_commit(ofull_bar(pb));
         tc::mma_commit(empty_bar(st));
@@ -349,27 +359,21 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
               reinterpret_cast<uint4*>(vb + rgn * kRegion + row * 128)[i] = make_uint4(0, 0, 0, 0);
       }
       if (t >= 2 && pv_seen <= t - 2) consume_pv(t - 2);  // P(t) reuses the buffer PV(t-2) read
-      uint8_t* prow = smem + Smem::p + (t & 1) * kKBytes;
-      // p = 2^(s * scale - m) (ex2 of -inf is +0); sums of the exact and of the rounded weights in
-      // packed pairs, two chains each
+      // p = 2^(s * scale - m) (ex2 of -inf is +0), bf16 pairs into this row's P columns in TMEM; sums
+      // of the exact and of the rounded weights in packed pairs, two chains each
       const uint64_t sc2 = pk2(a.scale_log2, a.scale_log2), nm2 = pk2(-m, -m);
       uint64_t la[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)}, lb[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)};
+      float pw[kH / 2];  // packed bf16 pairs (bit patterns)
 #pragma unroll
-      for (int c = 0; c < kH; c += 8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float x0, x1;
-          upk2(fma2(pk2(s[c + 2 * i], s[c + 2 * i + 1]), sc2, nm2), x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-          la[i & 1] = add2(la[i & 1], pk2(p0, p1));
-          lb[i & 1] = add2(lb[i & 1], pk2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u)));
-        }
-        // row r, keys 64 hf + c .. + 7: region hf, 16-byte chunk c / 8 swizzled by r % 8
-        const uint32_t off = (uint32_t)(hf * kRegion + r * 128 + ((((c >> 3) ^ (r & 7)) & 7) << 4));
-        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int c = 0; c < kH; c += 2) {
+        float x0, x1;
+        upk2(fma2(pk2(s[c], s[c + 1]), sc2, nm2), x0, x1);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+        const uint32_t u = *reinterpret_cast<uint32_t*>(&h2);
+        pw[c >> 1] = __uint_as_float(u);
+        la[(c >> 1) & 1] = add2(la[(c >> 1) & 1], pk2(p0, p1));
+        lb[(c >> 1) & 1] = add2(lb[(c >> 1) & 1], pk2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u)));
       }
       {
         float a0, a1, b0, b1;
@@ -378,7 +382,17 @@ gqa_tc_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         l += a0 + a1;
         lr += b0 + b1;
       }
-      tc::fence_proxy_async_smem();
+      const uint32_t pcol = tm_p + (t & 1) * (kTile / 2) + hf * (kH / 2);
+#pragma unroll
+      for (int c = 0; c < kH / 2; c += 16) {
+        float w16[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w16[i] = pw[c + i];
+        tc::tmem_st_x16(pcol + lane_base + c, w16);
+      }
+      tc::tmem_wait_st();
+      tc::fence_proxy_async_smem();  // V rows zeroed above are read by the PV MMA
+      tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(pfull_bar(t & 1));
     }
