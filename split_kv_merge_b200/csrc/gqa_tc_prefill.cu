@@ -12,13 +12,16 @@
 // B200 design: the standard (non-swapped) flash-attention tile with 128 query rows as M:
 //   S[128 rows, 128 keys] = Q[128, 128] . K^T      (rows = (query token, head of the group))
 //   O[128 rows, 128]     += P[128, 128 keys] . V  (V read MN-major from the same TMA tile)
-// S (double buffered) and O live in TMEM; P goes through shared memory as the A operand.  One
-// thread owns one row, so the row max / sum need no exchange; the running max is raised lazily
-// (only when a score passes it by more than 2^8) and O's row is rescaled in TMEM by its own
-// thread (warp-uniform decision, since TMEM access is warp-collective).  Roles: warp 4 TMA (2-stage
-// ring of 128-key K and V tiles, 3-D Q box), warp 5 TMEM + QK MMA issue, warp 6 PV MMA issue,
-// warps 0-3 softmax / epilogue.  Keys past the end of the item get s = -inf by selection and
-// their V rows are zeroed before the PV that reads them.  All waits are bounded.
+// S (double buffered), O and P (double buffered, bf16 pairs) all live in TMEM: the softmax writes
+// P with tcgen05.st and the PV MMA reads it as its A operand straight from TMEM, so P never
+// touches shared memory, which holds three 64 KB K+V stages instead.  A row is owned by two
+// threads of two warps on the same TMEM lane quarter (keys [64 hf, 64 hf + 64) of every tile and
+// head dims [64 hf, 64 hf + 64) of O each), exchanging row maxima and sums through shared memory;
+// the running max is raised lazily (only when a score passes it by more than 2^8) and O is
+// rescaled in TMEM (warp-uniform decision, since TMEM access is warp-collective).  Roles: warp 4
+// TMA (3-stage ring of 128-key K and V tiles, 3-D Q box), warp 5 TMEM + QK MMA issue, warp 6 PV
+// MMA issue, warps 0-3 and 7-10 softmax / epilogue.  Keys past the end of the item get s = -inf by
+// selection and their V rows are zeroed before the PV that reads them.  All waits are bounded.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
