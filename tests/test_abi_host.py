@@ -258,3 +258,36 @@ def test_mla_planner_kernel_choice(H, q_len, kv_dtype, page_size, kernel):
     assert plan.info.kernel == kernel
     rows = {12: 16, 13: 32}.get(kernel, 128)
     assert plan.info.q_tile == (skv.mla_fold_ratio(H, q_len, rows) if H <= rows else 1)
+
+
+@pytest.mark.parametrize("H,q_len", [(16, 1), (16, 4), (128, 1), (128, 4)])
+def test_mla_flat_plan_balances_tiles_and_pieces(H, q_len):
+    """The persistent MLA plan charges every work item a fixed cost (four 64-token tiles per query
+    unit: head groups x query tiles) on top of its tiles; per CTA, tiles + charges stay within a
+    few tiles of the mean, every page of every request is covered once, and no CTA is left with
+    the remainder of a degenerate cut."""
+    from workloads import mla_decode_case
+    c = mla_decode_case(H, q_len, "bf16")
+    plan = skv.plan_mla(q_len, c.kv_indptr, c.kv_last_page_len, 64, H, "balanced", 148, kv_dtype="bf16")
+    info = plan.info
+    assert info.kernel in (12, 13) and info.num_ctas == 148
+    rows = {12: 16, 13: 32}[info.kernel]
+    hg = H // rows if H > rows else 1
+    qt = -(-q_len // info.q_tile) * hg                       # query units per piece
+    w, _ = _items(plan)
+    cta = plan.words[info.cta_offset: info.cta_offset + info.num_ctas + 1]
+    L = c.kv_lengths()
+    n = np.diff(c.kv_indptr)
+    cost = []
+    for i in range(info.num_ctas):
+        items = w[cta[i]:cta[i + 1]]
+        # work items of one request piece differ only by query tile: count pieces once
+        pieces = {(int(r), int(a), int(b)) for r, _, _, a, b, *_ in items}
+        tiles = sum(-(-(min(b * 64, L[r]) - a * 64) // 64) for r, a, b in pieces)
+        cost.append(hg * tiles * -(-q_len // info.q_tile) + 4 * qt * len(pieces))
+    cost = np.array(cost)
+    assert cost.max() <= cost.mean() + 8 * qt + 8 * hg, (cost.max(), cost.mean())
+    for r in range(c.batch):
+        spans = sorted({(int(a), int(b)) for rr, _, _, a, b, *_ in w if rr == r})
+        assert spans[0][0] == 0 and spans[-1][1] == n[r]
+        assert all(spans[i][1] == spans[i + 1][0] for i in range(len(spans) - 1))
