@@ -430,8 +430,8 @@ def run_workload(args):
     resident; KV working sets above L2 except the tiny and shared-KV cases, which are noted)."""
     import torch
     import split_kv_merge_b200 as skv
-    from workloads import mla_decode_case, route_case, shared_kv_prefill_case, tiny_gqa_case
-    from workloads.device import mla_to_device, paged_to_device, route_to_device
+    from workloads import fetch_splice_case, mla_decode_case, route_case, shared_kv_prefill_case, tiny_gqa_case
+    from workloads.device import mla_to_device, paged_to_device, route_to_device, splice_to_device
     peaks, src = _peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]))
     tf = float(peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]))
@@ -440,7 +440,7 @@ def run_workload(args):
     names = args.workload.split(",")
     if names == ["all"]:
         names = ["tiny", "shared_kv"] + [f"mla_h{h}_q{q}_{d}" for h in (16, 128) for q in (1, 4)
-                                         for d in ("bf16", "e4m3")] + ["route"]
+                                         for d in ("bf16", "e4m3")] + ["route", "fetch_splice"]
     for name in names:
         line = {"workload": name, "peaks": src}
         if name in ("tiny", "shared_kv"):
@@ -494,6 +494,19 @@ def run_workload(args):
             kv_bytes = int(c.sel.size) * 1152              # gathered rows
             flops = float(c.sel.size) * c.num_heads * 2 * (576 + 512)
             line["kernel"] = rm.plan.info.kernel
+        elif name == "fetch_splice":
+            # fetch's local compute: every chunk of the route corpus moved into a requester's paged
+            # cache and re-rotated (all chunks in one call); bytes = each row read once and written once
+            c = fetch_splice_case()
+            d = splice_to_device(c, dev)
+            sp = skv.splice_params(d["src_ckv"], d["src_kpe"], d["src_pages"], d["dst_ckv"], d["dst_kpe"],
+                                   d["dst_pages"], rope_theta=c.rope_theta)
+            chunks = skv.splice_chunks([(int(c.src_start[ch]), int(c.dst_start[ch]), c.chunk_tokens, int(c.delta[ch]))
+                                        for ch in range(c.num_chunks)])
+            step = lambda: skv.splice_launch(sp, chunks, stream)
+            kv_bytes = 2 * c.num_chunks * c.chunk_tokens * 1152
+            flops = 0.0
+            line["kernel"] = "splice"
         else:
             raise SystemExit(f"unknown workload {name}")
         ms = _time_device(step, args.steps, args.warmup, torch, stream)
@@ -521,7 +534,7 @@ def main():
                                                           "smaller only for profiler captures)")
     ap.add_argument("--workload", default="llama70b",
                     help="llama70b (the benchmark line) | tiny | shared_kv | mla_h{16,128}_q{1,4}_{bf16,e4m3} | "
-                         "route | all (one line per configuration)")
+                         "route | fetch_splice | all (one line per configuration)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -16,6 +16,10 @@
  *                       partial attention at the KV holder merged "via online softmax",
  *                       "Move the Query, Not the Cache", Methodology; in-CTA split with
  *                       shared-memory merge, FlashInfer PR #5597 page, section 3).
+ *   skv_mla_splice      The fetch primitive's local compute: move a chunk's latent rows between
+ *                       page lists and re-rotate their RoPE part to the new positions ("Move
+ *                       the Query, Not the Cache", problem statement and Methodology: fetch
+ *                       adapts cached position encodings to new offsets, the "splice").
  *
  * Semantics shared by all calls (natural-log LSE of the scaled logits):
  *   s_t = sm_scale * q . k_t ;  O = sum_t softmax(s)_t v_t ;  LSE = ln sum_t exp(s_t).
@@ -257,6 +261,69 @@ SKV_API skv_status skv_merge_states(const float* o_states, const float* lse_stat
                             const int32_t* state_indptr, int32_t num_states, int64_t num_rows,
                             int32_t num_heads, int32_t head_dim, void* o_out, int32_t o_dtype,
                             float* lse_out, skv_stream_t stream);
+
+/* -------------------------------------------------------------------------------------------
+ * skv_mla_splice -- the fetch primitive's local compute.  "Move the Query, Not the Cache"
+ *   (Methodology, primitive comparison): fetch brings a whole KV chunk to the requester, adapts
+ *   its positions ("splice") and attends locally; the problem statement describes the
+ *   adaptation as re-rotating cached position encodings to new offsets.
+ *
+ *   For each chunk c and token t in [0, chunks_h[c].n_tokens): the latent row at logical
+ *   position chunks_h[c].src_start + t of the source page list (page
+ *   src_pages[pos / src_page_size], slot pos % src_page_size) is written at logical position
+ *   chunks_h[c].dst_start + t of the destination page list (same rule with the dst_ fields).
+ *   The 512-d latent (ckv) is copied bit for bit.  The 64-d rope part (kpe) holds keys rotated
+ *   to their old positions; each of its 32 pairs (a, b) turns by delta_pos * theta_i, with the
+ *   chunk's delta_pos (new position - old position):  a' = a cos - b sin, b' = a sin + b cos;
+ *   theta_i = inv_freq[i] when inv_freq (device, 32 floats) is given, else
+ *   rope_theta^(-2i/64).  Pairs are (2i, 2i+1) for SKV_ROPE_INTERLEAVED and (i, i+32) for
+ *   SKV_ROPE_HALVES.  Angles are formed in fp64, the rotation in fp32, results rounded to bf16
+ *   (nearest even).  All chunks of one call run in one launch (up to 64 chunks per launch).
+ *
+ *   Caches: bf16 only (kv_dtype SKV_BF16; anything else is SKV_ERR_UNSUPPORTED).  Layout as in
+ *   skv_mla_params: ckv(page, slot, d) = ckv[page*stride[0] + slot*stride[1] + d], strides in
+ *   elements and multiples of 8 (16 bytes), base pointers 16-byte aligned (SKV_ERR_ALIGNMENT).
+ *   The page lists must cover every position a chunk names.  A row may be read and written by
+ *   the same token (an in-place re-rotation, source = destination); otherwise no row written by
+ *   the call may be read or written by any other token of the call.  A page id outside
+ *   [0, *_num_pages) reports SKV_DEV_PAGE_OOB in *status and that token is skipped.  Chunks
+ *   with no tokens are allowed; a call with none launches nothing.  chunks_h is a host array
+ *   that the call reads before it returns.
+ * ----------------------------------------------------------------------------------------- */
+#define SKV_ROPE_INTERLEAVED 0
+#define SKV_ROPE_HALVES 1
+
+typedef struct {
+  const void* src_ckv;        /* bf16 latent rows of the source pages                          */
+  const void* src_kpe;        /* bf16 rope rows of the source pages                            */
+  int64_t src_ckv_stride[2];  /* (page, slot) strides in elements                              */
+  int64_t src_kpe_stride[2];
+  const int32_t* src_pages;   /* source page list                                              */
+  int32_t src_num_pages;      /* page ids must lie in [0, src_num_pages)                      */
+  int32_t src_page_size;
+  void* dst_ckv;
+  void* dst_kpe;
+  int64_t dst_ckv_stride[2];
+  int64_t dst_kpe_stride[2];
+  const int32_t* dst_pages;
+  int32_t dst_num_pages;
+  int32_t dst_page_size;
+  float rope_theta;           /* frequency base when inv_freq is NULL (> 0)                    */
+  int32_t rope_layout;        /* SKV_ROPE_INTERLEAVED or SKV_ROPE_HALVES                       */
+  const float* inv_freq;      /* optional device [32] per-pair frequencies                     */
+  int32_t kv_dtype;           /* SKV_BF16                                                      */
+  int32_t* status;            /* optional device status word                                   */
+} skv_splice_params;
+
+typedef struct {
+  int64_t src_start;          /* logical position of the chunk's first token, source list     */
+  int64_t dst_start;          /* logical position of its first token, destination list        */
+  int64_t n_tokens;
+  int64_t delta_pos;          /* new position - old position of every token of the chunk      */
+} skv_splice_chunk;
+
+SKV_API skv_status skv_mla_splice(const skv_splice_params* p, const skv_splice_chunk* chunks_h,
+                                  int32_t num_chunks, skv_stream_t stream);
 
 /* -------------------------------------------------------------------------------------------
  * skv_paged_kv_gather -- test hook for the page-table walk: copies the logical K and V of every

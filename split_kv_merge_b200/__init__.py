@@ -7,7 +7,7 @@ there is no fallback path.
 
 Functions mirror the C ABI in include/splitkv.h:
 ``plan_paged``, ``paged_attn_fwd``, ``plan_mla``, ``mla_decode_fwd``, ``merge_states``,
-``paged_kv_gather``, ``mla_fold_ratio``, ``status_str``, ``version``.
+``paged_kv_gather``, ``mla_splice``, ``mla_fold_ratio``, ``status_str``, ``version``.
 """
 from __future__ import annotations
 
@@ -27,6 +27,8 @@ _lib = ctypes.CDLL(_LIB_PATH)
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA = range(6)
 DEV_OK, DEV_TIMEOUT, DEV_PAGE_OOB, DEV_PLAN_BAD = 0, 16, 17, 18
 BF16, F32, E4M3 = 0, 1, 2
+ROPE_INTERLEAVED, ROPE_HALVES = 0, 1
+_ROPE = {"interleaved": ROPE_INTERLEAVED, "halves": ROPE_HALVES}
 SPLIT_NONE, SPLIT_FIXED, SPLIT_BALANCED, SPLIT_EXPLICIT = 0, 1, 2, 3
 _POLICY = {"none": SPLIT_NONE, "fixed": SPLIT_FIXED, "balanced": SPLIT_BALANCED, "explicit": SPLIT_EXPLICIT}
 
@@ -67,6 +69,22 @@ class MlaParams(ctypes.Structure):
                 ("status", _vp)]
 
 
+class SpliceParams(ctypes.Structure):
+    _fields_ = [("src_ckv", _vp), ("src_kpe", _vp),
+                ("src_ckv_stride", ctypes.c_int64 * 2), ("src_kpe_stride", ctypes.c_int64 * 2),
+                ("src_pages", _vp), ("src_num_pages", ctypes.c_int32), ("src_page_size", ctypes.c_int32),
+                ("dst_ckv", _vp), ("dst_kpe", _vp),
+                ("dst_ckv_stride", ctypes.c_int64 * 2), ("dst_kpe_stride", ctypes.c_int64 * 2),
+                ("dst_pages", _vp), ("dst_num_pages", ctypes.c_int32), ("dst_page_size", ctypes.c_int32),
+                ("rope_theta", ctypes.c_float), ("rope_layout", ctypes.c_int32), ("inv_freq", _vp),
+                ("kv_dtype", ctypes.c_int32), ("status", _vp)]
+
+
+class SpliceChunk(ctypes.Structure):
+    _fields_ = [("src_start", ctypes.c_int64), ("dst_start", ctypes.c_int64), ("n_tokens", ctypes.c_int64),
+                ("delta_pos", ctypes.c_int64)]
+
+
 def _proto(name, res, args):
     f = getattr(_lib, name)
     f.restype = res
@@ -97,6 +115,8 @@ _merge = _proto("skv_merge_states", ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int32
                                                     ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp])
 _gather = _proto("skv_paged_kv_gather", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp, ctypes.c_int64, _vp,
                                                         _vp, _vp])
+_splice = _proto("skv_mla_splice", ctypes.c_int, [ctypes.POINTER(SpliceParams), ctypes.POINTER(SpliceChunk),
+                                                   ctypes.c_int32, _vp])
 _wait_timeout = _proto("skv_test_wait_timeout", ctypes.c_int, [_vp, ctypes.c_int64, _vp])
 _fold = _proto("skv_mla_fold_ratio", ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32])
 _status_str = _proto("skv_status_str", ctypes.c_char_p, [ctypes.c_int32])
@@ -105,7 +125,7 @@ _version = _proto("skv_version", ctypes.c_int32, [])
 SYMBOLS = ["skv_plan_paged", "skv_paged_attn_fwd", "skv_paged_attn_partial", "skv_merge_plan", "skv_plan_mla",
            "skv_mla_decode_fwd", "skv_mla_decode_partial", "skv_merge_states", "skv_paged_kv_gather",
            "skv_mla_fold_ratio", "skv_status_str", "skv_version", "skv_paged_attn_fwd_static_scratch",
-           "skv_test_wait_timeout"]
+           "skv_test_wait_timeout", "skv_mla_splice"]
 
 
 class SkvError(RuntimeError):
@@ -326,6 +346,56 @@ def paged_kv_gather(k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, t
                       status, None, num_pages)
     _check(_gather(ctypes.byref(p), _dptr(token_indptr), total_tokens, _dptr(k_out), _dptr(v_out),
                    _stream_ptr(stream)), "skv_paged_kv_gather")
+
+
+def mla_splice(src_ckv, src_kpe, src_pages, dst_ckv, dst_kpe, dst_pages, chunks, rope_theta: float = 10000.0,
+               rope_layout: str = "interleaved", inv_freq=None, status=None, src_num_pages: Optional[int] = None,
+               dst_num_pages: Optional[int] = None, stream=None) -> None:
+    """skv_mla_splice (fetch primitive, local compute).  src/dst ckv [pages, P, 512] and kpe
+    [pages, P, 64] bf16 views; src_pages / dst_pages device int32 page lists; ``chunks`` a sequence
+    of (src_start, dst_start, n_tokens, delta_pos): token t of a chunk moves from logical position
+    src_start + t to dst_start + t and its rope pairs turn by delta_pos * theta_i."""
+    p = splice_params(src_ckv, src_kpe, src_pages, dst_ckv, dst_kpe, dst_pages, rope_theta, rope_layout, inv_freq,
+                      status, src_num_pages, dst_num_pages)
+    splice_launch(p, splice_chunks(chunks), stream)
+
+
+def splice_chunks(chunks) -> "ctypes.Array":
+    """Host array of skv_splice_chunk from (src_start, dst_start, n_tokens, delta_pos) rows."""
+    rows = np.asarray(chunks, dtype=np.int64).reshape(-1, 4)
+    arr = (SpliceChunk * max(1, len(rows)))()
+    for i, (s0, d0, n, dl) in enumerate(rows):
+        arr[i].src_start, arr[i].dst_start, arr[i].n_tokens, arr[i].delta_pos = int(s0), int(d0), int(n), int(dl)
+    arr._n = len(rows)
+    return arr
+
+
+def splice_launch(p: "SpliceParams", chunks: "ctypes.Array", stream=None) -> None:
+    """Launch skv_mla_splice on prepared arguments (``splice_params``, ``splice_chunks``)."""
+    _check(_splice(ctypes.byref(p), chunks, chunks._n, _stream_ptr(stream)), "skv_mla_splice")
+
+
+def splice_params(src_ckv, src_kpe, src_pages, dst_ckv, dst_kpe, dst_pages, rope_theta: float = 10000.0,
+                  rope_layout: str = "interleaved", inv_freq=None, status=None, src_num_pages: Optional[int] = None,
+                  dst_num_pages: Optional[int] = None) -> "SpliceParams":
+    """The skv_splice_params of an mla_splice call, for repeated launches."""
+    for t in (src_ckv, src_kpe, dst_ckv, dst_kpe):
+        if t.stride(-1) != 1:
+            raise ValueError("the innermost stride of every cache view must be 1")
+    p = SpliceParams()
+    p.src_ckv, p.src_kpe, p.dst_ckv, p.dst_kpe = _dptr(src_ckv), _dptr(src_kpe), _dptr(dst_ckv), _dptr(dst_kpe)
+    for i in range(2):
+        p.src_ckv_stride[i], p.src_kpe_stride[i] = src_ckv.stride(i), src_kpe.stride(i)
+        p.dst_ckv_stride[i], p.dst_kpe_stride[i] = dst_ckv.stride(i), dst_kpe.stride(i)
+    p.src_pages, p.dst_pages = _dptr(src_pages), _dptr(dst_pages)
+    p.src_num_pages = src_ckv.shape[0] if src_num_pages is None else src_num_pages
+    p.dst_num_pages = dst_ckv.shape[0] if dst_num_pages is None else dst_num_pages
+    p.src_page_size, p.dst_page_size = src_ckv.shape[1], dst_ckv.shape[1]
+    p.rope_theta, p.rope_layout = float(rope_theta), _ROPE[rope_layout]
+    p.inv_freq, p.kv_dtype, p.status = _dptr(inv_freq), _dtype_code(src_ckv), _dptr(status)
+    if _dtype_code(dst_ckv) != p.kv_dtype:
+        raise ValueError("source and destination caches must have the same dtype")
+    return p
 
 
 def test_wait_timeout(status, limit_ns: int, stream=None) -> None:

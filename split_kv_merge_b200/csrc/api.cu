@@ -540,6 +540,36 @@ skv_status skv_test_wait_timeout(int32_t* status, int64_t limit_ns, skv_stream_t
   return cuda_status(launch_wait_timeout(status, (uint64_t)limit_ns, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+skv_status skv_mla_splice(const skv_splice_params* p, const skv_splice_chunk* chunks_h, int32_t num_chunks,
+                          skv_stream_t stream) {
+  if (p == nullptr || num_chunks < 0 || (num_chunks > 0 && chunks_h == nullptr)) return SKV_ERR_INVALID;
+  int64_t total = 0;
+  for (int32_t c = 0; c < num_chunks; ++c) {
+    const skv_splice_chunk& ch = chunks_h[c];
+    if (ch.n_tokens < 0 || ch.src_start < 0 || ch.dst_start < 0) return SKV_ERR_INVALID;
+    if (ch.src_start > INT64_MAX / 2 - ch.n_tokens || ch.dst_start > INT64_MAX / 2 - ch.n_tokens ||
+        total > INT64_MAX / 4 - ch.n_tokens)
+      return SKV_ERR_INVALID;
+    total += ch.n_tokens;
+  }
+  if (total == 0) return SKV_OK;
+  if (!p->src_ckv || !p->src_kpe || !p->dst_ckv || !p->dst_kpe || !p->src_pages || !p->dst_pages)
+    return SKV_ERR_INVALID;
+  if (p->src_page_size < 1 || p->dst_page_size < 1 || p->src_num_pages < 1 || p->dst_num_pages < 1)
+    return SKV_ERR_INVALID;
+  if (p->rope_layout != SKV_ROPE_INTERLEAVED && p->rope_layout != SKV_ROPE_HALVES) return SKV_ERR_INVALID;
+  if (p->inv_freq == nullptr && !(p->rope_theta > 0.0f && p->rope_theta < INFINITY)) return SKV_ERR_INVALID;
+  if (p->kv_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
+  if (!aligned16(p->src_ckv) || !aligned16(p->src_kpe) || !aligned16(p->dst_ckv) || !aligned16(p->dst_kpe))
+    return SKV_ERR_ALIGNMENT;
+  const int64_t strides[8] = {p->src_ckv_stride[0], p->src_ckv_stride[1], p->src_kpe_stride[0],
+                              p->src_kpe_stride[1], p->dst_ckv_stride[0], p->dst_ckv_stride[1],
+                              p->dst_kpe_stride[0], p->dst_kpe_stride[1]};
+  for (int64_t st : strides)
+    if (st % 8 != 0) return SKV_ERR_ALIGNMENT;
+  return cuda_status(launch_splice(*p, chunks_h, num_chunks, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 skv_status skv_paged_kv_gather(const skv_paged_params* p, const int32_t* token_indptr,
                                int64_t total_tokens, void* k_out, void* v_out, skv_stream_t stream) {
   if (p == nullptr || total_tokens < 0) return SKV_ERR_INVALID;

@@ -63,6 +63,7 @@ int launch_wait_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t s);
 int launch_merge(const float* o_states, const float* lse_states, const int32_t* state_indptr,
                  int32_t num_states, const MergeItem* items, int64_t num_rows, int32_t num_heads,
                  int32_t head_dim, void* o_out, int32_t o_dtype, float* lse_out, cudaStream_t s);
+int launch_splice(const skv_splice_params& p, const skv_splice_chunk* chunks, int num_chunks, cudaStream_t s);
 int launch_gather(const skv_paged_params& p, const int32_t* token_indptr, int64_t total_tokens,
                   void* k_out, void* v_out, bool same_kv, cudaStream_t s);
 

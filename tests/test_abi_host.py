@@ -220,6 +220,47 @@ def test_mla_validation():
     assert fwd(ctypes.byref(bad), fake, ctypes.byref(info), None) == skv.ERR_ALIGNMENT
 
 
+def test_splice_validation():
+    """skv_mla_splice rejects bad arguments before launching (pointers never dereferenced)."""
+    fake = 1 << 20
+    p = skv.SpliceParams()
+    p.src_ckv = p.src_kpe = p.dst_ckv = p.dst_kpe = p.src_pages = p.dst_pages = fake
+    p.src_ckv_stride[0], p.src_ckv_stride[1] = 64 * 576, 576
+    p.src_kpe_stride[0], p.src_kpe_stride[1] = 64 * 576, 576
+    p.dst_ckv_stride[0], p.dst_ckv_stride[1] = 16 * 512, 512
+    p.dst_kpe_stride[0], p.dst_kpe_stride[1] = 16 * 64, 64
+    p.src_num_pages, p.src_page_size, p.dst_num_pages, p.dst_page_size = 8, 64, 40, 16
+    p.rope_theta = 10000.0
+    good = [(0, 10, 100, 4096), (100, 300, 50, -7)]
+
+    def call(chunks=good, **kw):
+        q = skv.SpliceParams.from_buffer_copy(p)
+        for k, v in kw.items():
+            setattr(q, k, v)
+        arr = skv.splice_chunks(chunks)
+        return skv._splice(ctypes.byref(q), arr, arr._n, None)
+
+    assert call([]) == skv.OK                          # nothing to move: no launch
+    assert call([(0, 0, 0, 5), (3, 9, 0, 1)]) == skv.OK
+    assert call([(0, 0, -1, 0)]) == skv.ERR_INVALID
+    assert call([(0, -2, 4, 0)]) == skv.ERR_INVALID
+    assert call([(2 ** 62, 0, 4, 0)]) == skv.ERR_INVALID
+    assert call(dst_pages=None) == skv.ERR_INVALID
+    assert call(src_page_size=0) == skv.ERR_INVALID
+    assert call(rope_layout=2) == skv.ERR_INVALID
+    assert call(rope_theta=0.0) == skv.ERR_INVALID
+    assert call(rope_theta=float("inf")) == skv.ERR_INVALID
+    assert call(kv_dtype=skv.E4M3) == skv.ERR_UNSUPPORTED
+    assert call(dst_kpe=fake + 8) == skv.ERR_ALIGNMENT
+    bad = skv.SpliceParams.from_buffer_copy(p)
+    bad.dst_ckv_stride[1] = 516
+    arr = skv.splice_chunks(good)
+    assert skv._splice(ctypes.byref(bad), arr, 2, None) == skv.ERR_ALIGNMENT
+    assert skv._splice(None, arr, 2, None) == skv.ERR_INVALID
+    assert skv._splice(ctypes.byref(p), None, 2, None) == skv.ERR_INVALID
+    assert skv._splice(ctypes.byref(p), arr, -1, None) == skv.ERR_INVALID
+
+
 # ----------------------------------------------------------------------------- kernel choice
 @pytest.mark.parametrize("hq,hk,q_len,page_size,kernel,q_tile", [
     (64, 8, 1, 16, 3, 1),     # Llama decode: all-KV-heads decode kernel

@@ -7,7 +7,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .gen import MlaCase, PagedCase, RouteCase
+from .gen import MlaCase, PagedCase, RouteCase, SpliceCase
 
 
 def bf16_tensor(bits: np.ndarray, device):
@@ -49,3 +49,16 @@ def route_to_device(c: RouteCase, device):
     return dict(q_nope=bf16_tensor(c.q_nope, device), q_pe=bf16_tensor(c.q_pe, device), cache=cache,
                 ckv=cache[..., :512], kpe=cache[..., 512:],
                 sel_cqk=i32_tensor(np.ascontiguousarray(c.sel.transpose(1, 0, 2)), device))
+
+
+def splice_to_device(c: SpliceCase, device, fill_bits: int = 0x40E0):
+    """Source cache views, a destination cache [dst_num_pages, Pd, 576] pre-filled with one bf16
+    pattern (7.0 by default, so rows the splice must not touch can be checked), page lists."""
+    import torch
+    src = bf16_tensor(c.src, device)
+    dst = torch.full((c.dst_num_pages, c.dst_page_size, 576), 0, dtype=torch.int16, device=device)
+    dst.fill_(int(np.int16(np.uint16(fill_bits))))
+    dst = dst.view(torch.bfloat16)
+    return dict(src=src, src_ckv=src[..., :512], src_kpe=src[..., 512:], dst=dst, dst_ckv=dst[..., :512],
+                dst_kpe=dst[..., 512:], src_pages=i32_tensor(c.src_pages, device),
+                dst_pages=i32_tensor(c.dst_pages, device))

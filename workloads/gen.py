@@ -20,6 +20,7 @@ decode with seqlen_q folding) and the "Move the Query, Not the Cache" summary
 3. ``shared_kv_prefill_case`` one 16384-token KV, P=64, 32/8 heads, 32 x 128 queries
 4. ``mla_decode_case``      32 requests, H in {16,128}, q_len in {1,4}, 512+64 latent
 5. ``route_case``           131072-token latent cache, 8 chunks, 256 queries x 16 heads
+6. ``fetch_splice_case``    the same corpus fetched chunk by chunk into a requester's paged cache
 """
 from __future__ import annotations
 
@@ -35,7 +36,7 @@ __all__ = [
     "BF16_NAN", "E4M3_NAN", "f32_to_bf16_bits", "bf16_bits_to_f32", "e4m3_encode",
     "normal_f32", "normal_bf16", "build_page_table", "PagedCase", "MlaCase", "RouteCase",
     "tiny_gqa_case", "llama70b_decode_case", "shared_kv_prefill_case", "mla_decode_case",
-    "route_case", "even_split_pages",
+    "route_case", "even_split_pages", "SpliceCase", "fetch_splice_case",
 ]
 
 BF16_NAN = np.uint16(0x7FC0)
@@ -399,3 +400,54 @@ def route_case(num_queries: int = 256, num_chunks: int = 8, chunk_tokens: int = 
             sel[q, c] = ids + c * chunk_tokens
     return RouteCase("route_merge", q_nope, q_pe, cache, sel, num_chunks, chunk_tokens, num_heads,
                      1.0 / math.sqrt(192.0))
+
+
+@dataclass
+class SpliceCase:
+    """Fetch-primitive input: a latent corpus held in a paged cache (the chunk holder) and a
+    requester's paged cache.  Chunk c is corpus positions [c*T, (c+1)*T) (logical positions
+    ``src_start[c]`` .. of ``src_pages``); it lands at logical position ``dst_start[c]`` of
+    ``dst_pages`` and moves by ``delta[c]`` positions."""
+    name: str
+    src: np.ndarray             # uint16 [src_num_pages, Ps, 576]
+    src_pages: np.ndarray       # int32 corpus page list (logical order)
+    dst_pages: np.ndarray       # int32 requester page list (logical order)
+    dst_num_pages: int
+    dst_page_size: int
+    chunk_tokens: int
+    src_start: np.ndarray       # int64 [C]
+    dst_start: np.ndarray       # int64 [C]
+    delta: np.ndarray           # int64 [C]
+    rope_theta: float
+
+    @property
+    def num_chunks(self) -> int:
+        return len(self.src_start)
+
+
+def fetch_splice_case(num_chunks: int = 8, chunk_tokens: int = 16384, src_page_size: int = 64,
+                      dst_page_size: int = 64, context: int = 1000, seed: int = 5,
+                      rope_theta: float = 10000.0) -> SpliceCase:
+    """The route corpus (same draws as ``route_case``: num_chunks x chunk_tokens rows of 576 bf16
+    values) placed on seeded random physical pages of size ``src_page_size``; the requester holds
+    ``context`` tokens of its own and fetches the chunks in a seeded random order, each appended
+    after the previous one, so chunk c moves by delta = new position - c * chunk_tokens."""
+    rng = np.random.Generator(np.random.PCG64(seed + 6000))
+    n_tok = num_chunks * chunk_tokens
+    corpus = normal_bf16(seed, 3, (n_tok, 576))
+    n_src = -(-n_tok // src_page_size)
+    pad = n_src * src_page_size - n_tok
+    if pad:
+        corpus = np.concatenate([corpus, np.zeros((pad, 576), np.uint16)])
+    src_pages = rng.permutation(n_src).astype(np.int32)
+    src = np.empty((n_src, src_page_size, 576), np.uint16)
+    src[src_pages] = corpus.reshape(n_src, src_page_size, 576)
+    n_dst_used = -(-(context + n_tok) // dst_page_size)
+    dst_num_pages = n_dst_used + 3
+    dst_pages = rng.permutation(dst_num_pages)[:n_dst_used].astype(np.int32)
+    order = rng.permutation(num_chunks)
+    src_start = np.arange(num_chunks, dtype=np.int64) * chunk_tokens
+    dst_start = np.empty(num_chunks, np.int64)
+    dst_start[order] = context + np.arange(num_chunks, dtype=np.int64) * chunk_tokens
+    return SpliceCase(f"fetch_splice_{num_chunks}x{chunk_tokens}", src, src_pages, dst_pages, dst_num_pages,
+                      dst_page_size, chunk_tokens, src_start, dst_start, dst_start - src_start, rope_theta)
