@@ -4,6 +4,8 @@ returns its error codes before anything is launched."""
 import ctypes
 import os
 import re
+import shutil
+import subprocess
 
 import numpy as np
 import pytest
@@ -30,6 +32,33 @@ def test_library_exports_every_declared_symbol():
     for name in declared:
         assert hasattr(lib, name), name
     assert set(skv.SYMBOLS) <= declared
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a C compiler")
+def test_binding_structs_match_the_c_header(tmp_path):
+    """Every ctypes structure of the binding has the size, field offsets and field sizes of the C
+    struct it mirrors (compiled from include/splitkv.h with gcc)."""
+    pairs = [(skv.PlanInfo, "skv_plan_info"), (skv.PagedParams, "skv_paged_params"),
+             (skv.MlaParams, "skv_mla_params"), (skv.SpliceParams, "skv_splice_params"),
+             (skv.SpliceChunk, "skv_splice_chunk")]
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "splitkv.h"', "int main(void) {"]
+    for cls, cname in pairs:
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {field} %zu %zu\\n", offsetof({cname}, {field}), '
+                         f'sizeof((({cname}*)0)->{field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    c_layout = {tuple(l.split()[:2]): [int(x) for x in l.split()[2:]] for l in out if l.strip()}
+    for cls, cname in pairs:
+        assert c_layout[(cname, "size")] == [ctypes.sizeof(cls)], cname
+        for field, _ in cls._fields_:
+            desc = getattr(cls, field)
+            assert c_layout[(cname, field)] == [desc.offset, desc.size], (cname, field)
 
 
 def test_version_and_status_strings():
