@@ -18,9 +18,14 @@ What it computes (definitions; every step is the plain formula, no tiling or onl
   pages do not name a map).
 * Attention per (request, query token, query head) -- s_t = scale * q . k_t,
   m = max_t s_t, l = sum_t exp(s_t - m), O = sum_t exp(s_t - m) v_t / l, LSE = m + ln l
-  (natural log of the scaled logits; reading: the pages never fix the base).  No causal mask:
-  every query token of a request attends to all L_r tokens (the shared-KV broadcast and the
-  MLA fold both rest on KV being shared by all queries and heads).  Empty KV: O = 0, LSE = -inf.
+  (natural log of the scaled logits; reading: the pages never fix the base).  By default no
+  causal mask: every query token of a request attends to all L_r tokens (the shared-KV broadcast
+  and the MLA fold both rest on KV being shared by all queries and heads).  Empty KV: O = 0,
+  LSE = -inf.
+* Causal / multi-token decode (``causal=True``) -- the request's n_q query tokens are its last
+  n_q positions; query token i sees keys t <= L_r - n_q + i, and a token that sees no key gets
+  O = 0, LSE = -inf.  The FlashInfer PR #3309 page (reviewer feedback) mentions MLA decode with
+  multi-token prediction (MTP) but gives no mask indexing; this is the plainest reading.
 * Split partials -- the same definition restricted to a page range [a, b) of the request
   ("route": partial attention per KV chunk, returned as (O, LSE), "Move the Query, Not the
   Cache" summary, Methodology / primitive comparison; in-CTA split of the SM110 XQA page,
@@ -43,7 +48,7 @@ from typing import Iterable, Optional, Sequence
 import numpy as np
 
 __all__ = [
-    "bf16_to_f64", "e4m3_to_f64", "request_kv_length", "request_token_slots",
+    "bf16_to_f64", "e4m3_to_f64", "request_kv_length", "request_token_slots", "causal_visible",
     "paged_attention", "paged_attention_partials", "merge_states", "mla_decode",
     "mla_decode_partials",
 ]
@@ -89,12 +94,40 @@ def request_token_slots(kv_indptr, kv_indices, kv_last_page_len, page_size: int,
     return pages, t % page_size
 
 
+def causal_visible(n_q: int, kv_len: int, t) -> np.ndarray:
+    """[n_q, len(t)] bool.  The n_q query tokens of a request are its last n_q positions, query
+    token i at position kv_len - n_q + i; it sees key t when t <= kv_len - n_q + i (its own key
+    and every earlier one).  Reading of causal prefill / multi-token (MTP) decode: the pages name
+    the mask but give no indexing."""
+    i = np.arange(n_q, dtype=np.int64)[:, None]
+    return np.asarray(t, dtype=np.int64)[None, :] <= kv_len - n_q + i
+
+
+def _token_range(kv_indptr, kv_last_page_len, page_size: int, r: int, page_begin: int, page_end):
+    """Logical token ids of request r whose page lies in [page_begin, page_end)."""
+    n = int(kv_indptr[r + 1]) - int(kv_indptr[r])
+    L = request_kv_length(kv_indptr, kv_last_page_len, page_size, r)
+    page_end = n if page_end is None else page_end
+    return np.arange(page_begin * page_size, min(page_end * page_size, L), dtype=np.int64), L
+
+
 # ----------------------------------------------------------------------------- attention core
-def _softmax_attend(s: np.ndarray, v: np.ndarray):
-    """s: [rows, L] scaled logits, v: [L, Dv] -> O [rows, Dv], LSE [rows] (definition)."""
+def _softmax_attend(s: np.ndarray, v: np.ndarray, visible: Optional[np.ndarray] = None):
+    """s: [rows, L] scaled logits, v: [L, Dv] -> O [rows, Dv], LSE [rows] (definition).  With
+    ``visible`` ([rows, L] bool) each row attends only to its visible keys; a row that sees no
+    key gets O = 0, LSE = -inf (the empty-KV convention)."""
     rows = s.shape[0]
     if s.shape[1] == 0:
         return np.zeros((rows, v.shape[1])), np.full(rows, -np.inf)
+    if visible is not None:
+        o = np.zeros((rows, v.shape[1]))
+        lse = np.full(rows, -np.inf)
+        for i in range(rows):
+            keys = np.flatnonzero(visible[i])
+            if keys.size:
+                oi, li = _softmax_attend(s[i:i + 1, keys], v[keys])
+                o[i], lse[i] = oi[0], li[0]
+        return o, lse
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
     l = e.sum(axis=1, keepdims=True)
@@ -111,13 +144,17 @@ def _decode_kv(x, kv_dtype: str, kv_scale: float) -> np.ndarray:
 
 
 def _gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, page_size, sm_scale,
-                 r, heads, page_begin=0, page_end=None):
+                 r, heads, page_begin=0, page_end=None, causal=False):
     hq, hk = q.shape[1], k.shape[2]
     g = hq // hk
     pages, slots = request_token_slots(kv_indptr, kv_indices, kv_last_page_len, page_size, r,
                                        page_begin, page_end)
     q_r = bf16_to_f64(q[int(qo_indptr[r]):int(qo_indptr[r + 1])])      # [n_q, Hq, D]
     n_q, dv = q_r.shape[0], v.shape[3]
+    vis = None
+    if causal:
+        t, L = _token_range(kv_indptr, kv_last_page_len, page_size, r, page_begin, page_end)
+        vis = causal_visible(n_q, L, t)
     o = np.zeros((n_q, len(heads), dv))
     lse = np.zeros((n_q, len(heads)))
     for kh in sorted({h // g for h in heads}):
@@ -127,18 +164,19 @@ def _gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, pa
             if h // g != kh:
                 continue
             s = sm_scale * (q_r[:, h, :] @ kk.T)                          # [n_q, L]
-            o[:, j], lse[:, j] = _softmax_attend(s, vv)
+            o[:, j], lse[:, j] = _softmax_attend(s, vv, vis)
     return o, lse
 
 
 def paged_attention(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, page_size: int,
                     sm_scale: float, requests: Optional[Iterable[int]] = None,
-                    heads: Optional[Sequence[int]] = None):
+                    heads: Optional[Sequence[int]] = None, causal: bool = False):
     """GQA attention over a paged bf16 KV cache.
 
     q: bf16 bits [total_q, Hq, D]; k, v: bf16 bits [num_pages, P, Hk, D] (any strides);
     returns O [total_q, |heads|, Dv] and LSE [total_q, |heads|] in float64 (rows of requests
-    not in ``requests`` are NaN)."""
+    not in ``requests`` are NaN).  ``causal``: each query token sees only keys up to its own
+    position (``causal_visible``)."""
     heads = list(range(q.shape[1])) if heads is None else list(heads)
     requests = range(len(kv_indptr) - 1) if requests is None else requests
     O = np.full((q.shape[0], len(heads), v.shape[3]), np.nan)
@@ -146,13 +184,13 @@ def paged_attention(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len,
     for r in requests:
         a, b = int(qo_indptr[r]), int(qo_indptr[r + 1])
         O[a:b], LSE[a:b] = _gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len,
-                                        page_size, sm_scale, r, heads)
+                                        page_size, sm_scale, r, heads, causal=causal)
     return O, LSE
 
 
 def paged_attention_partials(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len,
                              page_size: int, sm_scale: float, split_page_start,
-                             requests: Optional[Iterable[int]] = None):
+                             requests: Optional[Iterable[int]] = None, causal: bool = False):
     """Per request r and split j over logical pages [split_page_start[r][j], [j+1]): the
     partial (O_j, LSE_j) of every query token and head.  Returns {r: (O [S, n_q, Hq, Dv],
     LSE [S, n_q, Hq])}."""
@@ -162,7 +200,7 @@ def paged_attention_partials(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_
     for r in requests:
         b = split_page_start[r]
         parts = [_gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, page_size,
-                              sm_scale, r, heads, b[j], b[j + 1]) for j in range(len(b) - 1)]
+                              sm_scale, r, heads, b[j], b[j + 1], causal) for j in range(len(b) - 1)]
         out[r] = (np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
     return out
 
@@ -195,7 +233,7 @@ def merge_states(o_states, lse_states):
 
 # ----------------------------------------------------------------------------- MLA
 def _mla_request(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len, page_size,
-                 sm_scale, kv_dtype, kv_scale, r, heads, page_begin=0, page_end=None):
+                 sm_scale, kv_dtype, kv_scale, r, heads, page_begin=0, page_end=None, causal=False):
     pages, slots = request_token_slots(kv_indptr, kv_indices, kv_last_page_len, page_size, r,
                                        page_begin, page_end)
     c = _decode_kv(ckv[pages, slots], kv_dtype, kv_scale)                 # [L, 512]  (= V)
@@ -204,13 +242,18 @@ def _mla_request(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len
     qp = bf16_to_f64(q_pe[r])[:, heads]
     q_len, nh = qn.shape[0], qn.shape[1]
     s = sm_scale * (qn.reshape(q_len * nh, -1) @ c.T + qp.reshape(q_len * nh, -1) @ kr.T)
-    o, lse = _softmax_attend(s, c)
+    vis = None
+    if causal:   # rows are (decode position i, head): every head of position i shares its mask
+        t, L = _token_range(kv_indptr, kv_last_page_len, page_size, r, page_begin, page_end)
+        vis = np.repeat(causal_visible(q_len, L, t), nh, axis=0)
+    o, lse = _softmax_attend(s, c) if vis is None else _softmax_attend(s, c, vis)
     return o.reshape(q_len, nh, -1), lse.reshape(q_len, nh)
 
 
 def mla_decode(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len, page_size: int,
                sm_scale: float, kv_dtype: str = "bf16", kv_scale: float = 1.0,
-               requests: Optional[Iterable[int]] = None, heads: Optional[Sequence[int]] = None):
+               requests: Optional[Iterable[int]] = None, heads: Optional[Sequence[int]] = None,
+               causal: bool = False):
     """MLA latent attention.  q_nope [B, q_len, H, 512], q_pe [B, q_len, H, 64] (bf16 bits);
     ckv [num_pages, P, 512], kpe [num_pages, P, 64] (bf16 bits or e4m3 codes).  Returns
     O [B, q_len, |heads|, 512], LSE [B, q_len, |heads|] (unrequested requests NaN)."""
@@ -221,13 +264,14 @@ def mla_decode(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len, 
     LSE = np.full((B, q_len, len(heads)), np.nan)
     for r in requests:
         O[r], LSE[r] = _mla_request(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len,
-                                    page_size, sm_scale, kv_dtype, kv_scale, r, heads)
+                                    page_size, sm_scale, kv_dtype, kv_scale, r, heads, causal=causal)
     return O, LSE
 
 
 def mla_decode_partials(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len,
                         page_size: int, sm_scale: float, split_page_start, kv_dtype: str = "bf16",
-                        kv_scale: float = 1.0, requests: Optional[Iterable[int]] = None):
+                        kv_scale: float = 1.0, requests: Optional[Iterable[int]] = None,
+                        causal: bool = False):
     """Per request and split (logical page ranges), the MLA partial (O_j, LSE_j)."""
     heads = list(range(q_nope.shape[2]))
     requests = range(len(kv_indptr) - 1) if requests is None else requests
@@ -235,7 +279,7 @@ def mla_decode_partials(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_p
     for r in requests:
         b = split_page_start[r]
         parts = [_mla_request(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len,
-                              page_size, sm_scale, kv_dtype, kv_scale, r, heads, b[j], b[j + 1])
+                              page_size, sm_scale, kv_dtype, kv_scale, r, heads, b[j], b[j + 1], causal)
                  for j in range(len(b) - 1)]
         out[r] = (np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
     return out

@@ -11,6 +11,7 @@ other than itself:
   written into the rows;
 * mutation tests: plausible mistakes planted in the oracle (on the CPU) must each fail a pin.
 """
+import ast
 import contextlib
 import inspect
 import math
@@ -143,6 +144,16 @@ def test_pin(pin):
 
 
 # ----------------------------------------------------------------------------- mutation tests
+def _code_signature(src):
+    """The syntax tree of a function's source without its docstring (comments are not in it):
+    equal when only a docstring or a comment changed."""
+    body = ast.parse(src).body[0].body
+    if body and isinstance(body[0], ast.Expr) and isinstance(getattr(body[0], "value", None), ast.Constant) \
+            and isinstance(body[0].value.value, str):
+        body = body[1:]
+    return ast.dump(ast.Module(body=body, type_ignores=[]))
+
+
 @contextlib.contextmanager
 def _mutated(func_name, old, new):
     """Re-define oracle.splice.<func_name> with ``old`` replaced by ``new`` in its source."""
@@ -152,6 +163,8 @@ def _mutated(func_name, old, new):
     ns = OS.__dict__
     exec(compile(src.replace(old, new, 1), OS.__file__, "exec"), ns)
     try:
+        assert _code_signature(src.replace(old, new, 1)) != _code_signature(src), \
+            f"mutation of {func_name} changes no code"
         yield
     finally:
         ns[func_name] = fn
