@@ -19,18 +19,89 @@ def _dev_i32(a, device, non_blocking=False):
     return t.to(device, non_blocking=non_blocking)
 
 
+def causal_split_tables(q_lens, kv_indptr_h, kv_indices_h, kv_last_page_len_h, page_size: int) -> dict:
+    """Host tables that turn causal attention into two unmasked passes and a merge.
+
+    The n_q query tokens of request r are its last n_q positions: token i sees keys
+    t <= L_r - n_q + i.  Every token sees the common prefix t < L_r - n_q + 1 (``prefix``: the same
+    pages, a shorter length), and token i also sees the i keys t in [L_r - n_q + 1, L_r - n_q + 1 + i)
+    (``diag``: one pseudo-request per query token over token rows, page size 1, where row id =
+    page * page_size + slot).  Merging the two partial states of each query row gives the causal
+    result exactly; a token that sees nothing keeps LSE = -inf in both."""
+    q_lens = np.asarray(q_lens, dtype=np.int64)
+    kv_indptr_h = np.asarray(kv_indptr_h, dtype=np.int64)
+    kv_indices_h = np.asarray(kv_indices_h, dtype=np.int64)
+    last_h = np.asarray(kv_last_page_len_h, dtype=np.int64)
+    B, P = len(q_lens), int(page_size)
+    n = np.diff(kv_indptr_h)
+    L = np.where(n > 0, (n - 1) * P + last_h, 0)
+    Lp = np.maximum(L - q_lens + 1, 0)                        # prefix every token sees
+    n_p = (Lp + P - 1) // P
+    pre_indptr = np.concatenate([[0], np.cumsum(n_p)])
+    pre_indices = np.concatenate([kv_indices_h[kv_indptr_h[r]:kv_indptr_h[r] + n_p[r]] for r in range(B)]
+                                 + [np.zeros(0, np.int64)])
+    pre_last = np.where(n_p > 0, Lp - (n_p - 1) * P, 1)
+    counts, rows = [], []
+    for r in range(B):
+        for i in range(int(q_lens[r])):
+            t = np.arange(Lp[r], max(Lp[r], L[r] - q_lens[r] + 1 + i), dtype=np.int64)
+            counts.append(len(t))
+            rows.append(kv_indices_h[kv_indptr_h[r] + t // P] * P + t % P)
+    counts = np.asarray(counts, dtype=np.int64)
+    return {"prefix": (pre_indptr.astype(np.int32), pre_indices.astype(np.int32), pre_last.astype(np.int32)),
+            "diag": (np.concatenate([[0], np.cumsum(counts)]).astype(np.int32),
+                     np.concatenate(rows + [np.zeros(0, np.int64)]).astype(np.int32),
+                     np.ones(len(counts), dtype=np.int32))}
+
+
+def _rows_view(cache, page_size: int):
+    """[num_pages, P, ...] cache -> [num_pages * P, 1, ...] view of its token rows (pages must be
+    laid out back to back: stride[0] == P * stride[1])."""
+    st = list(cache.stride())
+    if st[0] != page_size * st[1]:
+        raise ValueError("causal attention needs each cache's pages back to back (stride[0] == P * stride[1])")
+    return cache.as_strided((cache.shape[0] * page_size, 1, *cache.shape[2:]), (st[1], st[1], *st[2:]))
+
+
 def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, kv_last_page_len_h, *,
                     sm_scale: Optional[float] = None, policy="balanced", param: int = 0,
                     split_page_start=None, o_dtype=None, num_pages: Optional[int] = None,
                     kv_indptr=None, kv_last_page_len=None, plan: Optional[Plan] = None,
-                    status=None, stream=None):
+                    status=None, stream=None, causal: bool = False, kv_indices_h=None, o_out=None,
+                    lse_out=None):
     """GQA attention over a paged cache.  Host page-table shape arrays (``*_h``) feed the planner;
     ``kv_indices`` (and optionally ``kv_indptr`` / ``kv_last_page_len``) are device tensors.
-    Returns (o, lse, extras) with extras = {"plan", "o_part", "lse_part"}."""
+    Returns (o, lse, extras) with extras = {"plan", "o_part", "lse_part"}.
+
+    ``causal``: a request's query tokens are its last positions and each sees keys up to its own
+    (needs the host page list ``kv_indices_h``); computed as a prefix pass, a diagonal pass over
+    token rows and an exact merge (``causal_split_tables``)."""
     import torch
     dev = q.device
     hq, d = q.shape[1], q.shape[2]
     hk = k_cache.shape[2]
+    if causal:
+        if kv_indices_h is None:
+            raise ValueError("causal attention needs the host page list kv_indices_h")
+        P = k_cache.shape[1]
+        qo = np.asarray(qo_indptr_h, dtype=np.int64)
+        tab = causal_split_tables(np.diff(qo), kv_indptr_h, kv_indices_h, kv_last_page_len_h, P)
+        rows = q.shape[0]
+        o_st = torch.empty(2, rows, hq, d, dtype=torch.float32, device=dev)
+        lse_st = torch.empty(2, rows, hq, dtype=torch.float32, device=dev)
+        pi, px, pl = tab["prefix"]
+        paged_attention(q, k_cache, v_cache, qo_indptr_h, pi, _dev_i32(px, dev), pl, sm_scale=sm_scale,
+                        policy=policy, param=param, num_pages=num_pages, status=status, stream=stream,
+                        o_out=o_st[0], lse_out=lse_st[0])
+        di, dx, dl = tab["diag"]
+        n_rows = (k_cache.shape[0] if num_pages is None else num_pages) * P
+        paged_attention(q, _rows_view(k_cache, P), _rows_view(v_cache, P), np.arange(rows + 1), di,
+                        _dev_i32(dx, dev), dl, sm_scale=sm_scale, policy="none", num_pages=n_rows, status=status,
+                        stream=stream, o_out=o_st[1], lse_out=lse_st[1])
+        o = torch.empty(rows, hq, d, dtype=o_dtype or torch.float32, device=dev)
+        lse = torch.empty(rows, hq, dtype=torch.float32, device=dev)
+        merge_states(o_st, lse_st, o, lse, stream=stream)
+        return o, lse, {"plan": None, "o_states": o_st, "lse_states": lse_st, "tables": tab}
     if plan is None:
         plan = plan_paged(qo_indptr_h, kv_indptr_h, kv_last_page_len_h, k_cache.shape[1], hq, hk, d, policy,
                           param, split_page_start)
@@ -38,8 +109,8 @@ def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, k
         plan.to(dev)
     kv_indptr = _dev_i32(kv_indptr_h, dev) if kv_indptr is None else kv_indptr
     kv_last_page_len = _dev_i32(kv_last_page_len_h, dev) if kv_last_page_len is None else kv_last_page_len
-    o = torch.empty(q.shape[0], hq, d, dtype=o_dtype or torch.float32, device=dev)
-    lse = torch.empty(q.shape[0], hq, dtype=torch.float32, device=dev)
+    o = torch.empty(q.shape[0], hq, d, dtype=o_dtype or torch.float32, device=dev) if o_out is None else o_out
+    lse = torch.empty(q.shape[0], hq, dtype=torch.float32, device=dev) if lse_out is None else lse_out
     n_part = plan.info.num_partial_rows
     o_part = torch.empty(n_part, hq, d, dtype=torch.float32, device=dev) if n_part else None
     lse_part = torch.empty(n_part, hq, dtype=torch.float32, device=dev) if n_part else None
@@ -51,11 +122,41 @@ def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, k
 def mla_decode(q_nope, q_pe, ckv, kpe, kv_indptr_h, kv_indices, kv_last_page_len_h, *,
                sm_scale: Optional[float] = None, kv_scale: float = 1.0, policy="balanced", param: int = 0,
                split_page_start=None, o_dtype=None, num_pages: Optional[int] = None, kv_indptr=None,
-               kv_last_page_len=None, plan: Optional[Plan] = None, status=None, stream=None, o=None, lse=None):
-    """MLA latent decode over a paged latent cache (bf16 or e4m3 codes).  Returns (o, lse, extras)."""
+               kv_last_page_len=None, plan: Optional[Plan] = None, status=None, stream=None, o=None, lse=None,
+               causal: bool = False, kv_indices_h=None):
+    """MLA latent decode over a paged latent cache (bf16 or e4m3 codes).  Returns (o, lse, extras).
+
+    ``causal`` (multi-token decode): the q_len decode positions are each request's last positions
+    and each sees keys up to its own (needs ``kv_indices_h``); a prefix pass keeps the fold of
+    q_len into rows, a diagonal pass over token rows adds the few keys only later positions see,
+    and ``merge_states`` combines them exactly."""
     import torch
     dev = q_nope.device
     B, q_len, H = q_nope.shape[:3]
+    if causal:
+        if kv_indices_h is None:
+            raise ValueError("causal attention needs the host page list kv_indices_h")
+        P = ckv.shape[1]
+        tab = causal_split_tables(np.full(B, q_len), kv_indptr_h, kv_indices_h, kv_last_page_len_h, P)
+        o_st = torch.empty(2, B, q_len, H, 512, dtype=torch.float32, device=dev)
+        lse_st = torch.empty(2, B, q_len, H, dtype=torch.float32, device=dev)
+        pi, px, pl = tab["prefix"]
+        mla_decode(q_nope, q_pe, ckv, kpe, pi, _dev_i32(px, dev), pl, sm_scale=sm_scale, kv_scale=kv_scale,
+                   policy=policy, param=param, num_pages=num_pages, status=status, stream=stream, o=o_st[0],
+                   lse=lse_st[0])
+        di, dx, dl = tab["diag"]
+        n_rows = (ckv.shape[0] if num_pages is None else num_pages) * P
+        mla_decode(q_nope.reshape(B * q_len, 1, H, 512), q_pe.reshape(B * q_len, 1, H, 64), _rows_view(ckv, P),
+                   _rows_view(kpe, P), di, _dev_i32(dx, dev), dl, sm_scale=sm_scale, kv_scale=kv_scale,
+                   policy="none", num_pages=n_rows, status=status, stream=stream,
+                   o=o_st[1].view(B * q_len, 1, H, 512), lse=lse_st[1].view(B * q_len, 1, H))
+        if o is None:
+            o = torch.empty(B, q_len, H, 512, dtype=o_dtype or torch.float32, device=dev)
+        if lse is None:
+            lse = torch.empty(B, q_len, H, dtype=torch.float32, device=dev)
+        merge_states(o_st.view(2, B * q_len, H, 512), lse_st.view(2, B * q_len, H), o.view(B * q_len, H, 512),
+                     lse.view(B * q_len, H), stream=stream)
+        return o, lse, {"plan": None, "o_states": o_st, "lse_states": lse_st, "tables": tab}
     if plan is None:
         kd = "bf16" if ckv.dtype == torch.bfloat16 else "e4m3"
         plan = plan_mla(q_len, kv_indptr_h, kv_last_page_len_h, ckv.shape[1], H, policy, param, split_page_start, kd)
