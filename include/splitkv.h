@@ -16,6 +16,8 @@
  *                       partial attention at the KV holder merged "via online softmax",
  *                       "Move the Query, Not the Cache", Methodology; in-CTA split with
  *                       shared-memory merge, FlashInfer PR #5597 page, section 3).
+ *   skv_causal_tables   Host planner that turns causal / multi-token attention into a prefix
+ *                       call, a diagonal call over token rows and an exact merge.
  *   skv_mla_splice      The fetch primitive's local compute: move a chunk's latent rows between
  *                       page lists and re-rotate their RoPE part to the new positions ("Move
  *                       the Query, Not the Cache", problem statement and Methodology: fetch
@@ -23,8 +25,9 @@
  *
  * Semantics shared by all calls (natural-log LSE of the scaled logits):
  *   s_t = sm_scale * q . k_t ;  O = sum_t softmax(s)_t v_t ;  LSE = ln sum_t exp(s_t).
- *   A request with no KV tokens gives O = 0, LSE = -inf.  No causal mask: every query token
- *   of a request attends to all of the request's KV tokens.
+ *   A request with no KV tokens gives O = 0, LSE = -inf.  The attention calls take no mask:
+ *   every query token of a request attends to all of the request's KV tokens; causal attention
+ *   is planned by skv_causal_tables on top of them.
  *
  * Page table (device int32 arrays): request r owns pages kv_indices[kv_indptr[r] ..
  *   kv_indptr[r+1]); its length is L_r = (n_r - 1) * page_size + kv_last_page_len[r] with
@@ -261,6 +264,30 @@ SKV_API skv_status skv_merge_states(const float* o_states, const float* lse_stat
                             const int32_t* state_indptr, int32_t num_states, int64_t num_rows,
                             int32_t num_heads, int32_t head_dim, void* o_out, int32_t o_dtype,
                             float* lse_out, skv_stream_t stream);
+
+/* -------------------------------------------------------------------------------------------
+ * skv_causal_tables -- host planner for causal / multi-token attention.  The n_q query tokens of
+ *   request r (rows qo_indptr[r] .. qo_indptr[r+1]) are its last n_q positions; query token i
+ *   sees keys t <= L_r - n_q + i (multi-token prediction decode, mentioned on the FlashInfer PR
+ *   #3309 page; causal prefill).  The call splits this into two unmasked problems whose exact
+ *   merge (skv_merge_states, two states per query row) is the causal result:
+ *     prefix -- request r keeps its first ceil(Lp_r / P) pages, Lp_r = max(0, L_r - n_q + 1): the
+ *               keys every query token of r sees (same query rows, same page size);
+ *     diag   -- one request per query row j = qo_indptr[r] + i, page size 1, whose "pages" are the
+ *               token rows page * P + slot of keys [Lp_r, L_r - n_q + 1 + i): the keys token i sees
+ *               beyond the prefix (none for i = 0).  Run it on a [num_pages * P, 1, ...] view of the
+ *               cache (pages back to back) with num_pages * P rows.
+ *   Outputs are host arrays the caller allocates: prefix_indptr [batch+1], prefix_indices
+ *   [kv_indptr_h[batch]], prefix_last [batch]; diag_indptr [total_q+1], diag_last [total_q] (all 1),
+ *   diag_rows [diag_capacity].  *diag_rows_needed receives the number of diagonal rows; if it
+ *   exceeds diag_capacity nothing else is written and SKV_ERR_WORKSPACE is returned (size the
+ *   buffer with a first call of capacity 0).  Token rows must fit int32 (SKV_ERR_UNSUPPORTED).
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_causal_tables(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
+                                     const int32_t* kv_indices_h, const int32_t* kv_last_page_len_h,
+                                     int32_t page_size, int32_t* prefix_indptr_h, int32_t* prefix_indices_h,
+                                     int32_t* prefix_last_h, int32_t* diag_indptr_h, int32_t* diag_rows_h,
+                                     int32_t* diag_last_h, int64_t diag_capacity, int64_t* diag_rows_needed);
 
 /* -------------------------------------------------------------------------------------------
  * skv_mla_splice -- the fetch primitive's local compute.  "Move the Query, Not the Cache"

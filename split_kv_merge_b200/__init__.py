@@ -117,6 +117,9 @@ _gather = _proto("skv_paged_kv_gather", ctypes.c_int, [ctypes.POINTER(PagedParam
                                                         _vp, _vp])
 _splice = _proto("skv_mla_splice", ctypes.c_int, [ctypes.POINTER(SpliceParams), ctypes.POINTER(SpliceChunk),
                                                    ctypes.c_int32, _vp])
+_causal = _proto("skv_causal_tables", ctypes.c_int, [ctypes.c_int32, _i32p, _i32p, _i32p, _i32p, ctypes.c_int32,
+                                                     _i32p, _i32p, _i32p, _i32p, _i32p, _i32p, ctypes.c_int64,
+                                                     ctypes.POINTER(ctypes.c_int64)])
 _wait_timeout = _proto("skv_test_wait_timeout", ctypes.c_int, [_vp, ctypes.c_int64, _vp])
 _fold = _proto("skv_mla_fold_ratio", ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32])
 _status_str = _proto("skv_status_str", ctypes.c_char_p, [ctypes.c_int32])
@@ -125,7 +128,7 @@ _version = _proto("skv_version", ctypes.c_int32, [])
 SYMBOLS = ["skv_plan_paged", "skv_paged_attn_fwd", "skv_paged_attn_partial", "skv_merge_plan", "skv_plan_mla",
            "skv_mla_decode_fwd", "skv_mla_decode_partial", "skv_merge_states", "skv_paged_kv_gather",
            "skv_mla_fold_ratio", "skv_status_str", "skv_version", "skv_paged_attn_fwd_static_scratch",
-           "skv_test_wait_timeout", "skv_mla_splice"]
+           "skv_test_wait_timeout", "skv_mla_splice", "skv_causal_tables"]
 
 
 class SkvError(RuntimeError):
@@ -396,6 +399,29 @@ def splice_params(src_ckv, src_kpe, src_pages, dst_ckv, dst_kpe, dst_pages, rope
     if _dtype_code(dst_ckv) != p.kv_dtype:
         raise ValueError("source and destination caches must have the same dtype")
     return p
+
+
+def causal_tables(qo_indptr, kv_indptr, kv_indices, kv_last_page_len, page_size: int) -> dict:
+    """skv_causal_tables on host arrays: {"prefix": (kv_indptr, kv_indices, kv_last_page_len),
+    "diag": (kv_indptr, token rows, kv_last_page_len)}, int32 numpy arrays."""
+    qo, ip, ix, la = _i32(qo_indptr), _i32(kv_indptr), _i32(kv_indices), _i32(kv_last_page_len)
+    B, total_q = len(ip) - 1, int(qo[-1])
+    pre_ip, pre_ix, pre_la = (np.zeros(B + 1, np.int32), np.zeros(max(1, int(ip[-1])), np.int32),
+                              np.zeros(max(1, B), np.int32))
+    d_ip, d_la = np.zeros(total_q + 1, np.int32), np.zeros(max(1, total_q), np.int32)
+    need = ctypes.c_int64(0)
+    args = lambda rows, cap: (B, _ptr_i32(qo), _ptr_i32(ip), _ptr_i32(ix), _ptr_i32(la), int(page_size),
+                              _ptr_i32(pre_ip), _ptr_i32(pre_ix), _ptr_i32(pre_la), _ptr_i32(d_ip), _ptr_i32(rows),
+                              _ptr_i32(d_la), cap, ctypes.byref(need))
+    code = _causal(*args(None, 0))
+    if code == ERR_WORKSPACE:
+        rows = np.zeros(int(need.value), np.int32)
+        code = _causal(*args(rows, int(need.value)))
+    else:
+        rows = np.zeros(0, np.int32)
+    _check(code, "skv_causal_tables")
+    return {"prefix": (pre_ip, pre_ix[:int(pre_ip[-1])], pre_la[:B]),
+            "diag": (d_ip, rows, d_la[:total_q])}
 
 
 def test_wait_timeout(status, limit_ns: int, stream=None) -> None:

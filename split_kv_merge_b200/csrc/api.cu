@@ -540,6 +540,59 @@ skv_status skv_test_wait_timeout(int32_t* status, int64_t limit_ns, skv_stream_t
   return cuda_status(launch_wait_timeout(status, (uint64_t)limit_ns, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+skv_status skv_causal_tables(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
+                             const int32_t* kv_indices_h, const int32_t* kv_last_page_len_h, int32_t page_size,
+                             int32_t* prefix_indptr_h, int32_t* prefix_indices_h, int32_t* prefix_last_h,
+                             int32_t* diag_indptr_h, int32_t* diag_rows_h, int32_t* diag_last_h,
+                             int64_t diag_capacity, int64_t* diag_rows_needed) {
+  if (batch < 0 || page_size < 1 || diag_capacity < 0 || !qo_indptr_h || !kv_indptr_h || !kv_last_page_len_h ||
+      !diag_rows_needed)
+    return SKV_ERR_INVALID;
+  if (qo_indptr_h[0] != 0 || kv_indptr_h[0] != 0) return SKV_ERR_INVALID;
+  // validate the table and count the diagonal rows
+  int64_t need = 0;
+  for (int32_t r = 0; r < batch; ++r) {
+    const int64_t nq = (int64_t)qo_indptr_h[r + 1] - qo_indptr_h[r];
+    const int64_t n = (int64_t)kv_indptr_h[r + 1] - kv_indptr_h[r];
+    if (nq < 0 || n < 0) return SKV_ERR_INVALID;
+    if (n > 0 && (kv_last_page_len_h[r] < 1 || kv_last_page_len_h[r] > page_size)) return SKV_ERR_INVALID;
+    const int64_t L = n == 0 ? 0 : (n - 1) * page_size + kv_last_page_len_h[r];
+    const int64_t lp = std::min<int64_t>(L, std::max<int64_t>(0, L - nq + 1));  // nq = 0: no row sees more than L
+    for (int64_t i = 0; i < nq; ++i) need += std::max<int64_t>(0, L - nq + 1 + i - lp);
+  }
+  *diag_rows_needed = need;
+  if (need > diag_capacity) return SKV_ERR_WORKSPACE;
+  if (need > INT32_MAX) return SKV_ERR_UNSUPPORTED;
+  if (!prefix_indptr_h || !prefix_last_h || !diag_indptr_h || !diag_last_h || (need > 0 && !diag_rows_h) ||
+      (kv_indptr_h[batch] > 0 && (!kv_indices_h || !prefix_indices_h)))
+    return SKV_ERR_INVALID;
+  prefix_indptr_h[0] = 0;
+  diag_indptr_h[0] = 0;
+  int64_t drow = 0;
+  for (int32_t r = 0; r < batch; ++r) {
+    const int64_t nq = (int64_t)qo_indptr_h[r + 1] - qo_indptr_h[r];
+    const int64_t n = (int64_t)kv_indptr_h[r + 1] - kv_indptr_h[r];
+    const int64_t L = n == 0 ? 0 : (n - 1) * page_size + kv_last_page_len_h[r];
+    const int64_t lp = std::min<int64_t>(L, std::max<int64_t>(0, L - nq + 1));
+    const int64_t np_ = (lp + page_size - 1) / page_size;  // <= n: the prefix stays inside the request
+    const int32_t* pages = kv_indices_h + kv_indptr_h[r];
+    for (int64_t j = 0; j < np_; ++j) prefix_indices_h[prefix_indptr_h[r] + j] = pages[j];
+    prefix_indptr_h[r + 1] = prefix_indptr_h[r] + (int32_t)np_;
+    prefix_last_h[r] = np_ > 0 ? (int32_t)(lp - (np_ - 1) * page_size) : 1;
+    for (int64_t i = 0; i < nq; ++i) {
+      const int64_t row = qo_indptr_h[r] + i;
+      for (int64_t t = lp; t < L - nq + 1 + i; ++t) {
+        const int64_t id = (int64_t)pages[t / page_size] * page_size + t % page_size;
+        if (id < 0 || id > INT32_MAX) return SKV_ERR_UNSUPPORTED;
+        diag_rows_h[drow++] = (int32_t)id;
+      }
+      diag_indptr_h[row + 1] = (int32_t)drow;
+      diag_last_h[row] = 1;
+    }
+  }
+  return SKV_OK;
+}
+
 skv_status skv_mla_splice(const skv_splice_params* p, const skv_splice_chunk* chunks_h, int32_t num_chunks,
                           skv_stream_t stream) {
   if (p == nullptr || num_chunks < 0 || (num_chunks > 0 && chunks_h == nullptr)) return SKV_ERR_INVALID;

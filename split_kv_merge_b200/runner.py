@@ -6,7 +6,7 @@ from typing import Optional
 
 import numpy as np
 
-from . import (Plan, mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged)
+from . import (Plan, causal_tables, mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged)
 
 
 def _dev_i32(a, device, non_blocking=False):
@@ -20,38 +20,12 @@ def _dev_i32(a, device, non_blocking=False):
 
 
 def causal_split_tables(q_lens, kv_indptr_h, kv_indices_h, kv_last_page_len_h, page_size: int) -> dict:
-    """Host tables that turn causal attention into two unmasked passes and a merge.
-
-    The n_q query tokens of request r are its last n_q positions: token i sees keys
-    t <= L_r - n_q + i.  Every token sees the common prefix t < L_r - n_q + 1 (``prefix``: the same
-    pages, a shorter length), and token i also sees the i keys t in [L_r - n_q + 1, L_r - n_q + 1 + i)
-    (``diag``: one pseudo-request per query token over token rows, page size 1, where row id =
-    page * page_size + slot).  Merging the two partial states of each query row gives the causal
-    result exactly; a token that sees nothing keeps LSE = -inf in both."""
-    q_lens = np.asarray(q_lens, dtype=np.int64)
-    kv_indptr_h = np.asarray(kv_indptr_h, dtype=np.int64)
-    kv_indices_h = np.asarray(kv_indices_h, dtype=np.int64)
-    last_h = np.asarray(kv_last_page_len_h, dtype=np.int64)
-    B, P = len(q_lens), int(page_size)
-    n = np.diff(kv_indptr_h)
-    L = np.where(n > 0, (n - 1) * P + last_h, 0)
-    Lp = np.maximum(L - q_lens + 1, 0)                        # prefix every token sees
-    n_p = (Lp + P - 1) // P
-    pre_indptr = np.concatenate([[0], np.cumsum(n_p)])
-    pre_indices = np.concatenate([kv_indices_h[kv_indptr_h[r]:kv_indptr_h[r] + n_p[r]] for r in range(B)]
-                                 + [np.zeros(0, np.int64)])
-    pre_last = np.where(n_p > 0, Lp - (n_p - 1) * P, 1)
-    counts, rows = [], []
-    for r in range(B):
-        for i in range(int(q_lens[r])):
-            t = np.arange(Lp[r], max(Lp[r], L[r] - q_lens[r] + 1 + i), dtype=np.int64)
-            counts.append(len(t))
-            rows.append(kv_indices_h[kv_indptr_h[r] + t // P] * P + t % P)
-    counts = np.asarray(counts, dtype=np.int64)
-    return {"prefix": (pre_indptr.astype(np.int32), pre_indices.astype(np.int32), pre_last.astype(np.int32)),
-            "diag": (np.concatenate([[0], np.cumsum(counts)]).astype(np.int32),
-                     np.concatenate(rows + [np.zeros(0, np.int64)]).astype(np.int32),
-                     np.ones(len(counts), dtype=np.int32))}
+    """Host tables that turn causal attention into two unmasked passes and a merge
+    (``skv_causal_tables``): ``prefix`` -- each request cut to the keys all its query tokens see;
+    ``diag`` -- one page-size-1 request per query token over the token rows (page * P + slot) it
+    sees beyond that prefix."""
+    qo = np.concatenate([[0], np.cumsum(np.asarray(q_lens, dtype=np.int64))])
+    return causal_tables(qo, kv_indptr_h, kv_indices_h, kv_last_page_len_h, page_size)
 
 
 def _rows_view(cache, page_size: int):

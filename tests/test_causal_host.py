@@ -3,6 +3,7 @@
 (two unmasked passes, token-row views of the caches, an exact merge) are run with the three
 launches replaced by float64 stand-ins built on the oracle, on CPU tensors, and must reproduce
 the oracle's causal attention.  What this leaves to the GPU tests is the kernels themselves."""
+import ctypes
 import math
 
 import numpy as np
@@ -10,6 +11,7 @@ import pytest
 import torch
 
 import oracle.attention as OA
+import split_kv_merge_b200 as skv
 import split_kv_merge_b200.runner as R
 from workloads import build_page_table, normal_bf16
 
@@ -114,7 +116,7 @@ def test_causal_tables_cover_each_visible_key_once():
         B = int(rng.integers(1, 6))
         P = int(rng.choice([1, 4, 16]))
         lengths = rng.integers(0, 60, size=B).tolist()
-        q_lens = rng.integers(1, 8, size=B)
+        q_lens = rng.integers(0, 8, size=B)      # requests without query tokens included
         kv_indptr, kv_indices, last, num_pages = build_page_table(rng, lengths, P, extra_pages=0)
         tab = R.causal_split_tables(q_lens, kv_indptr, kv_indices, last, P)
         pi, px, pl = tab["prefix"]
@@ -125,6 +127,7 @@ def test_causal_tables_cover_each_visible_key_once():
             pages = kv_indices[kv_indptr[r]:kv_indptr[r + 1]]
             n_p = pi[r + 1] - pi[r]
             Lp = 0 if n_p == 0 else (n_p - 1) * P + pl[r]
+            assert n_p <= len(pages) and Lp <= L          # the prefix never leaves the request
             assert np.array_equal(px[pi[r]:pi[r + 1]], pages[:n_p]) and 1 <= pl[r] <= P
             prefix_rows = [pages[t // P] * P + t % P for t in range(Lp)]
             for i in range(int(q_lens[r])):
@@ -133,6 +136,30 @@ def test_causal_tables_cover_each_visible_key_once():
                 assert got == want, (trial, r, i)
                 row += 1
         assert row == len(di) - 1 and np.all(dl == 1)
+
+
+def test_causal_tables_validation_and_sizing():
+    qo, ip, ix, la = [np.asarray(a, np.int32) for a in ([0, 2, 5], [0, 2, 3], [4, 1, 7], [3, 2])]
+    B = 2
+    outs = [np.zeros(B + 1, np.int32), np.zeros(3, np.int32), np.zeros(B, np.int32), np.zeros(6, np.int32),
+            np.zeros(64, np.int32), np.zeros(5, np.int32)]
+    need = ctypes.c_int64(-1)
+
+    def call(qo=qo, ip=ip, la=la, P=4, cap=64, rows=outs[4]):
+        p = skv._ptr_i32
+        return skv._causal(B, p(qo), p(ip), p(ix), p(la), P, p(outs[0]), p(outs[1]), p(outs[2]), p(outs[3]),
+                           p(rows), p(outs[5]), cap, ctypes.byref(need))
+
+    # request 0: L = 7, 2 query tokens -> prefix 6 keys, token 1 sees 1 more; request 1: L = 2 and
+    # 3 query tokens -> prefix 0 keys, tokens 1 and 2 see 1 and 2 keys: 4 diagonal rows
+    assert call(cap=0) == skv.ERR_WORKSPACE and need.value == 4
+    assert call() == skv.OK and need.value == 4
+    assert outs[0].tolist() == [0, 2, 2] and outs[2].tolist() == [2, 1]
+    assert outs[3].tolist() == [0, 0, 1, 1, 2, 4]
+    assert outs[4][:4].tolist() == [1 * 4 + 2, 7 * 4 + 0, 7 * 4 + 0, 7 * 4 + 1]
+    assert call(la=np.asarray([5, 2], np.int32)) == skv.ERR_INVALID      # last page length > page size
+    assert call(qo=np.asarray([0, 3, 2], np.int32)) == skv.ERR_INVALID   # decreasing query offsets
+    assert call(P=0) == skv.ERR_INVALID
 
 
 def test_causal_needs_host_page_list():
