@@ -1,0 +1,116 @@
+"""Randomised host checks of the planners (no GPU): for random page tables (empty requests, requests
+without query rows, ragged lengths), page sizes, head shapes, split policies and both MLA cache
+types, every plan must
+
+* cover, for every query row of every request, the request's pages exactly once, split by split in
+  order (page ranges contiguous from 0 to n_r);
+* write each query row either directly (one split) or through partial rows that its merge item
+  lists exactly, with no partial row written twice and every partial row inside the buffer;
+* hand the work to persistent CTAs through a monotone CTA index that ends at the work count."""
+import numpy as np
+import pytest
+
+import split_kv_merge_b200 as skv
+from workloads import build_page_table
+
+
+def _items(plan):
+    nw, nm = plan.info.num_work, plan.info.num_merge_rows
+    return plan.words[: 8 * nw].reshape(-1, 8), plan.words[8 * nw: 8 * nw + 4 * nm].reshape(-1, 4)
+
+
+def _check(plan, qo, n_pages):
+    info = plan.info
+    w, m = _items(plan)
+    B = len(n_pages)
+    part_owner = {}
+    direct = {}
+    spans = {}
+    for r, qs, qc, pb, pe, prow, pstride, j in w.tolist():
+        assert 0 <= r < B and qc >= 1 and qo[r] <= qs and qs + qc <= qo[r + 1], (r, qs, qc)
+        assert 0 <= pb <= pe <= n_pages[r]
+        for i in range(qc):
+            row = qs + i
+            spans.setdefault(row, []).append((j, pb, pe))
+            if prow < 0:
+                assert row not in direct, f"row {row} written directly twice"
+                direct[row] = True
+            else:
+                p = prow + i * pstride
+                assert 0 <= p < info.num_partial_rows and p not in part_owner, (row, p)
+                part_owner[p] = row
+    merged = {}
+    for out_row, sb, sc, _ in m.tolist():
+        assert out_row not in merged and out_row not in direct
+        assert sorted(p for p, row in part_owner.items() if row == out_row) == list(range(sb, sb + sc))
+        merged[out_row] = sc
+    assert len(part_owner) == sum(merged.values()) == info.num_partial_rows
+    for r in range(B):
+        for row in range(qo[r], qo[r + 1]):
+            assert (row in direct) != (row in merged), f"row {row}: direct and merged, or neither"
+            sp = sorted(spans[row])
+            assert [j for j, _, _ in sp] == list(range(len(sp)))
+            assert sp[0][1] == 0 and sp[-1][2] == n_pages[r]
+            assert all(sp[k][2] == sp[k + 1][1] for k in range(len(sp) - 1))
+    if info.num_ctas:
+        cta = plan.words[info.cta_offset: info.cta_offset + info.num_ctas + 1]
+        assert cta[0] == 0 and cta[-1] == info.num_work and np.all(np.diff(cta) >= 0)
+
+
+def _random_table(rng, P, max_len, q_max):
+    B = int(rng.integers(1, 30))
+    lengths = rng.integers(0, max_len + 1, size=B)
+    lengths[rng.random(B) < 0.15] = 0
+    q_lens = rng.integers(0, q_max + 1, size=B)
+    kv_indptr, kv_indices, last, _ = build_page_table(rng, lengths.tolist(), P, extra_pages=0)
+    return q_lens, kv_indptr, last
+
+
+def _policy(rng, n_pages):
+    kind = rng.choice(["none", "fixed", "balanced", "balanced_small", "explicit"])
+    if kind == "fixed":
+        return "fixed", int(rng.integers(1, 6)), None
+    if kind == "balanced":
+        return "balanced", 148, None
+    if kind == "balanced_small":
+        return "balanced", int(rng.integers(1, 40)), None
+    if kind == "explicit":
+        sps = []
+        for n in n_pages:
+            k = int(rng.integers(1, 4))
+            cuts = np.sort(rng.integers(0, n + 1, size=k - 1)) if n >= 0 else []
+            sps.append([0, *[int(x) for x in cuts], int(n)])
+        return "explicit", 0, sps
+    return "none", 0, None
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_paged_plans(seed):
+    rng = np.random.Generator(np.random.PCG64(1000 + seed))
+    for _ in range(15):
+        hq, hk, d = [(64, 8, 128), (32, 8, 128), (8, 2, 64), (16, 4, 128), (8, 8, 64)][int(rng.integers(0, 5))]
+        P = int(rng.choice([1, 4, 16, 64]))
+        q_max = int(rng.choice([1, 4, 40, 200]))
+        q_lens, kv_indptr, last = _random_table(rng, P, 3000, q_max)
+        qo = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+        n_pages = np.diff(kv_indptr)
+        policy, param, sps = _policy(rng, n_pages)
+        plan = skv.plan_paged(qo, kv_indptr, last, P, hq, hk, d, policy, param, sps)
+        _check(plan, qo, n_pages)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_mla_plans(seed):
+    rng = np.random.Generator(np.random.PCG64(2000 + seed))
+    for _ in range(15):
+        H = int(rng.choice([16, 32, 64, 128]))
+        q_len = int(rng.integers(1, 5))
+        P = int(rng.choice([1, 4, 16, 64, 128]))
+        kv_dtype = str(rng.choice(["bf16", "e4m3"]))
+        _, kv_indptr, last = _random_table(rng, P, 5000, 1)
+        B = len(kv_indptr) - 1
+        qo = (np.arange(B + 1) * q_len).astype(np.int32)
+        n_pages = np.diff(kv_indptr)
+        policy, param, sps = _policy(rng, n_pages)
+        plan = skv.plan_mla(q_len, kv_indptr, last, P, H, policy, param, sps, kv_dtype=kv_dtype)
+        _check(plan, qo, n_pages)
