@@ -61,6 +61,18 @@ def test_binding_structs_match_the_c_header(tmp_path):
             assert c_layout[(cname, field)] == [desc.offset, desc.size], (cname, field)
 
 
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a C compiler")
+def test_plain_c_consumer(tmp_path):
+    """tests/c/host_calls.c, compiled against include/splitkv.h and linked to libsplitkv.so, runs the
+    host-only entry points from C (planners, causal planner, validation, status strings)."""
+    lib_dir = os.path.dirname(skv.library_path())
+    exe = tmp_path / "host_calls"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "host_calls.c"),
+                    "-L", lib_dir, "-lsplitkv", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
 def test_version_and_status_strings():
     assert skv.version() >= 1
     assert skv.status_str(0) == "ok"
