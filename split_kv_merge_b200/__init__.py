@@ -168,6 +168,22 @@ def _dptr(t) -> Optional[int]:
     return None if t is None else int(t.data_ptr())
 
 
+_PLACEHOLDER = {}
+
+
+def _index_ptr(t) -> Optional[int]:
+    """Pointer of an int32 index tensor; an empty one (no page of any request) is passed as a small
+    zero buffer on its device, since torch gives empty tensors no storage and the library rejects
+    a NULL page list.  The kernels read no page id of a request without pages."""
+    if t is None or t.numel() > 0:
+        return _dptr(t)
+    import torch
+    key = str(t.device)
+    if key not in _PLACEHOLDER:
+        _PLACEHOLDER[key] = torch.zeros(4, dtype=torch.int32, device=t.device)
+    return _dptr(_PLACEHOLDER[key])
+
+
 def _stream_ptr(stream) -> Optional[int]:
     if stream is None:
         import torch
@@ -254,7 +270,7 @@ def _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, 
     for i in range(3):
         p.k_stride[i] = k_cache.stride(i)
         p.v_stride[i] = v_cache.stride(i)
-    p.kv_indptr, p.kv_indices, p.kv_last_page_len = _dptr(kv_indptr), _dptr(kv_indices), _dptr(kv_last_page_len)
+    p.kv_indptr, p.kv_indices, p.kv_last_page_len = _dptr(kv_indptr), _index_ptr(kv_indices), _dptr(kv_last_page_len)
     p.batch = kv_indptr.shape[0] - 1
     p.total_q = q.shape[0] if q is not None else 0
     p.num_pages = k_cache.shape[0] if num_pages is None else num_pages
@@ -309,7 +325,7 @@ def mla_decode_fwd(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_l
         p.kpe_stride[i] = kpe.stride(i)
     p.kv_dtype = _dtype_code(ckv)
     p.kv_scale = float(kv_scale)
-    p.kv_indptr, p.kv_indices, p.kv_last_page_len = _dptr(kv_indptr), _dptr(kv_indices), _dptr(kv_last_page_len)
+    p.kv_indptr, p.kv_indices, p.kv_last_page_len = _dptr(kv_indptr), _index_ptr(kv_indices), _dptr(kv_last_page_len)
     p.batch = kv_indptr.shape[0] - 1
     p.q_len = q_nope.shape[1]
     p.num_heads = q_nope.shape[2]

@@ -61,17 +61,23 @@ def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, k
         qo = np.asarray(qo_indptr_h, dtype=np.int64)
         tab = causal_split_tables(np.diff(qo), kv_indptr_h, kv_indices_h, kv_last_page_len_h, P)
         rows = q.shape[0]
-        o_st = torch.empty(2, rows, hq, d, dtype=torch.float32, device=dev)
-        lse_st = torch.empty(2, rows, hq, dtype=torch.float32, device=dev)
         pi, px, pl = tab["prefix"]
-        paged_attention(q, k_cache, v_cache, qo_indptr_h, pi, _dev_i32(px, dev), pl, sm_scale=sm_scale,
-                        policy=policy, param=param, num_pages=num_pages, status=status, stream=stream,
-                        o_out=o_st[0], lse_out=lse_st[0])
         di, dx, dl = tab["diag"]
         n_rows = (k_cache.shape[0] if num_pages is None else num_pages) * P
-        paged_attention(q, _rows_view(k_cache, P), _rows_view(v_cache, P), np.arange(rows + 1), di,
-                        _dev_i32(dx, dev), dl, sm_scale=sm_scale, policy="none", num_pages=n_rows, status=status,
-                        stream=stream, o_out=o_st[1], lse_out=lse_st[1])
+        prefix = lambda oo, ll: paged_attention(  # noqa: E731
+            q, k_cache, v_cache, qo_indptr_h, pi, _dev_i32(px, dev), pl, sm_scale=sm_scale, policy=policy,
+            param=param, o_dtype=o_dtype, num_pages=num_pages, status=status, stream=stream, o_out=oo, lse_out=ll)
+        diag = lambda oo, ll: paged_attention(  # noqa: E731
+            q, _rows_view(k_cache, P), _rows_view(v_cache, P), np.arange(rows + 1), di, _dev_i32(dx, dev), dl,
+            sm_scale=sm_scale, policy="none", o_dtype=o_dtype, num_pages=n_rows, status=status, stream=stream,
+            o_out=oo, lse_out=ll)
+        if int(di[-1]) == 0 or int(pi[-1]) == 0:  # one pass sees nothing: the other is the answer
+            o, lse, _ = (prefix if int(di[-1]) == 0 else diag)(None, None)
+            return o, lse, {"plan": None, "tables": tab}
+        o_st = torch.empty(2, rows, hq, d, dtype=torch.float32, device=dev)
+        lse_st = torch.empty(2, rows, hq, dtype=torch.float32, device=dev)
+        prefix(o_st[0], lse_st[0])
+        diag(o_st[1], lse_st[1])
         o = torch.empty(rows, hq, d, dtype=o_dtype or torch.float32, device=dev)
         lse = torch.empty(rows, hq, dtype=torch.float32, device=dev)
         merge_states(o_st, lse_st, o, lse, stream=stream)
@@ -112,22 +118,28 @@ def mla_decode(q_nope, q_pe, ckv, kpe, kv_indptr_h, kv_indices, kv_last_page_len
             raise ValueError("causal attention needs the host page list kv_indices_h")
         P = ckv.shape[1]
         tab = causal_split_tables(np.full(B, q_len), kv_indptr_h, kv_indices_h, kv_last_page_len_h, P)
-        o_st = torch.empty(2, B, q_len, H, 512, dtype=torch.float32, device=dev)
-        lse_st = torch.empty(2, B, q_len, H, dtype=torch.float32, device=dev)
         pi, px, pl = tab["prefix"]
-        mla_decode(q_nope, q_pe, ckv, kpe, pi, _dev_i32(px, dev), pl, sm_scale=sm_scale, kv_scale=kv_scale,
-                   policy=policy, param=param, num_pages=num_pages, status=status, stream=stream, o=o_st[0],
-                   lse=lse_st[0])
         di, dx, dl = tab["diag"]
         n_rows = (ckv.shape[0] if num_pages is None else num_pages) * P
-        mla_decode(q_nope.reshape(B * q_len, 1, H, 512), q_pe.reshape(B * q_len, 1, H, 64), _rows_view(ckv, P),
-                   _rows_view(kpe, P), di, _dev_i32(dx, dev), dl, sm_scale=sm_scale, kv_scale=kv_scale,
-                   policy="none", num_pages=n_rows, status=status, stream=stream,
-                   o=o_st[1].view(B * q_len, 1, H, 512), lse=lse_st[1].view(B * q_len, 1, H))
         if o is None:
             o = torch.empty(B, q_len, H, 512, dtype=o_dtype or torch.float32, device=dev)
         if lse is None:
             lse = torch.empty(B, q_len, H, dtype=torch.float32, device=dev)
+        prefix = lambda oo, ll: mla_decode(  # noqa: E731
+            q_nope, q_pe, ckv, kpe, pi, _dev_i32(px, dev), pl, sm_scale=sm_scale, kv_scale=kv_scale, policy=policy,
+            param=param, num_pages=num_pages, status=status, stream=stream, o=oo, lse=ll)
+        diag = lambda oo, ll: mla_decode(  # noqa: E731
+            q_nope.reshape(B * q_len, 1, H, 512), q_pe.reshape(B * q_len, 1, H, 64), _rows_view(ckv, P),
+            _rows_view(kpe, P), di, _dev_i32(dx, dev), dl, sm_scale=sm_scale, kv_scale=kv_scale, policy="none",
+            num_pages=n_rows, status=status, stream=stream, o=oo.view(B * q_len, 1, H, 512),
+            lse=ll.view(B * q_len, 1, H))
+        if int(di[-1]) == 0 or int(pi[-1]) == 0:  # one pass sees nothing: the other is the answer
+            (prefix if int(di[-1]) == 0 else diag)(o, lse)
+            return o, lse, {"plan": None, "tables": tab}
+        o_st = torch.empty(2, B, q_len, H, 512, dtype=torch.float32, device=dev)
+        lse_st = torch.empty(2, B, q_len, H, dtype=torch.float32, device=dev)
+        prefix(o_st[0], lse_st[0])
+        diag(o_st[1], lse_st[1])
         merge_states(o_st.view(2, B * q_len, H, 512), lse_st.view(2, B * q_len, H), o.view(B * q_len, H, 512),
                      lse.view(B * q_len, H), stream=stream)
         return o, lse, {"plan": None, "o_states": o_st, "lse_states": lse_st, "tables": tab}

@@ -87,6 +87,39 @@ def test_causal_gqa_composition(monkeypatch, indep_v):
     assert len(di) == int(qo[-1]) + 1
 
 
+@pytest.mark.parametrize("case", ["one_token_each", "all_prefix_empty"])
+def test_causal_single_pass_cases(monkeypatch, case):
+    """With one query token per request there are no diagonal keys, and with every request shorter
+    than its query block there is no common prefix: one pass gives the answer, no merge."""
+    _Fakes(monkeypatch)
+    rng = np.random.Generator(np.random.PCG64(54))
+    if case == "one_token_each":
+        lengths, q_lens = [13, 0, 40, 7], [1, 1, 1, 1]
+    else:
+        lengths, q_lens = [1, 0, 2, 3], [2, 3, 3, 5]
+    P, hq, hk, d = 4, 8, 2, 64
+    kv_indptr, kv_indices, last, num_pages = build_page_table(rng, lengths, P, extra_pages=1)
+    qo = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q, k, v = (normal_bf16(54, i, s) for i, s in ((1, (int(qo[-1]), hq, d)), (2, (num_pages, P, hk, d)),
+                                                   (3, (num_pages, P, hk, d))))
+    o, lse, ex = R.paged_attention(_tb(q), _tb(k), _tb(v), qo, kv_indptr, torch.from_numpy(kv_indices), last,
+                                   sm_scale=0.125, policy="none", causal=True, kv_indices_h=kv_indices)
+    assert "o_states" not in ex                      # a single pass, no merge
+    O, LSE = OA.paged_attention(q, k, v, qo, kv_indptr, kv_indices, last, P, 0.125, causal=True)
+    np.testing.assert_allclose(o.numpy(), O, rtol=0, atol=1e-6)
+    np.testing.assert_array_equal(np.isneginf(lse.numpy()), np.isneginf(LSE))
+    fin = np.isfinite(LSE)
+    np.testing.assert_allclose(lse.numpy()[fin], LSE[fin], rtol=0, atol=1e-6)
+
+
+def test_empty_page_list_is_passed_as_a_placeholder():
+    """An empty page list (no request has pages) reaches the library as a non-NULL buffer."""
+    empty = torch.zeros(0, dtype=torch.int32)
+    assert skv._index_ptr(empty) not in (None, 0)
+    full = torch.arange(3, dtype=torch.int32)
+    assert skv._index_ptr(full) == full.data_ptr() and skv._index_ptr(None) is None
+
+
 def test_causal_mla_composition(monkeypatch):
     _Fakes(monkeypatch)
     rng = np.random.Generator(np.random.PCG64(52))

@@ -30,12 +30,18 @@ def _cmp(o, lse, O, LSE, tol, where):
     assert err_l <= 1e-3, f"{where}: LSE max-abs {err_l}"
 
 
-@pytest.mark.parametrize("shape", ["mtp_decode", "prefill"])
+@pytest.mark.parametrize("shape", ["mtp_decode", "prefill", "one_token_each", "no_common_prefix"])
 def test_causal_gqa(shape):
     rng = np.random.Generator(np.random.PCG64(61))
     if shape == "mtp_decode":      # Llama-70B-shaped heads, 1-4 query tokens per request
         hq, hk, d, P = 64, 8, 128, 16
         lengths, q_lens = [1, 700, 0, 3, 257, 512], [2, 4, 1, 4, 3, 1]
+    elif shape == "one_token_each":  # no diagonal keys: the prefix pass alone
+        hq, hk, d, P = 64, 8, 128, 16
+        lengths, q_lens = [1, 700, 0, 257], [1, 1, 1, 1]
+    elif shape == "no_common_prefix":  # every request shorter than its query block: the diagonal pass alone
+        hq, hk, d, P = 64, 8, 128, 16
+        lengths, q_lens = [1, 0, 2, 3], [2, 3, 3, 4]
     else:                          # shared-KV prefill heads, 128-token query blocks
         hq, hk, d, P = 32, 8, 128, 64
         lengths, q_lens = [300, 500, 128], [128, 128, 128]
