@@ -435,6 +435,7 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
   if (info->kernel != KERNEL_GQA_SIMT && info->kernel != KERNEL_GQA_TC_DECODE && info->kernel != KERNEL_GQA_TC_WIDE &&
       info->kernel != KERNEL_GQA_TC_PREFILL)
     return SKV_ERR_INVALID;
+  if (info->num_work == 0) return SKV_OK;  // no query rows: nothing to launch
   const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
                        p->k_stride[2] == p->v_stride[2];
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -498,6 +499,7 @@ skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d
   if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
   const bool tc = info->kernel == KERNEL_MLA_TC16 || info->kernel == KERNEL_MLA_TC32;
   if (info->kernel != KERNEL_MLA_SIMT && !tc) return SKV_ERR_INVALID;
+  if (info->num_work == 0) return SKV_OK;  // no requests: nothing to launch
   if (tc && (info->num_ctas < 1 || info->cta_offset < 8LL * info->num_work + 4LL * info->num_merge_rows))
     return SKV_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

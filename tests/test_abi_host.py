@@ -261,6 +261,32 @@ def test_mla_validation():
     assert fwd(ctypes.byref(bad), fake, ctypes.byref(info), None) == skv.ERR_ALIGNMENT
 
 
+def test_empty_plans_launch_nothing():
+    """A batch without requests, or without query rows, plans no work; the launches then return OK
+    without touching the device (so this runs on a machine without a GPU)."""
+    fake = 1 << 20
+    for qo, ip, la in (([0], [0], []), ([0, 0, 0], [0, 2, 3], [5, 16])):
+        plan = skv.plan_paged(np.array(qo), np.array(ip), np.array(la), 16, 64, 8, 128, "balanced", 148)
+        assert plan.info.num_work == 0 and plan.info.num_merge_rows == 0
+        p = skv.PagedParams()
+        p.q = p.k_cache = p.v_cache = p.kv_indptr = p.kv_indices = p.kv_last_page_len = p.o = fake
+        for i in range(3):
+            p.k_stride[i] = p.v_stride[i] = [16 * 8 * 128, 8 * 128, 128][i]
+        p.batch, p.total_q, p.num_pages, p.page_size = len(ip) - 1, 0, 4, 16
+        p.num_qo_heads, p.num_kv_heads, p.head_dim, p.sm_scale = 64, 8, 128, 0.088
+        words = np.ascontiguousarray(plan.words)
+        assert skv._paged_fwd(ctypes.byref(p), words.ctypes.data, ctypes.byref(plan.info), None) == skv.OK
+    plan = skv.plan_mla(1, np.array([0]), np.array([], np.int32), 64, 16, "balanced", 148)
+    assert plan.info.num_work == 0
+    m = skv.MlaParams()
+    m.q_nope = m.q_pe = m.ckv = m.kpe = m.kv_indptr = m.kv_indices = m.kv_last_page_len = m.o = fake
+    m.ckv_stride[0], m.ckv_stride[1] = 64 * 576, 576
+    m.kpe_stride[0], m.kpe_stride[1] = 64 * 576, 576
+    m.batch, m.q_len, m.num_heads, m.num_pages, m.page_size, m.sm_scale = 0, 1, 16, 4, 64, 0.07
+    words = np.ascontiguousarray(plan.words)
+    assert skv._mla_fwd(ctypes.byref(m), words.ctypes.data, ctypes.byref(plan.info), None) == skv.OK
+
+
 def test_splice_validation():
     """skv_mla_splice rejects bad arguments before launching (pointers never dereferenced)."""
     fake = 1 << 20
