@@ -16,6 +16,8 @@
  *                       partial attention at the KV holder merged "via online softmax",
  *                       "Move the Query, Not the Cache", Methodology; in-CTA split with
  *                       shared-memory merge, FlashInfer PR #5597 page, section 3).
+ *   skv_plan_paged_subset  Planner for part of a batch (a mixed prefill + decode batch runs as two
+ *                       launches, each on the kernel that suits its requests).
  *   skv_causal_tables   Host planner that turns causal / multi-token attention into a prefix
  *                       call, a diagonal call over token rows and an exact merge.
  *   skv_mla_splice      The fetch primitive's local compute: move a chunk's latent rows between
@@ -264,6 +266,22 @@ SKV_API skv_status skv_merge_states(const float* o_states, const float* lse_stat
                             const int32_t* state_indptr, int32_t num_states, int64_t num_rows,
                             int32_t num_heads, int32_t head_dim, void* o_out, int32_t o_dtype,
                             float* lse_out, skv_stream_t stream);
+
+/* -------------------------------------------------------------------------------------------
+ * skv_plan_paged_subset -- skv_plan_paged for the requests listed in requests_h only (distinct
+ *   indices in [0, batch)); the others get no work, so a launch with this plan writes only the
+ *   listed requests' query rows and partial rows.  One batch that mixes prefill and decode
+ *   requests (a POD batch: prefill on decode, FlashInfer PR #4736 page, batch_pod.cu) is planned
+ *   as two subsets, each choosing its own kernel, and launched with the batch's own q, page table
+ *   and outputs -- no copy of any of them.  Every plan needs its own o_part / lse_part.  Explicit
+ *   splits are not accepted here (SKV_ERR_INVALID).
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_plan_paged_subset(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
+                                         const int32_t* kv_last_page_len_h, int32_t page_size,
+                                         int32_t num_qo_heads, int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t policy, int32_t param, const int32_t* requests_h,
+                                         int32_t num_requests, int32_t* plan_h, int64_t plan_capacity,
+                                         skv_plan_info* info);
 
 /* -------------------------------------------------------------------------------------------
  * skv_causal_tables -- host planner for causal / multi-token attention.  The n_q query tokens of

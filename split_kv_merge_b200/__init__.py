@@ -96,6 +96,10 @@ _plan_paged = _proto("skv_plan_paged", ctypes.c_int, [ctypes.c_int32, _i32p, _i3
                                                        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                        ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, _i32p,
                                                        ctypes.c_int64, ctypes.POINTER(PlanInfo)])
+_plan_subset = _proto("skv_plan_paged_subset", ctypes.c_int, [ctypes.c_int32, _i32p, _i32p, _i32p, ctypes.c_int32,
+                                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                             ctypes.c_int32, ctypes.c_int32, _i32p, ctypes.c_int32,
+                                                             _i32p, ctypes.c_int64, ctypes.POINTER(PlanInfo)])
 _plan_mla = _proto("skv_plan_mla", ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32,
                                                    ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                    _i32p, _i32p, _i32p, ctypes.c_int64, ctypes.POINTER(PlanInfo)])
@@ -128,7 +132,7 @@ _version = _proto("skv_version", ctypes.c_int32, [])
 SYMBOLS = ["skv_plan_paged", "skv_paged_attn_fwd", "skv_paged_attn_partial", "skv_merge_plan", "skv_plan_mla",
            "skv_mla_decode_fwd", "skv_mla_decode_partial", "skv_merge_states", "skv_paged_kv_gather",
            "skv_mla_fold_ratio", "skv_status_str", "skv_version", "skv_paged_attn_fwd_static_scratch",
-           "skv_test_wait_timeout", "skv_mla_splice", "skv_causal_tables"]
+           "skv_test_wait_timeout", "skv_mla_splice", "skv_causal_tables", "skv_plan_paged_subset"]
 
 
 class SkvError(RuntimeError):
@@ -245,6 +249,23 @@ def plan_paged(qo_indptr, kv_indptr, kv_last_page_len, page_size: int, num_qo_he
     return _plan(_plan_paged, lambda pol: (b, _ptr_i32(qo), _ptr_i32(ki), _ptr_i32(la), page_size, num_qo_heads,
                                            num_kv_heads, head_dim, pol, param),
                  policy, split_page_start, "skv_plan_paged")
+
+
+def plan_paged_subset(qo_indptr, kv_indptr, kv_last_page_len, page_size: int, num_qo_heads: int,
+                      num_kv_heads: int, head_dim: int, requests, policy="balanced", param: int = 0) -> Plan:
+    """Host planner for the listed requests of a batch only (skv_plan_paged_subset)."""
+    qo, ki, la, rq = _i32(qo_indptr), _i32(kv_indptr), _i32(kv_last_page_len), _i32(requests)
+    b = len(ki) - 1
+    pol = _POLICY[policy] if isinstance(policy, str) else int(policy)
+    info = PlanInfo()
+    args = (b, _ptr_i32(qo), _ptr_i32(ki), _ptr_i32(la), page_size, num_qo_heads, num_kv_heads, head_dim, pol,
+            param, _ptr_i32(rq), len(rq))
+    code = _plan_subset(*args, None, 0, ctypes.byref(info))
+    if code not in (OK, ERR_WORKSPACE):
+        _check(code, "skv_plan_paged_subset")
+    words = np.zeros(max(1, info.plan_words), dtype=np.int32)
+    _check(_plan_subset(*args, _ptr_i32(words), words.size, ctypes.byref(info)), "skv_plan_paged_subset")
+    return Plan(words[: info.plan_words] if info.plan_words else words[:0], info)
 
 
 def plan_mla(batch_q_len: int, kv_indptr, kv_last_page_len, page_size: int, num_heads: int,
@@ -449,4 +470,4 @@ def library_path() -> str:
     return _LIB_PATH
 
 
-from .runner import RouteMerge, mla_decode, paged_attention  # noqa: E402,F401
+from .runner import RouteMerge, mla_decode, paged_attention, pod_attention  # noqa: E402,F401

@@ -292,6 +292,63 @@ skv_status check_plan(const int32_t* plan_d, const skv_plan_info* info) {
   return SKV_OK;
 }
 
+// skv_plan_paged, optionally restricted to the requests marked in `include` (the others get no
+// work: no query rows, no pages), so one batch can be planned as several kernel launches.
+skv_status plan_paged_impl(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
+                           const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_qo_heads,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t policy, int32_t param,
+                           const int32_t* split_indptr_h, const int32_t* split_bounds_h,
+                           const std::vector<char>* include, int32_t* plan_h, int64_t plan_capacity,
+                           skv_plan_info* info) {
+  if (info != nullptr) std::memset(info, 0, sizeof(*info));
+  if (qo_indptr_h == nullptr || num_qo_heads < 1 || num_kv_heads < 1) return SKV_ERR_INVALID;
+  if (num_qo_heads % num_kv_heads != 0) return SKV_ERR_INVALID;
+  if (head_dim != 64 && head_dim != 128) return SKV_ERR_UNSUPPORTED;
+  std::vector<ReqShape> req;
+  skv_status st = check_table_h(batch, kv_indptr_h, kv_last_page_len_h, page_size, req);
+  if (st != SKV_OK) return st;
+  if (batch > 0 && qo_indptr_h[0] != 0) return SKV_ERR_INVALID;
+  for (int32_t r = 0; r < batch; ++r) {
+    req[r].q_start = qo_indptr_h[r];
+    req[r].q_len = qo_indptr_h[r + 1] - qo_indptr_h[r];
+    if (req[r].q_len < 0) return SKV_ERR_INVALID;
+    if (include != nullptr && !(*include)[r]) {
+      req[r].q_len = 0;
+      req[r].n_pages = 0;
+    }
+  }
+  const int32_t g = num_qo_heads / num_kv_heads;
+  int32_t max_q = 1;
+  for (const auto& q : req) max_q = std::max(max_q, q.q_len);
+  // all-KV-heads tensor-core decode when every request's query rows per KV head fit its 8
+  // columns (whole pages stream contiguously); else the per-KV-head tensor-core decode; else the
+  // generic CUDA-core kernel
+  const bool wide = g <= 8 && 8 % g == 0 && max_q * g <= 8 &&
+                    gqa_tc_wide_supported(head_dim, page_size, num_kv_heads, g, 8 / g);
+  // more query rows per KV head than one 16-column decode tile holds: 128-row prefill tiles
+  const bool prefill = !wide && (int64_t)max_q * g > 16 && gqa_tc_prefill_supported(head_dim, page_size, g);
+  const int32_t tc_q_tile = std::max<int32_t>(1, std::min<int32_t>(16 / std::max<int32_t>(g, 1), max_q));
+  const bool tc = !wide && !prefill && g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
+  const int32_t kernel = wide      ? KERNEL_GQA_TC_WIDE
+                         : prefill ? KERNEL_GQA_TC_PREFILL
+                         : tc      ? KERNEL_GQA_TC_DECODE
+                                   : KERNEL_GQA_SIMT;
+  const int32_t q_tile = wide ? 8 / g : prefill ? 128 / g : tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
+  std::vector<int64_t> kv_len(batch);
+  for (int32_t r = 0; r < batch; ++r)
+    kv_len[r] = req[r].n_pages == 0 ? 0
+                                    : (int64_t)(req[r].n_pages - 1) * page_size + kv_last_page_len_h[r];
+  PersistOpts po;
+  po.page_size = page_size;
+  if (wide) {  // persistent all-heads kernel: 16-token tiles, one CTA per SM
+    po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
+    po.tile_tokens = 16;
+  }
+  // per-KV-head tensor-core kernel: a few large units per SM; CUDA-core kernel: many small CTAs
+  return plan_common(batch, req, kv_len, q_tile, wide ? 1 : num_kv_heads, prefill ? 2 : tc ? 6 : 64, policy, param,
+                     split_indptr_h, split_bounds_h, kernel, po, plan_h, plan_capacity, info);
+}
+
 }  // namespace
 
 extern "C" {
@@ -327,49 +384,27 @@ skv_status skv_plan_paged(int32_t batch, const int32_t* qo_indptr_h, const int32
                           int32_t policy, int32_t param, const int32_t* split_indptr_h,
                           const int32_t* split_bounds_h, int32_t* plan_h,
                           int64_t plan_capacity, skv_plan_info* info) {
+  return plan_paged_impl(batch, qo_indptr_h, kv_indptr_h, kv_last_page_len_h, page_size, num_qo_heads, num_kv_heads,
+                         head_dim, policy, param, split_indptr_h, split_bounds_h, nullptr, plan_h, plan_capacity,
+                         info);
+}
+
+skv_status skv_plan_paged_subset(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
+                                 const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_qo_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t policy, int32_t param,
+                                 const int32_t* requests_h, int32_t num_requests, int32_t* plan_h,
+                                 int64_t plan_capacity, skv_plan_info* info) {
   if (info != nullptr) std::memset(info, 0, sizeof(*info));
-  if (qo_indptr_h == nullptr || num_qo_heads < 1 || num_kv_heads < 1) return SKV_ERR_INVALID;
-  if (num_qo_heads % num_kv_heads != 0) return SKV_ERR_INVALID;
-  if (head_dim != 64 && head_dim != 128) return SKV_ERR_UNSUPPORTED;
-  std::vector<ReqShape> req;
-  skv_status st = check_table_h(batch, kv_indptr_h, kv_last_page_len_h, page_size, req);
-  if (st != SKV_OK) return st;
-  if (batch > 0 && qo_indptr_h[0] != 0) return SKV_ERR_INVALID;
-  for (int32_t r = 0; r < batch; ++r) {
-    req[r].q_start = qo_indptr_h[r];
-    req[r].q_len = qo_indptr_h[r + 1] - qo_indptr_h[r];
-    if (req[r].q_len < 0) return SKV_ERR_INVALID;
+  if (batch < 0 || num_requests < 0 || (num_requests > 0 && requests_h == nullptr)) return SKV_ERR_INVALID;
+  if (policy == SKV_SPLIT_EXPLICIT) return SKV_ERR_INVALID;
+  std::vector<char> include(batch, 0);
+  for (int32_t i = 0; i < num_requests; ++i) {
+    const int32_t r = requests_h[i];
+    if (r < 0 || r >= batch || include[r]) return SKV_ERR_INVALID;  // out of range or listed twice
+    include[r] = 1;
   }
-  const int32_t g = num_qo_heads / num_kv_heads;
-  int32_t max_q = 1;
-  for (const auto& q : req) max_q = std::max(max_q, q.q_len);
-  // all-KV-heads tensor-core decode when every request's query rows per KV head fit its 8
-  // columns (whole pages stream contiguously); else the per-KV-head tensor-core decode; else the
-  // generic CUDA-core kernel
-  const bool wide = g <= 8 && 8 % g == 0 && max_q * g <= 8 &&
-                    gqa_tc_wide_supported(head_dim, page_size, num_kv_heads, g, 8 / g);
-  // more query rows per KV head than one 16-column decode tile holds: 128-row prefill tiles
-  const bool prefill = !wide && (int64_t)max_q * g > 16 && gqa_tc_prefill_supported(head_dim, page_size, g);
-  const int32_t tc_q_tile = std::max<int32_t>(1, std::min<int32_t>(16 / std::max<int32_t>(g, 1), max_q));
-  const bool tc = !wide && !prefill && g <= 16 && gqa_tc_decode_supported(head_dim, page_size, g, tc_q_tile);
-  const int32_t kernel = wide      ? KERNEL_GQA_TC_WIDE
-                         : prefill ? KERNEL_GQA_TC_PREFILL
-                         : tc      ? KERNEL_GQA_TC_DECODE
-                                   : KERNEL_GQA_SIMT;
-  const int32_t q_tile = wide ? 8 / g : prefill ? 128 / g : tc ? tc_q_tile : std::max<int32_t>(1, 16 / g);
-  std::vector<int64_t> kv_len(batch);
-  for (int32_t r = 0; r < batch; ++r)
-    kv_len[r] = req[r].n_pages == 0 ? 0
-                                    : (int64_t)(req[r].n_pages - 1) * page_size + kv_last_page_len_h[r];
-  PersistOpts po;
-  po.page_size = page_size;
-  if (wide) {  // persistent all-heads kernel: 16-token tiles, one CTA per SM
-    po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
-    po.tile_tokens = 16;
-  }
-  // per-KV-head tensor-core kernel: a few large units per SM; CUDA-core kernel: many small CTAs
-  return plan_common(batch, req, kv_len, q_tile, wide ? 1 : num_kv_heads, prefill ? 2 : tc ? 6 : 64, policy, param,
-                     split_indptr_h, split_bounds_h, kernel, po, plan_h, plan_capacity, info);
+  return plan_paged_impl(batch, qo_indptr_h, kv_indptr_h, kv_last_page_len_h, page_size, num_qo_heads, num_kv_heads,
+                         head_dim, policy, param, nullptr, nullptr, &include, plan_h, plan_capacity, info);
 }
 
 skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,

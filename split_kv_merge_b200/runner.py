@@ -6,7 +6,8 @@ from typing import Optional
 
 import numpy as np
 
-from . import (Plan, causal_tables, mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged)
+from . import (Plan, causal_tables, mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged,
+               plan_paged_subset)
 
 
 def _dev_i32(a, device, non_blocking=False):
@@ -97,6 +98,38 @@ def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, k
     paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan, o, lse, o_part, lse_part,
                    status, sm_scale, num_pages, stream)
     return o, lse, {"plan": plan, "o_part": o_part, "lse_part": lse_part}
+
+
+def pod_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, kv_last_page_len_h, *,
+                  decode_q_max: Optional[int] = None, sm_scale: Optional[float] = None, policy="balanced",
+                  param: int = 0, o_dtype=None, num_pages: Optional[int] = None, status=None, stream=None):
+    """A batch that mixes prefill and decode requests (POD: prefill on decode, FlashInfer PR #4736
+    page, batch_pod.cu), run as one launch per kind on the batch's own q, page table and outputs:
+    requests with at most ``decode_q_max`` query tokens (default: what the all-KV-heads decode
+    kernel holds, 8 // group) on the decode plan, the rest on the prefill plan
+    (``skv_plan_paged_subset``).  Returns (o, lse, {"plans": [...]})."""
+    import torch
+    dev = q.device
+    hq, d = q.shape[1], q.shape[2]
+    hk = k_cache.shape[2]
+    q_lens = np.diff(np.asarray(qo_indptr_h, dtype=np.int64))
+    if decode_q_max is None:
+        decode_q_max = max(1, 8 // max(1, hq // hk))
+    kv_indptr = _dev_i32(kv_indptr_h, dev)
+    kv_last = _dev_i32(kv_last_page_len_h, dev)
+    o = torch.empty(q.shape[0], hq, d, dtype=o_dtype or torch.float32, device=dev)
+    lse = torch.empty(q.shape[0], hq, dtype=torch.float32, device=dev)
+    plans = []
+    for reqs in (np.flatnonzero(q_lens <= decode_q_max), np.flatnonzero(q_lens > decode_q_max)):
+        if len(reqs) == 0:
+            continue
+        plan = plan_paged_subset(qo_indptr_h, kv_indptr_h, kv_last_page_len_h, k_cache.shape[1], hq, hk, d, reqs,
+                                 policy, param)
+        paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, kv_last_page_len_h,
+                        sm_scale=sm_scale, num_pages=num_pages, kv_indptr=kv_indptr, kv_last_page_len=kv_last,
+                        plan=plan, status=status, stream=stream, o_out=o, lse_out=lse)
+        plans.append(plan)
+    return o, lse, {"plans": plans}
 
 
 def mla_decode(q_nope, q_pe, ckv, kpe, kv_indptr_h, kv_indices, kv_last_page_len_h, *,

@@ -114,3 +114,59 @@ def test_mla_plans(seed):
         policy, param, sps = _policy(rng, n_pages)
         plan = skv.plan_mla(q_len, kv_indptr, last, P, H, policy, param, sps, kv_dtype=kv_dtype)
         _check(plan, qo, n_pages)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_paged_subset_plans(seed):
+    """A plan for a subset of the requests covers exactly those requests' query rows (pages once per
+    split, partials consistent) and nothing of the others; two complementary subsets together
+    cover the batch."""
+    rng = np.random.Generator(np.random.PCG64(3000 + seed))
+    for _ in range(12):
+        hq, hk, d = [(64, 8, 128), (32, 8, 128), (8, 2, 64)][int(rng.integers(0, 3))]
+        P = int(rng.choice([1, 16, 64]))
+        q_lens, kv_indptr, last = _random_table(rng, P, 2000, int(rng.choice([1, 8, 130])))
+        B = len(q_lens)
+        qo = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+        n_pages = np.diff(kv_indptr)
+        chosen = rng.random(B) < 0.5
+        policy = str(rng.choice(["none", "fixed", "balanced"]))
+        param = {"none": 0, "fixed": int(rng.integers(1, 4)), "balanced": 148}[policy]
+        covered = np.zeros(int(qo[-1]), bool)
+        for subset in (np.flatnonzero(chosen), np.flatnonzero(~chosen)):
+            plan = skv.plan_paged_subset(qo, kv_indptr, last, P, hq, hk, d, subset, policy, param)
+            w, _ = _items(plan)
+            assert set(w[:, 0].tolist()) <= set(subset.tolist())
+            # rows of the other requests must not appear: check against a table where they are empty
+            keep = np.zeros(B, bool)
+            keep[subset] = True
+            rows_sub = np.concatenate([np.arange(qo[r], qo[r + 1]) for r in subset] + [np.zeros(0, int)])
+            _check_subset(plan, qo, n_pages, keep)
+            assert not covered[rows_sub].any()
+            covered[rows_sub] = True
+        assert covered.all()
+
+
+def _check_subset(plan, qo, n_pages, keep):
+    """_check restricted to the requests in ``keep``: the others must have no rows at all."""
+    w, m = _items(plan)
+    for r, qs, qc, *_ in w.tolist():
+        assert keep[r] and qo[r] <= qs and qs + qc <= qo[r + 1]
+    q2 = [0]
+    for r in range(len(n_pages)):
+        q2.append(q2[-1] + (qo[r + 1] - qo[r] if keep[r] else 0))
+    # rebase the plan's rows onto the kept requests only, then run the full check on that table
+    shift = {}
+    for r in range(len(n_pages)):
+        shift[r] = q2[r] - qo[r]
+    w2 = w.copy()
+    for row in w2:
+        row[1] += shift[int(row[0])]
+    m2 = m.copy()
+    row_req = np.searchsorted(qo, np.arange(qo[-1]), side="right") - 1
+    for row in m2:
+        row[0] += shift[int(row_req[row[0]])]
+    words = plan.words.copy()
+    words[: w2.size] = w2.reshape(-1)
+    words[w2.size: w2.size + m2.size] = m2.reshape(-1)
+    _check(skv.Plan(words, plan.info), np.asarray(q2), np.where(keep, n_pages, 0))

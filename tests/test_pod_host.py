@@ -1,0 +1,79 @@
+"""Host logic of mixed prefill + decode (POD) batches (no GPU): ``runner.pod_attention`` plans the
+decode requests and the prefill requests of one batch separately (``skv_plan_paged_subset``) and
+launches both plans on the batch's own buffers.  With the launch replaced by a float64 stand-in
+that computes exactly the requests of the plan it is given (and writes only their rows), the two
+launches must together give the oracle's attention for the whole batch, each plan on the kernel
+that suits its requests."""
+import math
+
+import numpy as np
+import torch
+
+import oracle.attention as OA
+import split_kv_merge_b200 as skv
+import split_kv_merge_b200.runner as R
+from workloads import build_page_table, normal_bf16
+
+
+def _bits(t):
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _tb(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+def test_pod_batch_composition(monkeypatch):
+    launches = []
+    real_subset = R.plan_paged_subset
+
+    def plan_paged_subset(qo, *a, **k):
+        plan = real_subset(qo, *a, **k)
+        plan.qo = np.asarray(qo, dtype=np.int32)
+        return plan
+
+    def paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan, o, lse, o_part, lse_part,
+                       status, sm_scale, num_pages, stream):
+        w = plan.words[: 8 * plan.info.num_work].reshape(-1, 8)
+        reqs = sorted(set(w[:, 0].tolist()))
+        launches.append((plan.info.kernel, reqs))
+        O, LSE = OA.paged_attention(_bits(q), _bits(k_cache), _bits(v_cache), plan.qo, kv_indptr.numpy(),
+                                    kv_indices.numpy(), kv_last_page_len.numpy(), k_cache.shape[1], sm_scale,
+                                    requests=reqs)
+        for r in reqs:
+            a, b = int(plan.qo[r]), int(plan.qo[r + 1])
+            o[a:b] = torch.from_numpy(O[a:b])
+            lse[a:b] = torch.from_numpy(LSE[a:b])
+
+    monkeypatch.setattr(R, "plan_paged_subset", plan_paged_subset)
+    monkeypatch.setattr(R, "paged_attn_fwd", paged_attn_fwd)
+    rng = np.random.Generator(np.random.PCG64(71))
+    lengths, q_lens, P, hq, hk, d = [300, 17, 0, 64, 200, 5], [1, 40, 1, 1, 128, 0], 16, 64, 8, 128
+    kv_indptr, kv_indices, last, num_pages = build_page_table(rng, lengths, P, extra_pages=2)
+    qo = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q = normal_bf16(71, 1, (int(qo[-1]), hq, d))
+    k = normal_bf16(71, 2, (num_pages, P, hk, d))
+    v = normal_bf16(71, 3, (num_pages, P, hk, d))
+    scale = 1 / math.sqrt(d)
+    o, lse, ex = R.pod_attention(_tb(q), _tb(k), _tb(v), qo, kv_indptr, torch.from_numpy(kv_indices), last,
+                                 sm_scale=scale, policy="none")
+    # decode requests (one query token) on the all-KV-heads decode kernel, the rest on the prefill kernel
+    assert launches == [(3, [0, 2, 3]), (4, [1, 4])]
+    O, LSE = OA.paged_attention(q, k, v, qo, kv_indptr, kv_indices, last, P, scale)
+    np.testing.assert_allclose(o.numpy(), O, rtol=0, atol=1e-6)
+    np.testing.assert_array_equal(np.isneginf(lse.numpy()), np.isneginf(LSE))
+    fin = np.isfinite(LSE)
+    np.testing.assert_allclose(lse.numpy()[fin], LSE[fin], rtol=0, atol=1e-6)
+
+
+def test_subset_planner_rejects_bad_lists():
+    qo, ip, la = np.array([0, 1, 2]), np.array([0, 1, 2]), np.array([3, 3])
+    for bad in ([0, 0], [2], [-1]):
+        try:
+            skv.plan_paged_subset(qo, ip, la, 16, 8, 2, 64, bad, "none")
+        except skv.SkvError as e:
+            assert e.code == skv.ERR_INVALID
+        else:
+            raise AssertionError(f"accepted {bad}")
+    plan = skv.plan_paged_subset(qo, ip, la, 16, 8, 2, 64, [], "none")
+    assert plan.info.num_work == 0
