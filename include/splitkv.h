@@ -289,8 +289,8 @@ SKV_API skv_status skv_plan_paged_subset(int32_t batch, const int32_t* qo_indptr
  *   sees keys t <= L_r - n_q + i (multi-token prediction decode, mentioned on the FlashInfer PR
  *   #3309 page; causal prefill).  The call splits this into two unmasked problems whose exact
  *   merge (skv_merge_states, two states per query row) is the causal result:
- *     prefix -- request r keeps its first ceil(Lp_r / P) pages, Lp_r = max(0, L_r - n_q + 1): the
- *               keys every query token of r sees (same query rows, same page size);
+ *     prefix -- request r keeps its first ceil(Lp_r / P) pages, Lp_r = min(L_r, max(0, L_r - n_q + 1)):
+ *               the keys every query token of r sees (same query rows, same page size);
  *     diag   -- one request per query row j = qo_indptr[r] + i, page size 1, whose "pages" are the
  *               token rows page * P + slot of keys [Lp_r, L_r - n_q + 1 + i): the keys token i sees
  *               beyond the prefix (none for i = 0).  Run it on a [num_pages * P, 1, ...] view of the
