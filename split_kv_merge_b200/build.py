@@ -1,7 +1,6 @@
 """Build libsplitkv.so (sm_100a) in-tree with nvcc.
 
-    python split_kv_merge_b200/build.py [--force]      (SPLITKV_WAIT_LIMIT_NS=<ns> sets the kernels'
-                                                        bounded-wait limit; default 2 s)
+    python split_kv_merge_b200/build.py [--force]
 
 Each .cu under csrc/ compiles to _build/<name>.o (skipped when newer than its sources and the
 headers), then everything links into split_kv_merge_b200/libsplitkv.so with the CUDA runtime
@@ -24,8 +23,6 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
-if os.environ.get("SPLITKV_WAIT_LIMIT_NS"):  # bounded-wait limit of the kernels, in ns (default 2 s)
-    FLAGS.append(f"-DSPLITKV_WAIT_LIMIT_NS={int(os.environ['SPLITKV_WAIT_LIMIT_NS'])}ull")
 
 
 def _headers():

@@ -20,13 +20,8 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Every wait gives up after this long (device error SKV_DEV_TIMEOUT instead of a hang).  A build
-// may set another limit with -DSPLITKV_WAIT_LIMIT_NS=<ns> (SPLITKV_WAIT_LIMIT_NS in the build
-// environment).
-#ifndef SPLITKV_WAIT_LIMIT_NS
-#define SPLITKV_WAIT_LIMIT_NS 2000000000ull
-#endif
-constexpr uint64_t kWaitLimitNs = SPLITKV_WAIT_LIMIT_NS;
+// Every wait gives up after this long (device error SKV_DEV_TIMEOUT instead of a hang).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
