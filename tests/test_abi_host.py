@@ -35,7 +35,14 @@ def test_library_exports_every_declared_symbol():
 
 
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a C compiler")
-def test_binding_structs_match_the_c_header(tmp_path):
+def _scratch_dir():
+    """Build products of the C tests go to the repository's ignored build folder."""
+    d = os.path.join(ROOT, "_build", "c_tests")
+    os.makedirs(d, exist_ok=True)
+    return d
+
+
+def test_binding_structs_match_the_c_header():
     """Every ctypes structure of the binding has the size, field offsets and field sizes of the C
     struct it mirrors (compiled from include/splitkv.h with gcc)."""
     pairs = [(skv.PlanInfo, "skv_plan_info"), (skv.PagedParams, "skv_paged_params"),
@@ -48,10 +55,11 @@ def test_binding_structs_match_the_c_header(tmp_path):
             lines.append(f'  printf("{cname} {field} %zu %zu\\n", offsetof({cname}, {field}), '
                          f'sizeof((({cname}*)0)->{field}));')
     lines += ["  return 0;", "}"]
-    src = tmp_path / "layout.c"
-    src.write_text("\n".join(lines) + "\n")
-    exe = tmp_path / "layout"
-    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    src = os.path.join(_scratch_dir(), "layout.c")
+    with open(src, "w") as f:
+        f.write("\n".join(lines) + "\n")
+    exe = os.path.join(_scratch_dir(), "layout")
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), src, "-o", exe], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
     c_layout = {tuple(l.split()[:2]): [int(x) for x in l.split()[2:]] for l in out if l.strip()}
     for cls, cname in pairs:
@@ -62,11 +70,11 @@ def test_binding_structs_match_the_c_header(tmp_path):
 
 
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs a C compiler")
-def test_plain_c_consumer(tmp_path):
+def test_plain_c_consumer():
     """tests/c/host_calls.c, compiled against include/splitkv.h and linked to libsplitkv.so, runs the
     host-only entry points from C (planners, causal planner, validation, status strings)."""
     lib_dir = os.path.dirname(skv.library_path())
-    exe = tmp_path / "host_calls"
+    exe = os.path.join(_scratch_dir(), "host_calls")
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "host_calls.c"),
                     "-L", lib_dir, "-lsplitkv", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
