@@ -11,8 +11,8 @@
 // converted and a 64-token tile is 36 KB of shared memory (four or three of them in flight).
 //   * Both other operands are split into two e4m3 terms, hi = rn(x) and lo = rn(x - hi), stacked
 //     as 2 NR columns of N: queries (bf16, 8 significant bits) after a power-of-two scaling that
-//     puts the unit's largest |q| in [128, 256) -- exact for every |q| above 2^-10 of that maximum
-//     -- and the softmax weights p in [0, 2^8] (bf16-like precision, 8 significant bits).  The
+//     puts the unit's largest |q| in [128, 256) -- exact for every |q| of at least 2^-9 of that
+//     maximum, within 2^-17 of it below -- and the softmax weights p in [0, 2^8] (bf16-like precision, 8 significant bits).  The
 //     scaling goes back into the softmax scale; S and O sum their hi and lo columns.
 //   * S^T[64 tokens, 2 NR] = C . [Q_hi; Q_lo]^T, K = 32 per MMA: 16 ckv k-steps (128-byte
 //     swizzled rows) + 2 rope k-steps (64-byte swizzled rows); M = 64, so TMEM rows sit in lanes
