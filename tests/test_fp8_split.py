@@ -55,3 +55,17 @@ def test_random_units_at_many_scales():
         assert np.array_equal(back[big], qs[big])
         assert np.max(np.abs(back - qs)) <= 2.0 ** -10
         assert np.max(np.abs(back - qs)) / np.max(np.abs(qs)) <= 2.0 ** -17
+
+
+def test_softmax_weights_keep_eight_bits():
+    """Softmax weights p in [0, 2^8] (fp32, not scaled) split the same way: relative error at most
+    2^-8 from 2^-2 up (lo normal), absolute error at most 2^-10 below (lo on the subnormal grid)."""
+    rng = np.random.Generator(np.random.PCG64(8))
+    p = torch.from_numpy(np.concatenate([rng.random(200000) * 256.0, 2.0 ** rng.uniform(-20, 8, 200000),
+                                         [0.0, 1.0, 256.0]]).astype(np.float32))
+    hi = p.to(torch.float8_e4m3fn).float()
+    lo = (p - hi).to(torch.float8_e4m3fn).float()
+    err = (hi.double() + lo.double() - p.double()).abs()
+    normal = p >= 0.25
+    assert bool(torch.all(err[normal] <= 2.0 ** -8 * p[normal].double()))
+    assert float(err[~normal].max()) <= 2.0 ** -10
