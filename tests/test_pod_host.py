@@ -1,4 +1,4 @@
-"""Host logic of mixed prefill + decode (POD) batches (no GPU): ``runner.pod_attention`` plans the
+"""Host logic of the composed calls (no GPU).  Mixed prefill + decode (POD) batches: ``runner.pod_attention`` plans the
 decode requests and the prefill requests of one batch separately (``skv_plan_paged_subset``) and
 launches both plans on the batch's own buffers.  With the launch replaced by a float64 stand-in
 that computes exactly the requests of the plan it is given (and writes only their rows), the two
@@ -77,3 +77,35 @@ def test_subset_planner_rejects_bad_lists():
             raise AssertionError(f"accepted {bad}")
     plan = skv.plan_paged_subset(qo, ip, la, 16, 8, 2, 64, [], "none")
     assert plan.info.num_work == 0
+
+
+def test_route_merge_composition(monkeypatch):
+    """``RouteMerge``: one partial launch per KV chunk over each query's selected rows (page size 1,
+    a page id is a token row), then the merge over chunks -- with the launches replaced by oracle
+    stand-ins the result equals unsplit attention over the union of the selections."""
+    from workloads import route_case
+
+    def mla_decode_fwd(q_nope, q_pe, ckv, kpe, kv_indptr, kv_indices, kv_last_page_len, plan, o, lse, o_part,
+                       lse_part, status, sm_scale, kv_scale, num_pages, stream):
+        O, LSE = OA.mla_decode(_bits(q_nope), _bits(q_pe), _bits(ckv), _bits(kpe), kv_indptr.numpy(),
+                               kv_indices.reshape(-1).numpy(), kv_last_page_len.numpy(), ckv.shape[1], sm_scale)
+        o.copy_(torch.from_numpy(O))
+        lse.copy_(torch.from_numpy(LSE))
+
+    def merge_states(o_states, lse_states, o_out, lse_out=None, state_indptr=None, num_states=0, stream=None):
+        O, LSE = OA.merge_states(o_states.double().numpy(), lse_states.double().numpy())
+        o_out.copy_(torch.from_numpy(O))
+        lse_out.copy_(torch.from_numpy(LSE))
+
+    monkeypatch.setattr(R, "mla_decode_fwd", mla_decode_fwd)
+    monkeypatch.setattr(R, "merge_states", merge_states)
+    c = route_case(num_queries=5, num_chunks=3, chunk_tokens=64, per_chunk=10)
+    cache = _tb(c.cache).view(c.cache.shape[0], 1, 576)
+    rm = R.RouteMerge(c.sel, c.num_heads, "cpu")
+    sel_cqk = torch.from_numpy(np.ascontiguousarray(c.sel.transpose(1, 0, 2)).astype(np.int32))
+    o, lse = rm(_tb(c.q_nope), _tb(c.q_pe), cache[..., :512], cache[..., 512:], sel_cqk, sm_scale=c.sm_scale)
+    u = c.union_mla()
+    O, LSE = OA.mla_decode(u.q_nope, u.q_pe, u.ckv, u.kpe, u.kv_indptr, u.kv_indices, u.kv_last_page_len, 1,
+                           u.sm_scale)
+    np.testing.assert_allclose(o.numpy(), O[:, 0], rtol=0, atol=1e-6)
+    np.testing.assert_allclose(lse.numpy(), LSE[:, 0], rtol=0, atol=1e-6)
