@@ -38,7 +38,8 @@ What it computes (definitions; every step is the plain formula, no tiling or onl
   latent cache row per token holds a 512-d compressed KV (ckv) and a 64-d rope part (kpe),
   shared by every head; s_t = scale * (q_nope . ckv_t + q_pe . kpe_t), v_t = ckv_t.  Folding
   seqlen_q into heads only re-labels rows, so it does not appear here.
-* fp8 cache -- OCP e4m3fn codes decoded exactly and multiplied by the per-tensor scale.
+* fp8 cache -- OCP e4m3fn codes decoded exactly and multiplied by the per-tensor scale (the MLA
+  latent cache, and the GQA K/V cache: ``kv_dtype="e4m3"``).
 """
 from __future__ import annotations
 
@@ -144,7 +145,7 @@ def _decode_kv(x, kv_dtype: str, kv_scale: float) -> np.ndarray:
 
 
 def _gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, page_size, sm_scale,
-                 r, heads, page_begin=0, page_end=None, causal=False):
+                 r, heads, page_begin=0, page_end=None, causal=False, kv_dtype="bf16", kv_scale=1.0):
     hq, hk = q.shape[1], k.shape[2]
     g = hq // hk
     pages, slots = request_token_slots(kv_indptr, kv_indices, kv_last_page_len, page_size, r,
@@ -158,8 +159,8 @@ def _gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, pa
     o = np.zeros((n_q, len(heads), dv))
     lse = np.zeros((n_q, len(heads)))
     for kh in sorted({h // g for h in heads}):
-        kk = bf16_to_f64(k[pages, slots, kh])                            # [L, D]
-        vv = bf16_to_f64(v[pages, slots, kh])                            # [L, Dv]
+        kk = _decode_kv(k[pages, slots, kh], kv_dtype, kv_scale)         # [L, D]
+        vv = _decode_kv(v[pages, slots, kh], kv_dtype, kv_scale)         # [L, Dv]
         for j, h in enumerate(heads):
             if h // g != kh:
                 continue
@@ -170,10 +171,11 @@ def _gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, pa
 
 def paged_attention(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, page_size: int,
                     sm_scale: float, requests: Optional[Iterable[int]] = None,
-                    heads: Optional[Sequence[int]] = None, causal: bool = False):
-    """GQA attention over a paged bf16 KV cache.
+                    heads: Optional[Sequence[int]] = None, causal: bool = False, kv_dtype: str = "bf16",
+                    kv_scale: float = 1.0):
+    """GQA attention over a paged KV cache (bf16, or e4m3 codes times the per-tensor ``kv_scale``).
 
-    q: bf16 bits [total_q, Hq, D]; k, v: bf16 bits [num_pages, P, Hk, D] (any strides);
+    q: bf16 bits [total_q, Hq, D]; k, v: bf16 bits or e4m3 codes [num_pages, P, Hk, D] (any strides);
     returns O [total_q, |heads|, Dv] and LSE [total_q, |heads|] in float64 (rows of requests
     not in ``requests`` are NaN).  ``causal``: each query token sees only keys up to its own
     position (``causal_visible``)."""
@@ -184,13 +186,15 @@ def paged_attention(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len,
     for r in requests:
         a, b = int(qo_indptr[r]), int(qo_indptr[r + 1])
         O[a:b], LSE[a:b] = _gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len,
-                                        page_size, sm_scale, r, heads, causal=causal)
+                                        page_size, sm_scale, r, heads, causal=causal, kv_dtype=kv_dtype,
+                                        kv_scale=kv_scale)
     return O, LSE
 
 
 def paged_attention_partials(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len,
                              page_size: int, sm_scale: float, split_page_start,
-                             requests: Optional[Iterable[int]] = None, causal: bool = False):
+                             requests: Optional[Iterable[int]] = None, causal: bool = False,
+                             kv_dtype: str = "bf16", kv_scale: float = 1.0):
     """Per request r and split j over logical pages [split_page_start[r][j], [j+1]): the
     partial (O_j, LSE_j) of every query token and head.  Returns {r: (O [S, n_q, Hq, Dv],
     LSE [S, n_q, Hq])}."""
@@ -200,7 +204,8 @@ def paged_attention_partials(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_
     for r in requests:
         b = split_page_start[r]
         parts = [_gqa_request(q, k, v, qo_indptr, kv_indptr, kv_indices, kv_last_page_len, page_size,
-                              sm_scale, r, heads, b[j], b[j + 1], causal) for j in range(len(b) - 1)]
+                              sm_scale, r, heads, b[j], b[j + 1], causal, kv_dtype, kv_scale)
+                 for j in range(len(b) - 1)]
         out[r] = (np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
     return out
 

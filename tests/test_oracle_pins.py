@@ -308,6 +308,41 @@ def pin_e4m3():
     np.testing.assert_array_equal(e4m3_encode(got[ok]), codes[ok])
 
 
+def pin_gqa_e4m3():
+    """GQA over an e4m3 K/V cache with per-tensor scale 2^-3 equals GQA over the bf16 cache holding
+    the same dequantised values (exact in bf16: at most 4 significant bits), computed by torch's
+    float64 SDPA on the dense rows the test gathers itself -- and differs from ignoring the scale."""
+    c = _tiny_case(71, hq=4, hk=2, d=8, P=4)
+    rng = np.random.Generator(np.random.PCG64(72))
+    kc = e4m3_encode(rng.standard_normal(c["k"].shape) * 40)
+    vc = e4m3_encode(rng.standard_normal(c["v"].shape) * 40)
+    scale = 2.0 ** -3
+    O, LSE = OA.paged_attention(c["q"], kc, vc, c["qo_indptr"], c["kv_indptr"], c["kv_indices"],
+                                c["kv_last_page_len"], c["page_size"], c["sm_scale"], kv_dtype="e4m3", kv_scale=scale)
+    kf = torch.from_numpy(kc).view(torch.float8_e4m3fn).double() * scale
+    vf = torch.from_numpy(vc).view(torch.float8_e4m3fn).double() * scale
+    assert torch.equal(kf.bfloat16().double(), kf) and torch.equal(vf.bfloat16().double(), vf)
+    P, hq, hk = c["page_size"], 4, 2
+    for r in range(len(c["kv_indptr"]) - 1):
+        n = int(c["kv_indptr"][r + 1] - c["kv_indptr"][r])
+        L = 0 if n == 0 else (n - 1) * P + int(c["kv_last_page_len"][r])
+        a, b = int(c["qo_indptr"][r]), int(c["qo_indptr"][r + 1])
+        if L == 0 or a == b:
+            continue
+        pages = torch.from_numpy(c["kv_indices"][c["kv_indptr"][r]:c["kv_indptr"][r + 1]].astype(np.int64))
+        kd = kf[pages].reshape(n * P, hk, -1)[:L]
+        vd = vf[pages].reshape(n * P, hk, -1)[:L]
+        qd = torch.from_numpy(OA.bf16_to_f64(c["q"][a:b]))
+        for h in range(hq):
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qd[None, None, :, h], kd[None, None, :, h // 2], vd[None, None, :, h // 2], scale=c["sm_scale"])
+            np.testing.assert_allclose(O[a:b, h], ref[0, 0].numpy(), rtol=0, atol=1e-12)
+    O1, _ = OA.paged_attention(c["q"], kc, vc, c["qo_indptr"], c["kv_indptr"], c["kv_indices"],
+                               c["kv_last_page_len"], c["page_size"], c["sm_scale"], kv_dtype="e4m3", kv_scale=1.0)
+    fin = np.isfinite(LSE)
+    assert np.max(np.abs(O1[fin] - O[fin])) > 0.1
+
+
 def pin_bf16():
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     got = OA.bf16_to_f64(bits)
@@ -334,7 +369,7 @@ def test_e4m3_encoder_is_nearest_even():
 
 
 PINS = [pin_brute_force, pin_decimal, pin_sdpa_library, pin_closed_forms, pin_split_merge,
-        pin_merge_special, pin_permutation, pin_broadcast, pin_mla, pin_e4m3, pin_bf16]
+        pin_merge_special, pin_permutation, pin_broadcast, pin_mla, pin_e4m3, pin_gqa_e4m3, pin_bf16]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -383,6 +418,8 @@ MUTATIONS = [
     ("_mla_request", "+ qp.reshape(q_len * nh, -1) @ kr.T", ""),
     ("_mla_request", "o, lse = _softmax_attend(s, c)", "o, lse = _softmax_attend(s, np.concatenate([c[:, 64:], c[:, :64]], 1))"),
     ("bf16_to_f64", "<< np.uint32(16)", "<< np.uint32(15)"),
+    ("_gqa_request", "kk = _decode_kv(k[pages, slots, kh], kv_dtype, kv_scale)",
+     "kk = _decode_kv(k[pages, slots, kh], kv_dtype, 1.0)"),
 ]
 
 
