@@ -48,3 +48,26 @@ def test_committed_traffic_record_names_the_decode_kernel():
         rec = json.load(f)
     r = rec["gqa_tc_wide_kernel"]
     assert r["bytes_per_launch"] > 0 and 1.0 <= r["traffic_over_algorithmic"] < 1.1
+
+
+def test_physical_gpu_and_rank_environment(monkeypatch):
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3,5")
+    assert bench._physical_gpu(0) == 3 and bench._physical_gpu(1) == 5 and bench._physical_gpu(2) == 2
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "GPU-1234abcd")     # UUIDs: keep the local index
+    assert bench._physical_gpu(0) == 0
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES")
+    assert bench._physical_gpu(1) == 1
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench._dist() == (1, 0, 0)
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    monkeypatch.setenv("RANK", "2")
+    monkeypatch.setenv("LOCAL_RANK", "2")
+    assert bench._dist() == (4, 2, 2)
+
+
+def test_kv_bytes_counts_k_and_v_once():
+    from workloads import tiny_gqa_case
+    c = tiny_gqa_case()
+    # lengths {37, 128, 200, 256} x 2 KV heads x 64 dims x 2 bytes x (K, V)
+    assert bench._kv_bytes(c) == (37 + 128 + 200 + 256) * 2 * 64 * 2 * 2
