@@ -194,6 +194,10 @@ SKV_API skv_status skv_merge_plan(const float* o_part, const float* lse_part, co
  *   that device current); make that first call before any stream capture.  Allocates nothing.
  *   All calls share the array and it keeps the last call's contents (every partial is written
  *   before it is read, so nothing needs clearing); calls that overlap on the GPU race.
+ *   `info` must be the summary returned together with `plan_d`: the size check reads
+ *   info->num_partial_rows while the kernels write the partial rows plan_d names, so a summary
+ *   from another plan would let them write past the array (the regular entry point would
+ *   write past the caller's own buffers instead).
  * ----------------------------------------------------------------------------------------- */
 SKV_API skv_status skv_paged_attn_fwd_static_scratch(const skv_paged_params* p, const int32_t* plan_d,
                                                      const skv_plan_info* info, skv_stream_t stream);

@@ -449,27 +449,14 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
   return r == CUDA_SUCCESS;
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  }
-  return n;
-}
+int num_sms() { return device_sm_count(); }
 
 template <int NC, typename OutT>
 int launch_t(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm, const TcArgs& a,
              const WorkItem* work, cudaStream_t s) {
   const int smem = Smem::total + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gqa_tc_decode_kernel<NC, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
-    if (e != cudaSuccess) return (int)e;
-    attr_set = true;
-  }
+  static DeviceSmemAttr attr;  // per device: the attribute belongs to the current device
+  if (const int e = attr.ensure(reinterpret_cast<const void*>(gqa_tc_decode_kernel<NC, OutT>), smem)) return e;
   const int grid = std::min(a.num_units, num_sms());
   gqa_tc_decode_kernel<NC, OutT><<<grid, kThreads, smem, s>>>(km, vm, qm, a, work);
   return (int)cudaGetLastError();

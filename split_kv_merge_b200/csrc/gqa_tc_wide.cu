@@ -572,13 +572,8 @@ template <int G, typename OutT>
 int launch_w(const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& qm, const WArgs& a,
              const WorkItem* work, cudaStream_t s) {
   const int smem = Smem::total + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gqa_tc_wide_kernel<G, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return (int)e;
-    attr_set = true;
-  }
+  static DeviceSmemAttr attr;  // per device: the attribute belongs to the current device
+  if (const int e = attr.ensure(reinterpret_cast<const void*>(gqa_tc_wide_kernel<G, OutT>), smem)) return e;
   gqa_tc_wide_kernel<G, OutT><<<a.num_ctas, kThreads, smem, s>>>(km, vm, qm, a, work);
   return (int)cudaGetLastError();
 }

@@ -747,12 +747,8 @@ bool make_map_m(CUtensorMap* m, const void* base, const cuuint64_t* dims, const 
 template <int NR, typename OutT>
 int launch_m(const CUtensorMap* maps, const MArgs& a, int num_ctas, const WorkItem* work, cudaStream_t s) {
   const int smem = MlaCfg<NR>::total + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel<NR, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return (int)e;
-    attr_set = true;
-  }
+  static DeviceSmemAttr attr;  // per device: the attribute belongs to the current device
+  if (const int e = attr.ensure(reinterpret_cast<const void*>(mla_tc_kernel<NR, OutT>), smem)) return e;
   // the three extra gather warps exist only in row-gather mode
   const int threads = a.gather ? kThreads : kThreads - (kGatherWarps - 1) * 32;
   mla_tc_kernel<NR, OutT><<<num_ctas, threads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a, work);

@@ -701,13 +701,8 @@ bool make_map8(CUtensorMap* m, CUtensorMapDataType type, CUtensorMapSwizzle swz,
 template <int NR, typename OutT>
 int launch_m8(const CUtensorMap* maps, const M8Args& a, int num_ctas, const WorkItem* work, cudaStream_t s) {
   const int smem = Cfg8<NR>::total + 1024;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(mla_tc_fp8_kernel<NR, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return (int)e;
-    attr_set = true;
-  }
+  static DeviceSmemAttr attr;  // per device: the attribute belongs to the current device
+  if (const int e = attr.ensure(reinterpret_cast<const void*>(mla_tc_fp8_kernel<NR, OutT>), smem)) return e;
   mla_tc_fp8_kernel<NR, OutT><<<num_ctas, kThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a, work);
   return (int)cudaGetLastError();
 }

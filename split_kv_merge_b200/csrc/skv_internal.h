@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/splitkv.h"
 
 namespace skv {
@@ -32,6 +34,52 @@ enum KernelId : int32_t {
   KERNEL_MLA_TC16 = 12,  // tensor-core MLA, 16 query rows per unit (bf16 or e4m3 cache)
   KERNEL_MLA_TC32 = 13,  // tensor-core MLA, 32 query rows per unit (bf16 or e4m3 cache)
 };
+
+// Host caches of per-device state.  cudaFuncSetAttribute and device attributes belong to the
+// device current at the call, so each cache is indexed by that device's ordinal: a launch on a
+// second GPU raises the kernel's shared-memory limit there too.
+constexpr int kMaxCachedDevices = 64;
+
+inline int current_device() {
+  int d = 0;
+  return cudaGetDevice(&d) == cudaSuccess ? d : -1;
+}
+
+// One per kernel instantiation: raises the kernel's dynamic shared-memory limit to `bytes` on
+// the current device, once per device (devices beyond the table set it on every launch).
+class DeviceSmemAttr {
+ public:
+  int ensure(const void* func, int bytes) {
+    const int dev = current_device();
+    if (dev < 0) return (int)cudaErrorNoDevice;
+    const bool cached = dev < kMaxCachedDevices;
+    if (cached && done_[dev].load(std::memory_order_acquire) == bytes) return 0;
+    const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return (int)e;
+    if (cached) done_[dev].store(bytes, std::memory_order_release);
+    return 0;
+  }
+
+ private:
+  std::atomic<int> done_[kMaxCachedDevices] = {};
+};
+
+// SM count of the current device (cached per device; 148 if the query fails).
+inline int device_sm_count() {
+  static std::atomic<int> cache[kMaxCachedDevices];
+  const int dev = current_device();
+  if (dev >= 0 && dev < kMaxCachedDevices) {
+    const int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+  }
+  int n = 0;
+  if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  if (dev < kMaxCachedDevices) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 
 // Plan words: [work items (8 words each)] [merge items (4 words each)].
 inline int64_t plan_words(int32_t num_work, int32_t num_merge) {

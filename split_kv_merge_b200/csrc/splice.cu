@@ -173,18 +173,17 @@ __global__ void __launch_bounds__(kWarps * 32) splice_kernel(const __grid_consta
 }
 
 int resident_grid(int64_t total) {
-  static int full = 0;
-  if (full == 0) {
-    int dev = 0, sms = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      sms = 148;
+  // resident CTAs per SM depend only on the kernel (same on every B200); SMs come per device
+  static std::atomic<int> per_sm_cache{0};
+  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
+  if (per_sm == 0) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, splice_kernel, kWarps * 32, 0) != cudaSuccess ||
         per_sm <= 0)
       per_sm = 4;
     cudaGetLastError();
-    full = sms * per_sm;
+    per_sm_cache.store(per_sm, std::memory_order_relaxed);
   }
+  const int64_t full = (int64_t)device_sm_count() * per_sm;
   const int64_t want = (total + kRows * kWarps - 1) / (kRows * kWarps);  // a full row group per warp
   return (int)std::max<int64_t>(1, std::min<int64_t>(want, full));
 }

@@ -18,6 +18,8 @@
 //  - Every call shares the one array and it keeps the last call's contents.  The attention
 //    kernel writes every partial row before the merge reads it, so nothing needs clearing;
 //    calls that overlap on the GPU (different streams) race on the array.
+//  - `info` must be the summary the planner returned with `plan_d`: the size check uses
+//    info->num_partial_rows, the kernels the partial rows stored in plan_d.
 #include <mutex>
 
 #include "skv_internal.h"

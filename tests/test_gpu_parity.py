@@ -1,6 +1,11 @@
 """GPU parity: the CUDA path (through the C ABI) against the float64 oracle on the same seeded
-inputs.  Tolerances: O max-abs <= 1e-2 (3e-2 for the e4m3 MLA cache), LSE abs <= 1e-3; page
-gather bit-exact; broadcast KV vs replicated KV bit-exact; repeated runs bit-identical.
+inputs.  Tolerances: O max-abs <= 1e-2, LSE abs <= 1e-3; page gather bit-exact; broadcast KV vs
+replicated KV bit-exact; repeated runs bit-identical.  The e4m3 MLA cache is held to the same
+1e-2 as bf16 (its tensor-core path splits the bf16 operand into two exact e4m3 terms, so only the
+cache is fp8, and the oracle reads the same decoded cache), which is tighter than the 3e-2 the
+fp8 case is allowed.  bf16 outputs: the fp32 value a kernel rounds is checked at 1e-2 and the
+rounding to bf16 bit for bit (a bf16 number of magnitude 4 or more is up to 2^-6 from the real
+value it stands for, so no kernel's bf16 output can be held to 1e-2 there).
 
 Sizes: reduced workloads the oracle finishes in seconds (several tiles, ragged tails) checked
 element by element, and the full workload sizes checked on seeded samples of requests
@@ -20,6 +25,7 @@ from workloads.device import mla_to_device, paged_to_device, route_to_device
 pytestmark = pytest.mark.gpu
 
 O_TOL, LSE_TOL, O_TOL_FP8 = 1e-2, 1e-3, 3e-2
+assert O_TOL <= O_TOL_FP8   # the e4m3 cases below are held to O_TOL, inside the fp8 allowance
 DEV = "cuda:0"
 
 
@@ -195,7 +201,7 @@ def test_mla_reduced(H, q_len, kv_dtype):
     rows = {12: 16, 13: 32}.get(info.kernel, 128)   # rows per tile of the kernel the planner chose
     assert info.q_tile == (skv.mla_fold_ratio(H, q_len, rows) if H <= rows else 1)
     O, LSE = _oracle_mla(c)
-    _cmp(_np(o), _np(lse), O, LSE, O_TOL_FP8 if kv_dtype == "e4m3" else O_TOL, where=f"mla {H} {q_len} {kv_dtype}")
+    _cmp(_np(o), _np(lse), O, LSE, O_TOL, where=f"mla {H} {q_len} {kv_dtype}")
 
 
 @pytest.mark.parametrize("kv_dtype", ["bf16", "e4m3"])
@@ -206,8 +212,7 @@ def test_mla_full_sampled(H, q_len, kv_dtype):
     L = c.kv_lengths()
     reqs = sorted({int(np.argmin(L)), int(np.argmax(L)), 5})
     O, LSE = _oracle_mla(c, requests=reqs)
-    _cmp(_np(o)[reqs], _np(lse)[reqs], O[reqs], LSE[reqs], O_TOL_FP8 if kv_dtype == "e4m3" else O_TOL,
-         where=f"mla full {H} {q_len} {kv_dtype}")
+    _cmp(_np(o)[reqs], _np(lse)[reqs], O[reqs], LSE[reqs], O_TOL, where=f"mla full {H} {q_len} {kv_dtype}")
 
 
 def _empty_request(c, j):
@@ -231,8 +236,7 @@ def test_mla_tensor_core_page_sizes_and_edges(kv_dtype, page_size, policy, param
     o, lse, ex = _run_mla(c, policy, param)
     assert ex["plan"].info.kernel == 12
     O, LSE = _oracle_mla(c)
-    _cmp(_np(o), _np(lse), O, LSE, O_TOL_FP8 if kv_dtype == "e4m3" else O_TOL,
-         where=f"mla edges {kv_dtype} P{page_size} {policy}")
+    _cmp(_np(o), _np(lse), O, LSE, O_TOL, where=f"mla edges {kv_dtype} P{page_size} {policy}")
 
 
 @pytest.mark.parametrize("H,q_len", [(16, 1), (16, 2), (128, 1)])
@@ -461,11 +465,11 @@ def test_prefill_tensor_core_rising_scores_fp32_and_bf16_out():
     o, lse, ex, _ = _run_paged(c, "fixed", 2)
     assert ex["plan"].info.kernel == 4
     _cmp(_np(o), _np(lse), O, LSE, where="prefill rising")
-    # bf16 output: the final rounding adds up to half a bf16 ulp (|O| * 2^-8 bounds it) on top of
-    # the fp32 result's error; rows here are close to single V rows, so |O| reaches a few units
+    # bf16 output (rows here are close to single V rows, so |O| reaches 4 and more): the fp32
+    # value checked above, rounded once to bf16 (nearest even), bit for bit
     ob, lb, _, _ = _run_paged(c, "fixed", 2, o_dtype=torch.bfloat16)
-    err = np.abs(_np(ob) - O) - np.abs(O) * 2.0 ** -8
-    assert float(err.max()) <= O_TOL, f"prefill rising bf16: {float(err.max())}"
+    assert float(np.abs(O).max()) >= 4.0        # the case really has values bf16 cannot hold to 1e-2
+    assert torch.equal(ob.cpu(), o.cpu().to(torch.bfloat16)), "bf16 output is not the rounded fp32 output"
     assert float(np.max(np.abs(_np(lb) - LSE))) <= LSE_TOL
 
 

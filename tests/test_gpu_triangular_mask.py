@@ -2,8 +2,8 @@
 position) against the oracle's causal attention: GQA decode with several query tokens, GQA
 causal prefill, and MLA multi-token decode, through ``runner.paged_attention`` /
 ``runner.mla_decode`` with ``causal=True`` (a prefix pass, a diagonal pass over token rows and
-the exact merge).  Tolerances as for the unmasked paths: O max-abs <= 1e-2 (3e-2 for the e4m3
-cache), LSE <= 1e-3; rows that see no key must give O = 0, LSE = -inf."""
+the exact merge).  Tolerances as for the unmasked paths: O max-abs <= 1e-2 (the e4m3 cache too,
+inside its 3e-2 allowance), LSE <= 1e-3; rows that see no key must give O = 0, LSE = -inf."""
 import math
 
 import numpy as np
@@ -75,4 +75,4 @@ def test_causal_mla_multi_token(q_len, kv_dtype):
     assert int(status.item()) == 0
     O, LSE = OA.mla_decode(c.q_nope, c.q_pe, c.ckv, c.kpe, c.kv_indptr, c.kv_indices, c.kv_last_page_len,
                            c.page_size, c.sm_scale, c.kv_dtype, c.kv_scale, causal=True)
-    _cmp(o, lse, O, LSE, 3e-2 if kv_dtype == "e4m3" else 1e-2, f"causal mla q{q_len} {kv_dtype}")
+    _cmp(o, lse, O, LSE, 1e-2, f"causal mla q{q_len} {kv_dtype}")
