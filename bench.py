@@ -355,6 +355,10 @@ def run_ours(args):
     }
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = _cpu_baseline(cases)
+    if ws == 1 and not args.no_configs:
+        del runs
+        torch.cuda.empty_cache()
+        line["configs"] = all_configs(args, dev, stream, skv, torch)
     print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
@@ -412,113 +416,243 @@ def _e2e(args, runs, dev, stream, skv, torch):
 
 
 # ----------------------------------------------------------------------------- other configurations
-def _time_device(step, steps, warmup, torch, stream):
+CONFIG_NAMES = (["tiny", "shared_kv"] + [f"mla_h{h}_q{q}_{d}" for h in (16, 128) for q in (1, 4)
+                                         for d in ("bf16", "e4m3")]
+                + ["mla_h16_q4_bf16_causal", "route", "fetch_splice"])
+L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2: written before every timed call
+
+
+def _threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        return 1
+
+
+def _time_calls(step, steps, warmup, torch, stream, flush):
+    """Mean device time (ms) of one call: `warmup` untimed calls, then `steps` calls each
+    bracketed by CUDA events on the launching stream, with L2 flushed (a 512 MB write) before
+    every timed call."""
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
         step()
-    e1.record(stream)
+        b.record(stream)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
 
 
-def run_workload(args):
-    """One timed JSON line per configuration other than the Llama-70B decode (device time, inputs
-    resident; KV working sets above L2 except the tiny and shared-KV cases, which are noted)."""
-    import torch
-    import split_kv_merge_b200 as skv
+def _sampled(units, budget_s):
+    """Run oracle sample units (callables returning the (bytes, FLOPs) they covered) until
+    budget_s has passed; returns ((bytes, FLOPs) done, seconds, units run).  At least one runs."""
+    done, n, t0 = np.zeros(2), 0, time.perf_counter()
+    for u in units:
+        done += np.asarray(u(), dtype=np.float64)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return done, time.perf_counter() - t0, n
+
+
+def _setup_config(name, dev, skv, torch, stream):
+    """Device inputs, the timed call and its algorithmic bytes / FLOPs for one configuration, plus
+    the oracle sample units (each returns the algorithmic bytes and FLOPs it covered) and the
+    kernel it runs."""
+    import oracle.attention as OA
     from workloads import fetch_splice_case, mla_decode_case, route_case, shared_kv_prefill_case, tiny_gqa_case
     from workloads.device import mla_to_device, paged_to_device, route_to_device, splice_to_device
-    peaks, src = _peaks()
-    hbm = float(peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]))
-    tf = float(peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]))
-    dev = torch.device("cuda", 0)
-    stream = torch.cuda.current_stream(dev)
-    names = args.workload.split(",")
-    if names == ["all"]:
-        names = ["tiny", "shared_kv"] + [f"mla_h{h}_q{q}_{d}" for h in (16, 128) for q in (1, 4)
-                                         for d in ("bf16", "e4m3")] + ["route", "fetch_splice"]
-    for name in names:
-        line = {"workload": name, "peaks": src}
-        if name in ("tiny", "shared_kv"):
-            c = tiny_gqa_case() if name == "tiny" else shared_kv_prefill_case()
-            d = paged_to_device(c, dev)
-            pol, par = ("fixed", 2) if name == "tiny" else ("none", 0)
-            plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, c.page_size, c.num_qo_heads,
-                                  c.num_kv_heads, c.head_dim, pol, par).to(dev)
-            n = max(1, plan.info.num_partial_rows)
-            o = torch.empty(c.q.shape[0], c.num_qo_heads, c.head_dim, device=dev)
-            lse = torch.empty(c.q.shape[0], c.num_qo_heads, device=dev)
-            op = torch.empty(n, c.num_qo_heads, c.head_dim, device=dev)
-            lp = torch.empty(n, c.num_qo_heads, device=dev)
-            step = lambda: skv.paged_attn_fwd(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"],
-                                              d["kv_last_page_len"], plan, o, lse, op, lp, None, c.sm_scale,
-                                              c.num_pages, stream)
-            L = c.kv_lengths()
-            q_rows = np.diff(c.qo_indptr)
-            kv_bytes = int(L.sum()) * c.num_kv_heads * c.head_dim * 4
-            flops = float(np.sum(q_rows * L)) * c.num_qo_heads * 4 * c.head_dim
-            if name == "shared_kv":   # the one shared KV is read once
-                kv_bytes = int(L[0]) * c.num_kv_heads * c.head_dim * 4
-            line["kernel"] = plan.info.kernel
-        elif name.startswith("mla_"):
-            _, hs, qs, dt = name.split("_")
-            H, q = int(hs[1:]), int(qs[1:])
-            c = mla_decode_case(H, q, dt)
-            d = mla_to_device(c, dev)
+    e = {}
+    if name in ("tiny", "shared_kv"):
+        c = tiny_gqa_case() if name == "tiny" else shared_kv_prefill_case()
+        d = paged_to_device(c, dev)
+        pol, par = ("fixed", 2) if name == "tiny" else ("none", 0)
+        plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, c.page_size, c.num_qo_heads,
+                              c.num_kv_heads, c.head_dim, pol, par).to(dev)
+        n = max(1, plan.info.num_partial_rows)
+        o = torch.empty(c.q.shape[0], c.num_qo_heads, c.head_dim, device=dev)
+        lse = torch.empty(c.q.shape[0], c.num_qo_heads, device=dev)
+        op = torch.empty(n, c.num_qo_heads, c.head_dim, device=dev)
+        lp = torch.empty(n, c.num_qo_heads, device=dev)
+        e["step"] = lambda: skv.paged_attn_fwd(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"],
+                                               d["kv_last_page_len"], plan, o, lse, op, lp, None, c.sm_scale,
+                                               c.num_pages, stream)
+        L = c.kv_lengths()
+        q_rows = np.diff(c.qo_indptr)
+        per_tok = c.num_kv_heads * c.head_dim * 4
+        e["bytes"] = int(L[0] if name == "shared_kv" else L.sum()) * per_tok   # the shared KV is read once
+        e["flops"] = float(np.sum(q_rows * L)) * c.num_qo_heads * 4 * c.head_dim
+        e["launches"] = 1 + (1 if plan.info.num_merge_rows else 0)
+        e["kernel"] = plan.info.kernel
+        e["dtype"] = "bf16"
+        unit_work = lambda r: (float(L[r]) * per_tok, float(q_rows[r] * L[r]) * c.num_qo_heads * 4 * c.head_dim)
+        e["oracle_units"] = (lambda r=r: (OA.paged_attention(c.q, c.k, c.v, c.qo_indptr, c.kv_indptr, c.kv_indices,
+                                                            c.kv_last_page_len, c.page_size, c.sm_scale,
+                                                            requests=[r]), unit_work(r))[1]
+                             for r in range(c.batch))
+        e["oracle_what"] = "requests (query batches)" if name == "shared_kv" else "requests"
+    elif name.startswith("mla_"):
+        parts = name.split("_")
+        H, q, dt = int(parts[1][1:]), int(parts[2][1:]), parts[3]
+        causal = len(parts) > 4 and parts[4] == "causal"
+        c = mla_decode_case(H, q, dt)
+        d = mla_to_device(c, dev)
+        o = torch.empty(c.batch, q, H, 512, device=dev)
+        lse = torch.empty(c.batch, q, H, device=dev)
+        if causal:
+            cm = skv.CausalMlaDecode(q, H, c.kv_indptr, c.kv_indices, c.kv_last_page_len, c.page_size, c.num_pages,
+                                     dev, dt)
+            e["step"] = lambda: cm(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], o, lse, sm_scale=c.sm_scale,
+                                   kv_scale=c.kv_scale, stream=stream)
+            e["launches"] = cm.launches()
+            e["kernel"] = [cm.prefix_plan.info.kernel, cm.diag_plan.info.kernel]
+        else:
             plan = skv.plan_mla(q, c.kv_indptr, c.kv_last_page_len, c.page_size, H, "balanced", 0,
                                 kv_dtype=dt).to(dev)
             n = max(1, plan.info.num_partial_rows)
-            o = torch.empty(c.batch, q, H, 512, device=dev)
-            lse = torch.empty(c.batch, q, H, device=dev)
             op = torch.empty(n, H, 512, device=dev)
             lp = torch.empty(n, H, device=dev)
-            step = lambda: skv.mla_decode_fwd(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], d["kv_indptr"],
-                                              d["kv_indices"], d["kv_last_page_len"], plan, o, lse, op, lp, None,
-                                              c.sm_scale, c.kv_scale, c.num_pages, stream)
-            L = c.kv_lengths()
-            kv_bytes = int(L.sum()) * (1152 if dt == "bf16" else 576)
-            flops = float(L.sum()) * H * q * 2 * (576 + 512)
-            line["kernel"] = plan.info.kernel
-        elif name == "route":
-            c = route_case()
-            d = route_to_device(c, dev)
-            rm = skv.RouteMerge(c.sel, c.num_heads, dev)
-            out_o = torch.empty(c.sel.shape[0], c.num_heads, 512, device=dev)
-            out_l = torch.empty(c.sel.shape[0], c.num_heads, device=dev)
-            step = lambda: rm(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], d["sel_cqk"], sm_scale=c.sm_scale,
-                              stream=stream, o=out_o, lse=out_l)
-            kv_bytes = int(c.sel.size) * 1152              # gathered rows
-            flops = float(c.sel.size) * c.num_heads * 2 * (576 + 512)
-            line["kernel"] = rm.plan.info.kernel
-        elif name == "fetch_splice":
-            # fetch's local compute: every chunk of the route corpus moved into a requester's paged
-            # cache and re-rotated (all chunks in one call); bytes = each row read once and written once
-            c = fetch_splice_case()
-            d = splice_to_device(c, dev)
-            sp = skv.splice_params(d["src_ckv"], d["src_kpe"], d["src_pages"], d["dst_ckv"], d["dst_kpe"],
-                                   d["dst_pages"], rope_theta=c.rope_theta)
-            chunks = skv.splice_chunks([(int(c.src_start[ch]), int(c.dst_start[ch]), c.chunk_tokens, int(c.delta[ch]))
-                                        for ch in range(c.num_chunks)])
-            step = lambda: skv.splice_launch(sp, chunks, stream)
-            kv_bytes = 2 * c.num_chunks * c.chunk_tokens * 1152
-            flops = 0.0
-            line["kernel"] = "splice"
-        else:
-            raise SystemExit(f"unknown workload {name}")
-        ms = _time_device(step, args.steps, args.warmup, torch, stream)
-        t_mem, t_tc = kv_bytes / (hbm * 1e9), flops / (tf * 1e12)
-        line.update({"us": round(ms * 1e3, 2), "kv_bytes": kv_bytes, "flops": flops,
-                     "GBps": round(kv_bytes / (ms * 1e-3) / 1e9, 1), "TFLOPs": round(flops / (ms * 1e-3) / 1e12, 2),
-                     "bound": "hbm" if t_mem >= t_tc else "tensor",
-                     "roofline_frac": round(max(t_mem, t_tc) / (ms * 1e-3), 4),
-                     "pct_hbm_measured": round(100 * kv_bytes / (ms * 1e-3) / 1e9 / hbm, 1),
-                     "pct_tensor_burst": round(100 * flops / (ms * 1e-3) / 1e12 / tf, 1)})
+            e["step"] = lambda: skv.mla_decode_fwd(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], d["kv_indptr"],
+                                                   d["kv_indices"], d["kv_last_page_len"], plan, o, lse, op, lp,
+                                                   None, c.sm_scale, c.kv_scale, c.num_pages, stream)
+            e["launches"] = 1 + (1 if plan.info.num_merge_rows else 0)
+            e["kernel"] = plan.info.kernel
+        L = c.kv_lengths()
+        per_tok = 1152 if dt == "bf16" else 576
+        e["bytes"] = int(L.sum()) * per_tok
+        # causal: position i of q_len sees L - q_len + 1 + i keys
+        vis = (lambda l: q * l - q * (q - 1) / 2) if causal else (lambda l: q * l)
+        e["flops"] = float(sum(vis(float(x)) for x in L)) * H * 2 * (576 + 512)
+        e["dtype"] = dt
+        unit_work = lambda r: (float(L[r]) * per_tok, vis(float(L[r])) * H * 2 * (576 + 512))
+        e["oracle_units"] = (lambda r=r: (OA.mla_decode(c.q_nope, c.q_pe, c.ckv, c.kpe, c.kv_indptr, c.kv_indices,
+                                                       c.kv_last_page_len, c.page_size, c.sm_scale, c.kv_dtype,
+                                                       c.kv_scale, requests=[r], causal=causal), unit_work(r))[1]
+                             for r in range(c.batch))
+        e["oracle_what"] = "requests"
+    elif name == "route":
+        c = route_case()
+        d = route_to_device(c, dev)
+        rm = skv.RouteMerge(c.sel, c.num_heads, dev)
+        out_o = torch.empty(c.sel.shape[0], c.num_heads, 512, device=dev)
+        out_l = torch.empty(c.sel.shape[0], c.num_heads, device=dev)
+        e["step"] = lambda: rm(d["q_nope"], d["q_pe"], d["ckv"], d["kpe"], d["sel_cqk"], sm_scale=c.sm_scale,
+                               stream=stream, o=out_o, lse=out_l)
+        e["bytes"] = int(c.sel.size) * 1152              # gathered rows
+        e["flops"] = float(c.sel.size) * c.num_heads * 2 * (576 + 512)
+        e["launches"] = c.num_chunks + 1
+        e["kernel"] = rm.plan.info.kernel
+        e["dtype"] = "bf16"
+        u = c.union_mla()
+        per_q = (c.num_chunks * c.sel.shape[2] * 1152.0, c.num_chunks * c.sel.shape[2] * c.num_heads * 2.0 * 1088)
+        e["oracle_units"] = (lambda qq=qq: (OA.mla_decode(u.q_nope, u.q_pe, u.ckv, u.kpe, u.kv_indptr, u.kv_indices,
+                                                         u.kv_last_page_len, 1, u.sm_scale, requests=[qq]),
+                                            per_q)[1]
+                             for qq in range(c.sel.shape[0]))
+        e["oracle_what"] = "queries (attention over the union of their selections)"
+    elif name == "fetch_splice":
+        # fetch's local compute: every chunk of the route corpus moved into a requester's paged
+        # cache and re-rotated (all chunks in one call); bytes = each row read once and written once
+        import oracle.splice as OS
+        c = fetch_splice_case()
+        d = splice_to_device(c, dev)
+        sp = skv.splice_params(d["src_ckv"], d["src_kpe"], d["src_pages"], d["dst_ckv"], d["dst_kpe"],
+                               d["dst_pages"], rope_theta=c.rope_theta)
+        chunks = skv.splice_chunks([(int(c.src_start[ch]), int(c.dst_start[ch]), c.chunk_tokens, int(c.delta[ch]))
+                                    for ch in range(c.num_chunks)])
+        e["step"] = lambda: skv.splice_launch(sp, chunks, stream)
+        e["bytes"] = 2 * c.num_chunks * c.chunk_tokens * 1152
+        e["flops"] = 0.0
+        e["launches"] = 1
+        e["kernel"] = "splice"
+        e["dtype"] = "bf16"
+        freq = OS.rope_inv_freq(c.rope_theta)
+        blk = 256
+        e["oracle_units"] = (lambda ch=ch, t0=t0: (OS.splice_rows(
+            c.src[..., :512], c.src[..., 512:], c.src_pages, int(c.src_start[ch]) + t0, c.dst_pages, c.dst_page_size,
+            int(c.dst_start[ch]) + t0, blk, int(c.delta[ch]), freq), (2.0 * blk * 1152, 0.0))[1]
+            for t0 in range(0, c.chunk_tokens, blk) for ch in range(c.num_chunks))
+        e["oracle_what"] = f"blocks of {blk} tokens"
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    return e
+
+
+def _config_entry(name, args, dev, stream, skv, torch, flush, peaks, peak_src, cpu_budget):
+    """One configuration: device time per call (attention + merge, inputs resident, L2 flushed
+    before each timed call), roofline fraction against the measured peaks, and the oracle timed on
+    the host cores over a bounded sample of the same inputs."""
+    e = _setup_config(name, dev, skv, torch, stream)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK["hbm_gbs"]))
+    tf_bf16 = float(peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]))
+    fp8 = e["dtype"] == "e4m3"
+    tf = tf_bf16 * (2.0 if fp8 else 1.0)
+    tf_src = (f"{peak_src} bf16 x 2 (nominal fp8 : bf16 dense ratio; e4m3 MMAs)" if fp8
+              else f"{peak_src} bf16 burst")
+    steps = max(3, min(args.steps, args.config_steps))
+    ms = _time_calls(e["step"], steps, max(3, min(args.warmup, 5)), torch, stream, flush)
+    t_mem, t_tc = e["bytes"] / (hbm * 1e9), e["flops"] / (tf * 1e12)
+    bound = "hbm" if t_mem >= t_tc else "tensor"
+    gbs = e["bytes"] / (ms * 1e-3) / 1e9
+    tfs = e["flops"] / (ms * 1e-3) / 1e12
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(gbs / hbm, 4), "peak_source": f"{peak_src} hbm_gbs"}
+    else:
+        roof = {"bound": "tensor", "achieved": round(tfs, 1), "peak": round(tf, 1), "unit": "TFLOP/s",
+                "frac": round(tfs / tf, 4), "peak_source": tf_src}
+    out = {"us": round(ms * 1e3, 2), "GBps": round(gbs, 1), "TFLOPs": round(tfs, 2), "kv_bytes": e["bytes"],
+           "flops": e["flops"], "roofline": roof, "kernel": e["kernel"], "launches_per_call": e["launches"],
+           "dtype": e["dtype"], "timed_calls": steps, "l2": "flushed (512 MB write) before every timed call"}
+    if cpu_budget > 0:
+        done, dt, n = _sampled(e["oracle_units"], cpu_budget)
+        work, scale = (done[0], 1e9) if roof["unit"] == "GB/s" else (done[1], 1e12)
+        out["cpu_baseline"] = {"value": work / dt / scale, "unit": roof["unit"], "cores": int(_threads_used()),
+                               "kind": "oracle",
+                               "sample": f"{n} {e['oracle_what']} of the same inputs, float64 numpy oracle, "
+                                         f"{dt:.1f} s on {os.cpu_count()} visible host cores; rate extrapolates "
+                                         f"linearly to the whole configuration"}
+    return out
+
+
+def _flush_buffer(torch, dev):
+    return torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+
+def run_workload(args):
+    """One JSON line per named configuration (the entries of the default line's ``configs``)."""
+    import torch
+    import split_kv_merge_b200 as skv
+    peaks, src = _peaks()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = _flush_buffer(torch, dev)
+    names = args.workload.split(",")
+    if names == ["all"]:
+        names = list(CONFIG_NAMES)
+    for name in names:
+        line = {"workload": name, **_config_entry(name, args, dev, stream, skv, torch, flush, peaks, src,
+                                                  0.0 if args.no_cpu_baseline else args.config_cpu_budget)}
         print(json.dumps(line), flush=True)
     return 0
+
+
+def all_configs(args, dev, stream, skv, torch):
+    """The ``configs`` object of the default line: every configuration other than the headline."""
+    peaks, src = _peaks()
+    flush = _flush_buffer(torch, dev)
+    out = {}
+    for name in CONFIG_NAMES:
+        out[name] = _config_entry(name, args, dev, stream, skv, torch, flush, peaks, src,
+                                  0.0 if args.no_cpu_baseline else args.config_cpu_budget)
+        torch.cuda.empty_cache()
+    del flush
+    return out
 
 
 def main():
@@ -534,7 +668,11 @@ def main():
                                                           "smaller only for profiler captures)")
     ap.add_argument("--workload", default="llama70b",
                     help="llama70b (the benchmark line) | tiny | shared_kv | mla_h{16,128}_q{1,4}_{bf16,e4m3} | "
-                         "route | fetch_splice | all (one line per configuration)")
+                         "mla_h16_q4_bf16_causal | route | fetch_splice | all (one line per configuration)")
+    ap.add_argument("--no-configs", action="store_true", help="default line without the per-configuration block")
+    ap.add_argument("--config-steps", type=int, default=20, help="timed calls per configuration (at most --steps)")
+    ap.add_argument("--config-cpu-budget", type=float, default=2.0,
+                    help="seconds of oracle work per configuration for its cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

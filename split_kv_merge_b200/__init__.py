@@ -470,4 +470,4 @@ def library_path() -> str:
     return _LIB_PATH
 
 
-from .runner import RouteMerge, mla_decode, paged_attention, pod_attention  # noqa: E402,F401
+from .runner import CausalMlaDecode, RouteMerge, mla_decode, paged_attention, pod_attention  # noqa: E402,F401

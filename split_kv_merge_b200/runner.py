@@ -229,3 +229,63 @@ class RouteMerge:
         merge_states(self.o_states.view(self.C, self.Q, self.H, 512), self.lse_states.view(self.C, self.Q, self.H),
                      o, lse, stream=stream)
         return o, lse
+
+
+class CausalMlaDecode:
+    """Causal multi-token MLA decode planned once and launched many times (the per-call form of
+    ``mla_decode(causal=True)`` without host planning): every decode step of a fixed batch runs
+    the prefix pass (each request cut to the keys all its q_len positions see, q_len folded into
+    rows), the diagonal pass (one page-size-1 request per query position over the few keys only
+    later positions see) and the exact merge of the two states."""
+
+    def __init__(self, q_len: int, num_heads: int, kv_indptr_h, kv_indices_h, kv_last_page_len_h,
+                 page_size: int, num_pages: int, device, kv_dtype: str = "bf16", policy="balanced",
+                 param: int = 0):
+        import torch
+        B = len(kv_indptr_h) - 1
+        self.B, self.q_len, self.H, self.P, self.num_pages = B, q_len, num_heads, page_size, num_pages
+        tab = causal_split_tables(np.full(B, q_len), kv_indptr_h, kv_indices_h, kv_last_page_len_h, page_size)
+        pi, px, pl = tab["prefix"]
+        di, dx, dl = tab["diag"]
+        self.has_prefix, self.has_diag = int(pi[-1]) > 0, int(di[-1]) > 0
+        self.prefix = (_dev_i32(pi, device), _dev_i32(px, device), _dev_i32(pl, device))
+        self.diag = (_dev_i32(di, device), _dev_i32(dx, device), _dev_i32(dl, device))
+        self.prefix_plan = plan_mla(q_len, pi, pl, page_size, num_heads, policy, param, None, kv_dtype).to(device)
+        self.diag_plan = plan_mla(1, di, dl, 1, num_heads, "none", 0, None, kv_dtype).to(device)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.o_st = torch.empty(2, B, q_len, num_heads, 512, **f32)
+        self.lse_st = torch.empty(2, B, q_len, num_heads, **f32)
+        n_pre, n_diag = self.prefix_plan.info.num_partial_rows, self.diag_plan.info.num_partial_rows
+        self.pre_part = (torch.empty(n_pre, num_heads, 512, **f32), torch.empty(n_pre, num_heads, **f32)) \
+            if n_pre else (None, None)
+        self.diag_part = (torch.empty(n_diag, num_heads, 512, **f32), torch.empty(n_diag, num_heads, **f32)) \
+            if n_diag else (None, None)
+
+    def launches(self) -> int:
+        """Kernel launches per call (attention passes, their plans' merge passes, the final merge)."""
+        n = 0
+        for on, plan in ((self.has_prefix, self.prefix_plan), (self.has_diag, self.diag_plan)):
+            if on:
+                n += 1 + (1 if plan.info.num_merge_rows > 0 else 0)
+        return n + (1 if self.has_prefix and self.has_diag else 0)
+
+    def __call__(self, q_nope, q_pe, ckv, kpe, o, lse, *, sm_scale=None, kv_scale: float = 1.0, status=None,
+                 stream=None):
+        B, q, H = self.B, self.q_len, self.H
+        both = self.has_prefix and self.has_diag
+        o_pre, l_pre = (self.o_st[0], self.lse_st[0]) if both else (o, lse)
+        o_dg, l_dg = (self.o_st[1], self.lse_st[1]) if both else (o, lse)
+        if self.has_prefix:
+            ip, ix, la = self.prefix
+            mla_decode_fwd(q_nope, q_pe, ckv, kpe, ip, ix, la, self.prefix_plan, o_pre, l_pre, *self.pre_part, status,
+                           sm_scale, kv_scale, self.num_pages, stream)
+        if self.has_diag:
+            ip, ix, la = self.diag
+            mla_decode_fwd(q_nope.reshape(B * q, 1, H, 512), q_pe.reshape(B * q, 1, H, 64), _rows_view(ckv, self.P),
+                           _rows_view(kpe, self.P), ip, ix, la, self.diag_plan, o_dg.view(B * q, 1, H, 512),
+                           l_dg.view(B * q, 1, H), *self.diag_part, status, sm_scale, kv_scale,
+                           self.num_pages * self.P, stream)
+        if both:
+            merge_states(self.o_st.view(2, B * q, H, 512), self.lse_st.view(2, B * q, H), o.view(B * q, H, 512),
+                         lse.view(B * q, H), stream=stream)
+        return o, lse

@@ -63,7 +63,8 @@ def e4m3_encode(x: np.ndarray, chunk: int = 1 << 24) -> np.ndarray:
     x = np.asarray(x)
     flat = x.reshape(-1)
     out = np.empty(flat.shape, dtype=np.uint8)
-    for lo in range(0, flat.size, chunk):
+
+    def encode(lo: int) -> None:   # chunks are independent; numpy releases the GIL inside them
         v = flat[lo:lo + chunk].astype(np.float64)
         a = np.minimum(np.abs(v), 448.0)
         sub = a < 2.0 ** -6
@@ -77,6 +78,14 @@ def e4m3_encode(x: np.ndarray, chunk: int = 1 << 24) -> np.ndarray:
         code_s = np.rint(a * 2.0 ** 9).astype(np.int64)   # 0..8 (8 is the smallest normal, code 0x08)
         code = np.minimum(np.where(sub, code_s, code_n), 0x7E).astype(np.uint8)
         out[lo:lo + chunk] = code | np.where(np.signbit(v), np.uint8(0x80), np.uint8(0))
+
+    starts = range(0, flat.size, chunk)
+    if len(starts) <= 1:
+        for lo in starts:
+            encode(lo)
+    else:
+        with ThreadPoolExecutor(min(8, len(starts))) as ex:
+            list(ex.map(encode, starts))
     return out.reshape(x.shape)
 
 
