@@ -416,8 +416,8 @@ def _e2e(args, runs, dev, stream, skv, torch):
 
 
 # ----------------------------------------------------------------------------- other configurations
-CONFIG_NAMES = (["tiny", "shared_kv"] + [f"mla_h{h}_q{q}_{d}" for h in (16, 128) for q in (1, 4)
-                                         for d in ("bf16", "e4m3")]
+CONFIG_NAMES = (["tiny", "llama70b_e4m3", "shared_kv"] + [f"mla_h{h}_q{q}_{d}" for h in (16, 128) for q in (1, 4)
+                                                          for d in ("bf16", "e4m3")]
                 + ["mla_h16_q4_bf16_causal", "route", "fetch_splice"])
 L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2: written before every timed call
 
@@ -466,11 +466,13 @@ def _setup_config(name, dev, skv, torch, stream):
     import oracle.attention as OA
     from workloads import fetch_splice_case, mla_decode_case, route_case, shared_kv_prefill_case, tiny_gqa_case
     from workloads.device import mla_to_device, paged_to_device, route_to_device, splice_to_device
+    from workloads import llama70b_decode_case
     e = {}
-    if name in ("tiny", "shared_kv"):
-        c = tiny_gqa_case() if name == "tiny" else shared_kv_prefill_case()
+    if name in ("tiny", "shared_kv", "llama70b_e4m3"):
+        c = {"tiny": tiny_gqa_case, "shared_kv": shared_kv_prefill_case,
+             "llama70b_e4m3": lambda: llama70b_decode_case(kv_dtype="e4m3")}[name]()
         d = paged_to_device(c, dev)
-        pol, par = ("fixed", 2) if name == "tiny" else ("none", 0)
+        pol, par = {"tiny": ("fixed", 2), "shared_kv": ("none", 0), "llama70b_e4m3": ("balanced", 0)}[name]
         plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, c.page_size, c.num_qo_heads,
                               c.num_kv_heads, c.head_dim, pol, par).to(dev)
         n = max(1, plan.info.num_partial_rows)
@@ -480,19 +482,20 @@ def _setup_config(name, dev, skv, torch, stream):
         lp = torch.empty(n, c.num_qo_heads, device=dev)
         e["step"] = lambda: skv.paged_attn_fwd(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"],
                                                d["kv_last_page_len"], plan, o, lse, op, lp, None, c.sm_scale,
-                                               c.num_pages, stream)
+                                               c.num_pages, stream, kv_scale=c.kv_scale)
         L = c.kv_lengths()
         q_rows = np.diff(c.qo_indptr)
-        per_tok = c.num_kv_heads * c.head_dim * 4
+        per_tok = c.num_kv_heads * c.head_dim * 2 * (1 if c.kv_dtype == "e4m3" else 2)
         e["bytes"] = int(L[0] if name == "shared_kv" else L.sum()) * per_tok   # the shared KV is read once
         e["flops"] = float(np.sum(q_rows * L)) * c.num_qo_heads * 4 * c.head_dim
         e["launches"] = 1 + (1 if plan.info.num_merge_rows else 0)
         e["kernel"] = plan.info.kernel
-        e["dtype"] = "bf16"
+        e["dtype"] = c.kv_dtype
         unit_work = lambda r: (float(L[r]) * per_tok, float(q_rows[r] * L[r]) * c.num_qo_heads * 4 * c.head_dim)
         e["oracle_units"] = (lambda r=r: (OA.paged_attention(c.q, c.k, c.v, c.qo_indptr, c.kv_indptr, c.kv_indices,
                                                             c.kv_last_page_len, c.page_size, c.sm_scale,
-                                                            requests=[r]), unit_work(r))[1]
+                                                            requests=[r], kv_dtype=c.kv_dtype,
+                                                            kv_scale=c.kv_scale), unit_work(r))[1]
                              for r in range(c.batch))
         e["oracle_what"] = "requests (query batches)" if name == "shared_kv" else "requests"
     elif name.startswith("mla_"):
@@ -667,7 +670,8 @@ def main():
     ap.add_argument("--batch", type=int, default=64, help="requests per GPU (64 = the benchmark workload; "
                                                           "smaller only for profiler captures)")
     ap.add_argument("--workload", default="llama70b",
-                    help="llama70b (the benchmark line) | tiny | shared_kv | mla_h{16,128}_q{1,4}_{bf16,e4m3} | "
+                    help="llama70b (the benchmark line) | tiny | llama70b_e4m3 | shared_kv | "
+                         "mla_h{16,128}_q{1,4}_{bf16,e4m3} | "
                          "mla_h16_q4_bf16_causal | route | fetch_splice | all (one line per configuration)")
     ap.add_argument("--no-configs", action="store_true", help="default line without the per-configuration block")
     ap.add_argument("--config-steps", type=int, default=20, help="timed calls per configuration (at most --steps)")

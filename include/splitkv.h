@@ -7,7 +7,9 @@
  *                       independent strides (FlashInfer PR #4736 page, section 1
  *                       "batch_pod.cu: flexible stride handling" and section 2 "SAME_KV_STRIDES
  *                       template specialisation"); one KV sequence may be listed by many query
- *                       batches (PyTorch MPS FlexAttention page, "KV batch broadcast").
+ *                       batches (PyTorch MPS FlexAttention page, "KV batch broadcast").  The
+ *                       cache may be bf16 or fp8 e4m3 with a per-tensor scale (FP8 KV decode,
+ *                       FlashInfer PR #3309 page, introduction).
  *   skv_mla_decode_fwd  Multi-head latent attention decode: every head reads one 512+64-d latent
  *                       row per token, V is the 512-d latent; seqlen_q is folded into heads to
  *                       fill the MMA M tile (FlashInfer PR #3309 page, sections 1-2 and "why it
@@ -157,6 +159,12 @@ typedef struct {
   float* o_part;            /* [num_partial_rows, Hq, D] fp32, needed when the plan splits     */
   float* lse_part;          /* [num_partial_rows, Hq] fp32                                     */
   int32_t* status;          /* device status word (may be NULL)                                */
+  int32_t kv_dtype;         /* SKV_BF16 (0, the default) or SKV_E4M3: K and V hold OCP e4m3fn   */
+                            /*   codes (one byte per element; strides then multiples of 16),    */
+                            /*   k = kv_scale * code(k), v = kv_scale * code(v).  e4m3 runs on  */
+                            /*   plans whose kernel is 3 (all KV heads on the tensor cores);    */
+                            /*   other plans return SKV_ERR_UNSUPPORTED                          */
+  float kv_scale;           /* per-tensor dequantisation scale for SKV_E4M3 (finite, > 0)      */
 } skv_paged_params;
 
 /* -------------------------------------------------------------------------------------------

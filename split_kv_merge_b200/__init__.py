@@ -55,7 +55,7 @@ class PagedParams(ctypes.Structure):
                 ("page_size", ctypes.c_int32), ("num_qo_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("sm_scale", ctypes.c_float),
                 ("o", _vp), ("o_dtype", ctypes.c_int32), ("lse", _vp), ("o_part", _vp), ("lse_part", _vp),
-                ("status", _vp)]
+                ("status", _vp), ("kv_dtype", ctypes.c_int32), ("kv_scale", ctypes.c_float)]
 
 
 class MlaParams(ctypes.Structure):
@@ -283,7 +283,7 @@ def plan_mla(batch_q_len: int, kv_indptr, kv_last_page_len, page_size: int, num_
 
 # ----------------------------------------------------------------------------- launches
 def _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, o, lse, o_part, lse_part,
-                  status, sm_scale, num_pages, page_size=None):
+                  status, sm_scale, num_pages, page_size=None, kv_scale: float = 1.0):
     if k_cache.stride(-1) != 1 or v_cache.stride(-1) != 1:
         raise ValueError("the innermost (head_dim) stride of K and V must be 1")
     p = PagedParams()
@@ -303,18 +303,23 @@ def _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, 
     p.o = _dptr(o)
     p.o_dtype = _dtype_code(o) if o is not None else F32
     p.lse, p.o_part, p.lse_part, p.status = _dptr(lse), _dptr(o_part), _dptr(lse_part), _dptr(status)
+    p.kv_dtype = _dtype_code(k_cache)
+    if _dtype_code(v_cache) != p.kv_dtype:
+        raise ValueError("K and V caches must have the same dtype")
+    p.kv_scale = float(kv_scale)
     return p
 
 
 def paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan: Plan, o, lse=None,
                    o_part=None, lse_part=None, status=None, sm_scale: Optional[float] = None,
-                   num_pages: Optional[int] = None, stream=None, phase: str = "all") -> None:
-    """skv_paged_attn_fwd.  q [total_q, Hq, D] bf16; k_cache / v_cache [num_pages, P, Hk, D] bf16
-    views (any page/slot/head strides, head_dim contiguous); page-table tensors int32 on the
-    device; o [total_q, Hq, D] f32|bf16; lse [total_q, Hq] f32; o_part / lse_part sized by
-    ``plan.info.num_partial_rows`` when the plan splits."""
+                   num_pages: Optional[int] = None, stream=None, phase: str = "all", kv_scale: float = 1.0) -> None:
+    """skv_paged_attn_fwd.  q [total_q, Hq, D] bf16; k_cache / v_cache [num_pages, P, Hk, D] bf16,
+    or e4m3 codes (float8_e4m3fn / uint8) with the per-tensor ``kv_scale``, views (any page/slot/head
+    strides, head_dim contiguous); page-table tensors int32 on the device; o [total_q, Hq, D]
+    f32|bf16; lse [total_q, Hq] f32; o_part / lse_part sized by ``plan.info.num_partial_rows``
+    when the plan splits."""
     p = _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, o, lse, o_part, lse_part,
-                      status, sm_scale, num_pages)
+                      status, sm_scale, num_pages, kv_scale=kv_scale)
     fn = {"all": _paged_fwd, "partial": _paged_partial}[phase]
     _check(fn(ctypes.byref(p), _dptr(plan.device), ctypes.byref(plan.info), _stream_ptr(stream)),
            "skv_paged_attn_fwd" if phase == "all" else "skv_paged_attn_partial")

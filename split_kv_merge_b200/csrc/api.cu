@@ -460,9 +460,13 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
     if (!p->q || !p->k_cache || !p->v_cache || !p->kv_indptr || !p->kv_indices || !p->kv_last_page_len || !p->o)
       return SKV_ERR_INVALID;
   }
+  if (p->kv_dtype != SKV_BF16 && p->kv_dtype != SKV_E4M3) return SKV_ERR_UNSUPPORTED;
+  const bool fp8 = p->kv_dtype == SKV_E4M3;
+  if (fp8 && !(p->kv_scale > 0.f && std::isfinite(p->kv_scale))) return SKV_ERR_INVALID;
+  const int64_t stride_unit = fp8 ? 16 : 8;  // elements per 16 bytes
   for (int i = 0; i < 3; ++i) {
     if (p->k_stride[i] < 0 || p->v_stride[i] < 0) return SKV_ERR_INVALID;
-    if ((p->k_stride[i] % 8) || (p->v_stride[i] % 8)) return SKV_ERR_ALIGNMENT;
+    if ((p->k_stride[i] % stride_unit) || (p->v_stride[i] % stride_unit)) return SKV_ERR_ALIGNMENT;
   }
   if (!aligned16(p->q) || !aligned16(p->k_cache) || !aligned16(p->v_cache) || !aligned16(p->o))
     return SKV_ERR_ALIGNMENT;
@@ -470,6 +474,8 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
   if (info->kernel != KERNEL_GQA_SIMT && info->kernel != KERNEL_GQA_TC_DECODE && info->kernel != KERNEL_GQA_TC_WIDE &&
       info->kernel != KERNEL_GQA_TC_PREFILL)
     return SKV_ERR_INVALID;
+  // the e4m3 cache runs on the all-KV-heads tensor-core kernel only
+  if (fp8 && info->kernel != KERNEL_GQA_TC_WIDE) return SKV_ERR_UNSUPPORTED;
   if (info->num_work == 0) return SKV_OK;  // no query rows: nothing to launch
   const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
                        p->k_stride[2] == p->v_stride[2];
@@ -479,7 +485,8 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
       (info->num_ctas < 1 || info->cta_offset < 8LL * info->num_work + 4LL * info->num_merge_rows))
     return SKV_ERR_INVALID;
   int e = info->kernel == KERNEL_GQA_TC_WIDE
-              ? launch_gqa_tc_wide(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile, s)
+              ? (fp8 ? launch_gqa_tc_wide_fp8(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile, s)
+                     : launch_gqa_tc_wide(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile, s))
           : info->kernel == KERNEL_GQA_TC_PREFILL ? launch_gqa_tc_prefill(*p, work, info->num_work, info->q_tile, s)
           : info->kernel == KERNEL_GQA_TC_DECODE ? launch_gqa_tc_decode(*p, work, info->num_work, info->q_tile, s)
                                                  : launch_gqa_simt(*p, work, info->num_work, info->q_tile, same_kv, s);
@@ -668,7 +675,7 @@ skv_status skv_paged_kv_gather(const skv_paged_params* p, const int32_t* token_i
       !p->kv_last_page_len)
     return SKV_ERR_INVALID;
   if (p->batch < 1 || p->page_size < 1 || p->num_kv_heads < 1 || p->head_dim < 1) return SKV_ERR_INVALID;
-  if (total_tokens > INT32_MAX) return SKV_ERR_UNSUPPORTED;
+  if (total_tokens > INT32_MAX || p->kv_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
   const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
                        p->k_stride[2] == p->v_stride[2];
   return cuda_status(launch_gather(*p, token_indptr, total_tokens, k_out, v_out, same_kv,

@@ -12,15 +12,17 @@
 //   * Both other operands are split into two e4m3 terms, hi = rn(x) and lo = rn(x - hi), stacked
 //     as 2 NR columns of N: queries (bf16, 8 significant bits) after a power-of-two scaling that
 //     puts the unit's largest |q| in [128, 256) -- exact for every |q| of at least 2^-9 of that
-//     maximum, within 2^-17 of it below -- and the softmax weights p in [0, 2^8] (bf16-like precision, 8 significant bits).  The
-//     scaling goes back into the softmax scale; S and O sum their hi and lo columns.
+//     maximum, within 2^-17 of it below -- and the softmax weights, shifted up by 2^4 to
+//     p' in [0, 2^8] (2^-8 relative precision from 2^-6 of the running maximum's weight up, 2^-14
+//     absolute below).  The query scaling goes back into the softmax scale, the weight shift into
+//     the LSE; S and O sum their hi and lo columns.
 //   * S^T[64 tokens, 2 NR] = C . [Q_hi; Q_lo]^T, K = 32 per MMA: 16 ckv k-steps (128-byte
 //     swizzled rows) + 2 rope k-steps (64-byte swizzled rows); M = 64, so TMEM rows sit in lanes
 //     0-15 of each warp quarter.  The k-steps are split over two issuers into two partial
 //     accumulators that the softmax adds.
 //   * O^T[512, 2 NR] += V^T . [P_hi; P_lo]^T in four M = 128 blocks (V read MN-major from the same
 //     tile), one block per issuer.
-//   * Online softmax with a lazily raised maximum (only when a score passes it by more than 2^8),
+//   * Online softmax with a lazily raised maximum (only when a score passes it by more than 2^4),
 //     O^T rescaled in TMEM on a raise; tokens past the end of the unit get s = -inf by selection
 //     and their V rows are zeroed in the tile before the PV that reads them.
 // Roles: warps 0-3 softmax / query split / epilogue, warp 4 TMA, warps 5-8 MMA issue (one per SM
@@ -43,7 +45,13 @@ constexpr int kTileBytes = 4 * kCRegion + kKRegion;
 constexpr int kBlocks = 4;
 constexpr int kIssuers = 4;
 constexpr int kThreads = (5 + kIssuers) * 32;
-constexpr float kRaise = 8.f;
+// The running maximum is raised only when a score passes it by more than 2^4 (log2 units), and
+// every weight is formed as p' = 2^(s - m + 4) <= 2^8 (e4m3 holds up to 448): the shift moves the
+// small weights of a row up into the range where the hi + lo split is relative (2^-8 from
+// p' = 2^-2 up, 2^-10 absolute below -- 2^-14 of the unshifted weight).  O / l is unchanged by
+// the shift; the LSE subtracts it.
+constexpr float kRaise = 4.f;
+constexpr float kPShift = 4.f;
 
 template <int NR>
 struct Cfg8 {
@@ -566,8 +574,8 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
 #pragma unroll
             for (int jj = 0; jj < NH; jj += 2) {
               // masked scores give 0 (rows past the unit's rows have no finite maximum)
-              const float p0 = sv[jj] == -INFINITY ? 0.f : ex2(sv[jj] - mloc[jj]);
-              const float p1 = sv[jj + 1] == -INFINITY ? 0.f : ex2(sv[jj + 1] - mloc[jj + 1]);
+              const float p0 = sv[jj] == -INFINITY ? 0.f : ex2(sv[jj] - mloc[jj] + kPShift);
+              const float p1 = sv[jj + 1] == -INFINITY ? 0.f : ex2(sv[jj + 1] - mloc[jj + 1] + kPShift);
               l[jj] += p0;
               l[jj + 1] += p1;
               uint32_t h2, l2;
@@ -618,7 +626,7 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
           const int n = tid;
           const float lt = red[n] + red[NR + n] + red[2 * NR + n] + red[3 * NR + n];
           inv_s[n] = lt > 0.f ? a.kv_scale / lt : 0.f;
-          lse_s[n] = lt > 0.f ? (m_s[n] + log2f(lt)) * kLn2 : -INFINITY;
+          lse_s[n] = lt > 0.f ? (m_s[n] - kPShift + log2f(lt)) * kLn2 : -INFINITY;
         }
         tc::named_bar_sync(1, 128);
         // O^T block by block: thread tid holds head dim b * 128 + tid of every row (hi + lo)

@@ -95,6 +95,8 @@ int launch_gqa_tc_decode(const skv_paged_params& p, const WorkItem* work, int nu
 bool gqa_tc_wide_supported(int head_dim, int page_size, int num_kv_heads, int group, int q_tile);
 int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                        int q_tile, cudaStream_t s);
+int launch_gqa_tc_wide_fp8(const skv_paged_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
+                           int q_tile, cudaStream_t s);
 bool gqa_tc_prefill_supported(int head_dim, int page_size, int group);
 int launch_gqa_tc_prefill(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
                           cudaStream_t s);

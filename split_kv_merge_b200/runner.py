@@ -43,9 +43,10 @@ def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, k
                     split_page_start=None, o_dtype=None, num_pages: Optional[int] = None,
                     kv_indptr=None, kv_last_page_len=None, plan: Optional[Plan] = None,
                     status=None, stream=None, causal: bool = False, kv_indices_h=None, o_out=None,
-                    lse_out=None):
+                    lse_out=None, kv_scale: float = 1.0):
     """GQA attention over a paged cache.  Host page-table shape arrays (``*_h``) feed the planner;
     ``kv_indices`` (and optionally ``kv_indptr`` / ``kv_last_page_len``) are device tensors.
+    K/V are bf16, or e4m3 codes (float8_e4m3fn) with the per-tensor ``kv_scale``.
     Returns (o, lse, extras) with extras = {"plan", "o_part", "lse_part"}.
 
     ``causal``: a request's query tokens are its last positions and each sees keys up to its own
@@ -96,7 +97,7 @@ def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, k
     o_part = torch.empty(n_part, hq, d, dtype=torch.float32, device=dev) if n_part else None
     lse_part = torch.empty(n_part, hq, dtype=torch.float32, device=dev) if n_part else None
     paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan, o, lse, o_part, lse_part,
-                   status, sm_scale, num_pages, stream)
+                   status, sm_scale, num_pages, stream, kv_scale=kv_scale)
     return o, lse, {"plan": plan, "o_part": o_part, "lse_part": lse_part}
 
 

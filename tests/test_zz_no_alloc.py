@@ -42,10 +42,10 @@ def _static(c, d, plan, o, lse, status):
 def test_static_scratch_matches_regular_entry_point_and_oracle_twice(indep):
     # another batch and plan first, with more partial rows than the case under test: its values
     # stay in the shared array
-    c0 = llama70b_decode_case(independent_v=not indep, batch=24, seed=7, len_range=(1024, 4096))
+    c0 = llama70b_decode_case(independent_v=not indep, batch=32, seed=7, len_range=(1024, 4096))
     d0 = paged_to_device(c0, DEV)
     plan0 = skv.plan_paged(c0.qo_indptr, c0.kv_indptr, c0.kv_last_page_len, c0.page_size, c0.num_qo_heads,
-                           c0.num_kv_heads, c0.head_dim, "fixed", 6).to(DEV)
+                           c0.num_kv_heads, c0.head_dim, "fixed", 8).to(DEV)   # 256 partial rows
     o0 = torch.empty(c0.q.shape[0], c0.num_qo_heads, c0.head_dim, device=DEV)
     lse0 = torch.empty(c0.q.shape[0], c0.num_qo_heads, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)

@@ -20,10 +20,19 @@ def i32_tensor(a, device):
     return torch.from_numpy(np.ascontiguousarray(np.asarray(a, dtype=np.int32))).to(device)
 
 
+def _kv_tensor(codes: np.ndarray, kv_dtype: str, device):
+    import torch
+    if kv_dtype == "bf16":
+        return bf16_tensor(codes, device)
+    return torch.from_numpy(np.ascontiguousarray(codes)).to(device).view(torch.float8_e4m3fn)
+
+
 def paged_to_device(c: PagedCase, device):
-    """dict of device tensors for a PagedCase: q, k, v (views), k_store, v_store, page table."""
-    k_store = bf16_tensor(c.k_store, device)
-    v_store = bf16_tensor(c.v_store, device)
+    """dict of device tensors for a PagedCase: q, k, v (views), k_store, v_store, page table
+    (K/V as bf16, or as float8_e4m3fn codes for an e4m3 case)."""
+    kd = getattr(c, "kv_dtype", "bf16")
+    k_store = _kv_tensor(c.k_store, kd, device)
+    v_store = _kv_tensor(c.v_store, kd, device)
     d = c.head_dim
     v = v_store[..., :d] if c.v_store.shape[-1] != d else v_store
     return dict(q=bf16_tensor(c.q, device), k=k_store, v=v, k_store=k_store, v_store=v_store,

@@ -172,6 +172,8 @@ class PagedCase:
     num_pages: int
     split_page_start: Optional[list] = None   # per request list of page boundaries
     meta: dict = field(default_factory=dict)
+    kv_dtype: str = "bf16"      # "bf16": k/v hold bf16 bits; "e4m3": OCP e4m3fn codes (uint8)
+    kv_scale: float = 1.0       # per-tensor dequantisation scale of the e4m3 codes
 
     @property
     def batch(self) -> int:
@@ -251,23 +253,25 @@ class RouteCase:
 
 
 # ----------------------------------------------------------------------------- helpers
-def _poison_paged(k_view, v_view, kv_indptr, kv_indices, last, page_size, num_pages):
+def _poison_paged(k_view, v_view, kv_indptr, kv_indices, last, page_size, num_pages, kv_dtype="bf16"):
     used = np.zeros(num_pages, dtype=bool)
     used[kv_indices] = True
-    k_view[~used] = BF16_NAN
-    v_view[~used] = BF16_NAN
-    sentinel = f32_to_bf16_bits(np.array([1.0e4], dtype=np.float32))[0]
+    nan = BF16_NAN if kv_dtype == "bf16" else E4M3_NAN
+    k_view[~used] = nan
+    v_view[~used] = nan
+    # a huge V in the tail slots: 1e4 in bf16, the largest e4m3 code (448) otherwise
+    sentinel = f32_to_bf16_bits(np.array([1.0e4], dtype=np.float32))[0] if kv_dtype == "bf16" else np.uint8(0x7E)
     for r in range(len(kv_indptr) - 1):
         n = kv_indptr[r + 1] - kv_indptr[r]
         if n == 0:
             continue
         p = kv_indices[kv_indptr[r + 1] - 1]
-        k_view[p, last[r]:] = BF16_NAN
+        k_view[p, last[r]:] = nan
         v_view[p, last[r]:] = sentinel
 
 
 def _make_paged(name, seed, lengths, q_len, hq, hk, d, page_size, independent_v, extra_pages=0,
-                poison=False, qo_lens=None):
+                poison=False, qo_lens=None, kv_dtype="bf16"):
     rng = np.random.Generator(np.random.PCG64(seed))
     kv_indptr, kv_indices, last, num_pages = build_page_table(rng, lengths, page_size, extra_pages)
     b = len(lengths)
@@ -275,18 +279,26 @@ def _make_paged(name, seed, lengths, q_len, hq, hk, d, page_size, independent_v,
     qo_indptr = np.zeros(b + 1, dtype=np.int32)
     qo_indptr[1:] = np.cumsum(qo_lens)
     q = normal_bf16(seed, 1, (int(qo_indptr[-1]), hq, d))
-    k_store = normal_bf16(seed, 2, (num_pages, page_size, hk, d))
-    if independent_v:
-        v_store = normal_bf16(seed, 3, (num_pages, page_size, hk, 2 * d))
-        v = v_store[..., :d]
+    v_shape = (num_pages, page_size, hk, 2 * d if independent_v else d)
+    kv_scale = 1.0
+    if kv_dtype == "bf16":
+        k_store = normal_bf16(seed, 2, (num_pages, page_size, hk, d))
+        v_store = normal_bf16(seed, 3, v_shape)
+    elif kv_dtype == "e4m3":
+        # N(0,1) draws encoded as e4m3 codes with one scale for K and V: amax / 448
+        kf = normal_f32(seed, 2, num_pages * page_size * hk * d)
+        vf = normal_f32(seed, 3, int(np.prod(v_shape)))
+        kv_scale = float(np.float32(max(float(np.max(np.abs(kf))), float(np.max(np.abs(vf)))) / 448.0))
+        k_store = e4m3_encode(kf / np.float64(kv_scale)).reshape(num_pages, page_size, hk, d)
+        v_store = e4m3_encode(vf / np.float64(kv_scale)).reshape(v_shape)
     else:
-        v_store = normal_bf16(seed, 3, (num_pages, page_size, hk, d))
-        v = v_store
+        raise ValueError(kv_dtype)
+    v = v_store[..., :d] if independent_v else v_store
     k = k_store
     if poison:
-        _poison_paged(k, v, kv_indptr, kv_indices, last, page_size, num_pages)
+        _poison_paged(k, v, kv_indptr, kv_indices, last, page_size, num_pages, kv_dtype)
     return PagedCase(name, q, k_store, v_store, k, v, qo_indptr, kv_indptr, kv_indices, last, page_size,
-                     hq, hk, d, 1.0 / math.sqrt(d), num_pages)
+                     hq, hk, d, 1.0 / math.sqrt(d), num_pages, kv_dtype=kv_dtype, kv_scale=kv_scale)
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -300,13 +312,15 @@ def tiny_gqa_case(poison: bool = False, independent_v: bool = False, seed: int =
 
 
 def llama70b_decode_case(independent_v: bool = False, batch: int = 64, seed: int = 2,
-                         len_range=(1024, 8192), poison: bool = False) -> PagedCase:
+                         len_range=(1024, 8192), poison: bool = False, kv_dtype: str = "bf16",
+                         q_len: int = 1) -> PagedCase:
     """Llama-3.1-70B-shaped decode: q_len 1, 64 query / 8 KV heads, D=128, P=16,
-    L ~ U[1024, 8192]; V optionally a column slice of a [.., 8, 256] buffer."""
+    L ~ U[1024, 8192]; V optionally a column slice of a [.., 8, 256] buffer; K/V bf16, or e4m3
+    codes with one per-tensor scale (``kv_dtype="e4m3"``)."""
     rng = np.random.Generator(np.random.PCG64(seed + 1000))
     lengths = rng.integers(len_range[0], len_range[1] + 1, size=batch)
-    name = "llama70b_decode" + ("_indep_v" if independent_v else "")
-    return _make_paged(name, seed, lengths, 1, 64, 8, 128, 16, independent_v, poison=poison)
+    name = "llama70b_decode" + ("_indep_v" if independent_v else "") + ("_e4m3" if kv_dtype == "e4m3" else "")
+    return _make_paged(name, seed, lengths, q_len, 64, 8, 128, 16, independent_v, poison=poison, kv_dtype=kv_dtype)
 
 
 def shared_kv_prefill_case(replicated: bool = False, n_batches: int = 32, q_len: int = 128,
