@@ -33,7 +33,7 @@ class _Fakes:
             return plan
 
         def paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan, o, lse, o_part,
-                           lse_part, status, sm_scale, num_pages, stream):
+                           lse_part, status, sm_scale, num_pages, stream, kv_scale=1.0):
             O, LSE = OA.paged_attention(_bits(q), _bits(k_cache), _bits(v_cache), plan.qo, kv_indptr.numpy(),
                                         kv_indices.numpy(), kv_last_page_len.numpy(), k_cache.shape[1], sm_scale)
             o.copy_(torch.from_numpy(O))

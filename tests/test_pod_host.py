@@ -33,7 +33,7 @@ def test_pod_batch_composition(monkeypatch):
         return plan
 
     def paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan, o, lse, o_part, lse_part,
-                       status, sm_scale, num_pages, stream):
+                       status, sm_scale, num_pages, stream, kv_scale=1.0):
         w = plan.words[: 8 * plan.info.num_work].reshape(-1, 8)
         reqs = sorted(set(w[:, 0].tolist()))
         launches.append((plan.info.kernel, reqs))
