@@ -418,7 +418,7 @@ def _e2e(args, runs, dev, stream, skv, torch):
 # ----------------------------------------------------------------------------- other configurations
 CONFIG_NAMES = (["tiny", "llama70b_e4m3", "shared_kv"] + [f"mla_h{h}_q{q}_{d}" for h in (16, 128) for q in (1, 4)
                                                           for d in ("bf16", "e4m3")]
-                + ["mla_h16_q4_bf16_causal", "route", "fetch_splice"])
+                + ["mla_h16_q4_bf16_causal", "pod", "pod_two_launches", "route", "fetch_splice"])
 L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2: written before every timed call
 
 
@@ -537,6 +537,32 @@ def _setup_config(name, dev, skv, torch, stream):
                                                        c.kv_scale, requests=[r], causal=causal), unit_work(r))[1]
                              for r in range(c.batch))
         e["oracle_what"] = "requests"
+    elif name in ("pod", "pod_two_launches"):
+        # a Llama-shaped POD batch: 48 decode requests + 2 prefill requests (1024 query tokens over
+        # 2048 KV tokens each), one attention launch or one launch per kind
+        from workloads import pod_case
+        c = pod_case()
+        d = paged_to_device(c, dev)
+        pod = skv.PodAttention(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, c.page_size, c.num_qo_heads,
+                               c.num_kv_heads, c.head_dim, dev, fused=name == "pod")
+        o = torch.empty(c.q.shape[0], c.num_qo_heads, c.head_dim, device=dev)
+        lse = torch.empty(c.q.shape[0], c.num_qo_heads, device=dev)
+        e["step"] = lambda: pod(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"], d["kv_last_page_len"], o,
+                                lse, sm_scale=c.sm_scale, num_pages=c.num_pages, stream=stream)
+        L = c.kv_lengths()
+        q_rows = np.diff(c.qo_indptr)
+        per_tok = c.num_kv_heads * c.head_dim * 4
+        e["bytes"] = int(L.sum()) * per_tok
+        e["flops"] = float(np.sum(q_rows * L)) * c.num_qo_heads * 4 * c.head_dim
+        e["launches"] = pod.launches()
+        e["kernel"] = {"decode_sms": pod.decode_sms, "plans": [p.info.kernel for p in pod.plans]}
+        e["dtype"] = "bf16"
+        unit_work = lambda r: (float(L[r]) * per_tok, float(q_rows[r] * L[r]) * c.num_qo_heads * 4 * c.head_dim)
+        e["oracle_units"] = (lambda r=r: (OA.paged_attention(c.q, c.k, c.v, c.qo_indptr, c.kv_indptr, c.kv_indices,
+                                                            c.kv_last_page_len, c.page_size, c.sm_scale,
+                                                            requests=[r]), unit_work(r))[1]
+                             for r in list(range(c.batch - 2, c.batch)) + list(range(c.batch - 2)))
+        e["oracle_what"] = "requests (prefill first)"
     elif name == "route":
         c = route_case()
         d = route_to_device(c, dev)
@@ -672,7 +698,8 @@ def main():
     ap.add_argument("--workload", default="llama70b",
                     help="llama70b (the benchmark line) | tiny | llama70b_e4m3 | shared_kv | "
                          "mla_h{16,128}_q{1,4}_{bf16,e4m3} | "
-                         "mla_h16_q4_bf16_causal | route | fetch_splice | all (one line per configuration)")
+                         "mla_h16_q4_bf16_causal | pod | pod_two_launches | route | fetch_splice | all (one line "
+                         "per configuration)")
     ap.add_argument("--no-configs", action="store_true", help="default line without the per-configuration block")
     ap.add_argument("--config-steps", type=int, default=20, help="timed calls per configuration (at most --steps)")
     ap.add_argument("--config-cpu-budget", type=float, default=2.0,

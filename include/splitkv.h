@@ -18,8 +18,10 @@
  *                       partial attention at the KV holder merged "via online softmax",
  *                       "Move the Query, Not the Cache", Methodology; in-CTA split with
  *                       shared-memory merge, FlashInfer PR #5597 page, section 3).
- *   skv_plan_paged_subset  Planner for part of a batch (a mixed prefill + decode batch runs as two
- *                       launches, each on the kernel that suits its requests).
+ *   skv_plan_paged_subset  Planner for part of a batch: a mixed prefill + decode batch is planned
+ *                       as two subsets, each on the kernel that suits its requests.
+ *   skv_pod_attn_fwd    Such a batch in one attention launch (FlashInfer PR #4736 page, section 1,
+ *                       batch_pod.cu: prefill and decode work fused in one kernel).
  *   skv_causal_tables   Host planner that turns causal / multi-token attention into a prefix
  *                       call, a diagonal call over token rows and an exact merge.
  *   skv_mla_splice      The fetch primitive's local compute: move a chunk's latent rows between
@@ -285,8 +287,9 @@ SKV_API skv_status skv_merge_states(const float* o_states, const float* lse_stat
  *   listed requests' query rows and partial rows.  One batch that mixes prefill and decode
  *   requests (a POD batch: prefill on decode, FlashInfer PR #4736 page, batch_pod.cu) is planned
  *   as two subsets, each choosing its own kernel, and launched with the batch's own q, page table
- *   and outputs -- no copy of any of them.  Every plan needs its own o_part / lse_part.  Explicit
- *   splits are not accepted here (SKV_ERR_INVALID).
+ *   and outputs -- no copy of any of them -- in one launch by skv_pod_attn_fwd, or one launch per
+ *   plan.  Every plan needs its own o_part / lse_part.  Explicit splits are not accepted here
+ *   (SKV_ERR_INVALID).
  * ----------------------------------------------------------------------------------------- */
 SKV_API skv_status skv_plan_paged_subset(int32_t batch, const int32_t* qo_indptr_h, const int32_t* kv_indptr_h,
                                          const int32_t* kv_last_page_len_h, int32_t page_size,
@@ -294,6 +297,28 @@ SKV_API skv_status skv_plan_paged_subset(int32_t batch, const int32_t* qo_indptr
                                          int32_t policy, int32_t param, const int32_t* requests_h,
                                          int32_t num_requests, int32_t* plan_h, int64_t plan_capacity,
                                          skv_plan_info* info);
+
+/* -------------------------------------------------------------------------------------------
+ * skv_pod_attn_fwd -- one batch mixing decode and prefill requests in ONE attention launch (POD,
+ *   FlashInfer PR #4736 page, section 1: batch_pod.cu fuses prefill and decode work in one kernel).
+ *   decode_plan_d / decode_info: skv_plan_paged_subset over the batch's decode requests; it must
+ *     pick kernel 3 (all KV heads on the tensor cores; 8 query rows per KV head) and, with
+ *     SKV_SPLIT_BALANCED, its `param` is the number of SMs (persistent CTAs) given to decode.
+ *   prefill_plan_d / prefill_info: skv_plan_paged_subset over the prefill requests; it must pick
+ *     kernel 4 (128-row prefill tiles).  Either plan may be empty (then only the other runs).
+ *   p: the batch's q, K/V caches (bf16), page table and outputs o / lse; p->o_part / p->lse_part
+ *     hold the decode plan's split partials and prefill_o_part / prefill_lse_part the prefill
+ *     plan's (each sized by its plan's num_partial_rows).
+ *   The launch has decode_info->num_ctas + prefill units CTAs: the first num_ctas stream the decode
+ *   slices (HBM-bound) for the whole launch while the rest take the prefill units (tensor-bound) on
+ *   the other SMs.  Results equal skv_paged_attn_fwd on each plan.  The two plans' merge passes
+ *   follow on the same stream.  Errors: as skv_paged_attn_fwd; SKV_ERR_UNSUPPORTED for another
+ *   kernel choice or an e4m3 cache.
+ * ----------------------------------------------------------------------------------------- */
+SKV_API skv_status skv_pod_attn_fwd(const skv_paged_params* p, const int32_t* decode_plan_d,
+                                    const skv_plan_info* decode_info, const int32_t* prefill_plan_d,
+                                    const skv_plan_info* prefill_info, float* prefill_o_part,
+                                    float* prefill_lse_part, skv_stream_t stream);
 
 /* -------------------------------------------------------------------------------------------
  * skv_causal_tables -- host planner for causal / multi-token attention.  The n_q query tokens of

@@ -6,7 +6,7 @@ streams); host arrays are numpy.  Importing this package without the built libra
 there is no fallback path.
 
 Functions mirror the C ABI in include/splitkv.h:
-``plan_paged``, ``paged_attn_fwd``, ``plan_mla``, ``mla_decode_fwd``, ``merge_states``,
+``plan_paged``, ``paged_attn_fwd``, ``pod_attn_fwd``, ``plan_mla``, ``mla_decode_fwd``, ``merge_states``,
 ``paged_kv_gather``, ``mla_splice``, ``mla_fold_ratio``, ``status_str``, ``version``.
 """
 from __future__ import annotations
@@ -113,6 +113,8 @@ _mla_partial = _proto("skv_mla_decode_partial", ctypes.c_int, [ctypes.POINTER(Ml
                                                                 ctypes.POINTER(PlanInfo), _vp])
 _paged_static = _proto("skv_paged_attn_fwd_static_scratch", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp,
                                                                           ctypes.POINTER(PlanInfo), _vp])
+_pod_fwd = _proto("skv_pod_attn_fwd", ctypes.c_int, [ctypes.POINTER(PagedParams), _vp, ctypes.POINTER(PlanInfo), _vp,
+                                                     ctypes.POINTER(PlanInfo), _vp, _vp, _vp])
 _merge_plan = _proto("skv_merge_plan", ctypes.c_int, [_vp, _vp, _vp, ctypes.POINTER(PlanInfo), ctypes.c_int32,
                                                        ctypes.c_int32, _vp, ctypes.c_int32, _vp, _vp])
 _merge = _proto("skv_merge_states", ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
@@ -132,7 +134,8 @@ _version = _proto("skv_version", ctypes.c_int32, [])
 SYMBOLS = ["skv_plan_paged", "skv_paged_attn_fwd", "skv_paged_attn_partial", "skv_merge_plan", "skv_plan_mla",
            "skv_mla_decode_fwd", "skv_mla_decode_partial", "skv_merge_states", "skv_paged_kv_gather",
            "skv_mla_fold_ratio", "skv_status_str", "skv_version", "skv_paged_attn_fwd_static_scratch",
-           "skv_test_wait_timeout", "skv_mla_splice", "skv_causal_tables", "skv_plan_paged_subset"]
+           "skv_test_wait_timeout", "skv_mla_splice", "skv_causal_tables", "skv_plan_paged_subset",
+           "skv_pod_attn_fwd"]
 
 
 class SkvError(RuntimeError):
@@ -325,6 +328,19 @@ def paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len,
            "skv_paged_attn_fwd" if phase == "all" else "skv_paged_attn_partial")
 
 
+def pod_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, decode_plan: Plan, prefill_plan: Plan,
+                 o, lse=None, decode_o_part=None, decode_lse_part=None, prefill_o_part=None, prefill_lse_part=None,
+                 status=None, sm_scale: Optional[float] = None, num_pages: Optional[int] = None, stream=None) -> None:
+    """skv_pod_attn_fwd: the decode subset plan (all-KV-heads kernel) and the prefill subset plan
+    (128-row kernel) of one batch in one attention launch, then both plans' merge passes.  Each
+    plan's split partials go to its own o_part / lse_part."""
+    p = _paged_params(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, o, lse, decode_o_part,
+                      decode_lse_part, status, sm_scale, num_pages)
+    _check(_pod_fwd(ctypes.byref(p), _dptr(decode_plan.device), ctypes.byref(decode_plan.info),
+                    _dptr(prefill_plan.device), ctypes.byref(prefill_plan.info), _dptr(prefill_o_part),
+                    _dptr(prefill_lse_part), _stream_ptr(stream)), "skv_pod_attn_fwd")
+
+
 def paged_attn_fwd_static_scratch(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan: Plan, o,
                                   lse=None, status=None, sm_scale: Optional[float] = None,
                                   num_pages: Optional[int] = None, stream=None) -> None:
@@ -475,4 +491,5 @@ def library_path() -> str:
     return _LIB_PATH
 
 
-from .runner import CausalMlaDecode, RouteMerge, mla_decode, paged_attention, pod_attention  # noqa: E402,F401
+from .runner import (CausalMlaDecode, PodAttention, RouteMerge, mla_decode, paged_attention,  # noqa: E402,F401
+                     pod_attention, pod_decode_sms)

@@ -447,8 +447,12 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
                      kernel, po, plan_h, plan_capacity, info);
 }
 
-skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan_d,
-                              const skv_plan_info* info, skv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Host checks of a paged launch: the arguments, the plan summary and the kernel it names.
+skv_status check_paged(const skv_paged_params* p, const int32_t* plan_d, const skv_plan_info* info) {
   if (p == nullptr) return SKV_ERR_INVALID;
   skv_status st = check_plan(plan_d, info);
   if (st != SKV_OK) return st;
@@ -476,14 +480,26 @@ skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan
     return SKV_ERR_INVALID;
   // the e4m3 cache runs on the all-KV-heads tensor-core kernel only
   if (fp8 && info->kernel != KERNEL_GQA_TC_WIDE) return SKV_ERR_UNSUPPORTED;
+  if (info->num_work > 0 && info->kernel == KERNEL_GQA_TC_WIDE &&
+      (info->num_ctas < 1 || info->cta_offset < 8LL * info->num_work + 4LL * info->num_merge_rows))
+    return SKV_ERR_INVALID;
+  return SKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+skv_status skv_paged_attn_partial(const skv_paged_params* p, const int32_t* plan_d,
+                              const skv_plan_info* info, skv_stream_t stream) {
+  skv_status st = check_paged(p, plan_d, info);
+  if (st != SKV_OK) return st;
+  const bool fp8 = p->kv_dtype == SKV_E4M3;
   if (info->num_work == 0) return SKV_OK;  // no query rows: nothing to launch
   const bool same_kv = p->k_stride[0] == p->v_stride[0] && p->k_stride[1] == p->v_stride[1] &&
                        p->k_stride[2] == p->v_stride[2];
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  if (info->kernel == KERNEL_GQA_TC_WIDE &&
-      (info->num_ctas < 1 || info->cta_offset < 8LL * info->num_work + 4LL * info->num_merge_rows))
-    return SKV_ERR_INVALID;
   int e = info->kernel == KERNEL_GQA_TC_WIDE
               ? (fp8 ? launch_gqa_tc_wide_fp8(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile, s)
                      : launch_gqa_tc_wide(*p, work, plan_d + info->cta_offset, info->num_ctas, info->q_tile, s))
@@ -513,6 +529,40 @@ skv_status skv_paged_attn_fwd(const skv_paged_params* p, const int32_t* plan_d,
   if (st != SKV_OK) return st;
   return skv_merge_plan(p->o_part, p->lse_part, plan_d, info, p->num_qo_heads, p->head_dim, p->o, p->o_dtype,
                         p->lse, stream);
+}
+
+skv_status skv_pod_attn_fwd(const skv_paged_params* p, const int32_t* decode_plan_d,
+                            const skv_plan_info* decode_info, const int32_t* prefill_plan_d,
+                            const skv_plan_info* prefill_info, float* prefill_o_part, float* prefill_lse_part,
+                            skv_stream_t stream) {
+  if (p == nullptr || decode_info == nullptr || prefill_info == nullptr) return SKV_ERR_INVALID;
+  skv_paged_params pp = *p;  // the prefill plan's view: its own partial buffers
+  pp.o_part = prefill_o_part;
+  pp.lse_part = prefill_lse_part;
+  skv_status st = check_paged(p, decode_plan_d, decode_info);
+  if (st == SKV_OK) st = check_paged(&pp, prefill_plan_d, prefill_info);
+  if (st != SKV_OK) return st;
+  if (p->kv_dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
+  const bool has_dec = decode_info->num_work > 0, has_pre = prefill_info->num_work > 0;
+  if ((has_dec && decode_info->kernel != KERNEL_GQA_TC_WIDE) || (has_pre && prefill_info->kernel != KERNEL_GQA_TC_PREFILL))
+    return SKV_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (has_dec && has_pre) {
+    st = cuda_status(launch_gqa_pod(*p, reinterpret_cast<const WorkItem*>(decode_plan_d),
+                                    decode_plan_d + decode_info->cta_offset, decode_info->num_ctas,
+                                    decode_info->q_tile, pp, reinterpret_cast<const WorkItem*>(prefill_plan_d),
+                                    prefill_info->num_work, prefill_info->q_tile, s));
+  } else if (has_dec) {
+    st = skv_paged_attn_partial(p, decode_plan_d, decode_info, stream);
+  } else if (has_pre) {
+    st = skv_paged_attn_partial(&pp, prefill_plan_d, prefill_info, stream);
+  }
+  if (st != SKV_OK) return st;
+  st = skv_merge_plan(p->o_part, p->lse_part, decode_plan_d, decode_info, p->num_qo_heads, p->head_dim, p->o,
+                      p->o_dtype, p->lse, stream);
+  if (st != SKV_OK) return st;
+  return skv_merge_plan(pp.o_part, pp.lse_part, prefill_plan_d, prefill_info, p->num_qo_heads, p->head_dim, p->o,
+                        p->o_dtype, p->lse, stream);
 }
 
 skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d,

@@ -97,6 +97,9 @@ int launch_gqa_tc_wide(const skv_paged_params& p, const WorkItem* work, const in
                        int q_tile, cudaStream_t s);
 int launch_gqa_tc_wide_fp8(const skv_paged_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                            int q_tile, cudaStream_t s);
+int launch_gqa_pod(const skv_paged_params& dp, const WorkItem* dwork, const int32_t* cta_indptr, int num_ctas,
+                   int dq_tile, const skv_paged_params& pp, const WorkItem* pwork, int pnum_work, int pq_tile,
+                   cudaStream_t s);
 bool gqa_tc_prefill_supported(int head_dim, int page_size, int group);
 int launch_gqa_tc_prefill(const skv_paged_params& p, const WorkItem* work, int num_work, int q_tile,
                           cudaStream_t s);

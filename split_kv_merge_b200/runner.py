@@ -7,7 +7,7 @@ from typing import Optional
 import numpy as np
 
 from . import (Plan, causal_tables, mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged,
-               plan_paged_subset)
+               plan_paged_subset, pod_attn_fwd)
 
 
 def _dev_i32(a, device, non_blocking=False):
@@ -101,36 +101,101 @@ def paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, k
     return o, lse, {"plan": plan, "o_part": o_part, "lse_part": lse_part}
 
 
+def pod_decode_sms(decode_kv_bytes: float, prefill_flops: float, num_sms: int = 148) -> int:
+    """SMs a POD launch gives to its decode slices: the decode part's share of the two parts'
+    standalone times (decode KV bytes at 6.0 TB/s, prefill FLOPs at 0.9 PFLOP/s -- what the two
+    kernels reach alone on B200), kept within [16, num_sms - 16]."""
+    t_dec, t_pre = float(decode_kv_bytes) / 6.0e12, float(prefill_flops) / 0.9e15
+    share = t_dec / (t_dec + t_pre) if t_dec + t_pre > 0 else 0.5
+    return int(min(num_sms - 16, max(16, round(num_sms * share))))
+
+
+class PodAttention:
+    """One batch mixing prefill and decode requests (POD: prefill on decode, FlashInfer PR #4736
+    page, batch_pod.cu), planned once: requests with at most ``decode_q_max`` query tokens (default:
+    what the all-KV-heads decode kernel holds, 8 // group) on the decode plan, whose KV slices are
+    balanced over ``decode_sms`` persistent CTAs, and the rest on the 128-row prefill plan
+    (``skv_plan_paged_subset`` twice).  ``fused``: both plans run in ONE attention launch
+    (``skv_pod_attn_fwd``: the decode CTAs stream the KV cache while the prefill CTAs fill the
+    other SMs); otherwise one launch per plan.  Each call runs on the batch's own q, page table and
+    outputs; each plan keeps its own partial buffers."""
+
+    def __init__(self, qo_indptr_h, kv_indptr_h, kv_last_page_len_h, page_size: int, num_qo_heads: int,
+                 num_kv_heads: int, head_dim: int, device, *, decode_q_max: Optional[int] = None,
+                 decode_sms: Optional[int] = None, num_sms: int = 148, policy="balanced", fused: bool = True):
+        import torch
+        qo = np.asarray(qo_indptr_h, dtype=np.int64)
+        q_lens = np.diff(qo)
+        g = num_qo_heads // num_kv_heads
+        if decode_q_max is None:
+            decode_q_max = max(1, 8 // max(1, g))
+        dec, pre = np.flatnonzero(q_lens <= decode_q_max), np.flatnonzero(q_lens > decode_q_max)
+        kv_ip = np.asarray(kv_indptr_h, dtype=np.int64)
+        n_pages = np.diff(kv_ip)
+        lengths = np.where(n_pages > 0, (n_pages - 1) * page_size + np.asarray(kv_last_page_len_h, np.int64), 0)
+        if decode_sms is None:
+            dec_bytes = float(lengths[dec].sum()) * num_kv_heads * head_dim * 4
+            pre_flops = float(np.sum(q_lens[pre] * lengths[pre])) * num_qo_heads * 4 * head_dim
+            decode_sms = pod_decode_sms(dec_bytes, pre_flops, num_sms) if len(pre) else num_sms
+        self.decode_sms = int(decode_sms)
+        args = (qo_indptr_h, kv_indptr_h, kv_last_page_len_h, page_size, num_qo_heads, num_kv_heads, head_dim)
+        self.decode_plan = plan_paged_subset(*args, dec, policy, self.decode_sms).to(device)
+        self.prefill_plan = plan_paged_subset(*args, pre, policy, max(1, num_sms - self.decode_sms) if len(dec)
+                                              else num_sms).to(device)
+        self.requests = (dec, pre)
+        self.fused = bool(fused) and len(dec) > 0 and len(pre) > 0 and self.decode_plan.info.kernel == 3 \
+            and self.prefill_plan.info.kernel == 4
+        f32 = dict(dtype=torch.float32, device=device)
+
+        def parts(plan):
+            n = plan.info.num_partial_rows
+            return (torch.empty(n, num_qo_heads, head_dim, **f32), torch.empty(n, num_qo_heads, **f32)) if n \
+                else (None, None)
+        self.decode_part, self.prefill_part = parts(self.decode_plan), parts(self.prefill_plan)
+
+    @property
+    def plans(self):
+        return [p for p, r in ((self.decode_plan, self.requests[0]), (self.prefill_plan, self.requests[1])) if len(r)]
+
+    def launches(self) -> int:
+        """Kernel launches per call (attention, then each plan's merge pass if it has merge rows)."""
+        merges = sum(1 for p in self.plans if p.info.num_merge_rows > 0)
+        return (1 if self.fused else len(self.plans)) + merges
+
+    def __call__(self, q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, o, lse, *, sm_scale=None,
+                 num_pages: Optional[int] = None, status=None, stream=None):
+        if self.fused:
+            pod_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, self.decode_plan,
+                         self.prefill_plan, o, lse, *self.decode_part, *self.prefill_part, status, sm_scale, num_pages,
+                         stream)
+            return o, lse
+        for plan, (op, lp) in ((self.decode_plan, self.decode_part), (self.prefill_plan, self.prefill_part)):
+            if plan.info.num_work > 0:
+                paged_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, plan, o, lse, op, lp,
+                               status, sm_scale, num_pages, stream)
+        return o, lse
+
+
 def pod_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, kv_last_page_len_h, *,
                   decode_q_max: Optional[int] = None, sm_scale: Optional[float] = None, policy="balanced",
-                  param: int = 0, o_dtype=None, num_pages: Optional[int] = None, status=None, stream=None):
-    """A batch that mixes prefill and decode requests (POD: prefill on decode, FlashInfer PR #4736
-    page, batch_pod.cu), run as one launch per kind on the batch's own q, page table and outputs:
-    requests with at most ``decode_q_max`` query tokens (default: what the all-KV-heads decode
-    kernel holds, 8 // group) on the decode plan, the rest on the prefill plan
-    (``skv_plan_paged_subset``).  Returns (o, lse, {"plans": [...]})."""
+                  decode_sms: Optional[int] = None, o_dtype=None, num_pages: Optional[int] = None, status=None,
+                  stream=None, fused: bool = True):
+    """A batch that mixes prefill and decode requests (``PodAttention``), planned and run once: by
+    default in one attention launch, with ``fused=False`` one launch per plan.
+    Returns (o, lse, {"plans": [...], "pod": the PodAttention})."""
     import torch
     dev = q.device
     hq, d = q.shape[1], q.shape[2]
     hk = k_cache.shape[2]
-    q_lens = np.diff(np.asarray(qo_indptr_h, dtype=np.int64))
-    if decode_q_max is None:
-        decode_q_max = max(1, 8 // max(1, hq // hk))
+    pod = PodAttention(qo_indptr_h, kv_indptr_h, kv_last_page_len_h, k_cache.shape[1], hq, hk, d, dev,
+                       decode_q_max=decode_q_max, decode_sms=decode_sms, policy=policy, fused=fused)
     kv_indptr = _dev_i32(kv_indptr_h, dev)
     kv_last = _dev_i32(kv_last_page_len_h, dev)
     o = torch.empty(q.shape[0], hq, d, dtype=o_dtype or torch.float32, device=dev)
     lse = torch.empty(q.shape[0], hq, dtype=torch.float32, device=dev)
-    plans = []
-    for reqs in (np.flatnonzero(q_lens <= decode_q_max), np.flatnonzero(q_lens > decode_q_max)):
-        if len(reqs) == 0:
-            continue
-        plan = plan_paged_subset(qo_indptr_h, kv_indptr_h, kv_last_page_len_h, k_cache.shape[1], hq, hk, d, reqs,
-                                 policy, param)
-        paged_attention(q, k_cache, v_cache, qo_indptr_h, kv_indptr_h, kv_indices, kv_last_page_len_h,
-                        sm_scale=sm_scale, num_pages=num_pages, kv_indptr=kv_indptr, kv_last_page_len=kv_last,
-                        plan=plan, status=status, stream=stream, o_out=o, lse_out=lse)
-        plans.append(plan)
-    return o, lse, {"plans": plans}
+    pod(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last, o, lse, sm_scale=sm_scale, num_pages=num_pages,
+        status=status, stream=stream)
+    return o, lse, {"plans": pod.plans, "pod": pod}
 
 
 def mla_decode(q_nope, q_pe, ckv, kpe, kv_indptr_h, kv_indices, kv_last_page_len_h, *,

@@ -56,7 +56,7 @@ def test_pod_batch_composition(monkeypatch):
     v = normal_bf16(71, 3, (num_pages, P, hk, d))
     scale = 1 / math.sqrt(d)
     o, lse, ex = R.pod_attention(_tb(q), _tb(k), _tb(v), qo, kv_indptr, torch.from_numpy(kv_indices), last,
-                                 sm_scale=scale, policy="none")
+                                 sm_scale=scale, policy="none", fused=False)
     # decode requests (one query token) on the all-KV-heads decode kernel, the rest on the prefill kernel
     assert launches == [(3, [0, 2, 3]), (4, [1, 4])]
     O, LSE = OA.paged_attention(q, k, v, qo, kv_indptr, kv_indices, last, P, scale)
@@ -64,6 +64,62 @@ def test_pod_batch_composition(monkeypatch):
     np.testing.assert_array_equal(np.isneginf(lse.numpy()), np.isneginf(LSE))
     fin = np.isfinite(LSE)
     np.testing.assert_allclose(lse.numpy()[fin], LSE[fin], rtol=0, atol=1e-6)
+
+
+def test_pod_fused_composition(monkeypatch):
+    """The one-launch form: ``PodAttention`` hands both plans (decode subset on the all-KV-heads
+    kernel with its CTAs = the SMs given to decode, prefill subset on the 128-row kernel) and their
+    own partial buffers to ONE ``skv_pod_attn_fwd`` call; a stand-in computing exactly the requests
+    of each plan gives the oracle's attention for the whole batch."""
+    calls = []
+    real_subset = R.plan_paged_subset
+
+    def plan_paged_subset(qo, *a, **k):
+        plan = real_subset(qo, *a, **k)
+        plan.qo = np.asarray(qo, dtype=np.int32)
+        return plan
+
+    def pod_attn_fwd(q, k_cache, v_cache, kv_indptr, kv_indices, kv_last_page_len, dplan, pplan, o, lse, dop, dlp,
+                     pop, plp, status, sm_scale, num_pages, stream):
+        calls.append((dplan.info.kernel, dplan.info.num_ctas, pplan.info.kernel))
+        for plan in (dplan, pplan):
+            w = plan.words[: 8 * plan.info.num_work].reshape(-1, 8)
+            reqs = sorted(set(w[:, 0].tolist()))
+            O, LSE = OA.paged_attention(_bits(q), _bits(k_cache), _bits(v_cache), plan.qo, kv_indptr.numpy(),
+                                        kv_indices.numpy(), kv_last_page_len.numpy(), k_cache.shape[1], sm_scale,
+                                        requests=reqs)
+            for r in reqs:
+                a, b = int(plan.qo[r]), int(plan.qo[r + 1])
+                o[a:b] = torch.from_numpy(O[a:b])
+                lse[a:b] = torch.from_numpy(LSE[a:b])
+
+    monkeypatch.setattr(R, "plan_paged_subset", plan_paged_subset)
+    monkeypatch.setattr(R, "pod_attn_fwd", pod_attn_fwd)
+    rng = np.random.Generator(np.random.PCG64(72))
+    lengths, q_lens, P, hq, hk, d = [300, 170, 0, 640, 200, 5, 64], [1, 40, 1, 1, 128, 0, 1], 16, 64, 8, 128
+    kv_indptr, kv_indices, last, num_pages = build_page_table(rng, lengths, P, extra_pages=2)
+    qo = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    q = normal_bf16(72, 1, (int(qo[-1]), hq, d))
+    k = normal_bf16(72, 2, (num_pages, P, hk, d))
+    v = normal_bf16(72, 3, (num_pages, P, hk, d))
+    scale = 1 / math.sqrt(d)
+    o, lse, ex = R.pod_attention(_tb(q), _tb(k), _tb(v), qo, kv_indptr, torch.from_numpy(kv_indices), last,
+                                 sm_scale=scale, decode_sms=40)
+    assert calls == [(3, 40, 4)]                   # one launch; the decode slices on 40 CTAs
+    assert ex["pod"].fused and ex["pod"].launches() >= 1
+    O, LSE = OA.paged_attention(q, k, v, qo, kv_indptr, kv_indices, last, P, scale)
+    np.testing.assert_allclose(o.numpy(), O, rtol=0, atol=1e-6)
+    fin = np.isfinite(LSE)
+    np.testing.assert_array_equal(np.isneginf(lse.numpy()), np.isneginf(LSE))
+    np.testing.assert_allclose(lse.numpy()[fin], LSE[fin], rtol=0, atol=1e-6)
+
+
+def test_pod_decode_sms_share():
+    """The SMs given to decode follow the decode part's share of the two standalone times and stay
+    within [16, SMs - 16]."""
+    assert R.pod_decode_sms(6.0e12 * 100e-6, 0.9e15 * 100e-6) == 74        # equal times: half the SMs
+    assert R.pod_decode_sms(6.0e12 * 300e-6, 0.9e15 * 100e-6) == 111
+    assert R.pod_decode_sms(1.0, 1.0e15) == 16 and R.pod_decode_sms(1.0e13, 1.0) == 132
 
 
 def test_subset_planner_rejects_bad_lists():

@@ -34,7 +34,7 @@ import numpy as np
 
 __all__ = [
     "BF16_NAN", "E4M3_NAN", "f32_to_bf16_bits", "bf16_bits_to_f32", "e4m3_encode",
-    "normal_f32", "normal_bf16", "build_page_table", "PagedCase", "MlaCase", "RouteCase",
+    "normal_f32", "normal_bf16", "build_page_table", "PagedCase", "MlaCase", "RouteCase", "pod_case",
     "tiny_gqa_case", "llama70b_decode_case", "shared_kv_prefill_case", "mla_decode_case",
     "route_case", "even_split_pages", "SpliceCase", "fetch_splice_case",
 ]
@@ -321,6 +321,19 @@ def llama70b_decode_case(independent_v: bool = False, batch: int = 64, seed: int
     lengths = rng.integers(len_range[0], len_range[1] + 1, size=batch)
     name = "llama70b_decode" + ("_indep_v" if independent_v else "") + ("_e4m3" if kv_dtype == "e4m3" else "")
     return _make_paged(name, seed, lengths, q_len, 64, 8, 128, 16, independent_v, poison=poison, kv_dtype=kv_dtype)
+
+
+def pod_case(num_decode: int = 48, prefill_q=(1024, 1024), prefill_kv=(2048, 2048), seed: int = 6,
+             decode_len_range=(1024, 8192)) -> PagedCase:
+    """A POD batch (prefill on decode) with Llama-3.1-70B heads (64 query / 8 KV, D=128, P=16):
+    ``num_decode`` decode requests (one query token, KV lengths U[1024, 8192]) followed by prefill
+    requests of ``prefill_q`` query tokens over ``prefill_kv`` KV tokens (every query token sees the
+    request's whole KV), bf16 N(0,1), randomly permuted pages."""
+    rng = np.random.Generator(np.random.PCG64(seed + 3000))
+    dec_lens = rng.integers(decode_len_range[0], decode_len_range[1] + 1, size=num_decode)
+    lengths = np.concatenate([dec_lens, np.asarray(prefill_kv, np.int64)])
+    qo_lens = np.concatenate([np.ones(num_decode, np.int64), np.asarray(prefill_q, np.int64)])
+    return _make_paged("pod_llama70b", seed, lengths, 1, 64, 8, 128, 16, False, qo_lens=qo_lens)
 
 
 def shared_kv_prefill_case(replicated: bool = False, n_batches: int = 32, q_len: int = 128,
