@@ -103,14 +103,17 @@ typedef struct {
   int32_t kernel;           /* kernel variant the dispatcher picked (informational): 1 GQA on  */
                             /*   CUDA cores, 2 GQA tensor-core decode per KV head, 3 GQA      */
                             /*   tensor-core decode over all KV heads, 4 GQA tensor-core      */
-                            /*   prefill (128 query rows), 11 MLA on CUDA cores, 12 / 13 MLA  */
-                            /*   tensor cores with 16 / 32 query rows per tile                */
+                            /*   prefill (128 query rows), 11 MLA on CUDA cores, 12 / 13 / 14 */
+                            /*   MLA tensor cores with 16 / 32 / 64 query rows per tile       */
   int32_t q_tile;           /* query tokens per work item (MLA: the fold ratio F)             */
   int32_t plan_words;       /* int32 words of the plan actually used                          */
   int32_t max_splits;       /* largest split count of any request                             */
   int32_t total_splits;     /* sum over requests of their split counts                        */
   int32_t num_ctas;         /* persistent kernels: CTAs the plan was balanced for (else 0);  */
-                            /*   CTA c runs work items cta_indptr[c] .. cta_indptr[c+1]       */
+                            /*   CTA c runs work items cta_indptr[c] .. cta_indptr[c+1]; for  */
+                            /*   kernel 14 a group of R CTAs shares each KV slice s (CTA c    */
+                            /*   runs slice c / R), R = (q_len / q_tile) * head groups        */
+                            /*   (num_heads / 64 when num_heads > 64, else 1)                 */
   int32_t cta_offset;       /* int32 word offset of cta_indptr [num_ctas+1] in the plan       */
 } skv_plan_info;
 
@@ -217,10 +220,13 @@ SKV_API skv_status skv_paged_attn_fwd_static_scratch(const skv_paged_params* p, 
  *   the cache type (SKV_BF16 or SKV_E4M3) the plan will run on.  The fold ratio F (seqlen_q
  *   tokens folded into the query-row dimension of a work item) is reported in info->q_tile:
  *   F = skv_mla_fold_ratio(H, q_len, R) with R the rows the chosen kernel puts on one tile
- *   (16 or 32 for the tensor-core kernel, which splits H > R heads into groups of R; 128 for
- *   the CUDA-core kernel).  The tensor-core kernels take page sizes >= 8 that divide or are
- *   multiples of 64, and (bf16 cache only) page size 1, where every page id is a token row; other
- *   page sizes run on the CUDA-core kernel.  Run a plan on the kv_dtype it was made for.
+ *   (16 or 32 for the tensor-core kernels, and 64 for the bf16 cache when H * q_len > 32 and the
+ *   page size is not 1; they split H > R heads into groups of R; 128 for the CUDA-core kernel).
+ *   With R = 64 the (query tile, head group) units of a KV slice run on a group of co-resident
+ *   CTAs at once, so each slice is read from HBM about once.  The tensor-core kernels take page
+ *   sizes >= 8 that divide or are multiples of 64, and (bf16 cache only) page size 1, where every
+ *   page id is a token row; other page sizes run on the CUDA-core kernel.  Run a plan on the
+ *   kv_dtype it was made for.
  * ----------------------------------------------------------------------------------------- */
 SKV_API skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h,
                         const int32_t* kv_last_page_len_h, int32_t page_size, int32_t num_heads,

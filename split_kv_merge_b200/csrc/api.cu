@@ -47,6 +47,11 @@ struct PersistOpts {
   int32_t tile_tokens = 128;
   int32_t page_size = 1;
   int32_t piece_cost = 0;  // fixed cost of a work item (query load, pipeline refill, epilogue), in tiles
+  // CTAs per KV slice.  With group > 1 the work items cover query tile 0 only and every slice is
+  // run by `group` co-resident CTAs, each taking one (query tile, head group) of every item, so
+  // the slice streams from HBM about once and the other CTAs read it from L2.  The plan's
+  // num_ctas counts all CTAs (slices x group); cta_indptr has one entry per slice.
+  int32_t group = 1;
 };
 
 // Tiles of logical pages [a, b) of a request of length L (pages of `page_size` tokens).
@@ -101,7 +106,8 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
     double total = 0, piece_total = 0;
     int64_t nonempty = 0;
     for (int32_t r = 0; r < batch; ++r) {
-      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile * units_per_page;
+      const int64_t qt = po.group > 1 ? (req[r].q_len > 0 ? 1 : 0)
+                                      : (req[r].q_len + q_tile - 1) / q_tile * units_per_page;
       w[r] = qt * range_tiles(0, req[r].n_pages, kv_len[r], P, T);
       total += (double)w[r];
       if (w[r] > 0) {
@@ -117,7 +123,8 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
     int cta = 0;
     double cum = 0;
     for (int32_t r = 0; r < batch; ++r) {
-      const int64_t qt = (req[r].q_len + q_tile - 1) / q_tile * units_per_page;
+      const int64_t qt = po.group > 1 ? (req[r].q_len > 0 ? 1 : 0)
+                                      : (req[r].q_len + q_tile - 1) / q_tile * units_per_page;
       const int32_t n = req[r].n_pages;
       bounds[r].push_back(0);
       if (n == 0 || qt == 0) {  // nothing to stream: one (empty) piece on the current CTA
@@ -188,7 +195,8 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
     max_splits = std::max(max_splits, S);
     total_splits += S;
     if (q.q_len == 0) continue;
-    for (int32_t q0 = 0; q0 < q.q_len; q0 += q_tile) {
+    const int32_t q_items = po.group > 1 ? 1 : q.q_len;  // grouped: query tile 0 stands for all tiles
+    for (int32_t q0 = 0; q0 < q_items; q0 += q_tile) {
       const int32_t qc = std::min(q_tile, q.q_len - q0);
       for (int j = 0; j < S; ++j) {
         WorkItem w;
@@ -253,7 +261,7 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
   info->q_tile = q_tile;
   info->max_splits = max_splits;
   info->total_splits = total_splits;
-  info->num_ctas = num_ctas;
+  info->num_ctas = num_ctas * std::max<int32_t>(1, po.group);
   const int64_t base_words = plan_words(info->num_work, info->num_merge_rows);
   info->cta_offset = persistent ? (int32_t)base_words : 0;
   const int64_t words = base_words + (persistent ? num_ctas + 1 : 0);
@@ -426,9 +434,13 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
   for (int32_t r = 0; r < batch; ++r)
     kv_len[r] = req[r].n_pages == 0 ? 0
                                     : (int64_t)(req[r].n_pages - 1) * page_size + kv_last_page_len_h[r];
-  // tensor-core kernel: 16 query rows per tile when all of a request's rows fit, else 32 (heads
-  // beyond 32 in groups of 32); the fold puts as many query tokens as fit into those rows
-  const int32_t nr = (int64_t)num_heads * q_len <= 16 ? 16 : 32;
+  // tensor-core kernel: 16 query rows per tile when all of a request's rows fit, else 32; for the
+  // bf16 cache 64 rows when a request has more (heads beyond 64 in groups of 64, their units spread
+  // over a group of CTAs that share each KV slice); the fold puts as many query tokens as fit into
+  // those rows
+  const int64_t hq = (int64_t)num_heads * q_len;
+  int32_t nr = hq <= 16 ? 16 : 32;
+  if (kv_dtype == SKV_BF16 && hq > 32 && mla_tc_supported(kv_dtype, page_size, num_heads, 64)) nr = 64;
   const bool tc = kv_dtype == SKV_E4M3 ? mla_tc_fp8_supported(page_size, num_heads, nr)
                                        : mla_tc_supported(kv_dtype, page_size, num_heads, nr);
   PersistOpts po;
@@ -436,12 +448,17 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
   int32_t kernel = KERNEL_MLA_SIMT, fold = skv_mla_fold_ratio(num_heads, q_len, 128);
   int64_t head_groups = 1;
   if (tc) {
-    kernel = nr == 16 ? KERNEL_MLA_TC16 : KERNEL_MLA_TC32;
+    kernel = nr == 16 ? KERNEL_MLA_TC16 : nr == 32 ? KERNEL_MLA_TC32 : KERNEL_MLA_TC64;
     fold = num_heads <= nr ? skv_mla_fold_ratio(num_heads, q_len, nr) : 1;
     head_groups = num_heads <= nr ? 1 : num_heads / nr;
-    po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
+    const int32_t sms = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
+    po.flat_ctas = sms;
     po.tile_tokens = mla_tc_tile_tokens();
     po.piece_cost = 4;  // measured: a work item's start and end cost about four 64-token tiles
+    if (nr == 64) {
+      po.group = (int32_t)(head_groups * (q_len / fold));
+      po.flat_ctas = std::max<int32_t>(1, sms / po.group);
+    }
   }
   return plan_common(batch, req, kv_len, fold, head_groups, 8, policy, param, split_indptr_h, split_bounds_h,
                      kernel, po, plan_h, plan_capacity, info);
@@ -589,14 +606,15 @@ skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d
       !aligned16(p->o))
     return SKV_ERR_ALIGNMENT;
   if (info->num_partial_rows > 0 && (!p->o_part || !p->lse_part)) return SKV_ERR_WORKSPACE;
-  const bool tc = info->kernel == KERNEL_MLA_TC16 || info->kernel == KERNEL_MLA_TC32;
+  const bool tc = info->kernel == KERNEL_MLA_TC16 || info->kernel == KERNEL_MLA_TC32 || info->kernel == KERNEL_MLA_TC64;
   if (info->kernel != KERNEL_MLA_SIMT && !tc) return SKV_ERR_INVALID;
+  if (info->kernel == KERNEL_MLA_TC64 && p->kv_dtype != SKV_BF16) return SKV_ERR_INVALID;
   if (info->num_work == 0) return SKV_OK;  // no requests: nothing to launch
   if (tc && (info->num_ctas < 1 || info->cta_offset < 8LL * info->num_work + 4LL * info->num_merge_rows))
     return SKV_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  const int rows = info->kernel == KERNEL_MLA_TC16 ? 16 : 32;
+  const int rows = info->kernel == KERNEL_MLA_TC16 ? 16 : info->kernel == KERNEL_MLA_TC32 ? 32 : 64;
   int e = !tc                         ? launch_mla_simt(*p, work, info->num_work, info->q_tile, s)
           : p->kv_dtype == SKV_E4M3 ? launch_mla_tc_fp8(*p, work, plan_d + info->cta_offset, info->num_ctas,
                                                         info->q_tile, rows, s)

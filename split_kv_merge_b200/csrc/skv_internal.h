@@ -33,6 +33,7 @@ enum KernelId : int32_t {
   KERNEL_MLA_SIMT = 11,
   KERNEL_MLA_TC16 = 12,  // tensor-core MLA, 16 query rows per unit (bf16 or e4m3 cache)
   KERNEL_MLA_TC32 = 13,  // tensor-core MLA, 32 query rows per unit (bf16 or e4m3 cache)
+  KERNEL_MLA_TC64 = 14,  // tensor-core MLA, 64 query rows per unit, CTA groups per KV slice (bf16)
 };
 
 // Host caches of per-device state.  cudaFuncSetAttribute and device attributes belong to the

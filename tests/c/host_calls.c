@@ -35,7 +35,8 @@ int main(void) {
 
   CHECK(skv_plan_mla(2, 4, kv_indptr, last, 16, 16, SKV_BF16, SKV_SPLIT_NONE, 0, NULL, NULL, plan, 4096, &info) ==
         SKV_OK);
-  CHECK(info.num_work >= 2 && info.q_tile == skv_mla_fold_ratio(16, 4, info.kernel == 13 ? 32 : 16));
+  /* 16 heads x 4 tokens = 64 rows: the 64-row bf16 kernel folds all four tokens into one unit */
+  CHECK(info.num_work >= 2 && info.kernel == 14 && info.q_tile == skv_mla_fold_ratio(16, 4, 64));
 
   /* causal tables: request 0 (L = 37, 1 token) sees everything through the prefix; request 1
    * (L = 16, 2 tokens) has a 15-token prefix and its second token adds token 15 (page 4, slot 15) */

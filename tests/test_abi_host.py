@@ -361,7 +361,9 @@ def test_paged_planner_kernel_choice(hq, hk, q_len, page_size, kernel, q_tile):
 
 
 @pytest.mark.parametrize("H,q_len,kv_dtype,page_size,kernel", [
-    (16, 1, "bf16", 64, 12), (16, 4, "bf16", 64, 13), (128, 1, "bf16", 64, 13),
+    (16, 1, "bf16", 64, 12), (16, 4, "bf16", 64, 14), (128, 1, "bf16", 64, 14), (128, 4, "bf16", 64, 14),
+    (16, 2, "bf16", 64, 13), (96, 1, "bf16", 64, 13),   # 32 rows; 96 heads are no multiple of 64
+    (16, 4, "bf16", 1, 13),                              # page size 1 takes at most 32 rows
     (16, 1, "e4m3", 64, 12), (128, 4, "e4m3", 64, 13),   # native fp8 tensor-core kernel
     (16, 1, "bf16", 1, 12),                              # page size 1: row gather on the tensor cores
     (16, 1, "e4m3", 1, 11),                              # e4m3 with page size 1: CUDA-core kernel
@@ -372,8 +374,11 @@ def test_mla_planner_kernel_choice(H, q_len, kv_dtype, page_size, kernel):
     last = np.array([page_size, 1, max(1, page_size // 2)], np.int32)
     plan = skv.plan_mla(q_len, kv_indptr, last, page_size, H, "balanced", 148, kv_dtype=kv_dtype)
     assert plan.info.kernel == kernel
-    rows = {12: 16, 13: 32}.get(kernel, 128)
+    rows = {12: 16, 13: 32, 14: 64}.get(kernel, 128)
     assert plan.info.q_tile == (skv.mla_fold_ratio(H, q_len, rows) if H <= rows else 1)
+    if kernel == 14:   # a group of (query tiles x head groups) CTAs per KV slice
+        group = (q_len // plan.info.q_tile) * (H // 64 if H > 64 else 1)
+        assert plan.info.num_ctas % group == 0 and 1 <= plan.info.num_ctas // group <= 148 // group
 
 
 @pytest.mark.parametrize("H,q_len", [(16, 1), (16, 4), (128, 1), (128, 4)])
@@ -386,21 +391,31 @@ def test_mla_flat_plan_balances_tiles_and_pieces(H, q_len):
     c = mla_decode_case(H, q_len, "bf16")
     plan = skv.plan_mla(q_len, c.kv_indptr, c.kv_last_page_len, 64, H, "balanced", 148, kv_dtype="bf16")
     info = plan.info
-    assert info.kernel in (12, 13) and info.num_ctas == 148
-    rows = {12: 16, 13: 32}[info.kernel]
+    assert info.kernel in (12, 13, 14)
+    rows = {12: 16, 13: 32, 14: 64}[info.kernel]
     hg = H // rows if H > rows else 1
     qt = -(-q_len // info.q_tile) * hg                       # query units per piece
+    if info.kernel == 14:
+        # grouped: each of the `qt` CTAs of a slice's group runs one query unit of every piece, so a
+        # slice costs its tiles once per CTA; the items stand for query tile 0
+        group, hg, qt = qt, 1, 1
+        assert info.num_ctas == 148 // group * group
+        q_len_eff = info.q_tile
+    else:
+        group, q_len_eff = 1, q_len
+        assert info.num_ctas == 148
+    slices = info.num_ctas // group
     w, _ = _items(plan)
-    cta = plan.words[info.cta_offset: info.cta_offset + info.num_ctas + 1]
+    cta = plan.words[info.cta_offset: info.cta_offset + slices + 1]
     L = c.kv_lengths()
     n = np.diff(c.kv_indptr)
     cost = []
-    for i in range(info.num_ctas):
+    for i in range(slices):
         items = w[cta[i]:cta[i + 1]]
         # work items of one request piece differ only by query tile: count pieces once
         pieces = {(int(r), int(a), int(b)) for r, _, _, a, b, *_ in items}
         tiles = sum(-(-(min(b * 64, L[r]) - a * 64) // 64) for r, a, b in pieces)
-        cost.append(hg * tiles * -(-q_len // info.q_tile) + 4 * qt * len(pieces))
+        cost.append(hg * tiles * -(-q_len_eff // info.q_tile) + 4 * qt * len(pieces))
     cost = np.array(cost)
     assert cost.max() <= cost.mean() + 8 * qt + 8 * hg, (cost.max(), cost.mean())
     for r in range(c.batch):

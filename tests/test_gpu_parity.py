@@ -198,7 +198,7 @@ def test_mla_reduced(H, q_len, kv_dtype):
     c = mla_decode_case(H, q_len, kv_dtype, batch=3, len_range=(100, 900), poison=True)
     o, lse, ex = _run_mla(c, "fixed", 3)
     info = ex["plan"].info
-    rows = {12: 16, 13: 32}.get(info.kernel, 128)   # rows per tile of the kernel the planner chose
+    rows = {12: 16, 13: 32, 14: 64}.get(info.kernel, 128)   # rows per tile of the kernel the planner chose
     assert info.q_tile == (skv.mla_fold_ratio(H, q_len, rows) if H <= rows else 1)
     O, LSE = _oracle_mla(c)
     _cmp(_np(o), _np(lse), O, LSE, O_TOL, where=f"mla {H} {q_len} {kv_dtype}")
@@ -237,6 +237,22 @@ def test_mla_tensor_core_page_sizes_and_edges(kv_dtype, page_size, policy, param
     assert ex["plan"].info.kernel == 12
     O, LSE = _oracle_mla(c)
     _cmp(_np(o), _np(lse), O, LSE, O_TOL, where=f"mla edges {kv_dtype} P{page_size} {policy}")
+
+
+@pytest.mark.parametrize("H,q_len", [(64, 3), (128, 2), (32, 4)])
+@pytest.mark.parametrize("page_size", [16, 128])
+@pytest.mark.parametrize("policy,param", [("none", 0), ("balanced", 148), ("fixed", 2)])
+def test_mla_64_row_groups(H, q_len, page_size, policy, param):
+    """The 64-row kernel with CTA groups: every (query tile, head group) of a KV slice on its own
+    co-resident CTA (groups of 3, 4 and 2 CTAs here), ragged lengths around tile and page
+    boundaries, an empty request, poisoned unused pages and tails, split or whole KV."""
+    c = mla_decode_case(H, q_len, "bf16", batch=5, len_range=(1, 900), page_size=page_size, poison=True, seed=13)
+    c = _empty_request(c, 1)
+    o, lse, ex = _run_mla(c, policy, param)
+    info = ex["plan"].info
+    assert info.kernel == 14 and info.q_tile == (skv.mla_fold_ratio(H, q_len, 64) if H <= 64 else 1)
+    O, LSE = _oracle_mla(c)
+    _cmp(_np(o), _np(lse), O, LSE, O_TOL, where=f"mla 64-row H{H} q{q_len} P{page_size} {policy}")
 
 
 @pytest.mark.parametrize("H,q_len", [(16, 1), (16, 2), (128, 1)])

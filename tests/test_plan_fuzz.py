@@ -19,9 +19,31 @@ def _items(plan):
     return plan.words[: 8 * nw].reshape(-1, 8), plan.words[8 * nw: 8 * nw + 4 * nm].reshape(-1, 4)
 
 
-def _check(plan, qo, n_pages):
+def _grouped(plan, qo, num_heads):
+    """Work items as the CTAs run them.  A plan of the 64-row MLA kernel (kernel 14) lists query tile
+    0 of each piece only: the CTAs of a slice's group take query tile t = 0 .. q_len / q_tile - 1 by
+    shifting the item's rows by t * q_tile and its partial rows by t * q_tile * part_stride (every
+    head group of a tile runs the same rows).  Returns (items, CTAs per slice)."""
+    w, _ = _items(plan)
+    if plan.info.kernel != 14:
+        return w, 1
+    q_len = int(qo[1] - qo[0]) if len(qo) > 1 else 0
+    qt_count = q_len // plan.info.q_tile
+    assert q_len == qt_count * plan.info.q_tile and np.all(np.diff(qo) == q_len)
+    out = []
+    for row in w.tolist():
+        r, qs, qc, pb, pe, prow, pstride, j = row
+        assert qs == qo[r] and qc == plan.info.q_tile   # query tile 0 of the request
+        for t in range(qt_count):
+            out.append([r, qs + t * qc, qc, pb, pe, prow + t * qc * pstride if prow >= 0 else prow, pstride, j])
+    group = qt_count * (num_heads // 64 if num_heads > 64 else 1)
+    return np.array(out, dtype=np.int64).reshape(-1, 8), group
+
+
+def _check(plan, qo, n_pages, num_heads=0):
     info = plan.info
-    w, m = _items(plan)
+    w, group = _grouped(plan, qo, num_heads)
+    _, m = _items(plan)
     B = len(n_pages)
     part_owner = {}
     direct = {}
@@ -53,8 +75,10 @@ def _check(plan, qo, n_pages):
             assert sp[0][1] == 0 and sp[-1][2] == n_pages[r]
             assert all(sp[k][2] == sp[k + 1][1] for k in range(len(sp) - 1))
     if info.num_ctas:
-        cta = plan.words[info.cta_offset: info.cta_offset + info.num_ctas + 1]
+        assert info.num_ctas % group == 0
+        cta = plan.words[info.cta_offset: info.cta_offset + info.num_ctas // group + 1]
         assert cta[0] == 0 and cta[-1] == info.num_work and np.all(np.diff(cta) >= 0)
+        assert info.cta_offset + info.num_ctas // group + 1 == info.plan_words
 
 
 def _random_table(rng, P, max_len, q_max):
@@ -113,7 +137,7 @@ def test_mla_plans(seed):
         n_pages = np.diff(kv_indptr)
         policy, param, sps = _policy(rng, n_pages)
         plan = skv.plan_mla(q_len, kv_indptr, last, P, H, policy, param, sps, kv_dtype=kv_dtype)
-        _check(plan, qo, n_pages)
+        _check(plan, qo, n_pages, H)
 
 
 @pytest.mark.parametrize("seed", range(8))
