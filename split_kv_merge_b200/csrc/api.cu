@@ -440,8 +440,9 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
   // those rows
   const int64_t hq = (int64_t)num_heads * q_len;
   int32_t nr = hq <= 16 ? 16 : 32;
-  if (kv_dtype == SKV_BF16 && hq > 32 && mla_tc_supported(kv_dtype, page_size, num_heads, 64)) nr = 64;
+  if (kv_dtype == SKV_BF16 && hq > 32 && mla_tc64_supported(kv_dtype, page_size, num_heads)) nr = 64;
   const bool tc = kv_dtype == SKV_E4M3 ? mla_tc_fp8_supported(page_size, num_heads, nr)
+                  : nr == 64           ? true
                                        : mla_tc_supported(kv_dtype, page_size, num_heads, nr);
   PersistOpts po;
   po.page_size = page_size;
@@ -614,12 +615,14 @@ skv_status skv_mla_decode_partial(const skv_mla_params* p, const int32_t* plan_d
     return SKV_ERR_INVALID;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const WorkItem* work = reinterpret_cast<const WorkItem*>(plan_d);
-  const int rows = info->kernel == KERNEL_MLA_TC16 ? 16 : info->kernel == KERNEL_MLA_TC32 ? 32 : 64;
-  int e = !tc                         ? launch_mla_simt(*p, work, info->num_work, info->q_tile, s)
-          : p->kv_dtype == SKV_E4M3 ? launch_mla_tc_fp8(*p, work, plan_d + info->cta_offset, info->num_ctas,
-                                                        info->q_tile, rows, s)
-                                      : launch_mla_tc(*p, work, plan_d + info->cta_offset, info->num_ctas,
-                                                      info->q_tile, rows, s);
+  const int rows = info->kernel == KERNEL_MLA_TC16 ? 16 : 32;
+  int e = !tc                                  ? launch_mla_simt(*p, work, info->num_work, info->q_tile, s)
+          : info->kernel == KERNEL_MLA_TC64    ? launch_mla_tc64(*p, work, plan_d + info->cta_offset, info->num_ctas,
+                                                                 info->q_tile, s)
+          : p->kv_dtype == SKV_E4M3            ? launch_mla_tc_fp8(*p, work, plan_d + info->cta_offset, info->num_ctas,
+                                                                   info->q_tile, rows, s)
+                                               : launch_mla_tc(*p, work, plan_d + info->cta_offset, info->num_ctas,
+                                                               info->q_tile, rows, s);
   return cuda_status(e);
 }
 

@@ -52,20 +52,12 @@ constexpr float kRaise = 8.f;
 
 template <int NR>
 struct MlaCfg {
-  // 64 rows: the query copy doubles, so the ring keeps two whole tiles of ckv (8 slots) with one
-  // kpe slot and one P buffer, and QK is split over two issuers (two partial accumulators) so S
-  // and O^T fit the 512 TMEM columns
-  static constexpr int kQParts = NR == 64 ? 2 : kIssuers;  // QK partial accumulators
   static constexpr int kCStages = NR == 16 ? 9 : 8;
-  static constexpr int kKStages = NR == 64 ? 1 : 4;
+  static constexpr int kKStages = 4;
   static constexpr int kQRegion = NR * 128;             // one 64-column region of Q
   static constexpr int kQBytes = 9 * kQRegion;          // q_nope (8 regions) + q_pe
   static constexpr int kPBytes = kTile * 128;           // P^T MN-major: one 128-byte row per token
-  static constexpr int kPBufs = NR == 64 ? 1 : 3;       // P(t) reuses the buffer of PV(t - kPBufs)
-  // 64 rows: each CTA of a group of co-resident CTAs takes one (query tile, head group) of every
-  // work item of its KV slice (launched without the row-gather warps)
-  static constexpr bool kGrouped = NR == 64;
-  static constexpr int kBlockThreads = NR == 64 ? (5 + kIssuers) * 32 : kThreads;
+  static constexpr int kPBufs = 3;                      // P(t) reuses the buffer of PV(t - 3)
   static constexpr int cring = 0;
   static constexpr int kring = cring + kCStages * kCSlot;
   static constexpr int q = kring + kKStages * kKSlot;
@@ -79,8 +71,8 @@ struct MlaCfg {
   static constexpr int nbars = 2 * kCStages + 2 * kKStages + 14;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
-  // S: 2 buffers x kQParts partial accumulators x NR (M=64 lanes); O^T: 4 blocks x NR
-  static constexpr int s_cols = 2 * kQParts * NR;
+  // S: 2 buffers x 4 partial accumulators (one per issuer) x NR (M=64 lanes); O^T: 4 blocks x NR
+  static constexpr int s_cols = 2 * kIssuers * NR;
   static constexpr int tmem_cols = s_cols + 4 * NR <= 256 ? 256 : 512;
 };
 
@@ -91,7 +83,6 @@ struct MArgs {
   const int32_t* cta_indptr;
   int num_pages, page_size, heads, hc, hg, q_tile;
   int gather;  // page size 1: token rows fetched with 16-byte cp.async by four warps
-  int group;   // 64-row kernel: CTAs per KV slice, one (query tile, head group) each
   const uint8_t* ckv_rows;  // page size 1: row id i starts at ckv_rows + i * ckv_row_bytes
   const uint8_t* kpe_rows;
   int64_t ckv_row_bytes, kpe_row_bytes;
@@ -108,16 +99,15 @@ struct MUnit {
   int t0, t1, ntiles;
 };
 
-// qt: this CTA's query tile of a grouped plan (whose items stand for query tile 0), else 0
-__device__ __forceinline__ MUnit load_munit(const MArgs& a, const WorkItem* work, int u, int qt = 0) {
+__device__ __forceinline__ MUnit load_munit(const MArgs& a, const WorkItem* work, int u) {
   MUnit x;
   const WorkItem w = work[u];
   x.r = w.r;
-  x.q_start = w.q_start + qt * a.q_tile;
+  x.q_start = w.q_start;
   x.q_count = w.q_count;
   x.page_begin = w.page_begin;
   x.page_end = w.page_end;
-  x.part_row = w.part_row < 0 ? w.part_row : w.part_row + qt * a.q_tile * w.part_stride;
+  x.part_row = w.part_row;
   x.part_stride = w.part_stride;
   const int L = request_len(a.kv_indptr, a.last, w.r, a.page_size);
   x.t0 = w.page_begin * a.page_size;
@@ -148,12 +138,12 @@ __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint3
 }
 
 template <int NR, typename OutT>
-__global__ void __launch_bounds__(MlaCfg<NR>::kBlockThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant__ CUtensorMap kpe_map,
               const __grid_constant__ CUtensorMap qn_map, const __grid_constant__ CUtensorMap qp_map, MArgs a,
               const WorkItem* __restrict__ work) {
   using C = MlaCfg<NR>;
-  constexpr int NC = C::kCStages, NK = C::kKStages, NQ = C::kQParts;
+  constexpr int NC = C::kCStages, NK = C::kKStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = tc::smem_u32(smem);
@@ -184,12 +174,12 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     }
     for (int s = 0; s < NK; ++s) {
       tc::mbar_init(kfull_bar(s), a.gather ? kGatherWarps * 32 : 1);
-      tc::mbar_init(kempty_bar(s), NQ);
+      tc::mbar_init(kempty_bar(s), kIssuers);
     }
     tc::mbar_init(qfull_bar(), 1);
-    tc::mbar_init(qempty_bar(), NQ);
+    tc::mbar_init(qempty_bar(), kIssuers);
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(sfull_bar(b), NQ);
+      tc::mbar_init(sfull_bar(b), kIssuers);
       tc::mbar_init(sempty_bar(b), 4);
     }
     for (int b = 0; b < C::kPBufs; ++b) tc::mbar_init(pfull_bar(b), 4);
@@ -217,12 +207,7 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
   const uint32_t tmem = *tmem_holder;
   const uint32_t tm_s = tmem, tm_o = tmem + C::s_cols;
 
-  // grouped plans: CTA c runs slice c / group, query tile and head group from c % group
-  const int slice = C::kGrouped ? (int)blockIdx.x / a.group : (int)blockIdx.x;
-  const int gsel = C::kGrouped ? (int)blockIdx.x % a.group : 0;
-  const int my_qt = gsel / a.hg;
-  const int hg_lo = C::kGrouped ? gsel % a.hg : 0, hg_hi = C::kGrouped ? hg_lo + 1 : a.hg;
-  const int u_begin = a.cta_indptr[slice], u_end = a.cta_indptr[slice + 1];
+  const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
   const int P = a.page_size;
   const int box_rows = min(P, kTile);
 
@@ -231,11 +216,11 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
     int gc = 0, gk = 0, n_unit = 0;
     bool ok = true;
     for (int u = u_begin; u < u_end && ok; ++u) {
-      const MUnit x = load_munit(a, work, u, my_qt);
+      const MUnit x = load_munit(a, work, u);
       if (x.ntiles == 0) continue;
       const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
       const int npages = x.page_end - x.page_begin;
-      for (int hgi = hg_lo; hgi < hg_hi && ok; ++hgi) {
+      for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
         if (warp == 4 && lane == 0) {  // Q of this unit once the previous unit's last S MMA is done
           if (n_unit >= 1) ok = tc::mbar_wait_sleep(qempty_bar(), (n_unit + 1) & 1, abort_flag, a.status);
           if (ok) {
@@ -360,15 +345,15 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             win = pi0;
             pid = (win + lane < npages) ? __ldg(ids + win + lane) : 0;
           }
-          // lane 0 claims the tile's four ckv slots (waits + expected bytes) and eight lanes issue their
-          // TMA boxes at once (a single issuing thread serialises them); then the kpe slot.  The ckv
-          // blocks go first: their slots free as earlier tiles' PV finishes, the kpe slot only once
-          // the previous tile's QK is done, and the blocks must not wait behind it.
+          // lane 0 claims the tile's kpe slot and its four ckv slots (waits + expected bytes); then
+          // nine lanes issue the nine TMA boxes at once (a single issuing thread serialises them)
           const int sk = gk % NK;
           int sc[kBlocks];
 #pragma unroll
           for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
           if (lane == 0) {
+            if (gk >= NK) ok = tc::mbar_wait_sleep(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
+            if (ok) tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(npg * box_rows * 128));
             for (int b = 0; b < kBlocks && ok; ++b) {
               const int g = gc + b;
               if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
@@ -381,26 +366,16 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
             if (lane == 0 && (unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
             const uint32_t row_off = (uint32_t)(i * box_rows * 128);
-            if (lane < 8) {
+            if (lane == 8) {
+              tma3(sbase + C::kring + sk * kKSlot + row_off, &kpe_map, kfull_bar(sk), 0, slot0, page);
+            } else if (lane < 8) {
               const int b = lane >> 1, hf = lane & 1;
               tma3(sbase + C::cring + sc[b] * kCSlot + hf * kHalf + row_off, &ckv_map, cfull_bar(sc[b]),
                    b * 128 + hf * 64, slot0, page);
             }
           }
-          gc += kBlocks;
-          if (lane == 0) {
-            if (gk >= NK) ok = tc::mbar_wait_sleep(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
-            if (ok) tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(npg * box_rows * 128));
-          }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-          for (int i = 0; i < npg; ++i) {
-            const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
-            if (lane == 8)
-              tma3(sbase + C::kring + sk * kKSlot + (uint32_t)(i * box_rows * 128), &kpe_map, kfull_bar(sk), 0, slot0,
-                   page);
-          }
           ++gk;
+          gc += kBlocks;
         }
         ++n_unit;
       }
@@ -431,15 +406,14 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
       bool ok = true;
       const uint32_t qs = sbase + C::q;
       for (int u = u_begin; u < u_end && ok; ++u) {
-        const MUnit x = load_munit(a, work, u, my_qt);
+        const MUnit x = load_munit(a, work, u);
         if (x.ntiles == 0) continue;
-        for (int hgi = hg_lo; hgi < hg_hi && ok; ++hgi) {
+        for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
           const int T = x.ntiles;
           ok = tc::mbar_wait_sleep(qfull_bar(), n_unit & 1, abort_flag, a.status);
           if (ok) tc::tc_fence_after();
-          // issue whichever is ready: PV(pv) (frees the tile's ckv blocks: first) or QK(qk); issuers
-          // beyond the NQ QK parts only run PV
-          int qk = w < NQ ? 0 : T, pv = 0;
+          // issue whichever is ready: PV(pv) (frees the tile's ckv blocks: first) or QK(qk)
+          int qk = 0, pv = 0;
           tc::PollClock clk;
           while (ok && pv < T) {
             bool did = false;
@@ -464,38 +438,23 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
                 did = true;
               }
             }
-            if (!did && qk < T) {  // ---- QK(qk), part w: quarters w * QPW .. (rope k-step + ckv block each)
-              constexpr int QPW = kBlocks / NQ;
+            if (!did && qk < T) {  // ---- QK(qk), quarter w
               const int tt = n_tile + qk, sb = tt & 1, gk = g + qk, sk = gk % NK;
-              bool ready = (tt < 2 || tc::mbar_test_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1)) &&
-                           tc::mbar_test_wait(kfull_bar(sk), (gk / NK) & 1);
-#pragma unroll
-              for (int qq = 0; qq < QPW; ++qq) {
-                const int cb = kBlocks * (g + qk) + w * QPW + qq;
-                ready = ready && tc::mbar_test_wait(cfull_bar(cb % NC), (cb / NC) & 1);
-              }
-              if (ready) {
+              const int cb = kBlocks * (g + qk) + w, st = cb % NC;
+              if ((tt < 2 || tc::mbar_test_wait(sempty_bar(sb), ((tt >> 1) + 1) & 1)) &&
+                  tc::mbar_test_wait(kfull_bar(sk), (gk / NK) & 1) && tc::mbar_test_wait(cfull_bar(st), (cb / NC) & 1)) {
                 tc::tc_fence_after();
-                const uint32_t d = tm_s + (sb * NQ + w) * NR;
-#pragma unroll
-                for (int qq = 0; qq < QPW; ++qq) {  // rope k-steps first: the kpe slot frees early
-                  const int qw = w * QPW + qq;
-                  tc::mma_bf16(d, tc::sdesc_sw128(sbase + C::kring + sk * kKSlot + qw * 32, 16, 1024),
-                               tc::sdesc_sw128(qs + 8 * C::kQRegion + qw * 32, 16, 1024), idesc_s,
-                               qq > 0 ? 1u : 0u);
-                }
+                const uint32_t d = tm_s + (sb * kIssuers + w) * NR;
+                tc::mma_bf16(d, tc::sdesc_sw128(sbase + C::kring + sk * kKSlot + w * 32, 16, 1024),
+                             tc::sdesc_sw128(qs + 8 * C::kQRegion + w * 32, 16, 1024), idesc_s, 0u);
                 tc::mma_commit(kempty_bar(sk));
+                const uint32_t cbase = sbase + C::cring + st * kCSlot;
 #pragma unroll
-                for (int qq = 0; qq < QPW; ++qq) {  // then ckv block qw of every quarter
-                  const int qw = w * QPW + qq;
-                  const uint32_t cbase = sbase + C::cring + ((kBlocks * (g + qk) + qw) % NC) * kCSlot;
-#pragma unroll
-                  for (int k = 0; k < 8; ++k) {
-                    const uint64_t ad = tc::sdesc_sw128(cbase + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
-                    const uint64_t bd =
-                        tc::sdesc_sw128(qs + (2 * qw + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
-                    tc::mma_bf16(d, ad, bd, idesc_s, 1u);
-                  }
+                for (int k = 0; k < 8; ++k) {
+                  const uint64_t ad = tc::sdesc_sw128(cbase + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
+                  const uint64_t bd =
+                      tc::sdesc_sw128(qs + (2 * w + (k >> 2)) * C::kQRegion + (k & 3) * 32, 16, 1024);
+                  tc::mma_bf16(d, ad, bd, idesc_s, 1u);
                 }
                 tc::mma_commit(sfull_bar(sb));
                 if (qk + 1 == T) tc::mma_commit(qempty_bar());  // Q free after the unit's last QK
@@ -530,9 +489,9 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
       tc::tc_fence_after();
     };
     for (int u = u_begin; u < u_end && ok; ++u) {
-      const MUnit x = load_munit(a, work, u, my_qt);
+      const MUnit x = load_munit(a, work, u);
       const int rows = x.q_count * a.hc;
-      for (int hgi = hg_lo; hgi < hg_hi && ok; ++hgi) {
+      for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
         const int h0 = hgi * a.hc;
         if (x.ntiles == 0) {  // no tokens: O = 0, LSE = -inf
           for (int n = 0; n < rows; ++n) {
@@ -571,12 +530,12 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
           tc::tc_fence_after();
           float s[NR];
 #pragma unroll
-          for (int w = 0; w < NQ; ++w) {  // sum of the partial accumulators
+          for (int w = 0; w < kIssuers; ++w) {  // sum of the four partial accumulators
             float v[NR];
 #pragma unroll
             for (int c = 0; c < NR; c += 16) {
               float v16[16];
-              tc::tmem_ld_x16(tm_s + lane_base + (sb * NQ + w) * NR + c, v16);
+              tc::tmem_ld_x16(tm_s + lane_base + (sb * kIssuers + w) * NR + c, v16);
 #pragma unroll
               for (int i = 0; i < 16; ++i) v[c + i] = v16[i];
             }
@@ -710,68 +669,35 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             lse_s[n] = lt > 0.f ? (m_s[n] + log2f(lt)) * kLn2 : -INFINITY;
           }
         }
-        if constexpr (NR <= 32) {
-          float ov[kBlocks][NR];
+        float ov[kBlocks][NR];
 #pragma unroll
-          for (int b = 0; b < kBlocks; ++b)
+        for (int b = 0; b < kBlocks; ++b)
 #pragma unroll
-            for (int c = 0; c < NR; c += 16) {
-              float v16[16];
-              tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, v16);
-              tc::tmem_wait_ld();
+          for (int c = 0; c < NR; c += 16) {
+            float v16[16];
+            tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, v16);
+            tc::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 16; ++i) ov[b][c + i] = v16[i];
-            }
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(ofree_bar());
-          tc::named_bar_sync(1, 128);
-#pragma unroll
-          for (int n = 0; n < NR; ++n) {
-            if (n >= rows) break;
-            const int qi = n / a.hc, h = h0 + n % a.hc;
-            const float iv = inv_s[n];
-            if (x.part_row < 0) {
-              OutT* dst = reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.heads + h) * 512 + tid;
-#pragma unroll
-              for (int b = 0; b < kBlocks; ++b) store_out(dst + b * 128, ov[b][n] * iv);
-            } else {
-              float* dst =
-                  a.o_part + (((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h) * 512 + tid;
-#pragma unroll
-              for (int b = 0; b < kBlocks; ++b) dst[b * 128] = ov[b][n] * iv;
-            }
+            for (int i = 0; i < 16; ++i) ov[b][c + i] = v16[i];
           }
-        } else {
-          // 64 rows: O^T read and stored 16 columns at a time (every thread owns lane `tid` of the
-          // four blocks: head dim b * 128 + tid of each row), then its buffer is released
-          tc::named_bar_sync(1, 128);  // inv_s from thread 0
-#pragma unroll 1
-          for (int b = 0; b < kBlocks; ++b) {
-#pragma unroll 1
-            for (int c = 0; c < NR; c += 16) {
-              float v16[16];
-              tc::tmem_ld_x16(tm_o + lane_base + b * NR + c, v16);
-              tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(ofree_bar());
+        tc::named_bar_sync(1, 128);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const int n = c + i;
-                if (n >= rows) break;
-                const int qi = n / a.hc, h = h0 + n % a.hc;
-                const float val = v16[i] * inv_s[n];
-                if (x.part_row < 0)
-                  store_out(reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.heads + h) * 512 +
-                                b * 128 + tid,
-                            val);
-                else
-                  a.o_part[(((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h) * 512 + b * 128 +
-                           tid] = val;
-              }
-            }
+        for (int n = 0; n < NR; ++n) {
+          if (n >= rows) break;
+          const int qi = n / a.hc, h = h0 + n % a.hc;
+          const float iv = inv_s[n];
+          if (x.part_row < 0) {
+            OutT* dst = reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.heads + h) * 512 + tid;
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) store_out(dst + b * 128, ov[b][n] * iv);
+          } else {
+            float* dst = a.o_part + (((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.heads + h) * 512 + tid;
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) dst[b * 128] = ov[b][n] * iv;
           }
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(ofree_bar());
         }
         if (tid < rows) {
           const int qi = tid / a.hc, h = h0 + tid % a.hc;
@@ -823,9 +749,8 @@ int launch_m(const CUtensorMap* maps, const MArgs& a, int num_ctas, const WorkIt
   const int smem = MlaCfg<NR>::total + 1024;
   static DeviceSmemAttr attr;  // per device: the attribute belongs to the current device
   if (const int e = attr.ensure(reinterpret_cast<const void*>(mla_tc_kernel<NR, OutT>), smem)) return e;
-  // the three extra gather warps exist only in row-gather mode (never with 64 rows)
+  // the three extra gather warps exist only in row-gather mode
   const int threads = a.gather ? kThreads : kThreads - (kGatherWarps - 1) * 32;
-  if (threads > MlaCfg<NR>::kBlockThreads) return (int)cudaErrorInvalidValue;
   mla_tc_kernel<NR, OutT><<<num_ctas, threads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], a, work);
   return (int)cudaGetLastError();
 }
@@ -833,10 +758,9 @@ int launch_m(const CUtensorMap* maps, const MArgs& a, int num_ctas, const WorkIt
 }  // namespace
 
 bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit) {
-  const bool paged = page_size >= 8 && (page_size <= kTile ? kTile % page_size == 0 : page_size % kTile == 0);
-  // page size 1 (row gather) runs with 16 or 32 rows; 64 rows only on paged caches
-  const bool page_ok = rows_per_unit == 64 ? paged : (page_size == 1 || paged);
-  return kv_dtype == SKV_BF16 && page_ok && (rows_per_unit == 16 || rows_per_unit == 32 || rows_per_unit == 64) &&
+  const bool page_ok = page_size == 1 ||
+                       (page_size >= 8 && (page_size <= kTile ? kTile % page_size == 0 : page_size % kTile == 0));
+  return kv_dtype == SKV_BF16 && page_ok && (rows_per_unit == 16 || rows_per_unit == 32) &&
          (num_heads <= rows_per_unit || num_heads % rows_per_unit == 0);
 }
 
@@ -893,9 +817,6 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
   a.hg = p.num_heads / hc;
   a.q_tile = q_tile;
   a.gather = gather ? 1 : 0;
-  // 64 rows: a group of (query tiles x head groups) CTAs per KV slice, grid = slices x group
-  a.group = NR == 64 ? (p.q_len / q_tile) * a.hg : 1;
-  if (NR == 64 && (p.q_len % q_tile != 0 || num_ctas % a.group != 0)) return (int)cudaErrorInvalidValue;
   a.ckv_rows = static_cast<const uint8_t*>(p.ckv);
   a.kpe_rows = static_cast<const uint8_t*>(p.kpe);
   a.ckv_row_bytes = p.ckv_stride[0] * 2;
@@ -909,8 +830,6 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
   const bool bf = p.o_dtype == SKV_BF16;
   if (NR == 16)
     return bf ? launch_m<16, __nv_bfloat16>(maps, a, num_ctas, work, s) : launch_m<16, float>(maps, a, num_ctas, work, s);
-  if (NR == 64)
-    return bf ? launch_m<64, __nv_bfloat16>(maps, a, num_ctas, work, s) : launch_m<64, float>(maps, a, num_ctas, work, s);
   return bf ? launch_m<32, __nv_bfloat16>(maps, a, num_ctas, work, s) : launch_m<32, float>(maps, a, num_ctas, work, s);
 }
 

@@ -108,6 +108,9 @@ int launch_mla_simt(const skv_mla_params& p, const WorkItem* work, int num_work,
                     cudaStream_t s);
 bool mla_tc_supported(int kv_dtype, int page_size, int num_heads, int rows_per_unit);
 int mla_tc_tile_tokens();
+bool mla_tc64_supported(int kv_dtype, int page_size, int num_heads);
+int launch_mla_tc64(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
+                    int q_tile, cudaStream_t s);
 int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* cta_indptr, int num_ctas,
                   int q_tile, int rows_per_unit, cudaStream_t s);
 bool mla_tc_fp8_supported(int page_size, int num_heads, int rows_per_unit);
