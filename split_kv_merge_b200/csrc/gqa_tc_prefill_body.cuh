@@ -180,45 +180,54 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& kmap, const CUte
 
   if (warp == 4) {
     // ======================================================================= TMA producer
+    // The whole warp streams the tiles: lanes hold the ids of the next 32 pages of the item (one
+    // per lane), lane 0 claims the stage, and lane i issues the K and V boxes of page i of the tile
+    // (a 128-key tile of 16-token pages is eight pages: their boxes go out at once instead of one
+    // after another behind eight dependent page-id loads).
+    bool ok = true;
+    int issued = 0;
     if (lane == 0) {
-      bool ok = true;
-      int issued = 0;
       tc::prefetch_tmap(&kmap);
       tc::prefetch_tmap(&vmap);
       tc::mbar_arrive_expect_tx(qfull_bar(), (uint32_t)(kRows * kD * 2));
       for (int rgn = 0; rgn < 2; ++rgn)
         tc::tma_load_3d(sbase + Smem::q + rgn * kRegion, &qmap, qfull_bar(), rgn * 64, kh * a.g, w.q_start);
-      const int* ids = a.kv_indices + a.kv_indptr[w.r] + w.page_begin;
-      const int npages = w.page_end - w.page_begin;
-      const int P = a.page_size, box_rows = min(P, kTile);
-      const uint64_t pol = tc::policy_evict_first();
-      for (int t = 0; t < T && ok; ++t) {
-        const int st = t % kStages;
-        if (t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
-        if (!ok) break;
-        const int pi0 = (t * kTile) / P;
-        const int npg = P >= kTile ? 1 : min(kTile / P, npages - pi0);
-        const int slot0 = P >= kTile ? (t * kTile) % P : 0;
-        tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(2 * 2 * npg * box_rows * 128));
-        const uint32_t kdst = sbase + Smem::kv + st * kStageBytes;
-        for (int i = 0; i < npg; ++i) {
-          const int page = __ldg(ids + pi0 + i);
-          if ((unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
-          const uint32_t row_off = (uint32_t)(i * box_rows * 128);
-          for (int rgn = 0; rgn < 2; ++rgn) {
-            tc::tma_load_4d(kdst + rgn * kRegion + row_off, &kmap, full_bar(st), rgn * 64, kh, slot0, page, pol);
-            tc::tma_load_4d(kdst + kKBytes + rgn * kRegion + row_off, &vmap, full_bar(st), rgn * 64, kh, slot0, page,
-                            pol);
-          }
-        }
-        issued = t + 1;
+    }
+    const int* ids = a.kv_indices + a.kv_indptr[w.r] + w.page_begin;
+    const int npages = w.page_end - w.page_begin;
+    const int P = a.page_size, box_rows = min(P, kTile);
+    const uint64_t pol = tc::policy_evict_first();
+    int win = -1000000, pid = 0;  // lanes hold the ids of pages [win, win + 32) of the item
+    for (int t = 0; t < T && ok; ++t) {
+      const int st = t % kStages;
+      if (lane == 0 && t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      const int pi0 = (t * kTile) / P;
+      const int npg = P >= kTile ? 1 : min(kTile / P, npages - pi0);
+      const int slot0 = P >= kTile ? (t * kTile) % P : 0;
+      if (pi0 < win || pi0 + npg > win + 32) {
+        win = pi0;
+        pid = (win + lane < npages) ? __ldg(ids + win + lane) : 0;
       }
-      if (!ok) {  // the copies of the last tile in each stage may still be landing: wait (bounded)
-        for (int t = max(0, issued - kStages); t < issued; ++t) {
-          const uint64_t t_start = tc::globaltimer_ns();
-          while (!tc::mbar_try_wait(full_bar(t % kStages), (t / kStages) & 1) &&
-                 tc::globaltimer_ns() - t_start < 20000000ull) {
-          }
+      const int page = __shfl_sync(0xffffffffu, pid, (pi0 - win + lane) & 31);
+      if (lane == 0) tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(2 * 2 * npg * box_rows * 128));
+      __syncwarp();
+      if (lane < npg) {
+        if ((unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
+        const uint32_t kdst = sbase + Smem::kv + st * kStageBytes + (uint32_t)(lane * box_rows * 128);
+        for (int rgn = 0; rgn < 2; ++rgn) {
+          tc::tma_load_4d(kdst + rgn * kRegion, &kmap, full_bar(st), rgn * 64, kh, slot0, page, pol);
+          tc::tma_load_4d(kdst + kKBytes + rgn * kRegion, &vmap, full_bar(st), rgn * 64, kh, slot0, page, pol);
+        }
+      }
+      issued = t + 1;
+    }
+    if (!ok && lane == 0) {  // the copies of the last tile in each stage may still be landing: wait (bounded)
+      for (int t = max(0, issued - kStages); t < issued; ++t) {
+        const uint64_t t_start = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(full_bar(t % kStages), (t / kStages) & 1) &&
+               tc::globaltimer_ns() - t_start < 20000000ull) {
         }
       }
     }

@@ -31,9 +31,10 @@
 // log2 units here; O^T rescaled in TMEM by the four softmax warps on a raise).  Masked rows
 // get s = -inf by selection and their V rows are zeroed before the PV that reads them.
 //
-// Roles: warp 4 TMA producer (query staging copy + the K/V ring), warp 5 TMEM allocation + MMA
-// issue, warps 0-3 query split (at the start of each work item), softmax and epilogue.  All waits
-// are bounded (SKV_DEV_TIMEOUT); the roles leave together and TMEM is always released.
+// Roles: warp 4 TMA producer (query staging copy + the K/V ring), warp 5 TMEM allocation + QK
+// issue, warp 6 PV issue, warps 0-3 query split (at the start of each work item), softmax and
+// epilogue.  All waits are bounded (SKV_DEV_TIMEOUT); the roles leave together and TMEM is
+// always released.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
@@ -58,7 +59,7 @@ constexpr int kQStage = 2 * kQRegion;         // bf16 query copy (TMA)
 constexpr int kQOps = 2 * kN * 128;           // [Q_hi; Q_lo] e4m3, 64 rows x 128 B each
 constexpr int kPairBytes = 16 * 128;          // 16 rows x 128 B (64 bytes of K used)
 constexpr int kPBytes = 4 * kPairBytes;       // 8 KB per buffer
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;               // softmax 0-3, TMA 4, QK 5, PV 6
 constexpr int kTmemCols = 256;                // S0 S1 (64 each), O0 O1 (64 each)
 // The running maximum is raised only when a score passes it by more than 2^4 (log2 units), and
 // every weight is formed as p' = 2^(s - m + 4) <= 2^8 (e4m3 holds up to 448): the shift moves the
@@ -315,40 +316,19 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       }
     }
   } else if (warp == 5) {
-    // ======================================================================= MMA issuer
+    // ======================================================================= QK issuer
+    // S^T(t) for every tile as soon as its K tile and an S buffer are ready; PV has its own issuer
+    // (warp 6), so a tile's QK never waits behind the previous tile's PV (an MMA streaming from
+    // shared memory holds its issuing thread for tens of cycles).
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_e4m3(128, kN, false);
-      constexpr uint32_t idesc_o = idesc_e4m3(128, 16, true);  // V^T MN-major, P K-major
       int n_tile = 0, n_unit = 0;
       bool ok = true;
       const uint32_t qo = sbase + Smem::qops;
-      auto issue_pv = [&](int t, int j, uint32_t o_cols) -> bool {
-        const int st = t % kStages, pb = t & 1;
-        if (!tc::mbar_wait(pfull_bar(pb), (t >> 1) & 1, abort_flag, a.status)) return false;
-        tc::tc_fence_after();
-        const uint32_t vs = sbase + Smem::kv + st * kStageBytes + kKBytes;
-        const uint32_t ps = sbase + Smem::p + pb * kPBytes;
-#pragma unroll
-        for (int pr = 0; pr < 4; ++pr) {
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {  // k = 0: hi terms, k = 1: lo terms (bytes 32-63 of P)
-            const uint64_t ad = sw128(vs + pr * 32 * 128, 8192, 1024);
-            const uint64_t bd = sw128(ps + pr * kPairBytes + k * 32, 16, 1024);
-            mma_f8(o_cols + 16 * pr, ad, bd, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
-          }
-        }
-        tc::mma_commit(ofull_bar(t & 1));
-        tc::mma_commit(empty_bar(st));
-        return true;
-      };
       for (int u = u_begin; u < u_end && ok; ++u) {
         const WUnit8 x = load_wunit8(a, work, u);
         if (x.ntiles == 0) continue;
-        const int ob = n_unit & 1;
-        const uint32_t o_cols = tm_o + ob * kN;
         ok = tc::mbar_wait(qready_bar(), n_unit & 1, abort_flag, a.status);
-        // this unit's O^T buffer was last read by the finalize of unit n_unit - 2
-        if (ok && n_unit >= 2) ok = tc::mbar_wait(ofree_bar(ob), ((n_unit >> 1) + 1) & 1, abort_flag, a.status);
         if (!ok) break;
         tc::tc_fence_after();
         for (int j = 0; j < x.ntiles && ok; ++j) {
@@ -366,14 +346,49 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
                      idesc_s, (h > 0 || k > 0) ? 1u : 0u);
           tc::mma_commit(sfull_bar(sb));
           if (j == x.ntiles - 1) tc::mma_commit(qempty_bar());  // query terms free once the last S is done
-          if (j >= 1) ok = issue_pv(t - 1, j - 1, o_cols);
         }
-        if (ok) ok = issue_pv(n_tile + x.ntiles - 1, x.ntiles - 1, o_cols);
         n_tile += x.ntiles;
         ++n_unit;
       }
     }
-  } else {
+  } else if (warp == 6) {
+    // ======================================================================= PV issuer
+    // O^T(t) += V(t)^T . [P_hi; P_lo](t)^T once P(t) is written; then the K/V ring slot is free
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_e4m3(128, 16, true);  // V^T MN-major, P K-major
+      int n_tile = 0, n_unit = 0;
+      bool ok = true;
+      for (int u = u_begin; u < u_end && ok; ++u) {
+        const WUnit8 x = load_wunit8(a, work, u);
+        if (x.ntiles == 0) continue;
+        const int ob = n_unit & 1;
+        const uint32_t o_cols = tm_o + ob * kN;
+        // this unit's O^T buffer was last read by the finalize of unit n_unit - 2
+        if (n_unit >= 2) ok = tc::mbar_wait(ofree_bar(ob), ((n_unit >> 1) + 1) & 1, abort_flag, a.status);
+        for (int j = 0; j < x.ntiles && ok; ++j) {
+          const int t = n_tile + j, st = t % kStages, pb = t & 1;
+          ok = tc::mbar_wait(pfull_bar(pb), (t >> 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t vs = sbase + Smem::kv + st * kStageBytes + kKBytes;
+          const uint32_t ps = sbase + Smem::p + pb * kPBytes;
+#pragma unroll
+          for (int pr = 0; pr < 4; ++pr) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {  // k = 0: hi terms, k = 1: lo terms (bytes 32-63 of P)
+              const uint64_t ad = sw128(vs + pr * 32 * 128, 8192, 1024);
+              const uint64_t bd = sw128(ps + pr * kPairBytes + k * 32, 16, 1024);
+              mma_f8(o_cols + 16 * pr, ad, bd, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          tc::mma_commit(ofull_bar(t & 1));
+          tc::mma_commit(empty_bar(st));
+        }
+        n_tile += x.ntiles;
+        ++n_unit;
+      }
+    }
+  } else if (warp < 4) {
     // ======================================================================= split / softmax
     float* alpha_s = reinterpret_cast<float*>(smem + Smem::alpha);
     float* inv_s = reinterpret_cast<float*>(smem + Smem::inv);
