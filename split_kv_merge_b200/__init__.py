@@ -491,5 +491,5 @@ def library_path() -> str:
     return _LIB_PATH
 
 
-from .runner import (CausalMlaDecode, PodAttention, RouteMerge, mla_decode, paged_attention,  # noqa: E402,F401
-                     pod_attention, pod_decode_sms)
+from .runner import (CausalMlaDecode, PagedDecodePipeline, PodAttention, RouteMerge, mla_decode,  # noqa: E402,F401
+                     paged_attention, pod_attention, pod_decode_sms)

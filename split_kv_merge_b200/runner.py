@@ -2,12 +2,13 @@
 launch through the C ABI.  These are the calls a user makes; they add no arithmetic."""
 from __future__ import annotations
 
+import ctypes
 from typing import Optional
 
 import numpy as np
 
-from . import (Plan, causal_tables, mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged,
-               plan_paged_subset, pod_attn_fwd)
+from . import (OK, ERR_WORKSPACE, Plan, PlanInfo, _POLICY, _check, _plan_paged, _ptr_i32, causal_tables,
+               mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged, plan_paged_subset, pod_attn_fwd)
 
 
 def _dev_i32(a, device, non_blocking=False):
@@ -355,3 +356,127 @@ class CausalMlaDecode:
             merge_states(self.o_st.view(2, B * q, H, 512), self.lse_st.view(2, B * q, H), o.view(B * q, H, 512),
                          lse.view(B * q, H), stream=stream)
         return o, lse
+
+
+class PagedDecodePipeline:
+    """Serving-loop helper for repeated paged attention over a device-resident KV cache, with the
+    step's inputs and outputs in host memory.
+
+    ``submit`` takes one step's query (a pinned host bf16 tensor [rows, Hq, D]) and page table
+    (host int arrays), plans it on the host (``skv_plan_paged`` written straight into a pinned
+    plan buffer), copies query, page table and plan to the device on an input stream, runs the
+    attention and merge passes on a compute stream and copies O and LSE back into pinned host
+    buffers on an output stream; it returns a ticket and does not wait.  ``depth`` sets of host and
+    device buffers alternate, so the host planning and the copies of the next steps overlap the
+    kernels of the current one; ``result(ticket)`` waits for that step's output copy and returns
+    views of its pinned O and LSE (valid until the same buffer set is reused, ``depth`` submits
+    later).  Nothing is allocated per step once the buffers have grown to the largest step."""
+
+    def __init__(self, k_cache, v_cache, num_qo_heads: int, *, max_rows: int, max_batch: int, max_page_ids: int,
+                 sm_scale: Optional[float] = None, num_pages: Optional[int] = None, o_dtype=None, policy="balanced",
+                 param: int = 0, depth: int = 2, plan_words: int = 1 << 16):
+        import torch
+        self.torch = torch
+        self.k, self.v = k_cache, v_cache
+        dev = k_cache.device
+        self.dev = dev
+        self.hq, self.hk, self.d, self.P = num_qo_heads, k_cache.shape[2], k_cache.shape[3], k_cache.shape[1]
+        self.sm_scale, self.num_pages = sm_scale, num_pages
+        self.policy = _POLICY[policy] if isinstance(policy, str) else int(policy)
+        self.param = param
+        self.o_dtype = o_dtype or torch.float32
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        pin = dict(pin_memory=True)
+        self.slots = []
+        for _ in range(depth):
+            slot = dict(
+                plan_h=torch.empty(plan_words, dtype=torch.int32, **pin),
+                tab_h=[torch.empty(n, dtype=torch.int32, **pin) for n in (max_batch + 1, max_page_ids, max_batch)],
+                o_h=torch.empty(max_rows, num_qo_heads, self.d, dtype=self.o_dtype, **pin),
+                lse_h=torch.empty(max_rows, num_qo_heads, dtype=torch.float32, **pin),
+                q=torch.empty(max_rows, num_qo_heads, self.d, dtype=torch.bfloat16, device=dev),
+                plan=torch.empty(plan_words, dtype=torch.int32, device=dev),
+                tab=[torch.empty(n, dtype=torch.int32, device=dev) for n in (max_batch + 1, max_page_ids, max_batch)],
+                o=torch.empty(max_rows, num_qo_heads, self.d, dtype=self.o_dtype, device=dev),
+                lse=torch.empty(max_rows, num_qo_heads, dtype=torch.float32, device=dev),
+                o_part=torch.empty(0, device=dev), lse_part=torch.empty(0, device=dev),
+                ev_in=torch.cuda.Event(), ev_run=torch.cuda.Event(), ev_out=torch.cuda.Event(), rows=0, used=False)
+            self.slots.append(slot)
+        self.count = 0
+        self.h2d_bytes = self.d2h_bytes = 0
+
+    def _plan_into(self, slot, qo, ki, la):
+        """skv_plan_paged straight into the slot's pinned plan buffer (grown if too small)."""
+        b = len(ki) - 1
+        info = PlanInfo()
+        while True:
+            buf = slot["plan_h"]
+            code = _plan_paged(b, _ptr_i32(qo), _ptr_i32(ki), _ptr_i32(la), self.P, self.hq, self.hk, self.d,
+                               self.policy, self.param, None, None,
+                               ctypes.cast(ctypes.c_void_p(buf.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
+                               buf.numel(), ctypes.byref(info))
+            if code == OK:
+                return info
+            if code != ERR_WORKSPACE:
+                _check(code, "skv_plan_paged")
+            n = max(info.plan_words, 2 * buf.numel())
+            slot["plan_h"] = self.torch.empty(n, dtype=self.torch.int32, pin_memory=True)
+            slot["plan"] = self.torch.empty(n, dtype=self.torch.int32, device=self.dev)
+
+    def submit(self, q_h, qo_indptr_h, kv_indptr_h, kv_indices_h, kv_last_page_len_h) -> int:
+        torch = self.torch
+        slot = self.slots[self.count % len(self.slots)]
+        if slot["used"]:
+            slot["ev_out"].synchronize()  # the previous step of this buffer set has been read back
+        qo, ki, la = (np.ascontiguousarray(np.asarray(x, dtype=np.int32)) for x in (qo_indptr_h, kv_indptr_h,
+                                                                               kv_last_page_len_h))
+        kx = np.ascontiguousarray(np.asarray(kv_indices_h, dtype=np.int32))
+        rows = q_h.shape[0]
+        if (rows > slot["o_h"].shape[0] or ki.size > slot["tab_h"][0].numel() or kx.size > slot["tab_h"][1].numel()
+                or la.size > slot["tab_h"][2].numel()):
+            raise ValueError("step larger than the pipeline's max_rows / max_batch / max_page_ids")
+        info = self._plan_into(slot, qo, ki, la)
+        nw = max(1, info.plan_words)
+        np_views = [t.numpy() for t in slot["tab_h"]]
+        np_views[0][: ki.size] = ki
+        np_views[1][: kx.size] = kx
+        np_views[2][: la.size] = la
+        n_part = info.num_partial_rows
+        if n_part > slot["o_part"].shape[0]:  # grows to the largest plan seen, then stays
+            slot["o_part"] = torch.empty(n_part, self.hq, self.d, dtype=torch.float32, device=self.dev)
+            slot["lse_part"] = torch.empty(n_part, self.hq, dtype=torch.float32, device=self.dev)
+        with torch.cuda.stream(self.s_in):
+            if slot["used"]:
+                self.s_in.wait_event(slot["ev_run"])  # the device buffers are free again
+            slot["q"][:rows].copy_(q_h, non_blocking=True)
+            for src, dst, n in zip(slot["tab_h"], slot["tab"], (ki.size, kx.size, la.size)):
+                dst[:n].copy_(src[:n], non_blocking=True)
+            slot["plan"][:nw].copy_(slot["plan_h"][:nw], non_blocking=True)
+            slot["ev_in"].record(self.s_in)
+        plan = Plan(slot["plan_h"][:nw].numpy(), info, slot["plan"][:nw])
+        with torch.cuda.stream(self.s_run):
+            self.s_run.wait_event(slot["ev_in"])
+            paged_attn_fwd(slot["q"][:rows], self.k, self.v, slot["tab"][0][: ki.size], slot["tab"][1][: max(1, kx.size)],
+                           slot["tab"][2][: la.size], plan, slot["o"][:rows], slot["lse"][:rows],
+                           slot["o_part"] if n_part else None, slot["lse_part"] if n_part else None, None,
+                           self.sm_scale, self.num_pages, self.s_run)
+            slot["ev_run"].record(self.s_run)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(slot["ev_run"])
+            slot["o_h"][:rows].copy_(slot["o"][:rows], non_blocking=True)
+            slot["lse_h"][:rows].copy_(slot["lse"][:rows], non_blocking=True)
+            slot["ev_out"].record(self.s_out)
+        slot["used"], slot["rows"] = True, rows
+        self.h2d_bytes += q_h.numel() * q_h.element_size() + 4 * (ki.size + kx.size + la.size) + 4 * nw
+        self.d2h_bytes += rows * self.hq * (self.d * slot["o_h"].element_size() + 4)
+        self.count += 1
+        return self.count - 1
+
+    def result(self, ticket: int):
+        """Wait for step ``ticket``'s output copy; returns (O, LSE) views of its pinned host buffers."""
+        if ticket < self.count - len(self.slots):
+            raise ValueError("that step's buffers have been reused")
+        slot = self.slots[ticket % len(self.slots)]
+        slot["ev_out"].synchronize()
+        return slot["o_h"][: slot["rows"]], slot["lse_h"][: slot["rows"]]
+
