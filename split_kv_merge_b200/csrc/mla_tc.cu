@@ -83,6 +83,7 @@ struct MArgs {
   const int32_t* cta_indptr;
   int num_pages, page_size, heads, hc, hg, q_tile;
   int gather;  // page size 1: token rows fetched with 16-byte cp.async by four warps
+  int block_box;  // page size a multiple of 64: one 4-D box moves a whole 128-dim ckv block
   const uint8_t* ckv_rows;  // page size 1: row id i starts at ckv_rows + i * ckv_row_bytes
   const uint8_t* kpe_rows;
   int64_t ckv_row_bytes, kpe_row_bytes;
@@ -134,6 +135,15 @@ __device__ __forceinline__ void tma3(uint32_t dst, const CUtensorMap* map, uint3
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
       "[%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2,
+                                     int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 
@@ -368,6 +378,9 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             const uint32_t row_off = (uint32_t)(i * box_rows * 128);
             if (lane == 8) {
               tma3(sbase + C::kring + sk * kKSlot + row_off, &kpe_map, kfull_bar(sk), 0, slot0, page);
+            } else if (a.block_box) {  // one box per 128-dim block: both 64-column halves (fewer TMA issues)
+              if (lane < 4)
+                tma4(sbase + C::cring + sc[lane] * kCSlot, &ckv_map, cfull_bar(sc[lane]), 0, slot0, 2 * lane, page);
             } else if (lane < 8) {
               const int b = lane >> 1, hf = lane & 1;
               tma3(sbase + C::cring + sc[b] * kCSlot + hf * kHalf + row_off, &ckv_map, cfull_bar(sc[b]),
@@ -736,9 +749,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_m() {
 
 bool make_map_m(CUtensorMap* m, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
                 const cuuint32_t* box, int rank = 3) {
+  // rank 4 is the ckv block view (64 dims, slot, 64-dim chunk, page)
   auto fn = encode_fn_m();
   if (fn == nullptr) return false;
-  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -781,7 +795,15 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
     maps[0] = CUtensorMap{};
     maps[1] = CUtensorMap{};
   }
-  if (!gather) {
+  const bool block_box = !gather && p.page_size % kTile == 0;
+  if (block_box) {
+    // (64 dims, slot, 64-dim chunk, page): a box of 64 slots x 2 chunks is one 128-dim block, landing
+    // as its two 64-column swizzled halves one after the other
+    const cuuint64_t dims[4] = {64, (cuuint64_t)p.page_size, 8, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t st[3] = {(cuuint64_t)p.ckv_stride[1] * 2, 128, (cuuint64_t)p.ckv_stride[0] * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)kTile, 2, 1};
+    if (!make_map_m(&maps[0], p.ckv, dims, st, box, 4)) return (int)cudaErrorInvalidValue;
+  } else if (!gather) {
     const cuuint64_t dims[3] = {512, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
     const cuuint64_t st[2] = {(cuuint64_t)p.ckv_stride[1] * 2, (cuuint64_t)p.ckv_stride[0] * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
@@ -817,6 +839,7 @@ int launch_mla_tc(const skv_mla_params& p, const WorkItem* work, const int32_t* 
   a.hg = p.num_heads / hc;
   a.q_tile = q_tile;
   a.gather = gather ? 1 : 0;
+  a.block_box = block_box ? 1 : 0;
   a.ckv_rows = static_cast<const uint8_t*>(p.ckv);
   a.kpe_rows = static_cast<const uint8_t*>(p.kpe);
   a.ckv_row_bytes = p.ckv_stride[0] * 2;

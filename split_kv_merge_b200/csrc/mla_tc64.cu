@@ -85,6 +85,7 @@ struct M64Args {
   const int32_t* last;
   const int32_t* cta_indptr;  // per slice
   int num_pages, page_size, heads, hc, hg, q_tile, group;
+  int block_box;  // page size a multiple of 64: one 4-D box moves a whole 128-dim ckv block
   float scale_log2;
   void* o;
   float* lse;
@@ -126,6 +127,15 @@ __device__ __forceinline__ float redux_max(float v) {
   float r;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
+}
+
+__device__ __forceinline__ void tma4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1, int c2,
+                                     int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
 }
 
 template <typename OutT>
@@ -264,7 +274,9 @@ mla_tc64_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_consta
         for (int i = 0; i < npg; ++i) {
           const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
           if (lane == 0 && (unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
-          if (lane < 8) {
+          if (a.block_box) {  // one box per 128-dim block: both 64-column halves (fewer TMA issues)
+            if (lane < 4) tma4(sbase + C::cring + sc[lane] * kCSlot, &ckv_map, cfull_bar(sc[lane]), 0, slot0, 2 * lane, page);
+          } else if (lane < 8) {
             const int b = lane >> 1, hf = lane & 1;
             tc::tma_load_3d(sbase + C::cring + sc[b] * kCSlot + hf * kHalf + (uint32_t)(i * box_rows * 128), &ckv_map,
                             cfull_bar(sc[b]), b * 128 + hf * 64, slot0, page);
@@ -633,11 +645,11 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_m64() {
 }
 
 bool make_map_m64(CUtensorMap* m, const void* base, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
-                  const cuuint32_t* box) {
+                  const cuuint32_t* box, int rank = 3) {
   auto fn = encode_fn_m64();
   if (fn == nullptr) return false;
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides_bytes, box, estr,
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -672,7 +684,15 @@ int launch_mla_tc64(const skv_mla_params& p, const WorkItem* work, const int32_t
   const int box_rows = std::min(p.page_size, kTile);
   const int total_q = p.batch * p.q_len;
   CUtensorMap maps[4];
-  {
+  a.block_box = p.page_size % kTile == 0 ? 1 : 0;
+  if (a.block_box) {
+    // (64 dims, slot, 64-dim chunk, page): a box of 64 slots x 2 chunks is one 128-dim block, landing
+    // as its two 64-column swizzled halves one after the other
+    const cuuint64_t dims[4] = {64, (cuuint64_t)p.page_size, 8, (cuuint64_t)std::max(1, p.num_pages)};
+    const cuuint64_t st[3] = {(cuuint64_t)p.ckv_stride[1] * 2, 128, (cuuint64_t)p.ckv_stride[0] * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)kTile, 2, 1};
+    if (!make_map_m64(&maps[0], p.ckv, dims, st, box, 4)) return (int)cudaErrorInvalidValue;
+  } else {
     const cuuint64_t dims[3] = {512, (cuuint64_t)p.page_size, (cuuint64_t)std::max(1, p.num_pages)};
     const cuuint64_t st[2] = {(cuuint64_t)p.ckv_stride[1] * 2, (cuuint64_t)p.ckv_stride[0] * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
