@@ -59,6 +59,9 @@ constexpr int kRows = kHk * kTok;   // 128 = M of S^T
 constexpr int kD = 128;             // head dim = bytes per e4m3 row
 constexpr int kN = 64;              // query rows (columns of S^T): kHk * 8
 constexpr int kStages = 5;
+// work items of a CTA whose descriptors are staged in shared memory at kernel start, so no role
+// waits on dependent global loads (work item, then the request's page range) at a unit boundary
+constexpr int kUnitTab = 32;
 constexpr int kKBytes = kRows * kD;           // 16 KB per tensor per tile
 constexpr int kStageBytes = 2 * kKBytes;      // K + V
 constexpr int kQRegion = kN * 128;            // 8 KB: one 64-column bf16 half of the query copy
@@ -88,7 +91,8 @@ struct Smem {
   static constexpr int lsum = lse + kN * 4;                    // [2][64]
   static constexpr int msum = lsum + 2 * kN * 4;               // [2][64]
   static constexpr int qscale = msum + 2 * kN * 4;             // [2][64] float: 2^-e per query row, by unit parity
-  static constexpr int bars = qscale + 2 * kN * 4;
+  static constexpr int utab = qscale + 2 * kN * 4;             // [kUnitTab] work item descriptors
+  static constexpr int bars = utab + kUnitTab * 48;
   // ring, Q full / ready / ops empty, S full / empty (2 each), P full and O full (4 each), O free (2)
   static constexpr int nbars = 2 * kStages + 3 + 4 + 8 + 2;
   static constexpr int misc = bars + nbars * 8;
@@ -114,6 +118,8 @@ struct W8Args {
 struct WUnit8 {
   int r, q_start, q_count, page_begin, page_end, part_row, part_stride;
   int t0, t1, ntiles;
+  int ids_off;  // kv_indptr[r] + page_begin: the unit's first page id in kv_indices
+  int pad;
 };
 
 __device__ __forceinline__ WUnit8 load_wunit8(const W8Args& a, const WorkItem* work, int u) {
@@ -130,6 +136,8 @@ __device__ __forceinline__ WUnit8 load_wunit8(const W8Args& a, const WorkItem* w
   x.t0 = w.page_begin * a.page_size;
   x.t1 = min(w.page_end * a.page_size, L);
   x.ntiles = x.t1 > x.t0 ? (x.t1 - x.t0 + kTok - 1) / kTok : 0;
+  x.ids_off = a.kv_indptr[w.r] + w.page_begin;
+  x.pad = 0;
   return x;
 }
 
@@ -258,26 +266,36 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   for (int i = tid; i < 2 * kPBytes / 16; i += kThreads)
     reinterpret_cast<uint4*>(smem + Smem::p)[i] = make_uint4(0, 0, 0, 0);
   tc::fence_proxy_async_smem();
+  const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
+  WUnit8* utab = reinterpret_cast<WUnit8*>(smem + Smem::utab);
+  if (tid < min(kUnitTab, u_end - u_begin)) utab[tid] = load_wunit8(a, work, u_begin + tid);
   if (warp == kWarpQK) tc::tmem_alloc(tc::smem_u32(tmem_holder), kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t tm_s = tmem, tm_o = tmem + 2 * kN;  // O^T of (unit parity ob, group g): tm_o + (2 ob + g) kN
-
-  const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
+  auto unit = [&](int u) { return u - u_begin < kUnitTab ? utab[u - u_begin] : load_wunit8(a, work, u); };
+  // the next unit at or after u that has tiles (u_end if none)
+  auto next_with_tiles = [&](int u) {
+    while (u < u_end && unit(u).ntiles == 0) ++u;
+    return u;
+  };
   if (warp == kWarpTma) {
     // ======================================================================= TMA producer
     // Per unit: the query copy (once the previous unit's copy has been split), then the unit's
     // K/V tiles; lanes hold the page ids of the next 32 tiles while lane 0 issues.
     int n_tile = 0, n_unit = 0;
     bool ok = true;
+    bool have_pid = false;  // pid already holds this unit's first 32 page ids (fetched a unit ahead)
+    int pid = 0;
     for (int u = u_begin; u < u_end && ok; ++u) {
-      const WUnit8 x = load_wunit8(a, work, u);
+      const WUnit8 x = unit(u);
       if (x.ntiles == 0) continue;
-      const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
+      const int* ids = a.kv_indices + x.ids_off;
       const int tiles_per_page = a.page_size / kTok;
-      int pid = (lane < x.ntiles) ? __ldg(ids + lane * kTok / a.page_size) : 0;
+      if (!have_pid) pid = (lane < x.ntiles) ? __ldg(ids + lane * kTok / a.page_size) : 0;
+      have_pid = false;
       if (lane == 0) {
         if (n_unit >= 1) ok = tc::mbar_wait_sleep(qready_bar(), (n_unit - 1) & 1, abort_flag, a.status);
         if (ok) {
@@ -289,7 +307,15 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       for (int j0 = 0; j0 < x.ntiles && ok; j0 += 32) {
         const int jn = j0 + 32 + lane;
-        const int pid_next = (jn < x.ntiles) ? __ldg(ids + jn * kTok / a.page_size) : 0;
+        int pid_next = (jn < x.ntiles) ? __ldg(ids + jn * kTok / a.page_size) : 0;
+        if (j0 + 32 >= x.ntiles) {  // last batch: fetch the next unit's first page ids meanwhile
+          const int un = next_with_tiles(u + 1);
+          if (un < u_end) {
+            const WUnit8 xn = unit(un);
+            pid_next = (lane < xn.ntiles) ? __ldg(a.kv_indices + xn.ids_off + lane * kTok / a.page_size) : 0;
+            have_pid = true;
+          }
+        }
         const int nj = min(32, x.ntiles - j0);
         for (int jj = 0; jj < nj; ++jj) {
           const int j = j0 + jj, t = n_tile + j, st = t % kStages;
@@ -337,7 +363,7 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       bool ok = true;
       const uint32_t qo = sbase + Smem::qops;
       for (int u = u_begin; u < u_end && ok; ++u) {
-        const WUnit8 x = load_wunit8(a, work, u);
+        const WUnit8 x = unit(u);
         if (x.ntiles == 0) continue;
         ok = tc::mbar_wait(qready_bar(), n_unit & 1, abort_flag, a.status);
         if (!ok) break;
@@ -371,7 +397,7 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       int n_tile = 0, n_unit = 0;
       bool ok = true;
       for (int u = u_begin; u < u_end && ok; ++u) {
-        const WUnit8 x = load_wunit8(a, work, u);
+        const WUnit8 x = unit(u);
         if (x.ntiles == 0) continue;
         const int ob = n_unit & 1;
         // this unit's O^T pair was last read by the epilogue of unit n_unit - 2
@@ -475,17 +501,12 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(qready_bar());
     };
-    // the next unit at or after u that has tiles (u_end if none)
-    auto next_with_tiles = [&](int u) {
-      while (u < u_end && load_wunit8(a, work, u).ntiles == 0) ++u;
-      return u;
-    };
     // the first unit's query is split up front; every later one at the end of the previous unit's
     // tile loop, so its QKs start while that unit's last PV and epilogue are still running
     if (next_with_tiles(u_begin) < u_end) split_query(0);
     tc::named_bar_sync(3, 256);
     for (int u = u_begin; u < u_end && ok; ++u) {
-      const WUnit8 x = load_wunit8(a, work, u);
+      const WUnit8 x = unit(u);
       const int rows = x.q_count * G;      // valid columns per KV head
       if (x.ntiles == 0) {
         if (g == 0) {

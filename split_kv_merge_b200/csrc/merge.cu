@@ -29,16 +29,17 @@ merge_kernel(const float* __restrict__ o_states, const float* __restrict__ lse_s
   const int64_t row = blockIdx.x;
   const int h0 = blockIdx.y * hg;
   const int nh = min(hg, H - h0);
-  tc::grid_dependency_wait();  // the partials of the preceding attention grid are complete
-  int64_t out_row, base, jstride;
-  int S;
+  // a plan's merge items are written by the host before the attention launch, never by the
+  // preceding grid: read them before waiting on it, so only the partials' loads follow the wait
+  int64_t out_row = row, base = row, jstride = num_rows;
+  int S = num_states;
   if (items != nullptr) {
     const MergeItem it = items[row];
     out_row = it.out_row; base = it.state_begin; S = it.state_count; jstride = 1;
-  } else if (state_indptr != nullptr) {
-    out_row = row; base = state_indptr[row]; S = state_indptr[row + 1] - state_indptr[row]; jstride = 1;
-  } else {
-    out_row = row; base = row; S = num_states; jstride = num_rows;
+  }
+  tc::grid_dependency_wait();  // the partials of the preceding attention grid are complete
+  if (items == nullptr && state_indptr != nullptr) {
+    base = state_indptr[row]; S = state_indptr[row + 1] - state_indptr[row]; jstride = 1;
   }
   const int n4 = nh * D / 4;  // float4 of this block
   for (int e = threadIdx.x; e < n4; e += kMergeThreads) {
