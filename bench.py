@@ -265,12 +265,20 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def launch(run, ev=None):
+        # one skv_paged_attn_fwd call (attention, then the merge pass with programmatic dependent
+        # launch); with `ev`, the two phases as separate calls with `ev` recorded between them (an
+        # event between the kernels also ends the merge's early launch, so this form is used only
+        # to time the attention kernel alone)
         c, d = run["c"], run["d"]
+        if ev is None:
+            skv.paged_attn_fwd(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"], d["kv_last_page_len"],
+                               run["plan"], run["o"], run["lse"], run["o_part"], run["lse_part"], None, c.sm_scale,
+                               c.num_pages, stream)
+            return
         skv.paged_attn_fwd(d["q"], d["k"], d["v"], d["kv_indptr"], d["kv_indices"], d["kv_last_page_len"],
                            run["plan"], run["o"], run["lse"], run["o_part"], run["lse_part"], None, c.sm_scale,
                            c.num_pages, stream, phase="partial")
-        if ev is not None:
-            ev.record(stream)
+        ev.record(stream)
         skv.merge_plan(run["o_part"], run["lse_part"], run["plan"], c.num_qo_heads, c.head_dim, run["o"],
                        run["lse"], stream)
 
@@ -285,10 +293,14 @@ def run_ours(args):
             dist.barrier()
 
     # ---------------------------------------------------------------- device-timed region
+    # K steps of the public call (events only between runs), then -- for the roofline of the
+    # attention kernel -- the same K steps again as two phases with an event between them
     n_ev = args.steps * len(runs)
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     ev_c = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ra = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    rb = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    rc = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
@@ -299,16 +311,26 @@ def run_ours(args):
         for _ in range(args.steps):
             for run in runs:
                 ev_a[i].record(stream)
-                launch(run, ev_b[i])
+                launch(run)
                 ev_c[i].record(stream)
                 i += 1
         end.record(stream)
         torch.cuda.synchronize(dev)
+        barrier()
+        i = 0
+        for _ in range(args.steps):
+            for run in runs:
+                ra[i].record(stream)
+                launch(run, rb[i])
+                rc[i].record(stream)
+                i += 1
+        torch.cuda.synchronize(dev)
         time.sleep(0.1)
     barrier()
     total_ms = start.elapsed_time(end)
-    attn_ms = [ev_a[j].elapsed_time(ev_b[j]) for j in range(n_ev)]
-    merge_ms = [ev_b[j].elapsed_time(ev_c[j]) for j in range(n_ev)]
+    run_ms = [ev_a[j].elapsed_time(ev_c[j]) for j in range(n_ev)]
+    attn_ms = [ra[j].elapsed_time(rb[j]) for j in range(n_ev)]
+    merge_ms = [rb[j].elapsed_time(rc[j]) for j in range(n_ev)]
     total_ms, total_bytes = aggregate_over_ranks(total_ms, kv_bytes_step * args.steps, dev)
     value = total_bytes / (total_ms * 1e-3) / 1e9
     ms_per_step = total_ms / args.steps
@@ -336,10 +358,8 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": _config(cases, [r["plan"] for r in runs]),
         "us_per_step": round(ms_per_step * 1e3, 2),
-        "us_per_run": {"equal_strides": round(statistics.median(
-            [a + m for a, m in zip(attn_ms[0::2], merge_ms[0::2])]) * 1e3, 2),
-            "independent_v_strides": round(statistics.median(
-                [a + m for a, m in zip(attn_ms[1::2], merge_ms[1::2])]) * 1e3, 2)},
+        "us_per_run": {"equal_strides": round(statistics.median(run_ms[0::2]) * 1e3, 2),
+                       "independent_v_strides": round(statistics.median(run_ms[1::2]) * 1e3, 2)},
         "pct_hbm": {"of_nominal_8TBps": round(100 * value / ws / NOMINAL_HBM_GBS, 2),
                     f"of_{peak_src}_{hbm:.0f}GBps": round(100 * value / ws / hbm, 2)},
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
@@ -348,7 +368,11 @@ def run_ours(args):
                      "traffic": None if tr is None else tr["bytes_per_launch"],
                      "algorithmic_bytes_per_launch": int(per_launch_bytes),
                      "avg_launch_us": round(attn_avg_ms * 1e3, 2),
-                     "merge_avg_us": round(statistics.mean(merge_ms) * 1e3, 2)},
+                     "merge_avg_us": round(statistics.mean(merge_ms) * 1e3, 2),
+                     "how": "attention kernel timed with CUDA events around each of its launches in a second "
+                            "pass of the same steps right after the timed region (an event between the "
+                            "attention and merge kernels ends the merge's programmatic early launch, so the "
+                            "timed region itself records events only between runs)"},
         "e2e": e2e,
         "gpu_launches": args.steps * sum(1 + (1 if r["plan"].info.num_merge_rows > 0 else 0) for r in runs),
         "clocks": clk.summary(),
