@@ -435,7 +435,9 @@ def _e2e(args, runs, dev, stream, skv, torch):
             "h2d_bytes_per_step": h2d // steps, "d2h_bytes_per_step": d2h // steps,
             "ms_per_step": round(dt / steps * 1e3, 4),
             "how": "PagedDecodePipeline: host planning + pinned H2D of q, page table and plan + both phases + "
-                   "D2H of O and LSE every step; next step's host work and copies overlap this step's kernels"}
+                   "D2H of O and LSE every step; next step's host work and copies overlap this step's kernels, "
+                   "and the two runs of a step (one pipeline each, own streams) may overlap on the GPU where "
+                   "one kernel's tail leaves SMs free, which the device-timed region (one stream) does not do"}
 
 
 # ----------------------------------------------------------------------------- other configurations

@@ -145,7 +145,16 @@ skv_status plan_common(int32_t batch, const std::vector<ReqShape>& req, const st
         if (cta == G - 1) {
           b = n;
         } else {
-          while (b < n && (double)(qt * range_tiles(a, b + 1, kv_len[r], P, T)) <= room) ++b;
+          // the work of [a, b) grows with b: binary search for the last b that still fits
+          int32_t lo = a + 1, hi = n;
+          while (lo < hi) {
+            const int32_t mid = lo + (hi - lo + 1) / 2;
+            if ((double)(qt * range_tiles(a, mid, kv_len[r], P, T)) <= room)
+              lo = mid;
+            else
+              hi = mid - 1;
+          }
+          b = lo;
           if (qt * range_tiles(b, n, kv_len[r], P, T) < min_piece) b = n;  // no tiny remainder
         }
         const int64_t wt = qt * range_tiles(a, b, kv_len[r], P, T);

@@ -7,8 +7,9 @@ from typing import Optional
 
 import numpy as np
 
-from . import (OK, ERR_WORKSPACE, Plan, PlanInfo, _POLICY, _check, _plan_paged, _ptr_i32, causal_tables,
-               mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged, plan_paged_subset, pod_attn_fwd)
+from . import (OK, ERR_WORKSPACE, Plan, PlanInfo, _POLICY, _check, _paged_fwd, _paged_params, _plan_paged, _ptr_i32,
+               causal_tables, mla_decode_fwd, merge_states, paged_attn_fwd, plan_mla, plan_paged, plan_paged_subset,
+               pod_attn_fwd)
 
 
 def _dev_i32(a, device, non_blocking=False):
@@ -364,17 +365,19 @@ class PagedDecodePipeline:
 
     ``submit`` takes one step's query (a pinned host bf16 tensor [rows, Hq, D]) and page table
     (host int arrays), plans it on the host (``skv_plan_paged`` written straight into a pinned
-    plan buffer), copies query, page table and plan to the device on an input stream, runs the
-    attention and merge passes on a compute stream and copies O and LSE back into pinned host
-    buffers on an output stream; it returns a ticket and does not wait.  ``depth`` sets of host and
-    device buffers alternate, so the host planning and the copies of the next steps overlap the
-    kernels of the current one; ``result(ticket)`` waits for that step's output copy and returns
-    views of its pinned O and LSE (valid until the same buffer set is reused, ``depth`` submits
-    later).  Nothing is allocated per step once the buffers have grown to the largest step."""
+    buffer, followed there by the page table), copies query and [plan | page table] to the device
+    on an input stream (two copies), runs the attention and merge passes on a compute stream
+    (one ``skv_paged_attn_fwd`` call on launch arguments kept per buffer set) and copies O and LSE
+    back into pinned host buffers on an output stream; it returns a ticket and does not wait.
+    ``depth`` sets of host and device buffers alternate, so the host planning and the copies of
+    the next steps overlap the kernels of the current one; ``result(ticket)`` waits for that
+    step's output copy and returns views of its pinned O and LSE (valid until the same buffer set
+    is reused, ``depth`` submits later).  Nothing is allocated per step once the buffers have
+    grown to the largest step."""
 
     def __init__(self, k_cache, v_cache, num_qo_heads: int, *, max_rows: int, max_batch: int, max_page_ids: int,
                  sm_scale: Optional[float] = None, num_pages: Optional[int] = None, o_dtype=None, policy="balanced",
-                 param: int = 0, depth: int = 2, plan_words: int = 1 << 16):
+                 param: int = 0, depth: int = 2, plan_words: int = 1 << 14):
         import torch
         self.torch = torch
         self.k, self.v = k_cache, v_cache
@@ -385,43 +388,50 @@ class PagedDecodePipeline:
         self.policy = _POLICY[policy] if isinstance(policy, str) else int(policy)
         self.param = param
         self.o_dtype = o_dtype or torch.float32
+        self.max_rows, self.max_batch, self.max_page_ids = max_rows, max_batch, max_page_ids
         self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.p_in, self.p_run, self.p_out = (int(s.cuda_stream) for s in (self.s_in, self.s_run, self.s_out))
         pin = dict(pin_memory=True)
         self.slots = []
         for _ in range(depth):
             slot = dict(
-                plan_h=torch.empty(plan_words, dtype=torch.int32, **pin),
-                tab_h=[torch.empty(n, dtype=torch.int32, **pin) for n in (max_batch + 1, max_page_ids, max_batch)],
                 o_h=torch.empty(max_rows, num_qo_heads, self.d, dtype=self.o_dtype, **pin),
                 lse_h=torch.empty(max_rows, num_qo_heads, dtype=torch.float32, **pin),
                 q=torch.empty(max_rows, num_qo_heads, self.d, dtype=torch.bfloat16, device=dev),
-                plan=torch.empty(plan_words, dtype=torch.int32, device=dev),
-                tab=[torch.empty(n, dtype=torch.int32, device=dev) for n in (max_batch + 1, max_page_ids, max_batch)],
                 o=torch.empty(max_rows, num_qo_heads, self.d, dtype=self.o_dtype, device=dev),
                 lse=torch.empty(max_rows, num_qo_heads, dtype=torch.float32, device=dev),
                 o_part=torch.empty(0, device=dev), lse_part=torch.empty(0, device=dev),
                 ev_in=torch.cuda.Event(), ev_run=torch.cuda.Event(), ev_out=torch.cuda.Event(), rows=0, used=False)
+            self._size_inputs(slot, plan_words)
             self.slots.append(slot)
         self.count = 0
         self.h2d_bytes = self.d2h_bytes = 0
 
-    def _plan_into(self, slot, qo, ki, la):
-        """skv_plan_paged straight into the slot's pinned plan buffer (grown if too small)."""
-        b = len(ki) - 1
-        info = PlanInfo()
-        while True:
-            buf = slot["plan_h"]
-            code = _plan_paged(b, _ptr_i32(qo), _ptr_i32(ki), _ptr_i32(la), self.P, self.hq, self.hk, self.d,
-                               self.policy, self.param, None, None,
-                               ctypes.cast(ctypes.c_void_p(buf.data_ptr()), ctypes.POINTER(ctypes.c_int32)),
-                               buf.numel(), ctypes.byref(info))
-            if code == OK:
-                return info
-            if code != ERR_WORKSPACE:
-                _check(code, "skv_plan_paged")
-            n = max(info.plan_words, 2 * buf.numel())
-            slot["plan_h"] = self.torch.empty(n, dtype=self.torch.int32, pin_memory=True)
-            slot["plan"] = self.torch.empty(n, dtype=self.torch.int32, device=self.dev)
+    @staticmethod
+    def _align(n: int) -> int:
+        return (n + 15) & ~15  # 64-byte segments
+
+    def _size_inputs(self, slot, plan_cap: int):
+        """(Re)allocate the slot's pinned [plan | kv_indptr | kv_indices | last] buffer and its
+        device twin for a plan of up to plan_cap words; launch arguments are rebuilt."""
+        torch = self.torch
+        n = (self._align(plan_cap) + self._align(self.max_batch + 1) + self._align(self.max_page_ids)
+             + self._align(self.max_batch))
+        slot["in_h"] = torch.empty(n, dtype=torch.int32, pin_memory=True)
+        slot["in_np"] = slot["in_h"].numpy()
+        slot["in_d"] = torch.empty(n, dtype=torch.int32, device=self.dev)
+        slot["plan_cap"] = plan_cap
+        slot["params"] = None
+
+    def _params(self, slot):
+        """Launch arguments of the slot's fixed device buffers (built once, pointers patched per step)."""
+        if slot["params"] is None:
+            in_d = slot["in_d"]
+            slot["params"] = _paged_params(slot["q"], self.k, self.v, in_d[:2], in_d, in_d[:1], slot["o"], slot["lse"],
+                                           slot["o_part"] if slot["o_part"].numel() else None,
+                                           slot["lse_part"] if slot["lse_part"].numel() else None, None,
+                                           self.sm_scale, self.num_pages)
+        return slot["params"]
 
     def submit(self, q_h, qo_indptr_h, kv_indptr_h, kv_indices_h, kv_last_page_len_h) -> int:
         torch = self.torch
@@ -432,42 +442,53 @@ class PagedDecodePipeline:
                                                                                kv_last_page_len_h))
         kx = np.ascontiguousarray(np.asarray(kv_indices_h, dtype=np.int32))
         rows = q_h.shape[0]
-        if (rows > slot["o_h"].shape[0] or ki.size > slot["tab_h"][0].numel() or kx.size > slot["tab_h"][1].numel()
-                or la.size > slot["tab_h"][2].numel()):
+        if rows > self.max_rows or la.size > self.max_batch or kx.size > self.max_page_ids:
             raise ValueError("step larger than the pipeline's max_rows / max_batch / max_page_ids")
-        info = self._plan_into(slot, qo, ki, la)
+        b = len(ki) - 1
+        info = PlanInfo()
+        while True:  # plan straight into the front of the pinned input buffer
+            buf = slot["in_np"]
+            code = _plan_paged(b, _ptr_i32(qo), _ptr_i32(ki), _ptr_i32(la), self.P, self.hq, self.hk, self.d,
+                               self.policy, self.param, None, None, _ptr_i32(buf), slot["plan_cap"], ctypes.byref(info))
+            if code == OK:
+                break
+            if code != ERR_WORKSPACE:
+                _check(code, "skv_plan_paged")
+            self._size_inputs(slot, max(info.plan_words, 2 * slot["plan_cap"]))
         nw = max(1, info.plan_words)
-        np_views = [t.numpy() for t in slot["tab_h"]]
-        np_views[0][: ki.size] = ki
-        np_views[1][: kx.size] = kx
-        np_views[2][: la.size] = la
+        o_ki = self._align(nw)
+        o_kx = o_ki + self._align(ki.size)
+        o_la = o_kx + self._align(max(1, kx.size))
+        end = o_la + la.size
+        buf = slot["in_np"]
+        buf[o_ki: o_ki + ki.size] = ki
+        buf[o_kx: o_kx + kx.size] = kx
+        buf[o_la: end] = la
         n_part = info.num_partial_rows
         if n_part > slot["o_part"].shape[0]:  # grows to the largest plan seen, then stays
             slot["o_part"] = torch.empty(n_part, self.hq, self.d, dtype=torch.float32, device=self.dev)
             slot["lse_part"] = torch.empty(n_part, self.hq, dtype=torch.float32, device=self.dev)
+            slot["params"] = None
+        p = self._params(slot)
+        base = slot["in_d"].data_ptr()
+        p.kv_indptr, p.kv_indices, p.kv_last_page_len = base + 4 * o_ki, base + 4 * o_kx, base + 4 * o_la
+        p.batch, p.total_q = b, rows
+        if slot["used"]:
+            self.s_in.wait_event(slot["ev_run"])  # the slot's device buffers are free again
         with torch.cuda.stream(self.s_in):
-            if slot["used"]:
-                self.s_in.wait_event(slot["ev_run"])  # the device buffers are free again
             slot["q"][:rows].copy_(q_h, non_blocking=True)
-            for src, dst, n in zip(slot["tab_h"], slot["tab"], (ki.size, kx.size, la.size)):
-                dst[:n].copy_(src[:n], non_blocking=True)
-            slot["plan"][:nw].copy_(slot["plan_h"][:nw], non_blocking=True)
-            slot["ev_in"].record(self.s_in)
-        plan = Plan(slot["plan_h"][:nw].numpy(), info, slot["plan"][:nw])
-        with torch.cuda.stream(self.s_run):
-            self.s_run.wait_event(slot["ev_in"])
-            paged_attn_fwd(slot["q"][:rows], self.k, self.v, slot["tab"][0][: ki.size], slot["tab"][1][: max(1, kx.size)],
-                           slot["tab"][2][: la.size], plan, slot["o"][:rows], slot["lse"][:rows],
-                           slot["o_part"] if n_part else None, slot["lse_part"] if n_part else None, None,
-                           self.sm_scale, self.num_pages, self.s_run)
-            slot["ev_run"].record(self.s_run)
+            slot["in_d"][:end].copy_(slot["in_h"][:end], non_blocking=True)
+        slot["ev_in"].record(self.s_in)
+        self.s_run.wait_event(slot["ev_in"])
+        _check(_paged_fwd(ctypes.byref(p), base, ctypes.byref(info), self.p_run), "skv_paged_attn_fwd")
+        slot["ev_run"].record(self.s_run)
+        self.s_out.wait_event(slot["ev_run"])
         with torch.cuda.stream(self.s_out):
-            self.s_out.wait_event(slot["ev_run"])
             slot["o_h"][:rows].copy_(slot["o"][:rows], non_blocking=True)
             slot["lse_h"][:rows].copy_(slot["lse"][:rows], non_blocking=True)
-            slot["ev_out"].record(self.s_out)
+        slot["ev_out"].record(self.s_out)
         slot["used"], slot["rows"] = True, rows
-        self.h2d_bytes += q_h.numel() * q_h.element_size() + 4 * (ki.size + kx.size + la.size) + 4 * nw
+        self.h2d_bytes += q_h.numel() * q_h.element_size() + 4 * end
         self.d2h_bytes += rows * self.hq * (self.d * slot["o_h"].element_size() + 4)
         self.count += 1
         return self.count - 1

@@ -1,8 +1,8 @@
 """GPU parity of ``PagedDecodePipeline`` (the serving-loop helper: host planning into pinned buffers,
 input / compute / output streams, two alternating buffer sets): successive steps with different
 queries and page tables -- a step's host work and copies overlapping the previous step's kernels
--- give, step by step, the oracle's attention (O max-abs <= 1e-2, LSE <= 1e-3), and oversized
-steps are refused."""
+-- give, step by step, the oracle's attention (O max-abs <= 1e-2, LSE <= 1e-3), also when the
+pinned plan buffers start too small and grow, and oversized steps are refused."""
 import numpy as np
 import pytest
 import torch
@@ -17,7 +17,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def test_pipeline_steps_match_oracle():
+@pytest.mark.parametrize("plan_words", [1 << 14, 16])  # 16: the plan buffers grow on the first steps
+def test_pipeline_steps_match_oracle(plan_words):
     cases = [llama70b_decode_case(batch=b, seed=s, len_range=(200, 3000)) for b, s in ((6, 91), (9, 92), (6, 93), (3, 94))]
     # one cache holds every step's pages: steps use disjoint page ranges of a shared buffer
     offs = np.cumsum([0] + [c.num_pages for c in cases])
@@ -27,7 +28,7 @@ def test_pipeline_steps_match_oracle():
         k[o:o + c.num_pages] = bf16_tensor(c.k, DEV)
         v[o:o + c.num_pages] = bf16_tensor(c.v, DEV)
     pipe = skv.PagedDecodePipeline(k, v, 64, max_rows=9, max_batch=9, max_page_ids=max(len(c.kv_indices) for c in cases),
-                                   sm_scale=cases[0].sm_scale, num_pages=int(offs[-1]))
+                                   sm_scale=cases[0].sm_scale, num_pages=int(offs[-1]), plan_words=plan_words)
     qs = [torch.from_numpy(np.ascontiguousarray(c.q).view(np.int16)).view(torch.bfloat16).pin_memory() for c in cases]
     tickets = []
     results = {}
