@@ -232,6 +232,7 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& kmap, const CUtenso
         for (int jj = 0; jj < nj; ++jj) {
           const int j = j0 + jj, t = n_tile + j, st = t % kStages;
           const int page = __shfl_sync(0xffffffffu, pid, jj);
+          bool plain_wait = false;  // the slot wait without a pending Q copy: done by the whole warp
           if (lane == 0) {
             if (t >= kStages) {
               if (t - kStages >= n_tile) ok = flush_q();  // the slot holds a tile of this unit
@@ -251,9 +252,17 @@ __device__ __forceinline__ void wide_body(const CUtensorMap& kmap, const CUtenso
                   }
                 }
               } else if (ok) {
-                ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
+                plain_wait = true;
               }
             }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (__shfl_sync(0xffffffffu, plain_wait ? 1 : 0, 0)) {
+            // no lane waits alone while the others stand at a convergence point
+            ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
+            ok = __all_sync(0xffffffffu, ok);
+          }
+          if (lane == 0) {
             if (ok) {
               if ((unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
               const int slot0 = (j % tiles_per_page) * kTok;

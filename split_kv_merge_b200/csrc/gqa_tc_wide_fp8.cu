@@ -320,18 +320,18 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
         for (int jj = 0; jj < nj; ++jj) {
           const int j = j0 + jj, t = n_tile + j, st = t % kStages;
           const int page = __shfl_sync(0xffffffffu, pid, jj);
-          if (lane == 0) {
-            if (t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
-            if (ok) {
-              if ((unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
-              const int slot0 = (j % tiles_per_page) * kTok;
-              tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)kStageBytes);
-              const uint32_t kdst = sbase + Smem::kv + st * kStageBytes;
-              tma4(kdst, &kmap, full_bar(st), 0, slot0, 0, page);
-              tma4(kdst + kKBytes, &vmap, full_bar(st), 0, slot0, 0, page);
-            }
+          // the whole warp waits for the slot (no lane waits alone while the others stand at a
+          // convergence point); lane 0 posts the bytes and issues the two boxes
+          if (t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok && lane == 0) {
+            if ((unsigned)page >= (unsigned)a.num_pages) report(a.status, SKV_DEV_PAGE_OOB);
+            const int slot0 = (j % tiles_per_page) * kTok;
+            tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)kStageBytes);
+            const uint32_t kdst = sbase + Smem::kv + st * kStageBytes;
+            tma4(kdst, &kmap, full_bar(st), 0, slot0, 0, page);
+            tma4(kdst + kKBytes, &vmap, full_bar(st), 0, slot0, 0, page);
           }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
         }
         pid = pid_next;

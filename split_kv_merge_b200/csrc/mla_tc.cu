@@ -355,22 +355,24 @@ mla_tc_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_constant
             win = pi0;
             pid = (win + lane < npages) ? __ldg(ids + win + lane) : 0;
           }
-          // lane 0 claims the tile's kpe slot and its four ckv slots (waits + expected bytes); then
-          // nine lanes issue the nine TMA boxes at once (a single issuing thread serialises them)
+          // the whole warp waits for the tile's kpe slot and its four ckv slots (no lane waits
+          // alone while the others stand at a convergence point), lane 0 posts the expected bytes;
+          // then up to nine lanes issue the TMA boxes at once (a single issuing thread serialises them)
           const int sk = gk % NK;
           int sc[kBlocks];
 #pragma unroll
           for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
-          if (lane == 0) {
-            if (gk >= NK) ok = tc::mbar_wait_sleep(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
-            if (ok) tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(npg * box_rows * 128));
-            for (int b = 0; b < kBlocks && ok; ++b) {
-              const int g = gc + b;
-              if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
-              if (ok) tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * npg * box_rows * 128));
-            }
+          if (gk >= NK) ok = tc::mbar_wait_sleep(kempty_bar(sk), ((gk / NK) + 1) & 1, abort_flag, a.status);
+          for (int b = 0; b < kBlocks && ok; ++b) {
+            const int g = gc + b;
+            if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
           }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok && lane == 0) {
+            tc::mbar_arrive_expect_tx(kfull_bar(sk), (uint32_t)(npg * box_rows * 128));
+            for (int b = 0; b < kBlocks; ++b)
+              tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * npg * box_rows * 128));
+          }
           if (!ok) break;
           for (int i = 0; i < npg; ++i) {
             const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);

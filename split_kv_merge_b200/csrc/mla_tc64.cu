@@ -262,14 +262,15 @@ mla_tc64_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_consta
         int sc[kBlocks];
 #pragma unroll
         for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
-        if (lane == 0) {
-          for (int b = 0; b < kBlocks && ok; ++b) {
-            const int g = gc + b;
-            if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
-            if (ok) tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * npg * box_rows * 128));
-          }
+        // the whole warp waits for the slots (no lane waits alone while the others stand at a
+        // convergence point); lane 0 posts the expected bytes
+        for (int b = 0; b < kBlocks && ok; ++b) {
+          const int g = gc + b;
+          if (g >= NC) ok = tc::mbar_wait_sleep(cempty_bar(sc[b]), ((g / NC) + 1) & 1, abort_flag, a.status);
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && lane == 0)
+          for (int b = 0; b < kBlocks; ++b) tc::mbar_arrive_expect_tx(cfull_bar(sc[b]), (uint32_t)(2 * npg * box_rows * 128));
         if (!ok) break;
         for (int i = 0; i < npg; ++i) {
           const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);
@@ -283,11 +284,9 @@ mla_tc64_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_consta
           }
         }
         gc += kBlocks;
-        if (lane == 0) {
-          if (gk >= 1) ok = tc::mbar_wait_sleep(kempty_bar(), (gk + 1) & 1, abort_flag, a.status);
-          if (ok) tc::mbar_arrive_expect_tx(kfull_bar(), (uint32_t)(npg * box_rows * 128));
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (gk >= 1) ok = tc::mbar_wait_sleep(kempty_bar(), (gk + 1) & 1, abort_flag, a.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && lane == 0) tc::mbar_arrive_expect_tx(kfull_bar(), (uint32_t)(npg * box_rows * 128));
         if (!ok) break;
         for (int i = 0; i < npg; ++i) {
           const int page = __shfl_sync(0xffffffffu, pid, pi0 + i - win);

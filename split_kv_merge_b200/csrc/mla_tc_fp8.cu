@@ -266,11 +266,11 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
             pid = (win + lane < npages) ? __ldg(ids + win + lane) : 0;
           }
           const int st = g % NS;
-          if (lane == 0) {
-            if (g >= NS) ok = tc::mbar_wait_sleep(empty_bar(st), ((g / NS) + 1) & 1, abort_flag, a.status);
-            if (ok) tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(npg * box_rows * (4 * 128 + 64)));
-          }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          // the whole warp waits for the slot (no lane waits alone while the others stand at a
+          // convergence point); lane 0 posts the expected bytes
+          if (g >= NS) ok = tc::mbar_wait_sleep(empty_bar(st), ((g / NS) + 1) & 1, abort_flag, a.status);
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok && lane == 0) tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(npg * box_rows * (4 * 128 + 64)));
           if (!ok) break;
           const uint32_t tb = sbase + C::tiles + st * kTileBytes;
           for (int i = 0; i < npg; ++i) {  // five boxes per page, issued by five lanes at once
