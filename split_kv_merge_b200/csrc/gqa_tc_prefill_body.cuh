@@ -200,8 +200,10 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& kmap, const CUte
     int win = -1000000, pid = 0;  // lanes hold the ids of pages [win, win + 32) of the item
     for (int t = 0; t < T && ok; ++t) {
       const int st = t % kStages;
-      if (lane == 0 && t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      // the whole warp waits for the stage (no lane waits alone while the others stand at a
+      // convergence point)
+      if (t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       const int pi0 = (t * kTile) / P;
       const int npg = P >= kTile ? 1 : min(kTile / P, npages - pi0);
