@@ -5,7 +5,9 @@
 // (kpe), both stored as e4m3 with one per-tensor scale; s = sm_scale * kv_scale *
 // (q_nope . ckv + q_pe . kpe), V = kv_scale * ckv.  seqlen_q is folded into the row dimension as
 // in the bf16 kernel: rows n = qi * Hc + h of a unit, Hc = min(H, NR), F = q_tile tokens with
-// F * Hc <= NR; H > NR runs H / NR head groups.
+// F * Hc <= NR.  The (query tile, head group) units of a request -- q_len / F tiles times H / Hc
+// groups -- run on a group of that many co-resident CTAs that stream the same KV slice together
+// (as the 64-row bf16 kernel does), so the slice is read from HBM about once, not once per unit.
 //
 // B200 design: tcgen05.mma kind::f8f6f4 straight on the e4m3 cache tiles, so the cache is never
 // converted and a 64-token tile is 36 KB of shared memory (four or three of them in flight).
@@ -84,8 +86,9 @@ struct M8Args {
   const int32_t* kv_indptr;
   const int32_t* kv_indices;
   const int32_t* last;
-  const int32_t* cta_indptr;
+  const int32_t* cta_indptr;  // per KV slice
   int num_pages, page_size, heads, hc, hg, q_tile;
+  int group;                  // CTAs per KV slice: (q_len / q_tile) query tiles x hg head groups
   float scale_log2;                             // sm_scale * kv_scale * log2(e)
   float kv_scale;
   void* o;
@@ -100,15 +103,16 @@ struct MUnit8 {
   int t0, t1, ntiles;
 };
 
-__device__ __forceinline__ MUnit8 load_unit8(const M8Args& a, const WorkItem* work, int u) {
+// work item u as seen by the CTA of query tile qt of its group (the plan holds tile 0's item)
+__device__ __forceinline__ MUnit8 load_unit8(const M8Args& a, const WorkItem* work, int u, int qt) {
   MUnit8 x;
   const WorkItem w = work[u];
   x.r = w.r;
-  x.q_start = w.q_start;
+  x.q_start = w.q_start + qt * a.q_tile;
   x.q_count = w.q_count;
   x.page_begin = w.page_begin;
   x.page_end = w.page_end;
-  x.part_row = w.part_row;
+  x.part_row = w.part_row < 0 ? w.part_row : w.part_row + qt * a.q_tile * w.part_stride;
   x.part_stride = w.part_stride;
   const int L = request_len(a.kv_indptr, a.last, w.r, a.page_size);
   x.t0 = w.page_begin * a.page_size;
@@ -230,7 +234,11 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
   const uint32_t tmem = *tmem_holder;
   const uint32_t tm_s = tmem, tm_o = tmem + C::s_cols;
 
-  const int u_begin = a.cta_indptr[blockIdx.x], u_end = a.cta_indptr[blockIdx.x + 1];
+  // CTA c runs KV slice c / group for one (query tile, head group) unit, c % group: the group's
+  // CTAs stream the same pages at the same time, so each page comes from HBM about once
+  const int slice = (int)blockIdx.x / a.group, gsel = (int)blockIdx.x % a.group;
+  const int my_qt = gsel / a.hg, my_hg = gsel % a.hg;
+  const int u_begin = a.cta_indptr[slice], u_end = a.cta_indptr[slice + 1];
   const int P = a.page_size;
   const int box_rows = min(P, kTile);
 
@@ -239,11 +247,11 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
     int g = 0, n_unit = 0;
     bool ok = true;
     for (int u = u_begin; u < u_end && ok; ++u) {
-      const MUnit8 x = load_unit8(a, work, u);
+      const MUnit8 x = load_unit8(a, work, u, my_qt);
       if (x.ntiles == 0) continue;
       const int* ids = a.kv_indices + a.kv_indptr[x.r] + x.page_begin;
       const int npages = x.page_end - x.page_begin;
-      for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+      for (int hgi = my_hg; hgi == my_hg && ok; ++hgi) {
         if (lane == 0) {  // queries of this unit once the previous unit's copy has been split
           if (n_unit >= 1) ok = tc::mbar_wait_sleep(qready_bar(), (n_unit - 1) & 1, abort_flag, a.status);
           if (ok) {
@@ -311,9 +319,9 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
       bool ok = true;
       const uint32_t qo = sbase + C::qops;
       for (int u = u_begin; u < u_end && ok; ++u) {
-        const MUnit8 x = load_unit8(a, work, u);
+        const MUnit8 x = load_unit8(a, work, u, my_qt);
         if (x.ntiles == 0) continue;
-        for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+        for (int hgi = my_hg; hgi == my_hg && ok; ++hgi) {
           const int T = x.ntiles;
           ok = tc::mbar_wait_sleep(qready_bar(), n_unit & 1, abort_flag, a.status);
           if (ok) tc::tc_fence_after();
@@ -388,9 +396,9 @@ mla_tc_fp8_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_cons
       tc::tc_fence_after();
     };
     for (int u = u_begin; u < u_end && ok; ++u) {
-      const MUnit8 x = load_unit8(a, work, u);
+      const MUnit8 x = load_unit8(a, work, u, my_qt);
       const int rows = x.q_count * a.hc;
-      for (int hgi = 0; hgi < a.hg && ok; ++hgi) {
+      for (int hgi = my_hg; hgi == my_hg && ok; ++hgi) {
         const int h0 = hgi * a.hc;
         if (x.ntiles == 0) {  // no tokens: O = 0, LSE = -inf
           for (int n = 0; n < rows; ++n) {
@@ -773,6 +781,8 @@ int launch_mla_tc_fp8(const skv_mla_params& p, const WorkItem* work, const int32
   a.hc = hc;
   a.hg = p.num_heads / hc;
   a.q_tile = q_tile;
+  a.group = (p.q_len / q_tile) * a.hg;  // CTAs per KV slice, grid = slices x group
+  if (p.q_len % q_tile != 0 || num_ctas % a.group != 0) return (int)cudaErrorInvalidValue;
   a.kv_scale = p.kv_scale;
   a.scale_log2 = p.sm_scale * p.kv_scale * kLog2e;
   a.o = p.o;

@@ -19,13 +19,15 @@ def _items(plan):
     return plan.words[: 8 * nw].reshape(-1, 8), plan.words[8 * nw: 8 * nw + 4 * nm].reshape(-1, 4)
 
 
-def _grouped(plan, qo, num_heads):
-    """Work items as the CTAs run them.  A plan of the 64-row MLA kernel (kernel 14) lists query tile
-    0 of each piece only: the CTAs of a slice's group take query tile t = 0 .. q_len / q_tile - 1 by
-    shifting the item's rows by t * q_tile and its partial rows by t * q_tile * part_stride (every
-    head group of a tile runs the same rows).  Returns (items, CTAs per slice)."""
+def _grouped(plan, qo, num_heads, kv_dtype="bf16"):
+    """Work items as the CTAs run them.  A plan of the 64-row MLA kernel (kernel 14), or of the
+    e4m3 MLA kernels (12 / 13), lists query tile 0 of each piece only: the CTAs of a slice's group
+    take query tile t = 0 .. q_len / q_tile - 1 by shifting the item's rows by t * q_tile and its
+    partial rows by t * q_tile * part_stride (every head group of a tile runs the same rows).
+    Returns (items, CTAs per slice)."""
     w, _ = _items(plan)
-    if plan.info.kernel != 14:
+    rows = {12: 16, 13: 32, 14: 64}.get(plan.info.kernel, 0)
+    if not (plan.info.kernel == 14 or (rows and kv_dtype == "e4m3")):
         return w, 1
     q_len = int(qo[1] - qo[0]) if len(qo) > 1 else 0
     qt_count = q_len // plan.info.q_tile
@@ -36,13 +38,13 @@ def _grouped(plan, qo, num_heads):
         assert qs == qo[r] and qc == plan.info.q_tile   # query tile 0 of the request
         for t in range(qt_count):
             out.append([r, qs + t * qc, qc, pb, pe, prow + t * qc * pstride if prow >= 0 else prow, pstride, j])
-    group = qt_count * (num_heads // 64 if num_heads > 64 else 1)
+    group = qt_count * (num_heads // rows if num_heads > rows else 1)
     return np.array(out, dtype=np.int64).reshape(-1, 8), group
 
 
-def _check(plan, qo, n_pages, num_heads=0):
+def _check(plan, qo, n_pages, num_heads=0, kv_dtype="bf16"):
     info = plan.info
-    w, group = _grouped(plan, qo, num_heads)
+    w, group = _grouped(plan, qo, num_heads, kv_dtype)
     _, m = _items(plan)
     B = len(n_pages)
     part_owner = {}
@@ -137,7 +139,7 @@ def test_mla_plans(seed):
         n_pages = np.diff(kv_indptr)
         policy, param, sps = _policy(rng, n_pages)
         plan = skv.plan_mla(q_len, kv_indptr, last, P, H, policy, param, sps, kv_dtype=kv_dtype)
-        _check(plan, qo, n_pages, H)
+        _check(plan, qo, n_pages, H, kv_dtype)
 
 
 @pytest.mark.parametrize("seed", range(8))
