@@ -172,8 +172,8 @@ gqa_tc_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
   const int G = gridDim.x;
   if (warp == 4) {
     // ======================================================================= TMA producer
-    // The whole warp walks the units: lanes fetch the next tile's page ids (one per lane) while
-    // lane 0 waits for a free stage and issues the copies.
+    // The whole warp walks the units: lanes fetch the next tile's page ids (one per lane), the
+    // whole warp waits for a free stage, lane 0 issues the copies.
     const uint64_t pol = tc::policy_evict_first();
     const int ppt = kTile / a.page_size;  // pages per tile (<= 16)
     int n_tile = 0, n_unit = 0;
@@ -200,11 +200,10 @@ gqa_tc_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_cons
         const int npg = min(ppt, npages - j * ppt);
         const int nxt = (j + 1) * ppt;
         const int pid_next = (j + 1 < x.ntiles && lane < min(ppt, npages - nxt)) ? __ldg(ids + nxt + lane) : 0;
-        if (lane == 0) {
-          if (t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
-          if (ok) tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(npg * a.page_size * kD * 2 * 2));
-        }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        // no lane waits alone while the others stand at a convergence point
+        if (t >= kStages) ok = tc::mbar_wait(empty_bar(st), ((t / kStages) + 1) & 1, abort_flag, a.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && lane == 0) tc::mbar_arrive_expect_tx(full_bar(st), (uint32_t)(npg * a.page_size * kD * 2 * 2));
         if (!ok) break;
         const uint32_t kdst = sbase + Smem::kv + st * kStageBytes;
         const uint32_t vdst = kdst + kKBytes;

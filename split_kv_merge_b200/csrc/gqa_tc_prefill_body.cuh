@@ -181,9 +181,9 @@ __device__ __forceinline__ void prefill_body(const CUtensorMap& kmap, const CUte
   if (warp == 4) {
     // ======================================================================= TMA producer
     // The whole warp streams the tiles: lanes hold the ids of the next 32 pages of the item (one
-    // per lane), lane 0 claims the stage, and lane i issues the K and V boxes of page i of the tile
-    // (a 128-key tile of 16-token pages is eight pages: their boxes go out at once instead of one
-    // after another behind eight dependent page-id loads).
+    // per lane), the whole warp waits for the stage, and lane i issues the K and V boxes of page i
+    // of the tile (a 128-key tile of 16-token pages is eight pages: their boxes go out at once
+    // instead of one after another behind eight dependent page-id loads).
     bool ok = true;
     int issued = 0;
     if (lane == 0) {

@@ -284,7 +284,8 @@ gqa_tc_wide_fp8_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_co
   if (warp == kWarpTma) {
     // ======================================================================= TMA producer
     // Per unit: the query copy (once the previous unit's copy has been split), then the unit's
-    // K/V tiles; lanes hold the page ids of the next 32 tiles while lane 0 issues.
+    // K/V tiles; lanes hold the page ids of the next 32 tiles, the whole warp waits for a ring slot
+    // and lane 0 issues.
     int n_tile = 0, n_unit = 0;
     bool ok = true;
     bool have_pid = false;  // pid already holds this unit's first 32 page ids (fetched a unit ahead)

@@ -257,8 +257,9 @@ mla_tc64_kernel(const __grid_constant__ CUtensorMap ckv_map, const __grid_consta
           win = pi0;
           pid = (win + lane < npages) ? __ldg(ids + win + lane) : 0;
         }
-        // the four ckv slots first (lane 0 claims, eight lanes issue one box each per page), then
-        // the kpe slot, which frees only when the previous tile's QK is done
+        // the four ckv slots first (the whole warp waits, lane 0 posts the bytes, up to eight lanes
+        // issue one box each per page), then the kpe slot, which frees only when the previous
+        // tile's QK is done
         int sc[kBlocks];
 #pragma unroll
         for (int b = 0; b < kBlocks; ++b) sc[b] = (gc + b) % NC;
