@@ -467,7 +467,9 @@ skv_status skv_plan_mla(int32_t batch, int32_t q_len, const int32_t* kv_indptr_h
     const int32_t sms = device_sms(policy == SKV_SPLIT_BALANCED ? param : 0);
     po.flat_ctas = sms;
     po.tile_tokens = mla_tc_tile_tokens();
-    po.piece_cost = 4;  // measured: a work item's start and end cost about four 64-token tiles
+    // measured (bench A/B of the charge): a work item's start and end cost about four 64-token
+    // tiles on the e4m3 and 64-row kernels, about two on the bf16 16 / 32-row kernel
+    po.piece_cost = (kv_dtype == SKV_BF16 && nr < 64) ? 2 : 4;
     if (nr == 64 || kv_dtype == SKV_E4M3) {  // CTA groups per KV slice (64-row and e4m3 kernels)
       po.group = (int32_t)(head_groups * (q_len / fold));
       po.flat_ctas = std::max<int32_t>(1, sms / po.group);
