@@ -415,7 +415,7 @@ class PagedDecodePipeline:
         """(Re)allocate the slot's pinned [plan | kv_indptr | kv_indices | last] buffer and its
         device twin for a plan of up to plan_cap words; launch arguments are rebuilt."""
         torch = self.torch
-        n = (self._align(plan_cap) + self._align(self.max_batch + 1) + self._align(self.max_page_ids)
+        n = (self._align(plan_cap) + self._align(self.max_batch + 1) + self._align(max(1, self.max_page_ids))
              + self._align(self.max_batch))
         slot["in_h"] = torch.empty(n, dtype=torch.int32, pin_memory=True)
         slot["in_np"] = slot["in_h"].numpy()
