@@ -368,6 +368,7 @@ def test_paged_planner_kernel_choice(hq, hk, q_len, page_size, kernel, q_tile):
     (16, 2, "bf16", 64, 13), (96, 1, "bf16", 64, 13),   # 32 rows; 96 heads are no multiple of 64
     (16, 4, "bf16", 1, 13),                              # page size 1 takes at most 32 rows
     (16, 1, "e4m3", 64, 12), (128, 4, "e4m3", 64, 13),   # native fp8 tensor-core kernel
+    (128, 1, "e4m3", 64, 13), (16, 4, "e4m3", 64, 13),   # ... in CTA groups of 4 and 2 per KV slice
     (16, 1, "bf16", 1, 12),                              # page size 1: row gather on the tensor cores
     (16, 1, "e4m3", 1, 11),                              # e4m3 with page size 1: CUDA-core kernel
     (16, 1, "bf16", 4, 11),
@@ -379,17 +380,20 @@ def test_mla_planner_kernel_choice(H, q_len, kv_dtype, page_size, kernel):
     assert plan.info.kernel == kernel
     rows = {12: 16, 13: 32, 14: 64}.get(kernel, 128)
     assert plan.info.q_tile == (skv.mla_fold_ratio(H, q_len, rows) if H <= rows else 1)
-    if kernel == 14:   # a group of (query tiles x head groups) CTAs per KV slice
-        group = (q_len // plan.info.q_tile) * (H // 64 if H > 64 else 1)
+    if kernel == 14 or (kernel in (12, 13) and kv_dtype == "e4m3"):
+        # a group of (query tiles x head groups) CTAs per KV slice
+        group = (q_len // plan.info.q_tile) * (H // rows if H > rows else 1)
         assert plan.info.num_ctas % group == 0 and 1 <= plan.info.num_ctas // group <= 148 // group
+        w, _ = _items(plan)
+        assert np.all(w[:, 1] % q_len == 0)   # the items stand for query tile 0 of each request
 
 
 @pytest.mark.parametrize("H,q_len", [(16, 1), (16, 4), (128, 1), (128, 4)])
 def test_mla_flat_plan_balances_tiles_and_pieces(H, q_len):
-    """The persistent MLA plan charges every work item a fixed cost (four 64-token tiles per query
-    unit: head groups x query tiles) on top of its tiles; per CTA, tiles + charges stay within a
-    few tiles of the mean, every page of every request is covered once, and no CTA is left with
-    the remainder of a degenerate cut."""
+    """The persistent MLA plan charges every work item a fixed cost per query unit (head groups x
+    query tiles) on top of its tiles -- two 64-token tiles on the bf16 16 / 32-row kernel, four on
+    the 64-row kernel; per CTA, tiles + charges stay within a few tiles of the mean, every page of
+    every request is covered once, and no CTA is left with the remainder of a degenerate cut."""
     from workloads import mla_decode_case
     c = mla_decode_case(H, q_len, "bf16")
     plan = skv.plan_mla(q_len, c.kv_indptr, c.kv_last_page_len, 64, H, "balanced", 148, kv_dtype="bf16")
@@ -418,7 +422,8 @@ def test_mla_flat_plan_balances_tiles_and_pieces(H, q_len):
         # work items of one request piece differ only by query tile: count pieces once
         pieces = {(int(r), int(a), int(b)) for r, _, _, a, b, *_ in items}
         tiles = sum(-(-(min(b * 64, L[r]) - a * 64) // 64) for r, a, b in pieces)
-        cost.append(hg * tiles * -(-q_len_eff // info.q_tile) + 4 * qt * len(pieces))
+        charge = 4 if info.kernel == 14 else 2
+        cost.append(hg * tiles * -(-q_len_eff // info.q_tile) + charge * qt * len(pieces))
     cost = np.array(cost)
     assert cost.max() <= cost.mean() + 8 * qt + 8 * hg, (cost.max(), cost.mean())
     for r in range(c.batch):
